@@ -1,0 +1,461 @@
+/*
+ * blasst_oracle.c - plain, slow, fp64 CPU oracle for blocked attention with
+ * softmax thresholding. TEST INFRASTRUCTURE ONLY: the library and its kernels
+ * never call it; only the tests, the package's smoke check and the benchmark's
+ * CPU-baseline leg do.
+ *
+ * What it follows (citations name the web page and the paragraph on it; the
+ * paragraphs of the Telegram post are counted after its headline):
+ *
+ *   [T] "BLASST: Dynamic BLocked Attention Sparsity via Softmax Thresholding"
+ *       (Telegram channel seeallochnaya, post 3655):
+ *         para 2  - FlashAttention cuts the sequence into KV blocks and walks
+ *                   them left to right; the row max is subtracted before exp
+ *                   because softmax does not change under a shift.
+ *         para 3  - online softmax: keep the running max, compare each new
+ *                   block's local max with it, rescale the earlier partial
+ *                   results when it grows; after the last block the result is
+ *                   exact.
+ *         para 4  - FlashAttention 4 rescales lazily, only when precision is
+ *                   at risk; the result is still exact (ref_mode 1 below).
+ *         para 5  - BLASST: when a block's max is far below the max of the
+ *                   blocks before it, the block is dropped and its V vectors
+ *                   take no part in the computation.
+ *         para 6  - the figure: the first block is always processed.
+ *   [D] "BLASST wins Best Paper at MLSys 2026 ..." (digg.com/ai/al6mgdew),
+ *       the authors' announcement: one scalar threshold on the online-softmax
+ *       statistics decides the skip.
+ *
+ * The exact rule: a KV block is skipped when exp(m_blk - m_run) < lambda for
+ * every row of the query tile, where m_blk is the row's max score inside the
+ * block and m_run the row's running max over the blocks already computed.
+ * Readings taken where the pages are silent (listed with reasons in the
+ * design notes of the repository):
+ *   - scores are s = scale * q.k (natural units); the test is strict;
+ *   - a row with no valid key in the block votes "negligible";
+ *   - a skipped block adds nothing at all: not to m, not to l, not to O;
+ *   - blocks are visited in ascending order; block 0 of every query tile
+ *     (and of every decode split) is always computed;
+ *   - causal masking is bottom-right aligned: key j is visible from query
+ *     row i when j <= i + (Lkv - Lq);
+ *   - GQA maps query head hq to KV head hq / (Hq / Hkv);
+ *   - decode splits restart the running statistics at each split and are
+ *     combined by a log-sum-exp merge.
+ *
+ * Everything is computed in double. Inputs may be bf16 bit patterns, fp32 or
+ * fp64 and are widened exactly.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+enum { OR_BF16 = 0, OR_FP32 = 1, OR_FP64 = 2 };
+enum { MASK_COMPUTED = 0, MASK_SKIPPED = 1, MASK_NOT_VISITED = 2 };
+
+static double widen(const void *p, int dtype, int64_t i) {
+  if (dtype == OR_BF16) {
+    uint32_t u = (uint32_t)((const uint16_t *)p)[i] << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+  }
+  if (dtype == OR_FP32) return (double)((const float *)p)[i];
+  return ((const double *)p)[i];
+}
+
+static int resolve_threads(int n) {
+  if (n > 0) return n;
+  long c = sysconf(_SC_NPROCESSORS_ONLN);
+  return c > 0 ? (int)c : 1;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Prefill: one query tile of Br rows against the KV blocks of its head.     */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  const void *q, *k, *v;
+  int dtype;
+  int64_t B, Hq, Hkv, Lq, Lkv, d;
+  int causal;
+  double lambda;
+  int64_t Br, Bc;
+  double scale;
+  /* Reference point for the exponentials (shift invariance, [T] para 2/4):
+   *   0 - the running max itself (plain online softmax);
+   *   1 - lazy: the reference is moved to the running max only when the max
+   *       has grown past it by more than ref_param;
+   *   2 - fixed: the reference is the constant ref_param for the whole pass.
+   * The skip test always uses the exact running max. */
+  int ref_mode;
+  double ref_param;
+  const int64_t *items; /* flat tile ids (b*Hq + hq)*nQt + qt, or NULL = all */
+  int64_t n_items;
+  /* Outputs, one slot per listed item (item order):
+   *   o      [n_items, Br, d]
+   *   lse    [n_items, Br]       natural log; -inf for rows without keys
+   *   mask   [n_items, nKt]      0 computed, 1 skipped, 2 not visited
+   *   margin [n_items, nKt]      mu = max over rows of (m_blk - m_run),
+   *                              natural units; NaN where not visited
+   * Rows beyond Lq in a ragged last tile are left at 0. */
+  double *o, *lse;
+  uint8_t *mask;
+  double *margin;
+  int nthreads;
+} oracle_prefill_args;
+
+typedef struct {
+  const oracle_prefill_args *a;
+  int64_t next; /* shared work counter */
+  pthread_mutex_t mu;
+} prefill_ctx;
+
+static void prefill_tile(const oracle_prefill_args *a, int64_t slot,
+                         int64_t item, double *qrow, double *kblk,
+                         double *vblk, double *s, double *m, double *mref,
+                         double *l, double *acc, double *mb) {
+  const int64_t d = a->d, Br = a->Br, Bc = a->Bc;
+  const int64_t nQt = (a->Lq + Br - 1) / Br, nKt = (a->Lkv + Bc - 1) / Bc;
+  const int64_t g = a->Hq / a->Hkv;
+  const int64_t qt = item % nQt, bh = item / nQt;
+  const int64_t hq = bh % a->Hq, b = bh / a->Hq, hk = hq / g;
+  const int64_t r0 = qt * Br;
+  const int64_t r1 = r0 + Br < a->Lq ? r0 + Br : a->Lq;
+  const int64_t nr = r1 - r0;
+  const int64_t off = a->Lkv - a->Lq; /* bottom-right causal alignment */
+  const double log_lambda = a->lambda > 0.0 ? log(a->lambda) : -INFINITY;
+
+  /* Last KV block that holds a key visible from some row of the tile. */
+  int64_t kt_last = nKt - 1;
+  if (a->causal) {
+    int64_t last_key = (r1 - 1) + off;
+    if (last_key < 0) kt_last = -1;
+    else if (last_key / Bc < kt_last) kt_last = last_key / Bc;
+  }
+
+  const int64_t qbase = ((b * a->Hq + hq) * a->Lq) * d;
+  const int64_t kvbase = ((b * a->Hkv + hk) * a->Lkv) * d;
+  for (int64_t r = 0; r < nr; ++r)
+    for (int64_t x = 0; x < d; ++x)
+      qrow[r * d + x] = widen(a->q, a->dtype, qbase + (r0 + r) * d + x);
+
+  for (int64_t r = 0; r < Br; ++r) {
+    m[r] = -INFINITY;
+    mref[r] = -INFINITY;
+    l[r] = 0.0;
+    for (int64_t x = 0; x < d; ++x) acc[r * d + x] = 0.0;
+  }
+
+  uint8_t *mask = a->mask ? a->mask + slot * nKt : NULL;
+  double *margin = a->margin ? a->margin + slot * nKt : NULL;
+
+  /* [T] para 2: KV blocks are walked left to right. */
+  for (int64_t kt = 0; kt < nKt; ++kt) {
+    if (kt > kt_last) {
+      if (mask) mask[kt] = MASK_NOT_VISITED;
+      if (margin) margin[kt] = NAN;
+      continue;
+    }
+    const int64_t c0 = kt * Bc;
+    const int64_t c1 = c0 + Bc < a->Lkv ? c0 + Bc : a->Lkv;
+    const int64_t nc = c1 - c0;
+    for (int64_t j = 0; j < nc; ++j)
+      for (int64_t x = 0; x < d; ++x) {
+        kblk[j * d + x] = widen(a->k, a->dtype, kvbase + (c0 + j) * d + x);
+        vblk[j * d + x] = widen(a->v, a->dtype, kvbase + (c0 + j) * d + x);
+      }
+
+    /* Scores and the block's row max m_blk (the QK product is always
+     * formed: the block max cannot be known otherwise). */
+    double mu = -INFINITY;
+    for (int64_t r = 0; r < nr; ++r) {
+      mb[r] = -INFINITY;
+      for (int64_t j = 0; j < nc; ++j) {
+        int valid = !a->causal || (c0 + j) <= (r0 + r) + off;
+        double sv = -INFINITY;
+        if (valid) {
+          double dot = 0.0;
+          for (int64_t x = 0; x < d; ++x) dot += qrow[r * d + x] * kblk[j * d + x];
+          sv = a->scale * dot;
+        }
+        s[r * Bc + j] = sv;
+        if (sv > mb[r]) mb[r] = sv;
+      }
+      /* Row's distance to its running max; conventions for empty rows:
+       * a row with no valid key here votes "negligible" (-inf); a row that
+       * has seen no key yet but has one here is "not negligible" (+inf). */
+      double dr;
+      if (mb[r] == -INFINITY) dr = -INFINITY;
+      else if (m[r] == -INFINITY) dr = INFINITY;
+      else dr = mb[r] - m[r];
+      if (dr > mu) mu = dr;
+    }
+
+    /* [T] para 5 + [D]: skip when exp(m_blk - m_run) < lambda on every row,
+     * i.e. max_r (m_blk - m_run) < ln(lambda). [T] para 6: never block 0. */
+    int skip = (kt > 0) && (a->lambda > 0.0) && (mu < log_lambda);
+    if (mask) mask[kt] = skip ? MASK_SKIPPED : MASK_COMPUTED;
+    if (margin) margin[kt] = mu;
+    if (skip) continue; /* no V, no exp, no update of m, l or O */
+
+    /* [T] para 3: online softmax update with rescaling of earlier partials. */
+    for (int64_t r = 0; r < nr; ++r) {
+      if (mb[r] == -INFINITY) continue; /* nothing visible in this block */
+      double m_new = mb[r] > m[r] ? mb[r] : m[r];
+      double ref_new;
+      if (a->ref_mode == 2) ref_new = a->ref_param;
+      else if (a->ref_mode == 1)
+        ref_new = (mref[r] == -INFINITY || m_new > mref[r] + a->ref_param)
+                      ? m_new : mref[r];
+      else ref_new = m_new;
+      double alpha = (mref[r] == -INFINITY) ? 0.0 : exp(mref[r] - ref_new);
+      if (mref[r] == ref_new) alpha = 1.0;
+      l[r] *= alpha;
+      for (int64_t x = 0; x < d; ++x) acc[r * d + x] *= alpha;
+      for (int64_t j = 0; j < nc; ++j) {
+        double sv = s[r * Bc + j];
+        if (sv == -INFINITY) continue;
+        double p = exp(sv - ref_new);
+        l[r] += p;
+        for (int64_t x = 0; x < d; ++x) acc[r * d + x] += p * vblk[j * d + x];
+      }
+      m[r] = m_new;
+      mref[r] = ref_new;
+    }
+  }
+
+  /* Final normalisation; lse in natural log. */
+  for (int64_t r = 0; r < nr; ++r) {
+    double *orow = a->o ? a->o + (slot * Br + r) * d : NULL;
+    if (l[r] > 0.0) {
+      if (orow) for (int64_t x = 0; x < d; ++x) orow[x] = acc[r * d + x] / l[r];
+      if (a->lse) a->lse[slot * Br + r] = mref[r] + log(l[r]);
+    } else {
+      if (orow) for (int64_t x = 0; x < d; ++x) orow[x] = 0.0;
+      if (a->lse) a->lse[slot * Br + r] = -INFINITY;
+    }
+  }
+  for (int64_t r = nr; r < Br; ++r) {
+    if (a->o) for (int64_t x = 0; x < d; ++x) a->o[(slot * Br + r) * d + x] = 0.0;
+    if (a->lse) a->lse[slot * Br + r] = 0.0;
+  }
+}
+
+static void *prefill_worker(void *p) {
+  prefill_ctx *ctx = (prefill_ctx *)p;
+  const oracle_prefill_args *a = ctx->a;
+  const int64_t d = a->d, Br = a->Br, Bc = a->Bc;
+  double *qrow = malloc(sizeof(double) * Br * d);
+  double *kblk = malloc(sizeof(double) * Bc * d);
+  double *vblk = malloc(sizeof(double) * Bc * d);
+  double *s = malloc(sizeof(double) * Br * Bc);
+  double *acc = malloc(sizeof(double) * Br * d);
+  double *st = malloc(sizeof(double) * Br * 4);
+  if (!qrow || !kblk || !vblk || !s || !acc || !st) goto out;
+  for (;;) {
+    pthread_mutex_lock(&ctx->mu);
+    int64_t slot = ctx->next++;
+    pthread_mutex_unlock(&ctx->mu);
+    if (slot >= a->n_items) break;
+    int64_t item = a->items ? a->items[slot] : slot;
+    prefill_tile(a, slot, item, qrow, kblk, vblk, s, st, st + Br, st + 2 * Br,
+                 acc, st + 3 * Br);
+  }
+out:
+  free(qrow); free(kblk); free(vblk); free(s); free(acc); free(st);
+  return NULL;
+}
+
+int oracle_prefill(oracle_prefill_args *a) {
+  if (!a || a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Hq % a->Hkv ||
+      a->Lq <= 0 || a->Lkv <= 0 || a->d <= 0 || a->Br <= 0 || a->Bc <= 0 ||
+      a->lambda < 0.0 || a->lambda >= 1.0)
+    return -1;
+  const int64_t nQt = (a->Lq + a->Br - 1) / a->Br;
+  if (!a->items) a->n_items = a->B * a->Hq * nQt;
+  prefill_ctx ctx;
+  ctx.a = a;
+  ctx.next = 0;
+  pthread_mutex_init(&ctx.mu, NULL);
+  int nt = resolve_threads(a->nthreads);
+  if (nt > a->n_items) nt = (int)a->n_items;
+  if (nt < 1) nt = 1;
+  if (nt > 512) nt = 512;
+  pthread_t th[512];
+  int ok[512];
+  for (int t = 0; t < nt; ++t) ok[t] = pthread_create(&th[t], NULL, prefill_worker, &ctx) == 0;
+  for (int t = 0; t < nt; ++t) if (ok[t]) pthread_join(th[t], NULL);
+  /* Should every thread creation have failed, run inline. */
+  int any = 0;
+  for (int t = 0; t < nt; ++t) any |= ok[t];
+  if (!any) prefill_worker(&ctx);
+  pthread_mutex_destroy(&ctx.mu);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode: one query row per head, KV split into chunks, each chunk a pass   */
+/* of its own (running statistics restart), then a log-sum-exp merge.        */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  const void *q, *k, *v; /* q [B,Hq,1,d]; k, v [B,Hkv,Lkv,d] */
+  int dtype;
+  int64_t B, Hq, Hkv, Lkv, d;
+  double lambda;
+  int64_t Bc, num_splits;
+  double scale;
+  double *o_parts;   /* [B,Hq,S,d] normalised per split (0 for empty splits) */
+  double *lse_parts; /* [B,Hq,S] (-inf for empty splits) */
+  uint8_t *mask;     /* [B,Hq,nKt] */
+  double *margin;    /* [B,Hq,nKt] */
+  double *o, *lse;   /* merged: [B,Hq,d], [B,Hq] */
+  int nthreads;
+} oracle_decode_args;
+
+/* Keys per split: ceil(Lkv / S) rounded up to a whole number of blocks. */
+int64_t oracle_split_len(int64_t Lkv, int64_t Bc, int64_t S) {
+  int64_t per = (Lkv + S - 1) / S;
+  return ((per + Bc - 1) / Bc) * Bc;
+}
+
+void oracle_lse_merge(const double *o_parts, const double *lse_parts,
+                      int64_t n_rows, int64_t S, int64_t d, double *o,
+                      double *lse) {
+  for (int64_t r = 0; r < n_rows; ++r) {
+    double M = -INFINITY;
+    for (int64_t s = 0; s < S; ++s)
+      if (lse_parts[r * S + s] > M) M = lse_parts[r * S + s];
+    double wsum = 0.0;
+    for (int64_t x = 0; x < d; ++x) o[r * d + x] = 0.0;
+    if (M == -INFINITY) { lse[r] = -INFINITY; continue; }
+    for (int64_t s = 0; s < S; ++s) {
+      double ls = lse_parts[r * S + s];
+      double w = (ls == -INFINITY) ? 0.0 : exp(ls - M);
+      wsum += w;
+      for (int64_t x = 0; x < d; ++x) o[r * d + x] += w * o_parts[(r * S + s) * d + x];
+    }
+    for (int64_t x = 0; x < d; ++x) o[r * d + x] /= wsum;
+    lse[r] = M + log(wsum);
+  }
+}
+
+typedef struct {
+  const oracle_decode_args *a;
+  int64_t next;
+  pthread_mutex_t mu;
+} decode_ctx;
+
+static void decode_row_split(const oracle_decode_args *a, int64_t bh, int64_t sp,
+                             const double *qv, double *kv_k, double *kv_v,
+                             double *s, double *acc) {
+  const int64_t d = a->d, Bc = a->Bc, S = a->num_splits;
+  const int64_t nKt = (a->Lkv + Bc - 1) / Bc;
+  const int64_t g = a->Hq / a->Hkv;
+  const int64_t hq = bh % a->Hq, b = bh / a->Hq, hk = hq / g;
+  const int64_t Ls = oracle_split_len(a->Lkv, Bc, S);
+  const int64_t k0 = sp * Ls;
+  const int64_t k1 = k0 + Ls < a->Lkv ? k0 + Ls : a->Lkv;
+  const int64_t kvbase = ((b * a->Hkv + hk) * a->Lkv) * d;
+  const double log_lambda = a->lambda > 0.0 ? log(a->lambda) : -INFINITY;
+  double m = -INFINITY, l = 0.0;
+  for (int64_t x = 0; x < d; ++x) acc[x] = 0.0;
+  for (int64_t c0 = k0; c0 < k1; c0 += Bc) {
+    const int64_t kt = c0 / Bc;
+    const int64_t c1 = c0 + Bc < k1 ? c0 + Bc : k1;
+    const int64_t nc = c1 - c0;
+    double mb = -INFINITY;
+    for (int64_t j = 0; j < nc; ++j) {
+      double dot = 0.0;
+      for (int64_t x = 0; x < d; ++x) {
+        kv_k[j * d + x] = widen(a->k, a->dtype, kvbase + (c0 + j) * d + x);
+        dot += qv[x] * kv_k[j * d + x];
+      }
+      s[j] = a->scale * dot;
+      if (s[j] > mb) mb = s[j];
+    }
+    double mu = (m == -INFINITY) ? INFINITY : mb - m;
+    /* The first block of every split is always computed: the split starts
+     * its own pass with no running max. */
+    int skip = (c0 > k0) && (a->lambda > 0.0) && (mu < log_lambda);
+    if (a->mask) a->mask[bh * nKt + kt] = skip ? MASK_SKIPPED : MASK_COMPUTED;
+    if (a->margin) a->margin[bh * nKt + kt] = mu;
+    if (skip) continue;
+    for (int64_t j = 0; j < nc; ++j)
+      for (int64_t x = 0; x < d; ++x)
+        kv_v[j * d + x] = widen(a->v, a->dtype, kvbase + (c0 + j) * d + x);
+    double m_new = mb > m ? mb : m;
+    double alpha = (m == -INFINITY) ? 0.0 : exp(m - m_new);
+    l *= alpha;
+    for (int64_t x = 0; x < d; ++x) acc[x] *= alpha;
+    for (int64_t j = 0; j < nc; ++j) {
+      double p = exp(s[j] - m_new);
+      l += p;
+      for (int64_t x = 0; x < d; ++x) acc[x] += p * kv_v[j * d + x];
+    }
+    m = m_new;
+  }
+  double *op = a->o_parts + (bh * S + sp) * d;
+  if (l > 0.0) {
+    for (int64_t x = 0; x < d; ++x) op[x] = acc[x] / l;
+    a->lse_parts[bh * S + sp] = m + log(l);
+  } else {
+    for (int64_t x = 0; x < d; ++x) op[x] = 0.0;
+    a->lse_parts[bh * S + sp] = -INFINITY;
+  }
+}
+
+static void *decode_worker(void *p) {
+  decode_ctx *ctx = (decode_ctx *)p;
+  const oracle_decode_args *a = ctx->a;
+  const int64_t d = a->d, Bc = a->Bc, S = a->num_splits;
+  double *qv = malloc(sizeof(double) * d);
+  double *kk = malloc(sizeof(double) * Bc * d);
+  double *vv = malloc(sizeof(double) * Bc * d);
+  double *s = malloc(sizeof(double) * Bc);
+  double *acc = malloc(sizeof(double) * d);
+  const int64_t total = a->B * a->Hq * S;
+  if (!qv || !kk || !vv || !s || !acc) goto out;
+  for (;;) {
+    pthread_mutex_lock(&ctx->mu);
+    int64_t job = ctx->next++;
+    pthread_mutex_unlock(&ctx->mu);
+    if (job >= total) break;
+    int64_t bh = job / S, sp = job % S;
+    for (int64_t x = 0; x < d; ++x) qv[x] = widen(a->q, a->dtype, bh * d + x);
+    decode_row_split(a, bh, sp, qv, kk, vv, s, acc);
+  }
+out:
+  free(qv); free(kk); free(vv); free(s); free(acc);
+  return NULL;
+}
+
+int oracle_decode(oracle_decode_args *a) {
+  if (!a || a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Hq % a->Hkv ||
+      a->Lkv <= 0 || a->d <= 0 || a->Bc <= 0 || a->num_splits <= 0 ||
+      a->lambda < 0.0 || a->lambda >= 1.0 || !a->o_parts || !a->lse_parts)
+    return -1;
+  const int64_t nKt = (a->Lkv + a->Bc - 1) / a->Bc;
+  if (a->mask) memset(a->mask, MASK_NOT_VISITED, (size_t)(a->B * a->Hq * nKt));
+  decode_ctx ctx;
+  ctx.a = a;
+  ctx.next = 0;
+  pthread_mutex_init(&ctx.mu, NULL);
+  int64_t total = a->B * a->Hq * a->num_splits;
+  int nt = resolve_threads(a->nthreads);
+  if (nt > total) nt = (int)total;
+  if (nt > 512) nt = 512;
+  pthread_t th[512];
+  int ok[512], any = 0;
+  for (int t = 0; t < nt; ++t) { ok[t] = pthread_create(&th[t], NULL, decode_worker, &ctx) == 0; any |= ok[t]; }
+  for (int t = 0; t < nt; ++t) if (ok[t]) pthread_join(th[t], NULL);
+  if (!any) decode_worker(&ctx);
+  pthread_mutex_destroy(&ctx.mu);
+  if (a->o && a->lse)
+    oracle_lse_merge(a->o_parts, a->lse_parts, a->B * a->Hq, a->num_splits, a->d,
+                     a->o, a->lse);
+  return 0;
+}

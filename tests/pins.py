@@ -1,0 +1,359 @@
+"""Pins for the CPU oracle: checks against things the oracle does not compute
+itself (brute-force dense softmax attention written independently in numpy,
+closed-form error bounds, exact invariants of the method, a hand-worked
+example). Each ``pin_*`` raises AssertionError on failure; they take an
+``oracle.Oracle`` handle so the mutation test can run them against copies of
+the oracle with a planted mistake.
+
+Method statements these pins rest on ("BLASST: Dynamic BLocked Attention
+Sparsity via Softmax Thresholding", Telegram channel seeallochnaya, post 3655;
+paragraphs counted after the headline):
+  para 2/3 - blocked online softmax is exact once the last block is processed
+             (so lambda = 0 must give dense softmax attention);
+  para 2/4 - softmax is shift invariant, lazy rescaling keeps the result exact;
+  para 5   - a dropped block contributes nothing, its V is never used;
+  para 6   - the first block is always processed.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# --------------------------------------------------------------------------
+# Independent brute force: full score matrix, dense softmax, in float64.
+# --------------------------------------------------------------------------
+def dense_attention(q, k, v, causal, scale=None, keep=None):
+    """softmax(scale*Q K^T + mask) V over the full matrix. ``keep`` [B,Hq,Lq,Lkv]
+    optionally removes keys per row. Returns (o, lse)."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, Hq, Lq, d = q.shape
+    Hkv, Lkv = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    kk = np.repeat(k, g, axis=1)
+    vv = np.repeat(v, g, axis=1)
+    s = scale * np.einsum("bhid,bhjd->bhij", q, kk)
+    allowed = np.ones((Lq, Lkv), bool)
+    if causal:
+        i = np.arange(Lq)[:, None]
+        j = np.arange(Lkv)[None, :]
+        allowed = j <= i + (Lkv - Lq)
+    allowed = np.broadcast_to(allowed, s.shape)
+    if keep is not None:
+        allowed = allowed & keep
+    s = np.where(allowed, s, -np.inf)
+    m = s.max(-1, keepdims=True)
+    p = np.where(allowed, np.exp(s - m), 0.0)
+    lsum = p.sum(-1)
+    o = np.einsum("bhij,bhjd->bhid", p, vv) / lsum[..., None]
+    lse = m[..., 0] + np.log(lsum)
+    return o, lse
+
+
+def _dense_from(res):
+    import oracle
+    return oracle.prefill_dense(res)
+
+
+def rand_qkv(seed, B, Hq, Hkv, Lq, Lkv, d, planted=0.0, planted_blocks=(), Bc=16):
+    """fp64 inputs; optional planted direction on the query rows and on some
+    key blocks (to make the threshold skip actually fire)."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Hq, Lq, d))
+    k = rng.standard_normal((B, Hkv, Lkv, d))
+    v = rng.standard_normal((B, Hkv, Lkv, d))
+    if planted:
+        u = rng.standard_normal((B, Hkv, d))
+        u /= np.linalg.norm(u, axis=-1, keepdims=True)
+        g = Hq // Hkv
+        q += planted * np.repeat(u, g, axis=1)[:, :, None, :]
+        for blk in planted_blocks:
+            k[:, :, blk * Bc:(blk + 1) * Bc, :] += planted * u[:, :, None, :]
+    return q, k, v
+
+
+GEOMETRIES = [
+    # B, Hq, Hkv, Lq, Lkv, d, causal, Br, Bc
+    (1, 2, 2, 64, 64, 8, True, 16, 16),
+    (2, 4, 2, 100, 100, 8, True, 32, 16),     # GQA, ragged tail
+    (1, 2, 1, 37, 90, 8, True, 16, 32),       # Lq < Lkv, bottom-right causal
+    (1, 3, 3, 70, 130, 64, False, 32, 64),    # non-causal, ragged
+    (1, 2, 2, 256, 256, 64, True, 64, 64),
+    (1, 2, 2, 200, 200, 8, True, 64, 32),     # Br > Bc
+    (1, 2, 2, 1, 77, 8, False, 1, 16),        # one query row
+]
+
+
+def pin_lambda0_is_dense(orc):
+    """lambda = 0 never skips; blocked online softmax is then exactly dense
+    softmax attention (paras 2-3)."""
+    for n, (B, Hq, Hkv, Lq, Lkv, d, causal, Br, Bc) in enumerate(GEOMETRIES):
+        q, k, v = rand_qkv(100 + n, B, Hq, Hkv, Lq, Lkv, d, planted=2.0, planted_blocks=(0, 2), Bc=Bc)
+        res = orc.prefill(q, k, v, causal=causal, lam=0.0, Br=Br, Bc=Bc)
+        o, lse, mask, _ = _dense_from(res)
+        o_ref, lse_ref = dense_attention(q, k, v, causal)
+        assert np.all(mask != 1), "lambda=0 skipped a block"
+        np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-12)
+
+
+def _skipping_case(seed=7, d=16, L=256, Bc=16, Br=16, B=1, Hq=4, Hkv=2, causal=True, amp=6.0):
+    blocks = (0, 5, 11)
+    q, k, v = rand_qkv(seed, B, Hq, Hkv, L, L, d, planted=amp, planted_blocks=blocks, Bc=Bc)
+    return q, k, v, dict(causal=causal, Br=Br, Bc=Bc)
+
+
+def pin_first_block_always_computed(orc):
+    """para 6: block 0 of every query tile is processed, whatever lambda."""
+    q, k, v, kw = _skipping_case()
+    for lam in (1e-3, 0.5, 0.999):
+        res = orc.prefill(q, k, v, lam=lam, **kw)
+        assert np.all(res["mask"][:, 0] == 0)
+        assert np.any(res["mask"] == 1), "case did not skip anything"
+    # decode: every split starts with a computed block
+    qd = q[:, :, -1:, :]
+    S, Bc = 4, 16
+    out = orc.decode(qd, k, v, lam=0.5, Bc=Bc, num_splits=S)
+    Ls = orc.split_len(k.shape[2], Bc, S)
+    starts = [s * Ls // Bc for s in range(S) if s * Ls < k.shape[2]]
+    assert np.all(out["mask"][:, :, starts] == 0)
+    assert np.any(out["mask"] == 1)
+
+
+def _kept_keys(res, Lq, Lkv):
+    """Per-row key set implied by the oracle's own tile mask."""
+    B, Hq, Br, Bc, nQt, nKt = (res[x] for x in ("B", "Hq", "Br", "Bc", "nQt", "nKt"))
+    mask = res["mask"].reshape(B, Hq, nQt, nKt)
+    keep = np.zeros((B, Hq, Lq, Lkv), bool)
+    for qt in range(nQt):
+        for kt in range(nKt):
+            keep[:, :, qt * Br:(qt + 1) * Br, kt * Bc:(kt + 1) * Bc] = \
+                (mask[:, :, qt, kt] == 0)[:, :, None, None]
+    return keep
+
+
+def pin_kept_set_equivalence(orc):
+    """para 5: a skipped block contributes nothing. The output equals dense
+    softmax attention restricted to the kept blocks, exactly."""
+    for causal in (True, False):
+        q, k, v, kw = _skipping_case(causal=causal)
+        for lam in (1e-3, 1e-2, 0.2):
+            res = orc.prefill(q, k, v, lam=lam, **kw)
+            o, lse, mask, _ = _dense_from(res)
+            assert np.any(mask == 1)
+            keep = _kept_keys(res, q.shape[2], k.shape[2])
+            o_ref, lse_ref = dense_attention(q, k, v, causal, keep=keep)
+            np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-12)
+
+
+def pin_margins_independent_of_lambda(orc):
+    """A skipped block has m_blk < m_run on every row, so it would not have
+    moved the running max: the per-tile margins are the same for every lambda
+    in [0, 1) and the mask is [margin < ln lambda] (block 0 excepted), hence
+    monotone in lambda."""
+    q, k, v, kw = _skipping_case(seed=11)
+    base = orc.prefill(q, k, v, lam=0.0, **kw)
+    prev = None
+    for lam in (1e-6, 1e-4, 1e-3, 1e-2, 0.1, 0.5):
+        res = orc.prefill(q, k, v, lam=lam, **kw)
+        np.testing.assert_array_equal(res["margin"], base["margin"])
+        vis = res["mask"] != 2
+        pred = np.zeros_like(res["mask"])
+        mu = np.where(vis, base["margin"], 0.0)
+        pred[vis & (mu < np.log(lam))] = 1
+        pred[:, 0] = 0
+        pred[~vis] = 2
+        np.testing.assert_array_equal(res["mask"], pred)
+        if prev is not None:
+            assert np.all((prev == 1) <= (res["mask"] == 1)), "mask not monotone in lambda"
+        prev = res["mask"]
+
+
+def pin_shift_invariance(orc):
+    """paras 2/4: the reference point of the exponentials does not change the
+    result (lazy rescale with a large slack, or one fixed reference), and the
+    skip decisions are identical because they use the exact running max."""
+    q, k, v, kw = _skipping_case(seed=13)
+    for lam in (0.0, 1e-2):
+        a = orc.prefill(q, k, v, lam=lam, **kw)
+        for mode, par in ((1, 3.0), (1, 8.0), (2, 4.0)):
+            b = orc.prefill(q, k, v, lam=lam, ref_mode=mode, ref_param=par, **kw)
+            np.testing.assert_array_equal(a["mask"], b["mask"])
+            np.testing.assert_allclose(b["o"], a["o"], rtol=0, atol=1e-11)
+            np.testing.assert_allclose(b["lse"], a["lse"], rtol=0, atol=1e-11)
+
+
+def pin_permutation_invariance(orc):
+    """Reordering keys inside a block (with their values) or query rows
+    inside a tile (non-causal) changes nothing: the block max and the block's
+    sums do not depend on the order."""
+    q, k, v, kw = _skipping_case(seed=17, causal=False)
+    Bc, Br = kw["Bc"], kw["Br"]
+    rng = np.random.default_rng(5)
+    lam = 1e-2
+    a = orc.prefill(q, k, v, lam=lam, **kw)
+    perm = np.concatenate([blk * Bc + rng.permutation(Bc) for blk in range(k.shape[2] // Bc)])
+    b = orc.prefill(q, k[:, :, perm], v[:, :, perm], lam=lam, **kw)
+    np.testing.assert_array_equal(a["mask"], b["mask"])
+    np.testing.assert_allclose(b["o"], a["o"], rtol=0, atol=1e-12)
+    rperm = np.concatenate([t * Br + rng.permutation(Br) for t in range(q.shape[2] // Br)])
+    c = orc.prefill(q[:, :, rperm], k, v, lam=lam, **kw)
+    np.testing.assert_array_equal(a["mask"], c["mask"])
+    oa = _dense_from(a)[0]
+    oc = _dense_from(c)[0]
+    np.testing.assert_allclose(oc, oa[:, :, rperm], rtol=0, atol=1e-12)
+
+
+def pin_error_bound(orc):
+    """Every skipped score satisfies exp(s - m_final) <= exp(m_blk - m_run) <
+    lambda and the global row max lies in a kept block, so with n_skip(r)
+    skipped blocks of Bc keys: |O_lambda - O_exact| <= 2 max|v| lambda Bc
+    n_skip(r) and 0 <= lse_exact - lse_lambda <= -ln(1 - lambda Bc n_skip)."""
+    for causal in (True, False):
+        q, k, v, kw = _skipping_case(seed=19, causal=causal, amp=5.0)
+        o_ex, lse_ex = dense_attention(q, k, v, causal)
+        vmax = np.abs(v).max()
+        for lam in (1e-4, 1e-3, 1e-2):
+            res = orc.prefill(q, k, v, lam=lam, **kw)
+            o, lse, mask, _ = _dense_from(res)
+            Br = kw["Br"]
+            nskip = np.repeat((mask == 1).sum(-1), Br, axis=2)[:, :, : q.shape[2]]
+            bound = 2 * vmax * lam * kw["Bc"] * nskip
+            err = np.abs(o - o_ex).max(-1)
+            assert np.all(err <= bound + 1e-12), float((err - bound).max())
+            dl = lse_ex - lse
+            assert np.all(dl >= -1e-12)
+            frac = lam * kw["Bc"] * nskip
+            ok = frac < 1
+            assert np.all(dl[ok] <= -np.log1p(-frac[ok]) + 1e-12)
+
+
+def pin_gqa_replication(orc):
+    """Hq = g*Hkv with contiguous groups equals Hq = Hkv with each KV head
+    repeated g times (masks included)."""
+    q, k, v, kw = _skipping_case(seed=23, Hq=6, Hkv=2)
+    for lam in (0.0, 1e-2):
+        a = orc.prefill(q, k, v, lam=lam, **kw)
+        b = orc.prefill(q, np.repeat(k, 3, axis=1), np.repeat(v, 3, axis=1), lam=lam, **kw)
+        np.testing.assert_array_equal(a["mask"], b["mask"])
+        np.testing.assert_allclose(a["o"], b["o"], rtol=0, atol=0)
+
+
+def pin_decode_split_merge(orc):
+    """Split-KV decode: one split equals the single-row prefill pass; at
+    lambda = 0 any number of splits gives dense attention; merged partials
+    equal attention over the union of the splits' keys."""
+    q, k, v = rand_qkv(29, 2, 4, 2, 1, 300, 16, planted=5.0, planted_blocks=(0, 7, 12), Bc=16)
+    for lam in (0.0, 1e-3, 1e-1):
+        one = orc.decode(q, k, v, lam=lam, Bc=16, num_splits=1)
+        pre = orc.prefill(q, k, v, causal=False, lam=lam, Br=1, Bc=16)
+        np.testing.assert_array_equal(one["mask"].reshape(pre["mask"].shape), pre["mask"])
+        np.testing.assert_allclose(one["o"].reshape(-1, 16), pre["o"].reshape(-1, 16), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(one["lse"].reshape(-1), pre["lse"].reshape(-1), rtol=0, atol=1e-12)
+    o_ref, lse_ref = dense_attention(q, k, v, causal=False)
+    for S in (2, 3, 5, 19, 40):
+        out = orc.decode(q, k, v, lam=0.0, Bc=16, num_splits=S)
+        np.testing.assert_allclose(out["o"], o_ref[:, :, 0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(out["lse"], lse_ref[:, :, 0], rtol=0, atol=1e-12)
+        # each partial is dense attention over its own key range
+        Ls = orc.split_len(300, 16, S)
+        for s in range(S):
+            k0, k1 = s * Ls, min((s + 1) * Ls, 300)
+            if k0 >= k1:
+                assert np.all(out["lse_parts"][:, :, s] == -np.inf)
+                continue
+            op, lp = dense_attention(q, k[:, :, k0:k1], v[:, :, k0:k1], causal=False)
+            np.testing.assert_allclose(out["o_parts"][:, :, s], op[:, :, 0], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(out["lse_parts"][:, :, s], lp[:, :, 0], rtol=0, atol=1e-12)
+    # decode at lambda > 0: kept-set equivalence per split
+    S = 4
+    out = orc.decode(q, k, v, lam=1e-2, Bc=16, num_splits=S)
+    assert np.any(out["mask"] == 1)
+    keep = np.repeat(out["mask"] == 0, 16, axis=-1)[:, :, None, :300]
+    o_ref, lse_ref = dense_attention(q, k, v, causal=False, keep=keep)
+    # the merge over kept keys equals attention over all kept keys
+    np.testing.assert_allclose(out["o"], o_ref[:, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out["lse"], lse_ref[:, :, 0], rtol=0, atol=1e-12)
+
+
+def pin_lse_merge(orc):
+    """The log-sum-exp merge of partial softmax results over disjoint key sets
+    equals the softmax result over their union; empty parts (-inf) are ignored."""
+    rng = np.random.default_rng(31)
+    q, k, v = rand_qkv(37, 1, 3, 3, 1, 90, 8)
+    cuts = [0, 10, 10, 45, 90]
+    parts_o, parts_l = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        if a == b:
+            parts_o.append(np.zeros((1, 3, 8)))
+            parts_l.append(np.full((1, 3), -np.inf))
+            continue
+        o, l = dense_attention(q, k[:, :, a:b], v[:, :, a:b], causal=False)
+        parts_o.append(o[:, :, 0])
+        parts_l.append(l[:, :, 0])
+    o_parts = np.stack(parts_o, axis=2)
+    lse_parts = np.stack(parts_l, axis=2)
+    o, lse = orc.lse_merge(o_parts, lse_parts)
+    o_ref, lse_ref = dense_attention(q, k, v, causal=False)
+    np.testing.assert_allclose(o, o_ref[:, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref[:, :, 0], rtol=0, atol=1e-12)
+    del rng
+
+
+def pin_worked_example(orc):
+    """Hand-worked examples (tests/golden/skip_rule_worked_example.json): one
+    query row, d = 1, scores chosen by hand, expected masks derived on paper
+    from the rule, including an exact tie (a tie is computed: the test is
+    strict) and a row whose scores are all negative."""
+    with open(os.path.join(GOLDEN, "skip_rule_worked_example.json")) as f:
+        cases = json.load(f)["cases"]
+    for case in cases:
+        lam = case["lambda"]
+        keys = np.array(case["key_scores"], np.float64)
+        tie = case["tie_block"]
+        if tie:
+            # the tie block's max equals m_run + ln(lambda) exactly in double
+            keys[tie["index"] * case["Bc"]] = tie["running_max"] + np.log(lam)
+        L = keys.size
+        q = np.full((1, 1, 1, 1), 2.0)
+        k = keys.reshape(1, 1, L, 1)
+        v = np.array(case["values"], np.float64).reshape(1, 1, L, 1)
+        res = orc.prefill(q, k, v, causal=False, lam=lam, Br=1, Bc=case["Bc"], scale=0.5)
+        assert res["mask"][0].tolist() == case["expected_mask"], (case["name"], res["mask"][0].tolist())
+        kept = np.repeat(np.array(case["expected_mask"]) == 0, case["Bc"])
+        w = np.exp(keys[kept] - keys[kept].max())
+        o_ref = (w * v[0, 0, kept, 0]).sum() / w.sum()
+        lse_ref = keys[kept].max() + np.log(w.sum())
+        assert abs(res["o"][0, 0, 0] - o_ref) < 1e-14
+        assert abs(res["lse"][0, 0] - lse_ref) < 1e-14
+
+
+ALL_PINS = [
+    pin_lambda0_is_dense,
+    pin_first_block_always_computed,
+    pin_kept_set_equivalence,
+    pin_margins_independent_of_lambda,
+    pin_shift_invariance,
+    pin_permutation_invariance,
+    pin_error_bound,
+    pin_gqa_replication,
+    pin_decode_split_merge,
+    pin_lse_merge,
+    pin_worked_example,
+]
+
+
+def synth_small(name, **kw):
+    """A synthetic workload from the generator, shrunk for the CPU."""
+    return synth.CONFIGS[name].replace(**kw)
