@@ -1,0 +1,357 @@
+// blasst_capi.cu - the exported C ABI (include/blasst.h): argument checks,
+// TMA tensor maps, kernel selection and launch, the device error word.
+//
+// Single translation unit: the kernels are included here so that the error
+// word and every template instantiation live in one module.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/blasst.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+namespace {
+
+// Device error word: set (first error wins) by kernels whose bounded waits
+// gave up; read and cleared by blasst_check().
+__device__ int g_blasst_error = 0;
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+
+std::mutex g_mu;
+int* g_err_ptr[kMaxDevices] = {nullptr};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+// Address of the error word on the current device (looked up once per device).
+int* error_word() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_blasst_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int*>(ptr);
+  }
+  return g_err_ptr[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  return g_encode;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D map over a dense [heads, L, d] tensor: dims (d, L, heads), box
+// (64 columns, rows, 1), 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes,
+              int d, int L, int heads, int box_rows) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
+                           static_cast<cuuint64_t>(d) * elem_bytes * L};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes),
+                       static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int D, int BC, int BR>
+int launch_prefill_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const blasst::PrefillParams& p, cudaStream_t stream) {
+  using C = blasst::PrefillCfg<D, BC, BR>;
+  auto kernel = blasst::blasst_prefill_bf16_kernel<D, BC, BR>;
+  if (set_smem(kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
+  const dim3 grid(static_cast<unsigned>(p.nQblk) * p.B * p.Hq);
+  kernel<<<grid, 192, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? BLASST_OK : BLASST_ECUDA;
+}
+
+int dispatch_prefill_bf16(int d, int Bc, int Br, const CUtensorMap& mq, const CUtensorMap& mk,
+                          const CUtensorMap& mv, const blasst::PrefillParams& p,
+                          cudaStream_t s) {
+#define BLASST_PF(D_, BC_, BR_) \
+  if (d == D_ && Bc == BC_ && Br == BR_) return launch_prefill_bf16<D_, BC_, BR_>(mq, mk, mv, p, s);
+  BLASST_PF(128, 128, 128)
+  BLASST_PF(128, 128, 64)
+  BLASST_PF(128, 64, 128)
+  BLASST_PF(128, 64, 64)
+  BLASST_PF(64, 128, 128)
+  BLASST_PF(64, 128, 64)
+  BLASST_PF(64, 64, 128)
+  BLASST_PF(64, 64, 64)
+#undef BLASST_PF
+  return BLASST_EUNSUPPORTED;
+}
+
+template <int D, int BC, int G>
+int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const blasst::DecodeParams& p,
+                  cudaStream_t stream) {
+  using C = blasst::DecodeCfg<D, BC, G>;
+  auto kernel = blasst::blasst_decode_split_kernel<D, BC, G>;
+  if (set_smem(kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
+  const dim3 grid(p.S, p.Hkv, p.B);
+  kernel<<<grid, 128, C::SMEM_BYTES, stream>>>(mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? BLASST_OK : BLASST_ECUDA;
+}
+
+int dispatch_decode(int d, int Bc, int g, const CUtensorMap& mk, const CUtensorMap& mv,
+                    const blasst::DecodeParams& p, cudaStream_t s) {
+#define BLASST_DC(D_, BC_, G_) \
+  if (d == D_ && Bc == BC_ && g == G_) return launch_decode<D_, BC_, G_>(mk, mv, p, s);
+  BLASST_DC(128, 128, 1)
+  BLASST_DC(128, 128, 2)
+  BLASST_DC(128, 128, 4)
+  BLASST_DC(128, 128, 8)
+  BLASST_DC(128, 64, 1)
+  BLASST_DC(128, 64, 2)
+  BLASST_DC(128, 64, 4)
+  BLASST_DC(128, 64, 8)
+  BLASST_DC(64, 128, 1)
+  BLASST_DC(64, 128, 2)
+  BLASST_DC(64, 128, 4)
+  BLASST_DC(64, 128, 8)
+  BLASST_DC(64, 64, 1)
+  BLASST_DC(64, 64, 2)
+  BLASST_DC(64, 64, 4)
+  BLASST_DC(64, 64, 8)
+#undef BLASST_DC
+  return BLASST_EUNSUPPORTED;
+}
+
+float log2_lambda_of(float lambda) {
+  return lambda > 0.0f ? static_cast<float>(std::log2(static_cast<double>(lambda)))
+                       : -INFINITY;
+}
+
+}  // namespace
+
+extern "C" {
+
+int blasst_version(void) { return 100; }
+
+const char* blasst_status_string(int status) {
+  switch (status) {
+    case BLASST_OK: return "BLASST_OK";
+    case BLASST_EINVAL: return "BLASST_EINVAL: invalid argument";
+    case BLASST_EUNSUPPORTED: return "BLASST_EUNSUPPORTED: configuration not implemented";
+    case BLASST_ECUDA: return "BLASST_ECUDA: CUDA call failed";
+    case BLASST_ETIMEOUT: return "BLASST_ETIMEOUT: a device-side bounded wait gave up";
+    case BLASST_EWORKSPACE: return "BLASST_EWORKSPACE: workspace missing or too small";
+    default: return "BLASST: unknown status";
+  }
+}
+
+int blasst_fwd_ex(const blasst_fwd_args* a) {
+  if (!a) return BLASST_EINVAL;
+  if (!a->q || !a->k || !a->v || !a->o || !a->lse) return BLASST_EINVAL;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o) ||
+      !aligned16(a->lse))
+    return BLASST_EINVAL;
+  if (a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Lq <= 0 || a->Lkv <= 0) return BLASST_EINVAL;
+  if (a->Hq % a->Hkv != 0) return BLASST_EINVAL;
+  if (!(a->lambda >= 0.0f && a->lambda < 1.0f)) return BLASST_EINVAL;
+  if (a->d != 64 && a->d != 128) return BLASST_EUNSUPPORTED;
+  if ((a->Br != 64 && a->Br != 128) || (a->Bc != 64 && a->Bc != 128)) return BLASST_EUNSUPPORTED;
+  if (a->causal && a->Lq > a->Lkv) return BLASST_EUNSUPPORTED;
+  if (a->dtype != BLASST_BF16) return BLASST_EUNSUPPORTED;
+  if (static_cast<long long>(a->B) * a->Hq > (1ll << 24) ||
+      static_cast<long long>(a->B) * a->Hq * ((a->Lq + 127) / 128) > 0x7fffffffll)
+    return BLASST_EINVAL;
+
+  int* err = error_word();
+  if (!err) return BLASST_ECUDA;
+
+  blasst::PrefillParams p{};
+  p.o = a->o;
+  p.lse = a->lse;
+  p.mask = a->skip_mask_out;
+  p.stats = a->stats_out;
+  p.err = err;
+  p.B = a->B;
+  p.Hq = a->Hq;
+  p.Hkv = a->Hkv;
+  p.Lq = a->Lq;
+  p.Lkv = a->Lkv;
+  p.g = a->Hq / a->Hkv;
+  p.nQt = (a->Lq + a->Br - 1) / a->Br;
+  p.nKt = (a->Lkv + a->Bc - 1) / a->Bc;
+  p.nQblk = (a->Lq + 127) / 128;
+  p.causal = a->causal ? 1 : 0;
+  p.off = a->Lkv - a->Lq;
+  const double scale = a->scale > 0.0f ? static_cast<double>(a->scale)
+                                       : 1.0 / std::sqrt(static_cast<double>(a->d));
+  p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+  p.log2_lambda = log2_lambda_of(a->lambda);
+  p.timeout_ns = kTimeoutNs;
+
+  CUtensorMap mq, mk, mv;
+  const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&mq, a->q, dt, 2, a->d, a->Lq, a->B * a->Hq, 128) ||
+      !make_map(&mk, a->k, dt, 2, a->d, a->Lkv, a->B * a->Hkv, a->Bc) ||
+      !make_map(&mv, a->v, dt, 2, a->d, a->Lkv, a->B * a->Hkv, a->Bc))
+    return BLASST_ECUDA;
+  return dispatch_prefill_bf16(a->d, a->Bc, a->Br, mq, mk, mv, p,
+                               static_cast<cudaStream_t>(a->stream));
+}
+
+int blasst_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Lq, int Lkv, int d, int causal, float lambda, int Br, int Bc,
+               uint8_t* skip_mask_out) {
+  blasst_fwd_args a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Lq = Lq;
+  a.Lkv = Lkv;
+  a.d = d;
+  a.causal = causal;
+  a.lambda = lambda;
+  a.Br = Br;
+  a.Bc = Bc;
+  a.skip_mask_out = skip_mask_out;
+  a.dtype = BLASST_BF16;
+  a.scale = 0.0f;
+  a.stream = nullptr;
+  a.stats_out = nullptr;
+  return blasst_fwd_ex(&a);
+}
+
+size_t blasst_decode_workspace_bytes(int B, int Hq, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || d <= 0 || num_splits <= 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * Hq * num_splits;
+  const size_t o_bytes = rows * d * sizeof(float);
+  return o_bytes + rows * sizeof(float);
+}
+
+int blasst_lse_merge(const float* o_parts, const float* lse_parts, void* o, float* lse, int n_rows,
+                     int d, int num_splits, int out_dtype, void* stream) {
+  if (!o_parts || !lse_parts || !o || !lse || n_rows <= 0 || d <= 0 || num_splits <= 0)
+    return BLASST_EINVAL;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int threads = d >= 128 ? 128 : ((d + 31) / 32) * 32;
+  if (out_dtype == BLASST_BF16) {
+    blasst::blasst_lse_merge_kernel<__nv_bfloat16><<<n_rows, threads, 0, s>>>(
+        o_parts, lse_parts, static_cast<__nv_bfloat16*>(o), lse, d, num_splits);
+  } else if (out_dtype == BLASST_FP32) {
+    blasst::blasst_lse_merge_kernel<float><<<n_rows, threads, 0, s>>>(
+        o_parts, lse_parts, static_cast<float*>(o), lse, d, num_splits);
+  } else {
+    return BLASST_EINVAL;
+  }
+  return cudaGetLastError() == cudaSuccess ? BLASST_OK : BLASST_ECUDA;
+}
+
+int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                  int B, int Hq, int Hkv, int Lkv, int d, float lambda, int Bc, int num_splits,
+                  void* workspace, size_t workspace_bytes, uint8_t* skip_mask_out,
+                  blasst_stats* stats_out, void* stream) {
+  if (!q || !k_cache || !v_cache || !o || !lse) return BLASST_EINVAL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      !aligned16(lse))
+    return BLASST_EINVAL;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lkv <= 0 || num_splits <= 0) return BLASST_EINVAL;
+  if (Hq % Hkv != 0) return BLASST_EINVAL;
+  if (!(lambda >= 0.0f && lambda < 1.0f)) return BLASST_EINVAL;
+  if (d != 64 && d != 128) return BLASST_EUNSUPPORTED;
+  if (Bc != 64 && Bc != 128) return BLASST_EUNSUPPORTED;
+  const int g = Hq / Hkv;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return BLASST_EUNSUPPORTED;
+  if (num_splits > 65535 || B > 65535 || Hkv > 65535) return BLASST_EINVAL;
+  const size_t need = blasst_decode_workspace_bytes(B, Hq, d, num_splits);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return BLASST_EWORKSPACE;
+
+  int* err = error_word();
+  if (!err) return BLASST_ECUDA;
+
+  const size_t rows = static_cast<size_t>(B) * Hq * num_splits;
+  blasst::DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.o_parts = static_cast<float*>(workspace);
+  p.lse_parts = static_cast<float*>(workspace) + rows * d;
+  p.mask = skip_mask_out;
+  p.stats = stats_out;
+  p.err = err;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lkv = Lkv;
+  p.S = num_splits;
+  {
+    const long long per = (static_cast<long long>(Lkv) + num_splits - 1) / num_splits;
+    p.Ls = static_cast<int>(((per + Bc - 1) / Bc) * Bc);
+  }
+  p.nKt = (Lkv + Bc - 1) / Bc;
+  const double scale = 1.0 / std::sqrt(static_cast<double>(d));
+  p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+  p.log2_lambda = log2_lambda_of(lambda);
+  p.timeout_ns = kTimeoutNs;
+
+  CUtensorMap mk, mv;
+  const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&mk, k_cache, dt, 2, d, Lkv, B * Hkv, Bc) ||
+      !make_map(&mv, v_cache, dt, 2, d, Lkv, B * Hkv, Bc))
+    return BLASST_ECUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = dispatch_decode(d, Bc, g, mk, mv, p, s);
+  if (rc != BLASST_OK) return rc;
+  return blasst_lse_merge(p.o_parts, p.lse_parts, o, lse, B * Hq, d, num_splits, BLASST_BF16,
+                          stream);
+}
+
+int blasst_check(void* stream) {
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BLASST_ECUDA;
+  int* err = error_word();
+  if (!err) return BLASST_ECUDA;
+  int host = 0;
+  if (cudaMemcpy(&host, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return BLASST_ECUDA;
+  if (host != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return BLASST_ECUDA;
+  }
+  return host;
+}
+
+}  // extern "C"

@@ -1,0 +1,537 @@
+// prefill_sm100.cuh - forward prefill kernel for blocked attention with
+// softmax thresholding on sm_100a (tcgen05 + TMEM + TMA).
+//
+// Method ("BLASST: Dynamic BLocked Attention Sparsity via Softmax
+// Thresholding", Telegram channel seeallochnaya, post 3655, paragraphs 2-6
+// after the headline; "BLASST wins Best Paper at MLSys 2026 ...",
+// digg.com/ai/al6mgdew, the authors' announcement): KV blocks are walked
+// left to right with an online softmax; a block is dropped when
+// exp(m_blk - m_run) < lambda on every row of the query tile, in which case
+// its V is never loaded and no P.V product is formed; block 0 is always kept.
+// The lazy rescaling of FlashAttention 4 (paragraph 4) is used for the
+// output accumulator; the skip test always uses the exact running max.
+//
+// One CTA owns 128 query rows of one (batch, query head) and walks the KV
+// blocks of its KV head. Warp roles (192 threads):
+//   warps 0-3  softmax: thread t owns row t (TMEM lane t); row max, the vote,
+//              exp2, P -> TMEM, lazy O rescale, epilogue;
+//   warp 4     TMA producer: Q once, K ahead through a 3-stage ring, V only
+//              after the vote says the block is kept;
+//   warp 5     tcgen05 issuer: S = Q K^T into one of three TMEM S buffers,
+//              O += P V with P read from TMEM (P overwrites its S buffer).
+// With Br = 64 the 128 rows form two independent vote groups that share the
+// MMAs: a group that skips contributes zero rows of P and leaves its running
+// statistics untouched.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/blasst.h"
+#include "ptx_sm100.cuh"
+
+namespace blasst {
+
+struct PrefillParams {
+  void* o;
+  float* lse;
+  uint8_t* mask;
+  blasst_stats* stats;
+  int* err;
+  int B, Hq, Hkv, Lq, Lkv;
+  int g;      // Hq / Hkv
+  int nQt;    // ceil(Lq / Br)  (mask rows per head)
+  int nKt;    // ceil(Lkv / Bc)
+  int nQblk;  // ceil(Lq / 128) (CTAs per head)
+  int causal;
+  int off;    // Lkv - Lq
+  float scale_log2;   // scale * log2(e)
+  float log2_lambda;  // log2(lambda); -inf when lambda == 0
+  uint64_t timeout_ns;
+};
+
+constexpr int pow2_at_least(int x) {
+  int p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+template <int D, int BC, int BR>
+struct PrefillCfg {
+  static constexpr int BM = 128;
+  static constexpr int NG = BM / BR;   // vote groups
+  static constexpr int WPG = BR / 32;  // warps per vote group
+  static constexpr int NK = 3;
+  static constexpr int NV = 2;
+  static constexpr int NS = 3;
+  static constexpr int NSLOT = 4;
+  static constexpr int DBOX = D / 64;
+  static constexpr int Q_BOX = BM * 128;
+  static constexpr int KV_BOX = BC * 128;
+  static constexpr int Q_BYTES = Q_BOX * DBOX;
+  static constexpr int KV_BYTES = KV_BOX * DBOX;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NV * KV_BYTES;
+  // barrier indices
+  static constexpr int B_Q = 0;
+  static constexpr int B_KF = 1;
+  static constexpr int B_KE = B_KF + NK;
+  static constexpr int B_VF = B_KE + NK;
+  static constexpr int B_VE = B_VF + NV;
+  static constexpr int B_SF = B_VE + NV;
+  static constexpr int B_PV = B_SF + NS;
+  static constexpr int B_DEC = B_PV + NS;
+  static constexpr int B_P = B_DEC + NSLOT;
+  static constexpr int B_DRAIN = B_P + NSLOT;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  // misc words: [0] tmem base, [1] abort, [4..7] decisions, [8..15] votes
+  static constexpr int MISC_BYTES = 64;
+  static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+  static constexpr int S_COL = 0;        // S buffer b at column b * BC
+  static constexpr int O_COL = NS * BC;  // O accumulator
+  static constexpr int TMEM_COLS = pow2_at_least(NS * BC + D);
+  static constexpr uint32_t IDESC_QK = ptx::idesc_f32acc(1, 128, BC, false);
+  static constexpr uint32_t IDESC_PV = ptx::idesc_f32acc(1, 128, D, true);
+  static constexpr float TAU = 8.0f;  // lazy-rescale slack, log2 units
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(BC == 64 || BC == 128, "KV block");
+  static_assert(BR == 64 || BR == 128, "query tile");
+  static_assert(TMEM_COLS <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+__device__ __forceinline__ void record_error(int* err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+template <int D, int BC, int BR>
+__global__ void __launch_bounds__(192, 1)
+    blasst_prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
+                               const __grid_constant__ CUtensorMap tmK,
+                               const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+  using C = PrefillCfg<D, BC, BR>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = ptx::smem_u32(smem);
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = misc + 1;
+  volatile int* dec_val = misc + 4;
+  volatile int* votes = misc + 8;
+  auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: longest causal rows first ----------------------------
+  const int BH = p.B * p.Hq;
+  const int qblk = p.nQblk - 1 - static_cast<int>(blockIdx.x) / BH;
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int hq = bh % p.Hq;
+  const int b = bh / p.Hq;
+  const int bhk = b * p.Hkv + hq / p.g;
+  const int r0 = qblk * C::BM;
+
+  int kt_last[C::NG];
+  int nblk = 0;
+#pragma unroll
+  for (int gg = 0; gg < C::NG; ++gg) {
+    const int gr0 = r0 + gg * BR;
+    if (gr0 >= p.Lq) {
+      kt_last[gg] = -1;
+    } else {
+      const int gr1 = min(gr0 + BR, p.Lq);
+      int kl = p.nKt - 1;
+      if (p.causal) kl = min(kl, (gr1 - 1 + p.off) / BC);
+      kt_last[gg] = kl;
+    }
+    nblk = max(nblk, kt_last[gg] + 1);
+  }
+
+  // ---- set-up -------------------------------------------------------------
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar(C::B_Q), 1);
+    for (int i = 0; i < C::NK; ++i) {
+      ptx::mbar_init(bar(C::B_KF + i), 1);
+      ptx::mbar_init(bar(C::B_KE + i), 1);
+    }
+    for (int i = 0; i < C::NV; ++i) {
+      ptx::mbar_init(bar(C::B_VF + i), 1);
+      ptx::mbar_init(bar(C::B_VE + i), 1);
+    }
+    for (int i = 0; i < C::NS; ++i) {
+      ptx::mbar_init(bar(C::B_SF + i), 1);
+      ptx::mbar_init(bar(C::B_PV + i), 1);
+    }
+    for (int i = 0; i < C::NSLOT; ++i) {
+      ptx::mbar_init(bar(C::B_DEC + i), 1);
+      ptx::mbar_init(bar(C::B_P + i), 4);
+    }
+    ptx::mbar_init(bar(C::B_DRAIN), 1);
+    for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(ptx::smem_u32(const_cast<int*>(misc)), C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+
+  if (warp == 4) {
+    // ======================= TMA producer =================================
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmQ);
+      ptx::prefetch_tmap(&tmK);
+      ptx::prefetch_tmap(&tmV);
+      bool ok = true;
+      ptx::mbar_arrive_expect_tx(bar(C::B_Q), C::Q_BYTES);
+#pragma unroll
+      for (int bx = 0; bx < C::DBOX; ++bx)
+        ptx::tma_load_3d(sb + C::OFF_Q + bx * C::Q_BOX, &tmQ, bx * 64, r0, bh, bar(C::B_Q));
+      auto load_kv = [&](const CUtensorMap* tm, uint32_t dst, int blk, uint32_t fb) {
+        ptx::mbar_arrive_expect_tx(fb, C::KV_BYTES);
+#pragma unroll
+        for (int bx = 0; bx < C::DBOX; ++bx)
+          ptx::tma_load_3d(dst + bx * C::KV_BOX, tm, bx * 64, blk * BC, bhk, fb);
+      };
+      int kiss = 0;
+      for (; kiss < min(C::NK, nblk); ++kiss)
+        load_kv(&tmK, sb + C::OFF_K + kiss * C::KV_BYTES, kiss, bar(C::B_KF + kiss));
+      int vcount = 0;
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int slot = j % C::NSLOT;
+        ok = ptx::mbar_wait(bar(C::B_DEC + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        if (dec_val[slot] != 0) {
+          const int vs = vcount % C::NV;
+          if (vcount >= C::NV)
+            ok = ptx::mbar_wait(bar(C::B_VE + vs), ((vcount / C::NV) - 1) & 1, abort_flag,
+                                p.timeout_ns);
+          if (!ok) break;
+          load_kv(&tmV, sb + C::OFF_V + vs * C::KV_BYTES, j, bar(C::B_VF + vs));
+          ++vcount;
+        }
+        if (kiss < nblk) {
+          const int ks = kiss % C::NK;
+          ok = ptx::mbar_wait(bar(C::B_KE + ks), ((kiss / C::NK) - 1) & 1, abort_flag,
+                              p.timeout_ns);
+          if (!ok) break;
+          load_kv(&tmK, sb + C::OFF_K + ks * C::KV_BYTES, kiss, bar(C::B_KF + ks));
+          ++kiss;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_error(p.err, BLASST_ETIMEOUT);
+        // Let the copies already in flight land before the CTA exits.
+        ptx::mbar_wait(bar(C::B_Q), 0, abort_flag, p.timeout_ns);
+      }
+    }
+  } else if (warp == 5) {
+    // ======================= tcgen05 issuer ===============================
+    if (lane == 0) {
+      bool ok = ptx::mbar_wait(bar(C::B_Q), 0, abort_flag, p.timeout_ns);
+      ptx::tc_fence_after();
+      auto issue_qk = [&](int j) -> bool {
+        const int ks = j % C::NK;
+        if (!ptx::mbar_wait(bar(C::B_KF + ks), (j / C::NK) & 1, abort_flag, p.timeout_ns))
+          return false;
+        ptx::tc_fence_after();
+        const uint32_t d_tm = tmem + C::S_COL + (j % C::NS) * BC;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = ptx::sw128_desc(sb + C::OFF_Q + (kk >> 2) * C::Q_BOX + (kk & 3) * 32,
+                                             16, 1024);
+          const uint64_t bd = ptx::sw128_desc(
+              sb + C::OFF_K + ks * C::KV_BYTES + (kk >> 2) * C::KV_BOX + (kk & 3) * 32, 16, 1024);
+          ptx::mma_ss(d_tm, a, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar(C::B_KE + ks));
+        ptx::mma_commit(bar(C::B_SF + (j % C::NS)));
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      if (ok && nblk > 1) ok = issue_qk(1);
+      int pv_count = 0;
+      int pvn[C::NS] = {0, 0, 0};
+      bool kept_prev = false;
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int slot = j % C::NSLOT;
+        ok = ptx::mbar_wait(bar(C::B_P + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const bool keep = dec_val[slot] != 0;
+        if (keep) {
+          const int vs = pv_count % C::NV;
+          ok = ptx::mbar_wait(bar(C::B_VF + vs), (pv_count / C::NV) & 1, abort_flag,
+                              p.timeout_ns);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          const uint32_t p_tm = tmem + C::S_COL + (j % C::NS) * BC;
+#pragma unroll
+          for (int kk = 0; kk < BC / 16; ++kk) {
+            const uint64_t bd =
+                ptx::sw128_desc(sb + C::OFF_V + vs * C::KV_BYTES + kk * 2048, C::KV_BOX, 1024);
+            ptx::mma_ts(tmem + C::O_COL, p_tm + kk * 8, bd, C::IDESC_PV,
+                        (pv_count > 0 || kk > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(bar(C::B_VE + vs));
+          ptx::mma_commit(bar(C::B_PV + (j % C::NS)));
+          ++pvn[j % C::NS];
+          ++pv_count;
+        }
+        if (j + 2 < nblk) {
+          // S buffer (j+2)%3 last held block j-1: its P must have been read.
+          const int bp = (j + 2) % C::NS;
+          if (j >= 1 && kept_prev) {
+            ok = ptx::mbar_wait(bar(C::B_PV + bp), (pvn[bp] - 1) & 1, abort_flag, p.timeout_ns);
+            if (!ok) break;
+          }
+          ok = issue_qk(j + 2);
+        }
+        kept_prev = keep;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_error(p.err, BLASST_ETIMEOUT);
+      }
+      // Drain: every MMA issued above has completed before TMEM is freed.
+      ptx::mma_commit(bar(C::B_DRAIN));
+      ptx::mbar_wait(bar(C::B_DRAIN), 0, abort_flag, p.timeout_ns);
+    }
+  } else {
+    // ======================= softmax warps 0-3 ===========================
+    const int t = threadIdx.x;
+    const int row = r0 + t;
+    const bool row_exists = row < p.Lq;
+    const int gi = t / BR;
+    const int my_kt_last = kt_last[gi];
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int last_col = p.causal ? min(row + p.off, p.Lkv - 1) : p.Lkv - 1;
+    const float sl2 = p.scale_log2;
+    const bool thresholding = p.log2_lambda > -INFINITY;
+
+    float m = -INFINITY, mref = -INFINITY, l = 0.0f;
+    int pvn[C::NS] = {0, 0, 0};
+    int last_buf = -1, ncomp = 0;
+    unsigned long long st_vis = 0, st_skip = 0, st_vload = 0, st_flops = 0;
+    bool aborted = false;
+
+    for (int j = 0; j < nblk; ++j) {
+      const int sbuf = j % C::NS;
+      bool ok = true;
+      if (lane == 0) ok = ptx::mbar_wait(bar(C::B_SF + sbuf), (j / C::NS) & 1, abort_flag, p.timeout_ns);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ptx::tc_fence_after();
+
+      float s[BC];
+      float mb = -INFINITY;
+      bool rowskip = true;
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < BC / 32; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tmem + lane_base + C::S_COL + sbuf * BC + 32 * c, r);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[i]);
+        }
+        const int col0 = j * BC;
+        const bool need_mask = (col0 + BC > p.Lkv) || (p.causal && col0 + BC - 1 > r0 + p.off);
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < BC; ++c)
+            if (col0 + c > last_col) s[c] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BC; ++c) mx = fmaxf(mx, s[c]);
+        mb = mx * sl2;
+        const bool visited = j <= my_kt_last;
+        if (!row_exists || !visited) rowskip = true;
+        else if (j == 0 || !thresholding) rowskip = false;
+        else rowskip = (mb - m) < p.log2_lambda;
+      }
+      const unsigned all_skip = __all_sync(0xffffffffu, rowskip) ? 1u : 0u;
+      if (lane == 0) votes[(j & 1) * 4 + warp] = ok ? static_cast<int>(all_skip) : 2;
+      ptx::named_bar_sync(1, 128);
+      int keepmask = 0;
+      bool any_abort = false;
+#pragma unroll
+      for (int gg = 0; gg < C::NG; ++gg) {
+        bool gskip = true;
+#pragma unroll
+        for (int w = 0; w < C::WPG; ++w) {
+          const int v = votes[(j & 1) * 4 + gg * C::WPG + w];
+          if (v == 2) any_abort = true;
+          gskip = gskip && (v != 0);
+        }
+        if (j <= kt_last[gg] && !gskip) keepmask |= 1 << gg;
+      }
+      if (any_abort) {
+        aborted = true;
+        break;
+      }
+      if (t == 0) {
+        dec_val[j % C::NSLOT] = keepmask;
+        ptx::mbar_arrive(bar(C::B_DEC + (j % C::NSLOT)));
+        const unsigned long long tile_flops = 2ull * 128ull * BC * D;
+        st_flops += tile_flops + (keepmask ? tile_flops : 0ull);
+        st_vload += keepmask ? 1ull : 0ull;
+#pragma unroll
+        for (int gg = 0; gg < C::NG; ++gg) {
+          if (kt_last[gg] < 0) continue;
+          const int qt = r0 / BR + gg;
+          uint8_t code = 2;
+          if (j <= kt_last[gg]) {
+            ++st_vis;
+            code = ((keepmask >> gg) & 1) ? 0 : 1;
+            if (code == 1) ++st_skip;
+          }
+          if (p.mask) p.mask[(static_cast<size_t>(bh) * p.nQt + qt) * p.nKt + j] = code;
+        }
+      }
+      if (keepmask) {
+        const bool my_keep = (keepmask >> gi) & 1;
+        const float m_new = my_keep ? fmaxf(m, mb) : m;
+        const bool need = my_keep && (m_new > mref + C::TAU);
+        if (__any_sync(0xffffffffu, need)) {
+          const float mref_new = need ? m_new : mref;
+          if (ncomp > 0) {
+            // O must be quiescent: wait for the last issued P.V.
+            bool ok2 = true;
+            if (lane == 0)
+              ok2 = ptx::mbar_wait(bar(C::B_PV + last_buf), (pvn[last_buf] - 1) & 1, abort_flag,
+                                   p.timeout_ns);
+            ok2 = __shfl_sync(0xffffffffu, ok2 ? 1 : 0, 0) != 0;
+            if (!ok2) {
+              *abort_flag = 1;
+              record_error(p.err, BLASST_ETIMEOUT);
+            }
+            ptx::tc_fence_after();
+            const float alpha = need ? ptx::ex2(mref - mref_new) : 1.0f;
+            l *= alpha;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              const uint32_t ta = tmem + lane_base + C::O_COL + 32 * c;
+              ptx::tmem_ld32(ta, r);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              ptx::tmem_st32(ta, r);
+            }
+            ptx::tmem_wait_st();
+          }
+          mref = mref_new;
+        }
+        if (my_keep) m = m_new;
+
+        uint32_t pk[BC / 2];
+        if (my_keep) {
+          const float neg = -mref;
+          float rs = 0.0f;
+#pragma unroll
+          for (int c = 0; c < BC; c += 2) {
+            const float p0 = ptx::ex2(fmaf(s[c], sl2, neg));
+            const float p1 = ptx::ex2(fmaf(s[c + 1], sl2, neg));
+            rs += p0 + p1;
+            pk[c / 2] = ptx::pack_bf16x2(p0, p1);
+          }
+          l += rs;
+        } else {
+#pragma unroll
+          for (int c = 0; c < BC / 2; ++c) pk[c] = 0u;
+        }
+#pragma unroll
+        for (int c = 0; c < BC / 32; ++c)
+          ptx::tmem_st16(tmem + lane_base + C::S_COL + sbuf * BC + 16 * c, pk + 16 * c);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ++ncomp;
+        last_buf = sbuf;
+        ++pvn[sbuf];
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::B_P + (j % C::NSLOT)));
+    }
+
+    if (aborted) {
+      if (t == 0) {
+        *abort_flag = 1;
+        record_error(p.err, BLASST_ETIMEOUT);
+      }
+    } else {
+      // ---- epilogue: O / l -> bf16, lse, masks of unvisited blocks ------
+      bool ok = true;
+      if (ncomp > 0 && lane == 0)
+        ok = ptx::mbar_wait(bar(C::B_PV + last_buf), (pvn[last_buf] - 1) & 1, abort_flag,
+                            p.timeout_ns);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ptx::tc_fence_after();
+      if (!ok) {
+        *abort_flag = 1;
+        record_error(p.err, BLASST_ETIMEOUT);
+      } else {
+        const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
+                              (static_cast<size_t>(bh) * p.Lq + row) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tmem + lane_base + C::O_COL + 32 * c, r);
+          ptx::tmem_wait_ld();
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = ptx::pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
+                                    __uint_as_float(r[2 * i + 1]) * inv_l);
+          if (row_exists) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+        if (row_exists)
+          p.lse[static_cast<size_t>(bh) * p.Lq + row] = (mref + log2f(l)) * 0.6931471805599453f;
+        if (p.mask) {
+#pragma unroll
+          for (int gg = 0; gg < C::NG; ++gg) {
+            if (kt_last[gg] < 0) continue;
+            const int qt = r0 / BR + gg;
+            uint8_t* mrow = p.mask + (static_cast<size_t>(bh) * p.nQt + qt) * p.nKt;
+            for (int j = nblk + t; j < p.nKt; j += 128) mrow[j] = 2;
+          }
+        }
+        if (t == 0 && p.stats) {
+          const unsigned long long qbytes = 128ull * D * 2ull;
+          const unsigned long long kvb = static_cast<unsigned long long>(BC) * D * 2ull;
+          atomicAdd(&p.stats->tiles_visited, st_vis);
+          atomicAdd(&p.stats->tiles_skipped, st_skip);
+          atomicAdd(&p.stats->v_blocks_loaded, st_vload);
+          atomicAdd(&p.stats->mma_flops, st_flops);
+          atomicAdd(&p.stats->bytes_loaded, qbytes + kvb * (nblk + st_vload));
+        }
+      }
+    }
+  }
+
+  __syncwarp();  // role warps 4 and 5 reconverge (only lane 0 worked)
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace blasst

@@ -1,0 +1,165 @@
+/*
+ * blasst.h - C ABI of the B200 (sm_100a) library for blocked attention with
+ * softmax thresholding.
+ *
+ * The method: a FlashAttention-style forward pass walks the KV blocks of each
+ * query tile left to right with an online softmax (running row max m, running
+ * sum l, rescaled output accumulator). A KV block is skipped when its local
+ * score max is negligible against the running max, i.e. when
+ *     exp(m_blk - m_run) < lambda      for every row of the query tile;
+ * a skipped block's P.V product and V loads never happen, and the first block
+ * is always processed. Sources:
+ *   - "BLASST: Dynamic BLocked Attention Sparsity via Softmax Thresholding"
+ *     (Telegram channel seeallochnaya, post 3655), paragraphs 2-6 counted
+ *     after the headline: blocked left-to-right FlashAttention, online
+ *     softmax, FlashAttention-4 lazy rescaling, the skip rule (V of a dropped
+ *     block is not used), the first block always processed;
+ *   - "BLASST wins Best Paper at MLSys 2026 ..." (digg.com/ai/al6mgdew), the
+ *     authors' announcement: one scalar threshold on the online-softmax
+ *     statistics;
+ *   - "В тени длинного контекста ..." (denisavetisyan.com, LongCA-bench
+ *     review), section on masking strategies (causal and full masks) and the
+ *     closing section on the KV cache (the decode input).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them. Work is enqueued on `stream`
+ *     (a cudaStream_t; NULL means the legacy default stream) and the call
+ *     returns without synchronising.
+ *   - Layouts are dense row-major: q, o [B, Hq, Lq, d]; k, v [B, Hkv, Lkv, d];
+ *     lse [B, Hq, Lq] fp32 (natural log). Every tensor pointer must be 16-byte
+ *     aligned.
+ *   - GQA: query head hq reads KV head hq / (Hq / Hkv).
+ *   - Causal masks are bottom-right aligned: key j is visible from query row
+ *     i when j <= i + (Lkv - Lq).
+ *   - Scores are scale * q.k with scale = 1/sqrt(d) unless stated otherwise.
+ *   - A negative return value is an error from host-side validation or from
+ *     the launch; nothing is enqueued after a validation error. Errors raised
+ *     inside a kernel (a bounded wait that gave up) are recorded in a device
+ *     error word that blasst_check() reads and clears.
+ */
+#ifndef BLASST_H
+#define BLASST_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BLASST_API __attribute__((visibility("default")))
+#else
+#define BLASST_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BLASST_OK = 0,
+  BLASST_EINVAL = -1,        /* bad argument (shape, pointer, lambda, alignment) */
+  BLASST_EUNSUPPORTED = -2,  /* valid request this build does not implement */
+  BLASST_ECUDA = -3,         /* a CUDA runtime/driver call failed */
+  BLASST_ETIMEOUT = -4,      /* a device-side bounded wait gave up */
+  BLASST_EWORKSPACE = -5     /* workspace missing or too small */
+} blasst_status;
+
+typedef enum { BLASST_BF16 = 0, BLASST_FP32 = 1 } blasst_dtype;
+
+/* Telemetry counters, accumulated (atomically added) into a caller-owned
+ * DEVICE struct when one is passed; the library never clears it. */
+typedef struct blasst_stats {
+  unsigned long long tiles_visited;   /* (query tile, KV block) pairs whose scores were formed */
+  unsigned long long tiles_skipped;   /* of those, pairs dropped by the threshold */
+  unsigned long long v_blocks_loaded; /* KV blocks whose V was fetched */
+  unsigned long long mma_flops;       /* tensor-core / FMA flops actually executed (2 per MAC) */
+  unsigned long long bytes_loaded;    /* Q, K, V bytes requested from global memory */
+} blasst_stats;
+
+/* Forward prefill pass, bf16 in / bf16 out, fp32 lse, on the legacy default
+ * stream, scale 1/sqrt(d).
+ *   q, k, v, o  device pointers, layouts above. o may not alias q, k or v.
+ *   lse         [B, Hq, Lq] fp32, natural-log row log-sum-exp of the kept keys.
+ *   causal      1: bottom-right causal mask (requires Lq <= Lkv); 0: full.
+ *   lambda      threshold in [0, 1); 0 never skips (exact attention).
+ *   Br, Bc      query-tile rows and KV-block keys, each 64 or 128; the skip
+ *               decision is taken per (Br-row tile, Bc-key block).
+ *   d           head dimension, 64 or 128.
+ *   skip_mask_out  nullable device pointer to uint8 [B, Hq, ceil(Lq/Br),
+ *               ceil(Lkv/Bc)], fully written: 0 computed, 1 skipped,
+ *               2 not visited (causally invisible).
+ * Returns BLASST_OK or a negative blasst_status. */
+BLASST_API int blasst_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Lq, int Lkv, int d, int causal, float lambda, int Br, int Bc,
+               uint8_t* skip_mask_out);
+
+/* Extended form of blasst_fwd: same operation and arguments plus
+ *   dtype      BLASST_BF16 (q, k, v, o bf16) or BLASST_FP32 (fp32; d = 64 only;
+ *              scores use an error-compensated three-product tf32 split);
+ *   scale      score scale; <= 0 selects 1/sqrt(d);
+ *   stream     cudaStream_t to enqueue on (NULL = legacy default stream);
+ *   stats_out  nullable DEVICE pointer; counters are added to it. */
+typedef struct blasst_fwd_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int B, Hq, Hkv, Lq, Lkv, d;
+  int causal;
+  float lambda;
+  int Br, Bc;
+  uint8_t* skip_mask_out;
+  int dtype;
+  float scale;
+  void* stream;
+  blasst_stats* stats_out;
+} blasst_fwd_args;
+BLASST_API int blasst_fwd_ex(const blasst_fwd_args* args);
+
+/* Bytes of caller workspace that blasst_decode needs: fp32 partial outputs
+ * [B, Hq, num_splits, d] plus fp32 partial lse [B, Hq, num_splits]. */
+BLASST_API size_t blasst_decode_workspace_bytes(int B, int Hq, int d, int num_splits);
+
+/* Split-KV decode: one new query row per sequence and head against a
+ * contiguous KV cache, then a log-sum-exp merge of the splits.
+ *   q          [B, Hq, 1, d] bf16;  k_cache, v_cache [B, Hkv, Lkv, d] bf16.
+ *   o          [B, Hq, 1, d] bf16;  lse [B, Hq] fp32 (natural log).
+ *   Bc         KV block size (64 or 128); the skip decision is per (head, block).
+ *   num_splits S: keys are cut into S chunks of ceil(ceil(Lkv/S)/Bc)*Bc keys;
+ *              each chunk runs its own pass (its first block always
+ *              computed, running statistics restart), then chunks are merged.
+ *   workspace  device buffer of at least blasst_decode_workspace_bytes().
+ *   skip_mask_out nullable uint8 [B, Hq, ceil(Lkv/Bc)] (0 computed, 1 skipped).
+ *   stats_out  nullable device blasst_stats.
+ * A KV block's V rows are read only if at least one query head of its GQA
+ * group keeps the block; heads that skip it add nothing. */
+BLASST_API int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                  int B, int Hq, int Hkv, int Lkv, int d, float lambda, int Bc, int num_splits,
+                  void* workspace, size_t workspace_bytes, uint8_t* skip_mask_out,
+                  blasst_stats* stats_out, void* stream);
+
+/* Log-sum-exp merge of split partials (the second half of blasst_decode):
+ *   o_parts [n_rows, num_splits, d] fp32, normalised per split;
+ *   lse_parts [n_rows, num_splits] fp32, -inf marks an empty split;
+ *   o [n_rows, d] in `out_dtype` (BLASST_BF16 or BLASST_FP32); lse [n_rows].
+ * o = sum_s w_s o_s / sum_s w_s, lse = M + ln sum_s w_s, w_s = exp(lse_s - M),
+ * M = max_s lse_s. */
+BLASST_API int blasst_lse_merge(const float* o_parts, const float* lse_parts, void* o, float* lse, int n_rows,
+                     int d, int num_splits, int out_dtype, void* stream);
+
+/* Synchronises `stream`, then returns (and clears) the device error word:
+ * BLASST_OK, BLASST_ETIMEOUT if a kernel's bounded wait gave up, or
+ * BLASST_ECUDA if the stream reported a CUDA error. */
+BLASST_API int blasst_check(void* stream);
+
+/* Human-readable name of a blasst_status value (static storage). */
+BLASST_API const char* blasst_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+BLASST_API int blasst_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BLASST_H */

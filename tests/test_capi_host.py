@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/blasst.h declares, and rejects bad arguments before
+touching the device."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "blasst.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from dynamic_block_sparse_tiled_b200 import build
+    build.build()
+    import dynamic_block_sparse_tiled_b200 as bl
+    return bl.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"BLASST_API\s+[\w\s\*]+?\b(blasst_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("blasst_fwd", "blasst_fwd_ex", "blasst_decode", "blasst_decode_workspace_bytes",
+              "blasst_lse_merge", "blasst_check", "blasst_status_string", "blasst_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in blasst.h but not exported"
+
+
+def test_status_strings(lib):
+    import dynamic_block_sparse_tiled_b200 as bl
+    for code in (0, -1, -2, -3, -4, -5):
+        assert bl.blasst_status_string(code).startswith("BLASST")
+    assert bl.blasst_version() >= 100
+
+
+def _fwd(lib, **kw):
+    import dynamic_block_sparse_tiled_b200 as bl
+    base = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0x50000, B=1, Hq=4, Hkv=2,
+                Lq=256, Lkv=256, d=128, causal=1, lam=1e-3, Br=128, Bc=128, skip_mask_out=None,
+                dtype=0, scale=0.0, stream=None, stats_out=None)
+    base.update(kw)
+    args = bl._FwdArgs(*[base[f[0]] for f in bl._FwdArgs._fields_])
+    return lib.blasst_fwd_ex(C.byref(args))
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(q=None), -1),
+    (dict(q=0x10008), -1),          # misaligned
+    (dict(lse=0x50004), -1),        # misaligned lse
+    (dict(B=0), -1),
+    (dict(Hq=3, Hkv=2), -1),        # Hq % Hkv
+    (dict(lam=1.0), -1),
+    (dict(lam=-0.1), -1),
+    (dict(lam=float("nan")), -1),
+    (dict(d=96), -2),
+    (dict(Br=32), -2),
+    (dict(Bc=256), -2),
+    (dict(Lq=300, Lkv=256), -2),    # causal with Lq > Lkv
+    (dict(dtype=7), -2),
+])
+def test_fwd_rejects_bad_arguments_without_a_gpu(lib, bad, code):
+    assert _fwd(lib, **bad) == code
+
+
+def test_decode_workspace_and_rejections(lib):
+    ws = lib.blasst_decode_workspace_bytes(16, 32, 128, 64)
+    assert ws == 16 * 32 * 64 * (128 + 1) * 4
+    assert lib.blasst_decode_workspace_bytes(0, 32, 128, 64) == 0
+    vp = 0x10000
+    # too-small workspace
+    rc = lib.blasst_decode(vp, vp, vp, vp, vp, 16, 32, 8, 65536, 128, C.c_float(1e-3), 128, 64,
+                           vp, ws - 16, None, None, None)
+    assert rc == -5
+    # GQA group of 3 is not built
+    rc = lib.blasst_decode(vp, vp, vp, vp, vp, 1, 6, 2, 1024, 128, C.c_float(1e-3), 128, 4,
+                           vp, 1 << 30, None, None, None)
+    assert rc == -2
+    # lambda out of range
+    rc = lib.blasst_decode(vp, vp, vp, vp, vp, 1, 4, 1, 1024, 128, C.c_float(2.0), 128, 4,
+                           vp, 1 << 30, None, None, None)
+    assert rc == -1
+
+
+def test_merge_rejects_bad_arguments(lib):
+    assert lib.blasst_lse_merge(None, None, None, None, 1, 128, 2, 0, None) == -1
+    assert lib.blasst_lse_merge(0x1000, 0x2000, 0x3000, 0x4000, 4, 128, 2, 9, None) == -1
+
+
+def test_python_binding_fails_loudly_without_cuda_tensors():
+    import numpy as np
+    import torch
+    import dynamic_block_sparse_tiled_b200 as bl
+    q = torch.zeros((1, 1, 128, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        bl.attention_prefill(q, q, q)
+    del np

@@ -1,0 +1,151 @@
+"""GPU prefill kernel vs the CPU oracle, through the C ABI."""
+import numpy as np
+import pytest
+
+import oracle
+import parity
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    import dynamic_block_sparse_tiled_b200 as bl
+    return bl
+
+
+def run_case(w, lam, items=None, check_stats=True):
+    """Run GPU and oracle on workload ``w`` at threshold ``lam`` and compare."""
+    import torch
+    bl = _lib()
+    inp = synth.generate(w)
+    q, k, v = (parity.to_device(a) for a in (inp.q, inp.k, inp.v))
+    st = bl.new_stats()
+    lam32 = float(np.float32(lam))
+    o, lse, mask = bl.attention_prefill(q, k, v, causal=w.causal, lam=lam32, Br=w.Br, Bc=w.Bc,
+                                        with_mask=True, stats=st)
+    assert bl.blasst_check() == 0
+    torch.cuda.synchronize()
+    ref = oracle.prefill(inp.q, inp.k, inp.v, causal=w.causal, lam=lam32, Br=w.Br, Bc=w.Bc,
+                         items=items)
+    nQt, nKt = ref["nQt"], ref["nKt"]
+    o_g = parity.bf16_tensor_to_f64(o)
+    lse_g = lse.cpu().numpy().astype(np.float64)
+    mask_g = mask.cpu().numpy()
+    items_arr = ref["items"]
+    bh = items_arr // nQt
+    qt = items_arr % nQt
+    b, hq = bh // w.Hq, bh % w.Hq
+    # gather the GPU rows of the listed tiles: [n, Br, d]
+    rows = qt[:, None] * w.Br + np.arange(w.Br)[None, :]
+    valid = rows < w.Lq
+    rows_c = np.minimum(rows, w.Lq - 1)
+    o_gt = o_g[b[:, None], hq[:, None], rows_c]
+    lse_gt = lse_g[b[:, None], hq[:, None], rows_c]
+    mask_gt = mask_g.reshape(w.B * w.Hq, nQt, nKt)[bh, qt]
+    n_vis, n_dis, ok, dis = parity.compare_masks(mask_gt, ref["mask"], ref["margin"], lam32)
+    assert ok, f"mask: {n_dis} of {n_vis} visited tiles disagree outside the tie band"
+    row_ok = valid & ~dis.any(axis=1)[:, None]
+    stats = parity.compare_outputs(o_gt, lse_gt, ref["o"], ref["lse"], row_ok)
+    parity.assert_within(stats, w.name)
+    if check_stats and items is None:
+        sd = bl.stats_dict(st)
+        assert sd["tiles_visited"] == int((mask_g != 2).sum())
+        assert sd["tiles_skipped"] == int((mask_g == 1).sum())
+    return dict(stats, n_vis=n_vis, n_dis=n_dis, skip=float((ref["mask"] == 1).sum()) / max(n_vis, 1))
+
+
+BASE = synth.CONFIGS["prefill_32k"]
+
+SMALL = [
+    # name, overrides
+    ("gqa_2k_a12", dict(Hq=4, Hkv=2, Lq=2048, Lkv=2048, amp=12.0, window=256, n_needles=2)),
+    ("gqa_1k_literal", dict(Hq=4, Hkv=2, Lq=1024, Lkv=1024, window=256)),
+    ("ragged_1000", dict(Hq=2, Hkv=1, Lq=1000, Lkv=1000, amp=12.0, window=256, n_needles=2)),
+    ("br64", dict(Hq=2, Hkv=2, Lq=1024, Lkv=1024, Br=64, amp=12.0, window=256, n_needles=2)),
+    ("bc64", dict(Hq=2, Hkv=2, Lq=1024, Lkv=1024, Bc=64, amp=12.0, window=256, n_needles=2)),
+    ("br64_bc64_ragged", dict(Hq=2, Hkv=1, Lq=777, Lkv=777, Br=64, Bc=64, amp=12.0, window=256, n_needles=2)),
+    ("d64", dict(Hq=2, Hkv=2, Lq=1024, Lkv=1024, d=64, amp=12.0, window=256, n_needles=2)),
+    ("d64_br64_bc64", dict(Hq=2, Hkv=2, Lq=640, Lkv=640, d=64, Br=64, Bc=64, amp=12.0, window=256, n_needles=2)),
+    ("noncausal", dict(Hq=2, Hkv=2, Lq=512, Lkv=900, causal=False, amp=12.0, window=256, n_needles=2)),
+    ("bottom_right", dict(Hq=2, Hkv=1, Lq=300, Lkv=1100, amp=12.0, window=256, n_needles=2)),
+    ("batch2", dict(B=2, Hq=4, Hkv=1, Lq=768, Lkv=768, amp=12.0, window=256, n_needles=2)),
+    ("one_row", dict(Hq=2, Hkv=2, Lq=1, Lkv=700, causal=False, amp=12.0, n_needles=1)),
+    ("tiny_L", dict(Hq=1, Hkv=1, Lq=70, Lkv=70, amp=12.0)),
+]
+
+
+@pytest.mark.parametrize("name,over", SMALL, ids=[s[0] for s in SMALL])
+@pytest.mark.parametrize("lam", [0.0, 1e-3, 1e-2])
+def test_prefill_parity_small(name, over, lam):
+    w = BASE.replace(name=name, **over)
+    r = run_case(w, lam)
+    if lam >= 1e-3 and w.amp > 3 and w.Lkv >= 4 * w.Bc and w.causal:
+        assert r["skip"] > 0.05, f"skip path not exercised: {r}"
+
+
+@pytest.mark.parametrize("cfg", ["prefill_32k", "prefill_32k_a12"])
+def test_prefill_full_size_sampled(cfg):
+    """Full 32K, GQA 32/8, in the launch configuration the benchmark times;
+    the oracle computes a seeded sample of query tiles (first, last, random)."""
+    w = synth.CONFIGS[cfg]
+    nQt = -(-w.Lq // w.Br)
+    rng = np.random.default_rng(0)
+    items = set()
+    for bh in range(w.B * w.Hq):
+        items.add(bh * nQt + 0)
+        items.add(bh * nQt + nQt - 1)
+    items.update(int(x) for x in rng.integers(0, w.B * w.Hq * nQt, size=24))
+    items = sorted(items)[:80]
+    for lam in w.lambdas:
+        run_case(w, lam, items=items, check_stats=False)
+
+
+def test_prefill_lambda_monotone_full_size():
+    """Property at full size: the set of skipped tiles grows with lambda and
+    lambda = 0 skips nothing (the margins do not depend on lambda)."""
+    import torch
+    bl = _lib()
+    w = synth.CONFIGS["prefill_32k_a12"]
+    inp = synth.generate(w)
+    q, k, v = (parity.to_device(a) for a in (inp.q, inp.k, inp.v))
+    prev = None
+    for lam in (0.0, 1e-4, 1e-3, 1e-2):
+        _, _, mask = bl.attention_prefill(q, k, v, causal=True, lam=lam, Br=128, Bc=128,
+                                          with_mask=True)
+        m = mask.cpu().numpy()
+        if lam == 0.0:
+            assert not np.any(m == 1)
+        assert np.all(m[..., 0] == 0)
+        if prev is not None:
+            # allow tie-band flips: at most 0.1 % of tiles may go the other way
+            assert np.mean((prev == 1) & (m != 1)) < 1e-3
+        prev = m
+    torch.cuda.synchronize()
+
+
+def test_prefill_stats_and_skip_fraction():
+    bl = _lib()
+    w = BASE.replace(name="stats", Hq=4, Hkv=1, Lq=2048, Lkv=2048, amp=12.0, window=256, n_needles=2)
+    r = run_case(w, 1e-3)
+    assert r["skip"] > 0.3, r
+
+
+def test_c_entry_point_blasst_fwd_legacy_stream():
+    """The plain entry point blasst_fwd (bf16, legacy default stream) gives the same bits as blasst_fwd_ex."""
+    import torch
+    bl = _lib()
+    w = BASE.replace(name="legacy", Hq=2, Hkv=1, Lq=512, Lkv=512, amp=12.0, window=128)
+    inp = synth.generate(w)
+    q, k, v = (parity.to_device(a) for a in (inp.q, inp.k, inp.v))
+    o = torch.empty_like(q)
+    lse = torch.empty((1, 2, 512), dtype=torch.float32, device="cuda")
+    mask = torch.empty((1, 2, 4, 4), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    bl.blasst_fwd(q, k, v, o, lse, 1, 2, 1, 512, 512, 128, 1, float(np.float32(1e-3)), 128, 128,
+                  mask)
+    torch.cuda.synchronize()
+    o2, lse2, mask2 = bl.attention_prefill(q, k, v, causal=True, lam=float(np.float32(1e-3)),
+                                           Br=128, Bc=128, with_mask=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, lse2) and torch.equal(mask, mask2)
