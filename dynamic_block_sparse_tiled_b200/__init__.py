@@ -23,7 +23,7 @@ import threading
 __all__ = [
     "BlasstError", "Stats", "lib_path", "load_library",
     "blasst_fwd", "blasst_fwd_ex", "blasst_decode", "blasst_decode_workspace_bytes",
-    "blasst_lse_merge", "blasst_check", "blasst_status_string", "blasst_version",
+    "blasst_lse_merge", "blasst_check", "blasst_selftest_exp2", "blasst_status_string", "blasst_version",
     "attention_prefill", "attention_decode", "new_stats", "stats_dict",
     "BLASST_OK", "BLASST_EINVAL", "BLASST_EUNSUPPORTED", "BLASST_ECUDA", "BLASST_ETIMEOUT",
     "BLASST_EWORKSPACE", "BLASST_BF16", "BLASST_FP32",
@@ -94,6 +94,8 @@ def load_library(path: str | None = None):
         lib.blasst_check.restype = i
         lib.blasst_status_string.argtypes = [i]
         lib.blasst_status_string.restype = C.c_char_p
+        lib.blasst_selftest_exp2.argtypes = [vp, vp, vp, i, vp]
+        lib.blasst_selftest_exp2.restype = i
         lib.blasst_version.argtypes = []
         lib.blasst_version.restype = i
         if path is None:
@@ -185,6 +187,12 @@ def blasst_lse_merge(o_parts, lse_parts, o, lse, *, n_rows: int, d: int, num_spl
     rc = load_library().blasst_lse_merge(_ptr(o_parts), _ptr(lse_parts), _ptr(o), _ptr(lse),
                                          n_rows, d, num_splits, out_dtype, _stream(stream))
     _check(rc, "blasst_lse_merge")
+
+
+def blasst_selftest_exp2(x, y_mufu, y_poly, stream=None):
+    """The C self-test of the two exp2 paths (fp32 CUDA tensors of equal size)."""
+    _check(load_library().blasst_selftest_exp2(_ptr(x), _ptr(y_mufu), _ptr(y_poly), x.numel(),
+                                               _stream(stream)), "blasst_selftest_exp2")
 
 
 def blasst_check(stream=None) -> int:

@@ -96,7 +96,7 @@ int launch_prefill_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   auto kernel = blasst::blasst_prefill_bf16_kernel<D, BC, BR>;
   if (set_smem(kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
   const dim3 grid(static_cast<unsigned>(p.nQblk) * p.B * p.Hq);
-  kernel<<<grid, 192, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? BLASST_OK : BLASST_ECUDA;
 }
 
@@ -150,6 +150,15 @@ int dispatch_decode(int d, int Bc, int g, const CUtensorMap& mk, const CUtensorM
   BLASST_DC(64, 64, 8)
 #undef BLASST_DC
   return BLASST_EUNSUPPORTED;
+}
+
+__global__ void selftest_exp2_kernel(const float* x, float* y_mufu, float* y_poly, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    y_mufu[i] = blasst::ptx::ex2(x[i]);
+    float y1;
+    blasst::ptx::exp2_poly2(y_poly[i], y1, x[i], -x[i]);  // the two-wide form the kernel uses
+  }
 }
 
 float log2_lambda_of(float lambda) {
@@ -336,6 +345,13 @@ int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void*
   if (rc != BLASST_OK) return rc;
   return blasst_lse_merge(p.o_parts, p.lse_parts, o, lse, B * Hq, d, num_splits, BLASST_BF16,
                           stream);
+}
+
+int blasst_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n, void* stream) {
+  if (!x || !y_mufu || !y_poly || n <= 0) return BLASST_EINVAL;
+  selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_mufu,
+                                                                                     y_poly, n);
+  return cudaGetLastError() == cudaSuccess ? BLASST_OK : BLASST_ECUDA;
 }
 
 int blasst_check(void* stream) {

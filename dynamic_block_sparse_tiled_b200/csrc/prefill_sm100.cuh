@@ -12,13 +12,22 @@
 // output accumulator; the skip test always uses the exact running max.
 //
 // One CTA owns 128 query rows of one (batch, query head) and walks the KV
-// blocks of its KV head. Warp roles (192 threads):
-//   warps 0-3  softmax: thread t owns row t (TMEM lane t); row max, the vote,
-//              exp2, P -> TMEM, lazy O rescale, epilogue;
-//   warp 4     TMA producer: Q once, K ahead through a 3-stage ring, V only
-//              after the vote says the block is kept;
-//   warp 5     tcgen05 issuer: S = Q K^T into one of three TMEM S buffers,
-//              O += P V with P read from TMEM (P overwrites its S buffer).
+// blocks of its KV head. Warp roles (352 threads):
+//   warps 0-7  softmax: warps w and w+4 share the 32 rows of TMEM lanes
+//              32*(w%4).. and split the block's columns in halves; each takes
+//              its half-row max, the half-row skip test, exp2, its half of P
+//              (into TMEM), its half of the lazy O rescale and of the
+//              epilogue. The row skip test is exact on halves:
+//              max(a, b) - m < t  <=>  a - m < t  and  b - m < t;
+//   warp 8     TMA producer for Q and K (K runs ahead through a 3-stage ring,
+//              independent of the votes);
+//   warp 9     TMA producer for V: loads V of block j only after the vote on
+//              block j says some row group keeps it;
+//   warp 10    tcgen05 issuer: S = Q K^T into one of two TMEM S buffers,
+//              issued two blocks ahead, then O += P V with P read from one of
+//              two TMEM P buffers. P has TMEM of its own so that the issuer
+//              never waits for an MMA to finish: it waits only for the
+//              softmax (P ready), for K and for V.
 // With Br = 64 the 128 rows form two independent vote groups that share the
 // MMAs: a group that skips contributes zero rows of P and leaves its running
 // statistics untouched.
@@ -61,11 +70,17 @@ constexpr int pow2_at_least(int x) {
 template <int D, int BC, int BR>
 struct PrefillCfg {
   static constexpr int BM = 128;
-  static constexpr int NG = BM / BR;   // vote groups
-  static constexpr int WPG = BR / 32;  // warps per vote group
+  static constexpr int NTHREADS = 352;
+  static constexpr int NSOFT = 256;      // softmax threads (warps 0-7)
+  static constexpr int WARP_K = 8, WARP_V = 9, WARP_MMA = 10;
+  static constexpr int NG = BM / BR;     // vote groups
+  static constexpr int WPG = BR / 32;    // TMEM lane quarters per vote group
+  static constexpr int HALF = BC / 2;    // S columns per softmax warp
+  static constexpr int DHALF = D / 2;    // O columns per softmax warp
   static constexpr int NK = 3;
   static constexpr int NV = 2;
-  static constexpr int NS = 3;
+  static constexpr int NS = 2;   // S buffers (fp32, BC columns each)
+  static constexpr int NP = 2;   // P buffers (bf16 pairs, BC/2 columns each)
   static constexpr int NSLOT = 4;
   static constexpr int DBOX = D / 64;
   static constexpr int Q_BOX = BM * 128;
@@ -83,18 +98,21 @@ struct PrefillCfg {
   static constexpr int B_VF = B_KE + NK;
   static constexpr int B_VE = B_VF + NV;
   static constexpr int B_SF = B_VE + NV;
-  static constexpr int B_PV = B_SF + NS;
-  static constexpr int B_DEC = B_PV + NS;
+  static constexpr int B_PV = B_SF + NS;   // P.V done, one barrier per P buffer
+  static constexpr int B_DEC = B_PV + NP;
   static constexpr int B_P = B_DEC + NSLOT;
   static constexpr int B_DRAIN = B_P + NSLOT;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // misc words: [0] tmem base, [1] abort, [4..7] decisions, [8..15] votes
-  static constexpr int MISC_BYTES = 64;
-  static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-  static constexpr int S_COL = 0;        // S buffer b at column b * BC
-  static constexpr int O_COL = NS * BC;  // O accumulator
-  static constexpr int TMEM_COLS = pow2_at_least(NS * BC + D);
+  // misc words: [0] tmem base, [1] abort, [4..7] decisions, [8..23] votes (2 x 8 warps)
+  static constexpr int MISC_BYTES = 128;
+  static constexpr int OFF_PMAX = OFF_MISC + MISC_BYTES;  // [2][2 halves][128 rows] floats
+  static constexpr int OFF_LSUM = OFF_PMAX + 2 * 2 * 128 * 4;  // [2 halves][128 rows] floats
+  static constexpr int SMEM_BYTES = OFF_LSUM + 2 * 128 * 4 + 1024;  // + alignment slack
+  static constexpr int S_COL = 0;                   // S buffer b at column b * BC
+  static constexpr int P_COL = NS * BC;             // P buffer b at P_COL + b * BC / 2
+  static constexpr int O_COL = P_COL + NP * BC / 2; // O accumulator
+  static constexpr int TMEM_COLS = pow2_at_least(O_COL + D);
   static constexpr uint32_t IDESC_QK = ptx::idesc_f32acc(1, 128, BC, false);
   static constexpr uint32_t IDESC_PV = ptx::idesc_f32acc(1, 128, D, true);
   static constexpr float TAU = 8.0f;  // lazy-rescale slack, log2 units
@@ -110,7 +128,7 @@ __device__ __forceinline__ void record_error(int* err, int code) {
 }
 
 template <int D, int BC, int BR>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(352, 1)
     blasst_prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                                const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -123,18 +141,24 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = misc + 1;
   volatile int* dec_val = misc + 4;
   volatile int* votes = misc + 8;
+  volatile float* pmax = reinterpret_cast<volatile float*>(smem + C::OFF_PMAX);
+  volatile float* lsum = reinterpret_cast<volatile float*>(smem + C::OFF_LSUM);
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: longest causal rows first ----------------------------
-  const int BH = p.B * p.Hq;
-  const int qblk = p.nQblk - 1 - static_cast<int>(blockIdx.x) / BH;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  const int hq = bh % p.Hq;
-  const int b = bh / p.Hq;
-  const int bhk = b * p.Hkv + hq / p.g;
+  // ---- work item ----------------------------------------------------------
+  // KV-head major: the CTAs in flight share one KV head's K/V in L2; within
+  // a KV head, the longest causal rows go first and the g query heads of the
+  // group are adjacent.
+  const int per_kv = p.nQblk * p.g;
+  const int bhk = static_cast<int>(blockIdx.x) / per_kv;
+  const int rem = static_cast<int>(blockIdx.x) % per_kv;
+  const int qblk = p.nQblk - 1 - rem / p.g;
+  const int b = bhk / p.Hkv;
+  const int hq = (bhk % p.Hkv) * p.g + rem % p.g;
+  const int bh = b * p.Hq + hq;
   const int r0 = qblk * C::BM;
 
   int kt_last[C::NG];
@@ -164,19 +188,17 @@ __global__ void __launch_bounds__(192, 1)
       ptx::mbar_init(bar(C::B_VF + i), 1);
       ptx::mbar_init(bar(C::B_VE + i), 1);
     }
-    for (int i = 0; i < C::NS; ++i) {
-      ptx::mbar_init(bar(C::B_SF + i), 1);
-      ptx::mbar_init(bar(C::B_PV + i), 1);
-    }
+    for (int i = 0; i < C::NS; ++i) ptx::mbar_init(bar(C::B_SF + i), 1);
+    for (int i = 0; i < C::NP; ++i) ptx::mbar_init(bar(C::B_PV + i), 1);
     for (int i = 0; i < C::NSLOT; ++i) {
       ptx::mbar_init(bar(C::B_DEC + i), 1);
-      ptx::mbar_init(bar(C::B_P + i), 4);
+      ptx::mbar_init(bar(C::B_P + i), 8);
     }
     ptx::mbar_init(bar(C::B_DRAIN), 1);
     for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == C::WARP_MMA) {
     ptx::tmem_alloc(ptx::smem_u32(const_cast<int*>(misc)), C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
@@ -185,48 +207,30 @@ __global__ void __launch_bounds__(192, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
 
-  if (warp == 4) {
-    // ======================= TMA producer =================================
+  auto load_kv = [&](const CUtensorMap* tm, uint32_t dst, int blk, uint32_t fb) {
+    ptx::mbar_arrive_expect_tx(fb, C::KV_BYTES);
+#pragma unroll
+    for (int bx = 0; bx < C::DBOX; ++bx)
+      ptx::tma_load_3d(dst + bx * C::KV_BOX, tm, bx * 64, blk * BC, bhk, fb);
+  };
+
+  if (warp == C::WARP_K) {
+    // ======================= TMA producer: Q and K ========================
     if (lane == 0) {
       ptx::prefetch_tmap(&tmQ);
       ptx::prefetch_tmap(&tmK);
-      ptx::prefetch_tmap(&tmV);
       bool ok = true;
       ptx::mbar_arrive_expect_tx(bar(C::B_Q), C::Q_BYTES);
 #pragma unroll
       for (int bx = 0; bx < C::DBOX; ++bx)
         ptx::tma_load_3d(sb + C::OFF_Q + bx * C::Q_BOX, &tmQ, bx * 64, r0, bh, bar(C::B_Q));
-      auto load_kv = [&](const CUtensorMap* tm, uint32_t dst, int blk, uint32_t fb) {
-        ptx::mbar_arrive_expect_tx(fb, C::KV_BYTES);
-#pragma unroll
-        for (int bx = 0; bx < C::DBOX; ++bx)
-          ptx::tma_load_3d(dst + bx * C::KV_BOX, tm, bx * 64, blk * BC, bhk, fb);
-      };
-      int kiss = 0;
-      for (; kiss < min(C::NK, nblk); ++kiss)
-        load_kv(&tmK, sb + C::OFF_K + kiss * C::KV_BYTES, kiss, bar(C::B_KF + kiss));
-      int vcount = 0;
       for (int j = 0; j < nblk && ok; ++j) {
-        const int slot = j % C::NSLOT;
-        ok = ptx::mbar_wait(bar(C::B_DEC + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
-        if (!ok) break;
-        if (dec_val[slot] != 0) {
-          const int vs = vcount % C::NV;
-          if (vcount >= C::NV)
-            ok = ptx::mbar_wait(bar(C::B_VE + vs), ((vcount / C::NV) - 1) & 1, abort_flag,
-                                p.timeout_ns);
-          if (!ok) break;
-          load_kv(&tmV, sb + C::OFF_V + vs * C::KV_BYTES, j, bar(C::B_VF + vs));
-          ++vcount;
-        }
-        if (kiss < nblk) {
-          const int ks = kiss % C::NK;
-          ok = ptx::mbar_wait(bar(C::B_KE + ks), ((kiss / C::NK) - 1) & 1, abort_flag,
+        const int ks = j % C::NK;
+        if (j >= C::NK)
+          ok = ptx::mbar_wait(bar(C::B_KE + ks), ((j / C::NK) - 1) & 1, abort_flag,
                               p.timeout_ns);
-          if (!ok) break;
-          load_kv(&tmK, sb + C::OFF_K + ks * C::KV_BYTES, kiss, bar(C::B_KF + ks));
-          ++kiss;
-        }
+        if (!ok) break;
+        load_kv(&tmK, sb + C::OFF_K + ks * C::KV_BYTES, j, bar(C::B_KF + ks));
       }
       if (!ok) {
         *abort_flag = 1;
@@ -235,7 +239,57 @@ __global__ void __launch_bounds__(192, 1)
         ptx::mbar_wait(bar(C::B_Q), 0, abort_flag, p.timeout_ns);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == C::WARP_V) {
+    // ======================= TMA producer: V (after the vote) ==============
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmV);
+      bool ok = true;
+      int vcount = 0;
+      unsigned long long st_vis = 0, st_skip = 0, st_flops = 0;
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int slot = j % C::NSLOT;
+        ok = ptx::mbar_wait(bar(C::B_DEC + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        const int keepmask = dec_val[slot];
+        // skip-mask entries and counters for block j (off the softmax path)
+        const unsigned long long tile_flops = 2ull * 128ull * BC * D;
+        st_flops += tile_flops + (keepmask ? tile_flops : 0ull);
+#pragma unroll
+        for (int gg = 0; gg < C::NG; ++gg) {
+          if (kt_last[gg] < 0) continue;
+          uint8_t code = 2;
+          if (j <= kt_last[gg]) {
+            ++st_vis;
+            code = ((keepmask >> gg) & 1) ? 0 : 1;
+            if (code == 1) ++st_skip;
+          }
+          if (p.mask)
+            p.mask[(static_cast<size_t>(bh) * p.nQt + (r0 / BR + gg)) * p.nKt + j] = code;
+        }
+        if (keepmask != 0) {
+          const int vs = vcount % C::NV;
+          if (vcount >= C::NV)
+            ok = ptx::mbar_wait(bar(C::B_VE + vs), ((vcount / C::NV) - 1) & 1, abort_flag,
+                                p.timeout_ns);
+          if (!ok) break;
+          load_kv(&tmV, sb + C::OFF_V + vs * C::KV_BYTES, j, bar(C::B_VF + vs));
+          ++vcount;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_error(p.err, BLASST_ETIMEOUT);
+      } else if (p.stats) {
+        const unsigned long long qbytes = 128ull * D * 2ull;
+        const unsigned long long kvb = static_cast<unsigned long long>(BC) * D * 2ull;
+        atomicAdd(&p.stats->tiles_visited, st_vis);
+        atomicAdd(&p.stats->tiles_skipped, st_skip);
+        atomicAdd(&p.stats->v_blocks_loaded, static_cast<unsigned long long>(vcount));
+        atomicAdd(&p.stats->mma_flops, st_flops);
+        atomicAdd(&p.stats->bytes_loaded, qbytes + kvb * (nblk + vcount));
+      }
+    }
+  } else if (warp == C::WARP_MMA) {
     // ======================= tcgen05 issuer ===============================
     if (lane == 0) {
       bool ok = ptx::mbar_wait(bar(C::B_Q), 0, abort_flag, p.timeout_ns);
@@ -261,21 +315,26 @@ __global__ void __launch_bounds__(192, 1)
       if (ok) ok = issue_qk(0);
       if (ok && nblk > 1) ok = issue_qk(1);
       int pv_count = 0;
-      int pvn[C::NS] = {0, 0, 0};
-      bool kept_prev = false;
       for (int j = 0; j < nblk && ok; ++j) {
         const int slot = j % C::NSLOT;
         ok = ptx::mbar_wait(bar(C::B_P + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         ptx::tc_fence_after();
         const bool keep = dec_val[slot] != 0;
+        // Look-ahead first: S = Q K^T of block j+2 goes into the S buffer that
+        // block j's softmax has just finished reading, and keeps the tensor
+        // pipe busy while V_j (requested only after block j's vote) lands.
+        if (j + 2 < nblk) {
+          ok = issue_qk(j + 2);
+          if (!ok) break;
+        }
         if (keep) {
           const int vs = pv_count % C::NV;
           ok = ptx::mbar_wait(bar(C::B_VF + vs), (pv_count / C::NV) & 1, abort_flag,
                               p.timeout_ns);
           if (!ok) break;
           ptx::tc_fence_after();
-          const uint32_t p_tm = tmem + C::S_COL + (j % C::NS) * BC;
+          const uint32_t p_tm = tmem + C::P_COL + (j % C::NP) * (BC / 2);
 #pragma unroll
           for (int kk = 0; kk < BC / 16; ++kk) {
             const uint64_t bd =
@@ -284,20 +343,9 @@ __global__ void __launch_bounds__(192, 1)
                         (pv_count > 0 || kk > 0) ? 1u : 0u);
           }
           ptx::mma_commit(bar(C::B_VE + vs));
-          ptx::mma_commit(bar(C::B_PV + (j % C::NS)));
-          ++pvn[j % C::NS];
+          ptx::mma_commit(bar(C::B_PV + (j % C::NP)));
           ++pv_count;
         }
-        if (j + 2 < nblk) {
-          // S buffer (j+2)%3 last held block j-1: its P must have been read.
-          const int bp = (j + 2) % C::NS;
-          if (j >= 1 && kept_prev) {
-            ok = ptx::mbar_wait(bar(C::B_PV + bp), (pvn[bp] - 1) & 1, abort_flag, p.timeout_ns);
-            if (!ok) break;
-          }
-          ok = issue_qk(j + 2);
-        }
-        kept_prev = keep;
       }
       if (!ok) {
         *abort_flag = 1;
@@ -308,96 +356,99 @@ __global__ void __launch_bounds__(192, 1)
       ptx::mbar_wait(bar(C::B_DRAIN), 0, abort_flag, p.timeout_ns);
     }
   } else {
-    // ======================= softmax warps 0-3 ===========================
-    const int t = threadIdx.x;
+    // ======================= softmax warps 0-7 ===========================
+    const int quad = warp & 3;        // TMEM lane quarter
+    const int half = warp >> 2;       // column half
+    const int t = quad * 32 + lane;   // row within the CTA tile
     const int row = r0 + t;
     const bool row_exists = row < p.Lq;
     const int gi = t / BR;
     const int my_kt_last = kt_last[gi];
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int last_col = p.causal ? min(row + p.off, p.Lkv - 1) : p.Lkv - 1;
     const float sl2 = p.scale_log2;
     const bool thresholding = p.log2_lambda > -INFINITY;
+    const bool leader = threadIdx.x == 0;
 
-    float m = -INFINITY, mref = -INFINITY, l = 0.0f;
-    int pvn[C::NS] = {0, 0, 0};
+    float m = -INFINITY, mref = -INFINITY, l = 0.0f;  // l: this half's partial sum
+    int pvn[C::NP] = {0, 0};  // P.V products issued on each P buffer
     int last_buf = -1, ncomp = 0;
-    unsigned long long st_vis = 0, st_skip = 0, st_vload = 0, st_flops = 0;
     bool aborted = false;
 
     for (int j = 0; j < nblk; ++j) {
       const int sbuf = j % C::NS;
+      const int pbuf = j % C::NP;
       bool ok = true;
-      if (lane == 0) ok = ptx::mbar_wait(bar(C::B_SF + sbuf), (j / C::NS) & 1, abort_flag, p.timeout_ns);
+      if (lane == 0)
+        ok = ptx::mbar_wait(bar(C::B_SF + sbuf), (j / C::NS) & 1, abort_flag, p.timeout_ns);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       ptx::tc_fence_after();
 
-      float s[BC];
-      float mb = -INFINITY;
+      float s[C::HALF];
+      float mbh = -INFINITY;  // this half-row's max (log2 units)
       bool rowskip = true;
+      const int col0 = j * BC + half * C::HALF;
       if (ok) {
+        uint32_t sr[C::HALF];
 #pragma unroll
-        for (int c = 0; c < BC / 32; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tmem + lane_base + C::S_COL + sbuf * BC + 32 * c, r);
-          ptx::tmem_wait_ld();
+        for (int c = 0; c < C::HALF / 32; ++c)
+          ptx::tmem_ld32p(tmem + lane_base + C::S_COL + sbuf * BC + half * C::HALF + 32 * c,
+                          sr + 32 * c);
+        ptx::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[i]);
-        }
-        const int col0 = j * BC;
-        const bool need_mask = (col0 + BC > p.Lkv) || (p.causal && col0 + BC - 1 > r0 + p.off);
+        for (int c = 0; c < C::HALF; ++c) s[c] = __uint_as_float(sr[c]);
+        const bool need_mask =
+            (j * BC + BC > p.Lkv) || (p.causal && j * BC + BC - 1 > r0 + p.off);
         if (need_mask) {
 #pragma unroll
-          for (int c = 0; c < BC; ++c)
+          for (int c = 0; c < C::HALF; ++c)
             if (col0 + c > last_col) s[c] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // half-row max: 8 independent chains of three-input max, then a tree
+        float mc[8];
 #pragma unroll
-        for (int c = 0; c < BC; ++c) mx = fmaxf(mx, s[c]);
-        mb = mx * sl2;
+        for (int i = 0; i < 8; ++i) {
+          constexpr int W = C::HALF / 8;
+          float a = s[i * W];
+#pragma unroll
+          for (int c = 1; c + 1 < W; c += 2) a = ptx::fmax3(a, s[i * W + c], s[i * W + c + 1]);
+          if ((W - 1) % 2) a = fmaxf(a, s[i * W + W - 1]);
+          mc[i] = a;
+        }
+        mbh = ptx::fmax3(ptx::fmax3(mc[0], mc[1], mc[2]), ptx::fmax3(mc[3], mc[4], mc[5]),
+                         fmaxf(mc[6], mc[7])) * sl2;
         const bool visited = j <= my_kt_last;
         if (!row_exists || !visited) rowskip = true;
         else if (j == 0 || !thresholding) rowskip = false;
-        else rowskip = (mb - m) < p.log2_lambda;
+        else rowskip = (mbh - m) < p.log2_lambda;
       }
+      pmax[((j & 1) * 2 + half) * 128 + t] = mbh;
       const unsigned all_skip = __all_sync(0xffffffffu, rowskip) ? 1u : 0u;
-      if (lane == 0) votes[(j & 1) * 4 + warp] = ok ? static_cast<int>(all_skip) : 2;
-      ptx::named_bar_sync(1, 128);
+      if (lane == 0) votes[(j & 1) * 8 + warp] = ok ? static_cast<int>(all_skip) : 2;
+      ptx::named_bar_sync(1, C::NSOFT);
+      const float mb = fmaxf(mbh, pmax[((j & 1) * 2 + (half ^ 1)) * 128 + t]);
       int keepmask = 0;
       bool any_abort = false;
 #pragma unroll
       for (int gg = 0; gg < C::NG; ++gg) {
         bool gskip = true;
 #pragma unroll
-        for (int w = 0; w < C::WPG; ++w) {
-          const int v = votes[(j & 1) * 4 + gg * C::WPG + w];
-          if (v == 2) any_abort = true;
-          gskip = gskip && (v != 0);
-        }
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int w = 0; w < C::WPG; ++w) {
+            const int v = votes[(j & 1) * 8 + hh * 4 + gg * C::WPG + w];
+            if (v == 2) any_abort = true;
+            gskip = gskip && (v != 0);
+          }
         if (j <= kt_last[gg] && !gskip) keepmask |= 1 << gg;
       }
       if (any_abort) {
         aborted = true;
         break;
       }
-      if (t == 0) {
+      if (leader) {
         dec_val[j % C::NSLOT] = keepmask;
         ptx::mbar_arrive(bar(C::B_DEC + (j % C::NSLOT)));
-        const unsigned long long tile_flops = 2ull * 128ull * BC * D;
-        st_flops += tile_flops + (keepmask ? tile_flops : 0ull);
-        st_vload += keepmask ? 1ull : 0ull;
-#pragma unroll
-        for (int gg = 0; gg < C::NG; ++gg) {
-          if (kt_last[gg] < 0) continue;
-          const int qt = r0 / BR + gg;
-          uint8_t code = 2;
-          if (j <= kt_last[gg]) {
-            ++st_vis;
-            code = ((keepmask >> gg) & 1) ? 0 : 1;
-            if (code == 1) ++st_skip;
-          }
-          if (p.mask) p.mask[(static_cast<size_t>(bh) * p.nQt + qt) * p.nKt + j] = code;
-        }
       }
       if (keepmask) {
         const bool my_keep = (keepmask >> gi) & 1;
@@ -420,9 +471,9 @@ __global__ void __launch_bounds__(192, 1)
             const float alpha = need ? ptx::ex2(mref - mref_new) : 1.0f;
             l *= alpha;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < C::DHALF / 32; ++c) {
               uint32_t r[32];
-              const uint32_t ta = tmem + lane_base + C::O_COL + 32 * c;
+              const uint32_t ta = tmem + lane_base + C::O_COL + half * C::DHALF + 32 * c;
               ptx::tmem_ld32(ta, r);
               ptx::tmem_wait_ld();
 #pragma unroll
@@ -435,37 +486,62 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (my_keep) m = m_new;
 
-        uint32_t pk[BC / 2];
+        uint32_t pk[C::HALF / 2];
         if (my_keep) {
           const float neg = -mref;
-          float rs = 0.0f;
+          float rs[8];
 #pragma unroll
-          for (int c = 0; c < BC; c += 2) {
-            const float p0 = ptx::ex2(fmaf(s[c], sl2, neg));
-            const float p1 = ptx::ex2(fmaf(s[c + 1], sl2, neg));
-            rs += p0 + p1;
+          for (int i = 0; i < 8; ++i) rs[i] = 0.0f;
+#pragma unroll
+          for (int c = 0; c < C::HALF; c += 2) {
+            float x0, x1, p0, p1;
+            ptx::fma2(x0, x1, s[c], s[c + 1], sl2, sl2, neg, neg);
+            // every fourth pair of columns takes the FMA-pipe exp2
+            if (((c >> 1) & 3) == 3) {
+              ptx::exp2_poly2(p0, p1, x0, x1);
+            } else {
+              p0 = ptx::ex2(x0);
+              p1 = ptx::ex2(x1);
+            }
+            const int a = ((c >> 1) & 3) * 2;
+            ptx::add2(rs[a], rs[a + 1], rs[a], rs[a + 1], p0, p1);
             pk[c / 2] = ptx::pack_bf16x2(p0, p1);
           }
-          l += rs;
+          l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
         } else {
 #pragma unroll
-          for (int c = 0; c < BC / 2; ++c) pk[c] = 0u;
+          for (int c = 0; c < C::HALF / 2; ++c) pk[c] = 0u;
+        }
+        // P buffer pbuf was last read by the P.V of block j-2 (if computed).
+        if (pvn[pbuf] > 0 && last_buf != -1) {
+          bool ok3 = true;
+          if (lane == 0)
+            ok3 = ptx::mbar_wait(bar(C::B_PV + pbuf), (pvn[pbuf] - 1) & 1, abort_flag,
+                                 p.timeout_ns);
+          ok3 = __shfl_sync(0xffffffffu, ok3 ? 1 : 0, 0) != 0;
+          if (!ok3) {
+            *abort_flag = 1;
+            record_error(p.err, BLASST_ETIMEOUT);
+          }
+          ptx::tc_fence_after();
         }
 #pragma unroll
-        for (int c = 0; c < BC / 32; ++c)
-          ptx::tmem_st16(tmem + lane_base + C::S_COL + sbuf * BC + 16 * c, pk + 16 * c);
+        for (int c = 0; c < C::HALF / 32; ++c)
+          ptx::tmem_st16(tmem + lane_base + C::P_COL + pbuf * (BC / 2) + half * (C::HALF / 2) +
+                             16 * c,
+                         pk + 16 * c);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ++ncomp;
-        last_buf = sbuf;
-        ++pvn[sbuf];
+        last_buf = pbuf;
+        ++pvn[pbuf];
       }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(C::B_P + (j % C::NSLOT)));
     }
 
     if (aborted) {
-      if (t == 0) {
+      if (leader) {
         *abort_flag = 1;
         record_error(p.err, BLASST_ETIMEOUT);
       }
@@ -477,17 +553,20 @@ __global__ void __launch_bounds__(192, 1)
                             p.timeout_ns);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       ptx::tc_fence_after();
+      lsum[half * 128 + t] = l;
+      ptx::named_bar_sync(1, C::NSOFT);
+      const float ltot = l + lsum[(half ^ 1) * 128 + t];
       if (!ok) {
         *abort_flag = 1;
         record_error(p.err, BLASST_ETIMEOUT);
       } else {
-        const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+        const float inv_l = (ltot > 0.0f) ? 1.0f / ltot : 0.0f;
         __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                              (static_cast<size_t>(bh) * p.Lq + row) * D;
+                              (static_cast<size_t>(bh) * p.Lq + row) * D + half * C::DHALF;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < C::DHALF / 32; ++c) {
           uint32_t r[32];
-          ptx::tmem_ld32(tmem + lane_base + C::O_COL + 32 * c, r);
+          ptx::tmem_ld32(tmem + lane_base + C::O_COL + half * C::DHALF + 32 * c, r);
           ptx::tmem_wait_ld();
           uint32_t w[16];
 #pragma unroll
@@ -501,34 +580,26 @@ __global__ void __launch_bounds__(192, 1)
               dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
           }
         }
-        if (row_exists)
-          p.lse[static_cast<size_t>(bh) * p.Lq + row] = (mref + log2f(l)) * 0.6931471805599453f;
+        if (row_exists && half == 0)
+          p.lse[static_cast<size_t>(bh) * p.Lq + row] = (mref + log2f(ltot)) * 0.6931471805599453f;
         if (p.mask) {
 #pragma unroll
           for (int gg = 0; gg < C::NG; ++gg) {
             if (kt_last[gg] < 0) continue;
             const int qt = r0 / BR + gg;
             uint8_t* mrow = p.mask + (static_cast<size_t>(bh) * p.nQt + qt) * p.nKt;
-            for (int j = nblk + t; j < p.nKt; j += 128) mrow[j] = 2;
+            for (int jj = nblk + static_cast<int>(threadIdx.x); jj < p.nKt; jj += C::NSOFT)
+              mrow[jj] = 2;
           }
-        }
-        if (t == 0 && p.stats) {
-          const unsigned long long qbytes = 128ull * D * 2ull;
-          const unsigned long long kvb = static_cast<unsigned long long>(BC) * D * 2ull;
-          atomicAdd(&p.stats->tiles_visited, st_vis);
-          atomicAdd(&p.stats->tiles_skipped, st_skip);
-          atomicAdd(&p.stats->v_blocks_loaded, st_vload);
-          atomicAdd(&p.stats->mma_flops, st_flops);
-          atomicAdd(&p.stats->bytes_loaded, qbytes + kvb * (nblk + st_vload));
         }
       }
     }
   }
 
-  __syncwarp();  // role warps 4 and 5 reconverge (only lane 0 worked)
+  __syncwarp();  // role warps reconverge (only their lane 0 worked)
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == C::WARP_MMA) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -184,6 +184,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
+// Same as tmem_ld32, writing into r[0..31] of a larger register array.
+__device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -232,10 +247,69 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t ab_format, int M, i
 }
 
 // ------------------------------------------------------------------- math
+// Three-input max (sm_100 form of max.f32).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA/ALU pipes (keeps part of the exponentials off the MUFU
+// pipe). x = n + f with n = round(x) (the 1.5*2^23 shifter), f in [-1/2, 1/2];
+// 2^f by the degree-3 Chebyshev interpolant whose coefficients
+// gen_exp2_poly.py derives (relative error <= 1.0e-4); 2^n by adding n to the
+// exponent field. Below x = -125 the result leaves the normal range (and
+// inputs under -126 are clamped): it is then some value under 2^-125 instead
+// of the exact one, far below what an fp32 row sum or a bf16 P registers.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(5.583828315e-02f, f, 2.426394820e-01f);
+  p = fmaf(p, f, 6.931367517e-01f);
+  p = fmaf(p, f, 9.999245405e-01f);
+  const int n = __float_as_int(t) - 0x4B400000;
+  return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// ---- two-wide fp32 arithmetic (sm_100 f32x2 forms), on pairs of registers.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// exp2_poly on a pair, with two-wide arithmetic. The exponent insert uses
+// (bits(t) << 23) mod 2^32 == n << 23, because the shifter's own bits
+// (0x4B400000) vanish under the shift: one integer multiply-add per element.
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  float t0, t1, u0, u1, f0, f1, q0, q1;
+  add2(t0, t1, x0, x1, 12582912.0f, 12582912.0f);
+  add2(u0, u1, t0, t1, -12582912.0f, -12582912.0f);
+  fma2(f0, f1, u0, u1, -1.0f, -1.0f, x0, x1);
+  fma2(q0, q1, 5.583828315e-02f, 5.583828315e-02f, f0, f1, 2.426394820e-01f, 2.426394820e-01f);
+  fma2(q0, q1, q0, q1, f0, f1, 6.931367517e-01f, 6.931367517e-01f);
+  fma2(q0, q1, q0, q1, f0, f1, 9.999245405e-01f, 9.999245405e-01f);
+  y0 = __uint_as_float(__float_as_uint(t0) * (1u << 23) + __float_as_uint(q0));
+  y1 = __uint_as_float(__float_as_uint(t1) * (1u << 23) + __float_as_uint(q1));
 }
 
 // Two fp32 -> packed bf16x2, round to nearest even; `lo` lands in bits 0-15.

@@ -149,3 +149,23 @@ def test_c_entry_point_blasst_fwd_legacy_stream():
                                            Br=128, Bc=128, with_mask=True)
     torch.cuda.synchronize()
     assert torch.equal(o, o2) and torch.equal(lse, lse2) and torch.equal(mask, mask2)
+
+
+def test_exp2_paths_against_float64():
+    """The hardware exp2 and the FMA-pipe polynomial used for a quarter of the
+    softmax exponentials, against float64 2^x over the range where both give
+    normal floats (the kernel feeds x <= 8, the lazy-rescale slack)."""
+    import torch
+    bl = _lib()
+    x = np.concatenate([np.linspace(-125.0, 64.0, 200001), np.linspace(-1, 1, 20001),
+                        np.arange(-125, 65, dtype=np.float64)]).astype(np.float32)
+    xt = torch.from_numpy(x).cuda()
+    ym = torch.empty_like(xt)
+    yp = torch.empty_like(xt)
+    bl.blasst_selftest_exp2(xt, ym, yp)
+    torch.cuda.synchronize()
+    ref = np.exp2(x.astype(np.float64))
+    rel_p = np.abs(yp.cpu().numpy().astype(np.float64) / ref - 1.0)
+    rel_m = np.abs(ym.cpu().numpy().astype(np.float64) / ref - 1.0)
+    assert rel_p.max() < 1.1e-4, rel_p.max()
+    assert rel_m.max() < 1e-5, rel_m.max()
