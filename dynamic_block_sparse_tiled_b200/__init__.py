@@ -23,7 +23,8 @@ import threading
 __all__ = [
     "BlasstError", "Stats", "lib_path", "load_library",
     "blasst_fwd", "blasst_fwd_ex", "blasst_decode", "blasst_decode_workspace_bytes",
-    "blasst_lse_merge", "blasst_check", "blasst_selftest_exp2", "blasst_status_string", "blasst_version",
+    "blasst_lse_merge", "blasst_check", "blasst_selftest_exp2",
+    "blasst_decode_noalloc", "blasst_decode_noalloc_max_bytes", "blasst_status_string", "blasst_version",
     "attention_prefill", "attention_decode", "new_stats", "stats_dict",
     "BLASST_OK", "BLASST_EINVAL", "BLASST_EUNSUPPORTED", "BLASST_ECUDA", "BLASST_ETIMEOUT",
     "BLASST_EWORKSPACE", "BLASST_BF16", "BLASST_FP32",
@@ -88,6 +89,10 @@ def load_library(path: str | None = None):
         lib.blasst_decode_workspace_bytes.restype = sz
         lib.blasst_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp, vp, vp]
         lib.blasst_decode.restype = i
+        lib.blasst_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp, vp]
+        lib.blasst_decode_noalloc.restype = i
+        lib.blasst_decode_noalloc_max_bytes.argtypes = []
+        lib.blasst_decode_noalloc_max_bytes.restype = sz
         lib.blasst_lse_merge.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         lib.blasst_lse_merge.restype = i
         lib.blasst_check.argtypes = [vp]
@@ -180,6 +185,23 @@ def blasst_decode(q, k_cache, v_cache, o, lse, *, lam: float, Bc: int, num_split
         float(lam), Bc, num_splits, _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(skip_mask_out), _ptr(stats_out), _stream(stream))
     _check(rc, "blasst_decode")
+
+
+def blasst_decode_noalloc(q, k_cache, v_cache, o, lse, *, lam: float, Bc: int, num_splits: int,
+                          skip_mask_out=None, stats_out=None, stream=None):
+    """The C entry point of the same name: blasst_decode without a caller
+    workspace (the split partials live in a fixed array inside the library)."""
+    B, Hq = q.shape[0], q.shape[1]
+    d = q.shape[-1]
+    _, Hkv, Lkv, _ = k_cache.shape
+    rc = load_library().blasst_decode_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
+        float(lam), Bc, num_splits, _ptr(skip_mask_out), _ptr(stats_out), _stream(stream))
+    _check(rc, "blasst_decode_noalloc")
+
+
+def blasst_decode_noalloc_max_bytes() -> int:
+    return int(load_library().blasst_decode_noalloc_max_bytes())
 
 
 def blasst_lse_merge(o_parts, lse_parts, o, lse, *, n_rows: int, d: int, num_splits: int,

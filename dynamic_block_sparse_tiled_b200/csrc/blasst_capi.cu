@@ -371,3 +371,64 @@ int blasst_check(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode.
+//
+// Some callers cannot allocate device memory at the point where they run
+// decode: a plugin inside a framework that owns every device allocation
+// through its own pool, a serving loop that has planned its memory once at
+// start-up and must not touch the allocator afterwards, or a host thread for
+// which cudaMalloc would be too costly or would synchronise the device. For
+// them blasst_decode_noalloc keeps the split partials in the fixed array
+// below, which every GPU that loads this library holds (32 MiB) until the
+// process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+
+// Split partials of blasst_decode_noalloc. Host code must not use the
+// symbol's host-side shadow as a device address: the device address comes
+// from cudaGetSymbolAddress, looked up once per device below.
+__device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_decode_scratch on the current device, looked up (and
+// cached) on the first call made with that device current.
+void* decode_scratch() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || ptr == nullptr)
+      return nullptr;
+    g_scratch_ptr[dev] = ptr;
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t blasst_decode_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
+
+int blasst_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o,
+                          float* lse, int B, int Hq, int Hkv, int Lkv, int d, float lambda, int Bc,
+                          int num_splits, uint8_t* skip_mask_out, blasst_stats* stats_out,
+                          void* stream) {
+  if (B <= 0 || Hq <= 0 || d <= 0 || num_splits <= 0) return BLASST_EINVAL;
+  const size_t need = blasst_decode_workspace_bytes(B, Hq, d, num_splits);
+  if (need == 0 || need > kNoAllocScratchBytes) return BLASST_EWORKSPACE;
+  void* scratch = decode_scratch();
+  if (!scratch) return BLASST_ECUDA;
+  // Every partial the merge reads is written by the split kernel of the same
+  // call (empty splits included), so nothing in the array needs clearing.
+  return blasst_decode(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, d, lambda, Bc, num_splits,
+                       scratch, kNoAllocScratchBytes, skip_mask_out, stats_out, stream);
+}
+
+}  // extern "C"

@@ -138,6 +138,34 @@ BLASST_API int blasst_decode(const void* q, const void* k_cache, const void* v_c
                   void* workspace, size_t workspace_bytes, uint8_t* skip_mask_out,
                   blasst_stats* stats_out, void* stream);
 
+/* Allocation-free form of blasst_decode. The pages have no counterpart: this
+ * is for callers that cannot allocate device memory where they run decode
+ * (a plugin inside a framework that owns all device allocations, a serving
+ * loop whose memory was planned once at start-up, a host thread for which a
+ * cudaMalloc would be too costly or would synchronise the device).
+ * Same operation and arguments as blasst_decode, minus the workspace: the
+ * split partials live in a fixed device array inside the library, of
+ * blasst_decode_noalloc_max_bytes() bytes (32 MiB), which every GPU that loads
+ * the library holds until the process exits. The call allocates nothing and
+ * frees nothing.
+ *   - Requests whose partials, blasst_decode_workspace_bytes(B, Hq, d,
+ *     num_splits), exceed that size are rejected with BLASST_EWORKSPACE.
+ *   - The first call on a device looks up the array's device address (one
+ *     cudaGetSymbolAddress with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     every value a call reads back is written earlier in the same call.
+ *     Calls that may run concurrently on the GPU (different streams, or
+ *     different host threads on the same device) race on the array: order
+ *     them on one stream. */
+BLASST_API int blasst_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                     void* o, float* lse, int B, int Hq, int Hkv, int Lkv, int d,
+                                     float lambda, int Bc, int num_splits, uint8_t* skip_mask_out,
+                                     blasst_stats* stats_out, void* stream);
+
+/* Size in bytes of the fixed array blasst_decode_noalloc uses. */
+BLASST_API size_t blasst_decode_noalloc_max_bytes(void);
+
 /* Log-sum-exp merge of split partials (the second half of blasst_decode):
  *   o_parts [n_rows, num_splits, d] fp32, normalised per split;
  *   lse_parts [n_rows, num_splits] fp32, -inf marks an empty split;
