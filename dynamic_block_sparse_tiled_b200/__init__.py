@@ -101,6 +101,8 @@ def load_library(path: str | None = None):
         lib.blasst_status_string.restype = C.c_char_p
         lib.blasst_selftest_exp2.argtypes = [vp, vp, vp, i, vp]
         lib.blasst_selftest_exp2.restype = i
+        lib.blasst_last_cuda_error.argtypes = []
+        lib.blasst_last_cuda_error.restype = C.c_char_p
         lib.blasst_version.argtypes = []
         lib.blasst_version.restype = i
         if path is None:
@@ -143,6 +145,8 @@ def _stream(stream):
 
 def _check(rc: int, where: str):
     if rc != 0:
+        if rc == BLASST_ECUDA:
+            where = f"{where} [{load_library().blasst_last_cuda_error().decode()}]"
         raise BlasstError(rc, where)
 
 

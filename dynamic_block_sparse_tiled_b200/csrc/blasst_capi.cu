@@ -65,6 +65,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Text of the last failing CUDA call made by this library on this host thread.
+thread_local const char* g_last_cuda_error = "no error";
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return BLASST_OK;
+  g_last_cuda_error = cudaGetErrorString(e);
+  return BLASST_ECUDA;
+}
+
 // 3-D map over a dense [heads, L, d] tensor: dims (d, L, heads), box
 // (64 columns, rows, 1), 128-byte swizzle, zero fill outside the tensor.
 bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes,
@@ -86,7 +95,10 @@ bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int el
 
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) g_last_cuda_error = cudaGetErrorString(e);
+  return e;
 }
 
 template <int D, int BC, int BR>
@@ -97,7 +109,7 @@ int launch_prefill_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   if (set_smem(kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
   const dim3 grid(static_cast<unsigned>(p.nQblk) * p.B * p.Hq);
   kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? BLASST_OK : BLASST_ECUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 int dispatch_prefill_bf16(int d, int Bc, int Br, const CUtensorMap& mq, const CUtensorMap& mk,
@@ -125,7 +137,7 @@ int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const blasst::De
   if (set_smem(kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
   const dim3 grid(p.S, p.Hkv, p.B);
   kernel<<<grid, 128, C::SMEM_BYTES, stream>>>(mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? BLASST_OK : BLASST_ECUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 int dispatch_decode(int d, int Bc, int g, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -171,6 +183,8 @@ float log2_lambda_of(float lambda) {
 extern "C" {
 
 int blasst_version(void) { return 100; }
+
+const char* blasst_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char* blasst_status_string(int status) {
   switch (status) {
@@ -287,7 +301,7 @@ int blasst_lse_merge(const float* o_parts, const float* lse_parts, void* o, floa
   } else {
     return BLASST_EINVAL;
   }
-  return cudaGetLastError() == cudaSuccess ? BLASST_OK : BLASST_ECUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
@@ -351,7 +365,7 @@ int blasst_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n, vo
   if (!x || !y_mufu || !y_poly || n <= 0) return BLASST_EINVAL;
   selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_mufu,
                                                                                      y_poly, n);
-  return cudaGetLastError() == cudaSuccess ? BLASST_OK : BLASST_ECUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 int blasst_check(void* stream) {

@@ -24,8 +24,9 @@
 //   warp 9     TMA producer for V: loads V of block j only after the vote on
 //              block j says some row group keeps it;
 //   warp 10    tcgen05 issuer: S = Q K^T into one of two TMEM S buffers,
-//              issued two blocks ahead, then O += P V with P read from one of
-//              two TMEM P buffers. P has TMEM of its own so that the issuer
+//              issued two blocks ahead as soon as the softmax has read the
+//              buffer, then O += P V with P read from one of two TMEM P
+//              buffers. P has TMEM of its own so that the issuer
 //              never waits for an MMA to finish: it waits only for the
 //              softmax (P ready), for K and for V.
 // With Br = 64 the 128 rows form two independent vote groups that share the
@@ -97,14 +98,16 @@ struct PrefillCfg {
   static constexpr int B_KE = B_KF + NK;
   static constexpr int B_VF = B_KE + NK;
   static constexpr int B_VE = B_VF + NV;
-  static constexpr int B_SF = B_VE + NV;
-  static constexpr int B_PV = B_SF + NS;   // P.V done, one barrier per P buffer
+  static constexpr int B_SF = B_VE + NV;   // S written (tcgen05 commit)
+  static constexpr int B_SC = B_SF + NS;   // S read by all softmax warps (buffer reusable)
+  static constexpr int B_PV = B_SC + NS;   // P.V done, one barrier per P buffer
   static constexpr int B_DEC = B_PV + NP;
   static constexpr int B_P = B_DEC + NSLOT;
   static constexpr int B_DRAIN = B_P + NSLOT;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // misc words: [0] tmem base, [1] abort, [4..7] decisions, [8..23] votes (2 x 8 warps)
+  // misc words: [0] tmem base, [1] abort, [4..7] decisions, [8..23] votes (2 x 8 warps),
+  // [24..25] softmax-only abort words (by block parity)
   static constexpr int MISC_BYTES = 128;
   static constexpr int OFF_PMAX = OFF_MISC + MISC_BYTES;  // [2][2 halves][128 rows] floats
   static constexpr int OFF_LSUM = OFF_PMAX + 2 * 2 * 128 * 4;  // [2 halves][128 rows] floats
@@ -141,6 +144,7 @@ __global__ void __launch_bounds__(352, 1)
   volatile int* abort_flag = misc + 1;
   volatile int* dec_val = misc + 4;
   volatile int* votes = misc + 8;
+  volatile int* sm_abort = misc + 24;
   volatile float* pmax = reinterpret_cast<volatile float*>(smem + C::OFF_PMAX);
   volatile float* lsum = reinterpret_cast<volatile float*>(smem + C::OFF_LSUM);
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
@@ -188,7 +192,10 @@ __global__ void __launch_bounds__(352, 1)
       ptx::mbar_init(bar(C::B_VF + i), 1);
       ptx::mbar_init(bar(C::B_VE + i), 1);
     }
-    for (int i = 0; i < C::NS; ++i) ptx::mbar_init(bar(C::B_SF + i), 1);
+    for (int i = 0; i < C::NS; ++i) {
+      ptx::mbar_init(bar(C::B_SF + i), 1);
+      ptx::mbar_init(bar(C::B_SC + i), 8);
+    }
     for (int i = 0; i < C::NP; ++i) ptx::mbar_init(bar(C::B_PV + i), 1);
     for (int i = 0; i < C::NSLOT; ++i) {
       ptx::mbar_init(bar(C::B_DEC + i), 1);
@@ -316,18 +323,22 @@ __global__ void __launch_bounds__(352, 1)
       if (ok && nblk > 1) ok = issue_qk(1);
       int pv_count = 0;
       for (int j = 0; j < nblk && ok; ++j) {
+        // Look-ahead first: S = Q K^T of block j+2 goes into the S buffer of
+        // block j as soon as every softmax warp has read S_j (well before
+        // block j's exponentials are done), keeping the tensor pipe busy
+        // while V_j (requested only after block j's vote) lands.
+        if (j + 2 < nblk) {
+          ok = ptx::mbar_wait(bar(C::B_SC + (j % C::NS)), (j / C::NS) & 1, abort_flag,
+                              p.timeout_ns);
+          if (!ok) break;
+          ok = issue_qk(j + 2);
+          if (!ok) break;
+        }
         const int slot = j % C::NSLOT;
         ok = ptx::mbar_wait(bar(C::B_P + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         ptx::tc_fence_after();
         const bool keep = dec_val[slot] != 0;
-        // Look-ahead first: S = Q K^T of block j+2 goes into the S buffer that
-        // block j's softmax has just finished reading, and keeps the tensor
-        // pipe busy while V_j (requested only after block j's vote) lands.
-        if (j + 2 < nblk) {
-          ok = issue_qk(j + 2);
-          if (!ok) break;
-        }
         if (keep) {
           const int vs = pv_count % C::NV;
           ok = ptx::mbar_wait(bar(C::B_VF + vs), (pv_count / C::NV) & 1, abort_flag,
@@ -371,7 +382,7 @@ __global__ void __launch_bounds__(352, 1)
     const bool leader = threadIdx.x == 0;
 
     float m = -INFINITY, mref = -INFINITY, l = 0.0f;  // l: this half's partial sum
-    int pvn[C::NP] = {0, 0};  // P.V products issued on each P buffer
+    int pvn0 = 0, pvn1 = 0;  // P.V products issued on P buffer 0 / 1
     int last_buf = -1, ncomp = 0;
     bool aborted = false;
 
@@ -395,6 +406,10 @@ __global__ void __launch_bounds__(352, 1)
           ptx::tmem_ld32p(tmem + lane_base + C::S_COL + sbuf * BC + half * C::HALF + 32 * c,
                           sr + 32 * c);
         ptx::tmem_wait_ld();
+        // S_j is in registers: its TMEM buffer may take block j+2's scores.
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_SC + sbuf));
 #pragma unroll
         for (int c = 0; c < C::HALF; ++c) s[c] = __uint_as_float(sr[c]);
         const bool need_mask =
@@ -423,25 +438,35 @@ __global__ void __launch_bounds__(352, 1)
         else rowskip = (mbh - m) < p.log2_lambda;
       }
       pmax[((j & 1) * 2 + half) * 128 + t] = mbh;
-      const unsigned all_skip = __all_sync(0xffffffffu, rowskip) ? 1u : 0u;
-      if (lane == 0) votes[(j & 1) * 8 + warp] = ok ? static_cast<int>(all_skip) : 2;
-      ptx::named_bar_sync(1, C::NSOFT);
-      const float mb = fmaxf(mbh, pmax[((j & 1) * 2 + (half ^ 1)) * 128 + t]);
       int keepmask = 0;
       bool any_abort = false;
+      if constexpr (C::NG == 1) {
+        // One vote group: the barrier itself ANDs the half-row tests of all
+        // 256 softmax threads. A warp whose wait gave up marks the
+        // softmax-private abort word of this block parity before the barrier.
+        if (!ok && lane == 0) sm_abort[j & 1] = 1;
+        const bool all_skip = ptx::named_bar_and(1, C::NSOFT, rowskip);
+        any_abort = sm_abort[j & 1] != 0;
+        if (j <= kt_last[0] && !all_skip) keepmask = 1;
+      } else {
+        const unsigned all_skip = __all_sync(0xffffffffu, rowskip) ? 1u : 0u;
+        if (lane == 0) votes[(j & 1) * 8 + warp] = ok ? static_cast<int>(all_skip) : 2;
+        ptx::named_bar_sync(1, C::NSOFT);
 #pragma unroll
-      for (int gg = 0; gg < C::NG; ++gg) {
-        bool gskip = true;
+        for (int gg = 0; gg < C::NG; ++gg) {
+          bool gskip = true;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
+          for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-          for (int w = 0; w < C::WPG; ++w) {
-            const int v = votes[(j & 1) * 8 + hh * 4 + gg * C::WPG + w];
-            if (v == 2) any_abort = true;
-            gskip = gskip && (v != 0);
-          }
-        if (j <= kt_last[gg] && !gskip) keepmask |= 1 << gg;
+            for (int w = 0; w < C::WPG; ++w) {
+              const int v = votes[(j & 1) * 8 + hh * 4 + gg * C::WPG + w];
+              if (v == 2) any_abort = true;
+              gskip = gskip && (v != 0);
+            }
+          if (j <= kt_last[gg] && !gskip) keepmask |= 1 << gg;
+        }
       }
+      const float mb = fmaxf(mbh, pmax[((j & 1) * 2 + (half ^ 1)) * 128 + t]);
       if (any_abort) {
         aborted = true;
         break;
@@ -460,8 +485,8 @@ __global__ void __launch_bounds__(352, 1)
             // O must be quiescent: wait for the last issued P.V.
             bool ok2 = true;
             if (lane == 0)
-              ok2 = ptx::mbar_wait(bar(C::B_PV + last_buf), (pvn[last_buf] - 1) & 1, abort_flag,
-                                   p.timeout_ns);
+              ok2 = ptx::mbar_wait(bar(C::B_PV + last_buf),
+                                   ((last_buf ? pvn1 : pvn0) - 1) & 1, abort_flag, p.timeout_ns);
             ok2 = __shfl_sync(0xffffffffu, ok2 ? 1 : 0, 0) != 0;
             if (!ok2) {
               *abort_flag = 1;
@@ -496,8 +521,8 @@ __global__ void __launch_bounds__(352, 1)
           for (int c = 0; c < C::HALF; c += 2) {
             float x0, x1, p0, p1;
             ptx::fma2(x0, x1, s[c], s[c + 1], sl2, sl2, neg, neg);
-            // every fourth pair of columns takes the FMA-pipe exp2
-            if (((c >> 1) & 3) == 3) {
+            // every eighth pair of columns takes the FMA-pipe exp2
+            if (((c >> 1) & 7) == 7) {
               ptx::exp2_poly2(p0, p1, x0, x1);
             } else {
               p0 = ptx::ex2(x0);
@@ -513,10 +538,11 @@ __global__ void __launch_bounds__(352, 1)
           for (int c = 0; c < C::HALF / 2; ++c) pk[c] = 0u;
         }
         // P buffer pbuf was last read by the P.V of block j-2 (if computed).
-        if (pvn[pbuf] > 0 && last_buf != -1) {
+        const int pv_here = pbuf ? pvn1 : pvn0;
+        if (pv_here > 0) {
           bool ok3 = true;
           if (lane == 0)
-            ok3 = ptx::mbar_wait(bar(C::B_PV + pbuf), (pvn[pbuf] - 1) & 1, abort_flag,
+            ok3 = ptx::mbar_wait(bar(C::B_PV + pbuf), (pv_here - 1) & 1, abort_flag,
                                  p.timeout_ns);
           ok3 = __shfl_sync(0xffffffffu, ok3 ? 1 : 0, 0) != 0;
           if (!ok3) {
@@ -534,7 +560,8 @@ __global__ void __launch_bounds__(352, 1)
         ptx::tc_fence_before();
         ++ncomp;
         last_buf = pbuf;
-        ++pvn[pbuf];
+        if (pbuf) ++pvn1;
+        else ++pvn0;
       }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(C::B_P + (j % C::NSLOT)));
@@ -549,8 +576,8 @@ __global__ void __launch_bounds__(352, 1)
       // ---- epilogue: O / l -> bf16, lse, masks of unvisited blocks ------
       bool ok = true;
       if (ncomp > 0 && lane == 0)
-        ok = ptx::mbar_wait(bar(C::B_PV + last_buf), (pvn[last_buf] - 1) & 1, abort_flag,
-                            p.timeout_ns);
+        ok = ptx::mbar_wait(bar(C::B_PV + last_buf), ((last_buf ? pvn1 : pvn0) - 1) & 1,
+                            abort_flag, p.timeout_ns);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       ptx::tc_fence_after();
       lsum[half * 128 + t] = l;

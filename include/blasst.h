@@ -183,10 +183,14 @@ BLASST_API int blasst_check(void* stream);
 /* Self-test of the two exponentials the prefill kernel uses, so that a test
  * can check them against float64: y_mufu[i] = 2^x[i] from the hardware
  * approximation (ex2.approx), y_poly[i] = 2^x[i] from the FMA-pipe
- * polynomial that takes a quarter of the softmax exponentials (relative
+ * polynomial that takes part of the softmax exponentials (relative
  * error <= 1.1e-4 for x in [-125, 64]). x, y_mufu, y_poly: device fp32 [n]. */
 BLASST_API int blasst_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n,
                                     void* stream);
+
+/* Text of the last CUDA error this library saw on the calling host thread
+ * (the reason behind the latest BLASST_ECUDA), or "no error". */
+BLASST_API const char* blasst_last_cuda_error(void);
 
 /* Human-readable name of a blasst_status value (static storage). */
 BLASST_API const char* blasst_status_string(int status);
