@@ -135,8 +135,13 @@ int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const blasst::De
   using C = blasst::DecodeCfg<D, BC, G>;
   auto kernel = blasst::blasst_decode_split_kernel<D, BC, G>;
   if (set_smem(kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
-  const dim3 grid(p.S, p.Hkv, p.B);
-  kernel<<<grid, 128, C::SMEM_BYTES, stream>>>(mk, mv, p);
+  // persistent: one CTA per SM, each streaming its share of the splits
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long nsplits = static_cast<long long>(p.B) * p.Hkv * p.S;
+  const unsigned grid = static_cast<unsigned>(nsplits < sms ? nsplits : sms);
+  kernel<<<grid, C::NT, C::SMEM_BYTES, stream>>>(mk, mv, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -11,11 +11,24 @@
 // split is always computed. A block's V rows are fetched only if some head of
 // the GQA group keeps the block.
 //
-// Work split: one CTA of 128 threads per (split, KV head, sequence), holding
-// the G = Hq/Hkv query heads of the group. K blocks stream through a TMA ring
-// (128-byte swizzled tiles, so a thread reading one key row is bank-conflict
-// free); scores on the FMA pipes (M = G rows is far too short for the tensor
-// cores, and the kernel is bound by HBM bytes, not by arithmetic).
+// The kernel is bound by HBM bytes (K always, V of kept blocks), so it is
+// built to keep loads in flight:
+//   - persistent CTAs, one per SM, each streaming a fixed sequence of tasks
+//     (a task = one KV block of one split of one (sequence, KV head)), so the
+//     K prefetch runs across split boundaries without pipeline drains;
+//   - a producer warp streams K through a TMA ring (128-byte swizzled tiles:
+//     a thread reading one key row is bank-conflict free);
+//   - the votes run LA = 2 tasks ahead of the P.V accumulation. A vote needs
+//     only K and the running max, so the arithmetic is unchanged: task n is
+//     scored and voted (its V load issued at once if some head keeps it)
+//     while the P.V of task n-2 is accumulated from a V tile that had two
+//     scoring steps to arrive.
+// The two contractions of a task (q K^T with G = Hq/Hkv rows, and P V) run as
+// warp-level bf16 mma.sync tiles with the G rows padded to 16: far too thin
+// for tcgen05, but one tile instruction replaces hundreds of dependent FMAs
+// and shared-memory loads, which keeps four warps ahead of the HBM stream.
+// Each of the four compute warps owns a quarter of the block's keys; P stays
+// in the accumulator layout of q K^T, which is the operand layout of P V.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -43,32 +56,81 @@ struct DecodeParams {
 
 template <int D, int BC, int G>
 struct DecodeCfg {
-  static constexpr int NT = 128;
-  static constexpr int NK = 2;          // K ring stages
+  static constexpr int NC = 128;        // compute threads (warps 0-3)
+  static constexpr int NT = NC + 32;    // + producer warp 4
+  static constexpr int LA = 2;          // votes run LA tasks ahead of P.V
   static constexpr int DBOX = D / 64;
   static constexpr int KV_BOX = BC * 128;
   static constexpr int KV_BYTES = KV_BOX * DBOX;
-  static constexpr int CPR = D / 8;     // 16-byte chunks per key row
-  static constexpr int KG = NT / CPR;   // key groups in the P.V phase
-  static constexpr int RPT = BC / KG;   // rows per thread in the P.V phase
+  static constexpr int NK = 3;          // K ring stages
+  static constexpr int NV = LA + 1;     // V ring stages
+  static constexpr int NP = LA + 1;     // task records (P fragments, alpha, keep)
+  static constexpr int NFIN = 4;        // split finals ring (> LA + 1 open splits)
+  static constexpr int KW = BC / 4;     // keys per warp
+  static constexpr int NTQ = KW / 8;    // q K^T n-tiles (8 keys) per warp
+  static constexpr int KSP = KW / 16;   // P V k-steps (16 keys) per warp
+  static constexpr int NTO = D / 8;     // P V n-tiles (8 dims)
+  static constexpr int PREGS = KSP * 2; // bf16x2 P registers per thread per task
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
-  // After the last block the K/V ring is idle and holds the final reduction
-  // of the KG partial O accumulators (KG x G x D fp32).
-  static constexpr int RING_BYTES = (NK + 1) * KV_BYTES > KG * G * D * 4 ? (NK + 1) * KV_BYTES
-                                                                         : KG * G * D * 4;
-  static constexpr int OFF_Q = OFF_K + RING_BYTES;         // G x D fp32 (pre-scaled)
-  static constexpr int OFF_P = OFF_Q + G * D * 4;          // G x BC fp32 weights
-  // block maxima (2 x 4 warps x G, double-buffered) then block sums (4 x G)
-  static constexpr int OFF_RED = OFF_P + G * BC * 4;
-  static constexpr int OFF_BAR = (OFF_RED + 12 * G * 4 + 7) & ~7;
-  static constexpr int NBAR = NK + 1;
-  static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static_assert(BC % KG == 0, "rows per thread");
+  static constexpr int OFF_PF = OFF_V + NV * KV_BYTES;              // NP x NC x PREGS words
+  static constexpr int OFF_TASK = OFF_PF + NP * NC * PREGS * 4;      // NP x (G alpha, G keep)
+  static constexpr int OFF_RED = OFF_TASK + NP * 2 * G * 4;          // 4 warps x G max, x G sums
+  static constexpr int OFF_FIN = OFF_RED + 2 * 4 * G * 4;            // NFIN x (G m, G l)
+  static constexpr int OFF_FLAG = OFF_FIN + NFIN * 2 * G * 4;        // abort words
+  static constexpr int OFF_OACC = (OFF_FLAG + 64 + 15) & ~15;        // 4 warps x G x D fp32
+  static constexpr int OFF_BAR = (OFF_OACC + 4 * G * D * 4 + 7) & ~7;
+  static constexpr int NBAR = 2 * NK + NV;                           // K full/empty, V full
+  static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
+  static_assert(G <= 8, "rows of the padded tile");
+  static_assert(KW % 16 == 0 && (D / 16) % 2 == 0 && NTO % 2 == 0, "tile shapes");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
+// Position in the task sequence of one persistent CTA: splits cta,
+// cta + nctas, ... in order, each contributing its blocks.
+struct TaskCursor {
+  int split_id;  // flat (b, hk, split) index; >= nsplits: sequence finished
+  int blk;       // block within the split
+  int nblk;      // blocks in this split
+};
+
+namespace dmma {
+// D = A * B + C, m16n8k16, bf16 inputs, fp32 accumulation (rows 8-15 unused
+// here: a1 = a3 = 0 and c2/c3 discarded).
+__device__ __forceinline__ void mma16816(float& d0, float& d1, uint32_t a0, uint32_t a2, uint32_t b0,
+                                         uint32_t b1, float c0, float c1) {
+  float d2, d3;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%11,%12,%13};"
+      : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(0.0f),
+        "f"(0.0f));
+  (void)d2;
+  (void)d3;
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// Byte offset of the 16-byte chunk holding dims [8*chunk, 8*chunk+8) of row
+// `row` in a 128B-swizzled tile made of 64-column boxes of `box_bytes`.
+__device__ __forceinline__ uint32_t sw_chunk(int row, int chunk, int box_bytes) {
+  return static_cast<uint32_t>((chunk >> 3) * box_bytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+}  // namespace dmma
+
 template <int D, int BC, int G>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(160, 1)
     blasst_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   using C = DecodeCfg<D, BC, G>;
@@ -76,232 +138,358 @@ __global__ void __launch_bounds__(128)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sb = ptx::smem_u32(smem);
-  float* qs = reinterpret_cast<float*>(smem + C::OFF_Q);
-  float* ps = reinterpret_cast<float*>(smem + C::OFF_P);
-  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  uint32_t* pfrag = reinterpret_cast<uint32_t*>(smem + C::OFF_PF);          // [NP][NC][PREGS]
+  float* task_alpha = reinterpret_cast<float*>(smem + C::OFF_TASK);         // [NP][G]
+  int* task_keep = reinterpret_cast<int*>(smem + C::OFF_TASK) + C::NP * G;  // [NP][G]
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);                 // [2][4][G]
+  float* split_fin = reinterpret_cast<float*>(smem + C::OFF_FIN);           // [NFIN][2][G]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
+  volatile int* abort_seen = abort_flag + 2;  // [2], decided by thread 0 per task parity
+  float* oacc = reinterpret_cast<float*>(smem + C::OFF_OACC);               // [4][G][D]
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + C::NBAR * 8);
+  const int B_KF = 0, B_KE = C::NK, B_VF = 2 * C::NK;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-  const int bhk = b * p.Hkv + hk;
-  const int k0 = split * p.Ls;
-  const int k1 = min(k0 + p.Ls, p.Lkv);
-  const int nblk = k1 > k0 ? (k1 - k0 + BC - 1) / BC : 0;
+  const int g = lane >> 2, c4 = lane & 3;  // mma fragment row (head) and column pair
+  const int nsplits = p.B * p.Hkv * p.S;
   const bool thresholding = p.log2_lambda > -INFINITY;
+
+  auto split_blocks = [&](int sid) -> int {
+    const int sp = sid % p.S;
+    const int k0 = sp * p.Ls;
+    const int k1 = min(k0 + p.Ls, p.Lkv);
+    return k1 > k0 ? (k1 - k0 + BC - 1) / BC : 0;
+  };
+  // First split from `sid` on (stepping by the grid) with at least one
+  // block; the compute side writes the partials of the empty ones it passes
+  // (o = 0, lse = -inf).
+  auto advance_split = [&](int sid, bool write_empty) -> TaskCursor {
+    for (; sid < nsplits; sid += gridDim.x) {
+      const int nb = split_blocks(sid);
+      if (nb > 0) return TaskCursor{sid, 0, nb};
+      if (write_empty) {
+        const int sp = sid % p.S, bhk = sid / p.S;
+        const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
+        for (int i = t; i < G * D; i += C::NC) {
+          const int h = i / D, x = i % D;
+          const size_t prow = (static_cast<size_t>(b) * p.Hq + hk * G + h) * p.S + sp;
+          p.o_parts[prow * D + x] = 0.0f;
+          if (x == 0) p.lse_parts[prow] = -INFINITY;
+        }
+      }
+    }
+    return TaskCursor{nsplits, 0, 0};
+  };
+  auto next_task = [&](TaskCursor c, bool write_empty) -> TaskCursor {
+    if (c.blk + 1 < c.nblk) return TaskCursor{c.split_id, c.blk + 1, c.nblk};
+    return advance_split(c.split_id + static_cast<int>(gridDim.x), write_empty);
+  };
+  auto task_key0 = [&](const TaskCursor& c) -> int {
+    return (c.split_id % p.S) * p.Ls + c.blk * BC;
+  };
 
   if (t == 0) {
     for (int i = 0; i < C::NBAR; ++i) ptx::mbar_init(bar(i), 1);
-    *abort_flag = 0;
+    abort_flag[0] = 0;
+    abort_seen[0] = 0;
+    abort_seen[1] = 0;
     ptx::fence_mbar_init();
-  }
-  // Q rows of the group, pre-multiplied by scale*log2(e).
-  for (int i = t; i < G * D; i += C::NT) {
-    const int h = i / D, x = i % D;
-    const int hq = hk * G + h;
-    qs[i] = __bfloat162float(p.q[(static_cast<size_t>(b) * p.Hq + hq) * D + x]) * p.scale_log2;
   }
   __syncthreads();
 
-  auto load_tile = [&](const CUtensorMap* tm, uint32_t dst, int key0, uint32_t fb) {
+  auto load_tile = [&](const CUtensorMap* tm, uint32_t dst, int key0, int bhk, uint32_t fb) {
     ptx::mbar_arrive_expect_tx(fb, C::KV_BYTES);
 #pragma unroll
-    for (int bx = 0; bx < C::DBOX; ++bx) ptx::tma_load_3d(dst + bx * C::KV_BOX, tm, bx * 64, key0, bhk, fb);
+    for (int bx = 0; bx < C::DBOX; ++bx)
+      ptx::tma_load_3d(dst + bx * C::KV_BOX, tm, bx * 64, key0, bhk, fb);
   };
-  if (t == 0) {
-    for (int i = 0; i < min(C::NK, nblk); ++i)
-      load_tile(&tmK, sb + C::OFF_K + i * C::KV_BYTES, k0 + i * BC, bar(i));
+
+  if (warp == 4) {
+    // ======================= K producer ====================================
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmK);
+      TaskCursor c = advance_split(blockIdx.x, false);
+      int n = 0;
+      for (; c.split_id < nsplits; ++n) {
+        const int ks = n % C::NK;
+        if (n >= C::NK &&
+            !ptx::mbar_wait(bar(B_KE + ks), ((n / C::NK) - 1) & 1, abort_flag, p.timeout_ns)) {
+          *abort_flag = 1;
+          break;
+        }
+        load_tile(&tmK, sb + C::OFF_K + ks * C::KV_BYTES, task_key0(c), c.split_id / p.S,
+                  bar(B_KF + ks));
+        c = next_task(c, false);
+      }
+      // Let the last copies land before this warp leaves (they normally have).
+      for (int m = (n > C::NK ? n - C::NK : 0); m < n; ++m)
+        ptx::mbar_wait(bar(B_KF + m % C::NK), (m / C::NK) & 1, abort_flag, p.timeout_ns);
+    }
+    return;  // the producer warp takes no part in the compute barriers
   }
 
-  float m[G], l[G];
+  // ======================= compute warps 0-3 ================================
+  // Warp w owns keys [w*KW, w*KW + KW) of every block; thread (g, c4) holds,
+  // for head g < G, the scores of keys 8j + 2c4, 8j + 2c4 + 1 of each n-tile j
+  // and the outputs of dims 8nn + 2c4, 8nn + 2c4 + 1 of each n-tile nn.
+  float oa[C::NTO][2];
+#pragma unroll
+  for (int i = 0; i < C::NTO; ++i) oa[i][0] = oa[i][1] = 0.0f;
+  uint32_t qa[D / 16][2];  // q fragments (bf16 pairs) of head g for each k-step
+  float m[G], l[G];        // running statistics of the split being voted
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     m[h] = -INFINITY;
     l[h] = 0.0f;
   }
-  // P.V accumulators: thread owns chunk c (8 dims) of rows kg, kg+KG, ...
-  const int c = t % C::CPR, kg = t / C::CPR;
-  float acc[G][8];
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[h][i] = 0.0f;
+  unsigned long long st_vis = 0, st_skip = 0, st_flops = 0, st_bytes = 0;
+  int vcount = 0;     // V tiles issued (thread 0)
+  int vconsumed = 0;  // V tiles consumed by the P.V side
+  bool aborted = false;
 
-  int vphase = 0;
-  unsigned long long st_vis = 0, st_skip = 0, st_vload = 0, st_flops = 0;
-  bool ok = true;
+  TaskCursor pend[C::LA + 1];  // voted tasks awaiting their P.V, oldest first
+  int npend = 0;
+  int q_split = -1;  // split whose q rows are in qa
+  int vote_seq = 0;  // splits finished on the vote side
+  int pv_seq = 0;    // splits finished on the P.V side
 
-  for (int i = 0; i < nblk; ++i) {
-    const int key0 = k0 + i * BC;
-    const int stage = i % C::NK;
-    bool w = true;
-    if (lane == 0) w = ptx::mbar_wait(bar(stage), (i / C::NK) & 1, abort_flag, p.timeout_ns);
-    w = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
-    if (!w) *abort_flag = 1;
-    // ---- scores: thread t <-> key t of the block --------------------------
-    float s[G];
+  auto compute_barrier = [&]() { ptx::named_bar_sync(1, C::NC); };
+
+  // P.V of one voted task, then the split's epilogue if it was its last block.
+  auto do_pv = [&](const TaskCursor& c, int slot) {
+    const int* keep = task_keep + slot * G;
+    int any = 0;
 #pragma unroll
-    for (int h = 0; h < G; ++h) s[h] = 0.0f;
-    const bool key_ok = (t < BC) && (key0 + t < k1);
-    if (t < BC) {
-      const uint8_t* kst = smem + C::OFF_K + stage * C::KV_BYTES;
+    for (int h = 0; h < G; ++h) any |= keep[h];
+    if (c.blk == 0) {
 #pragma unroll
-      for (int bx = 0; bx < C::DBOX; ++bx) {
+      for (int i = 0; i < C::NTO; ++i) oa[i][0] = oa[i][1] = 0.0f;
+    }
+    if (any) {
+      const int vs = vconsumed % C::NV;
+      bool w = true;
+      if (lane == 0)
+        w = ptx::mbar_wait(bar(B_VF + vs), (vconsumed / C::NV) & 1, abort_flag, p.timeout_ns);
+      w = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+      if (!w) *abort_flag = 1;
+      ++vconsumed;
+      const float alpha = g < G ? task_alpha[slot * G + g] : 1.0f;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(kst + bx * C::KV_BOX + t * 128 +
-                                                            ((ch ^ (t & 7)) << 4));
-          const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-          float kf[8];
+      for (int i = 0; i < C::NTO; ++i) {
+        oa[i][0] *= alpha;
+        oa[i][1] *= alpha;
+      }
+      uint32_t pr[C::PREGS];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            kf[2 * e] = __uint_as_float(wds[e] << 16);
-            kf[2 * e + 1] = __uint_as_float(wds[e] & 0xffff0000u);
-          }
-          const int x0 = bx * 64 + ch * 8;
+      for (int i = 0; i < C::PREGS; ++i) pr[i] = pfrag[(slot * C::NC + t) * C::PREGS + i];
+      const uint32_t vst = sb + C::OFF_V + vs * C::KV_BYTES;
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float4 qa = *reinterpret_cast<const float4*>(qs + h * D + x0);
-            const float4 qb = *reinterpret_cast<const float4*>(qs + h * D + x0 + 4);
-            float a = s[h];
-            a = fmaf(qa.x, kf[0], a);
-            a = fmaf(qa.y, kf[1], a);
-            a = fmaf(qa.z, kf[2], a);
-            a = fmaf(qa.w, kf[3], a);
-            a = fmaf(qb.x, kf[4], a);
-            a = fmaf(qb.y, kf[5], a);
-            a = fmaf(qb.z, kf[6], a);
-            a = fmaf(qb.w, kf[7], a);
-            s[h] = a;
-          }
+      for (int k2 = 0; k2 < C::KSP; ++k2) {
+        // keys of this k-step: warp*KW + 16*k2 + [0, 16)
+        const int key = warp * C::KW + 16 * k2 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int nn = 0; nn < C::NTO; nn += 2) {
+          uint32_t b0, b1, b2, b3;
+          dmma::ldsm_x4_t(vst + dmma::sw_chunk(key, nn + (lane >> 4), C::KV_BOX), b0, b1, b2, b3);
+          dmma::mma16816(oa[nn][0], oa[nn][1], pr[2 * k2], pr[2 * k2 + 1], b0, b1, oa[nn][0],
+                         oa[nn][1]);
+          dmma::mma16816(oa[nn + 1][0], oa[nn + 1][1], pr[2 * k2], pr[2 * k2 + 1], b2, b3,
+                         oa[nn + 1][0], oa[nn + 1][1]);
         }
       }
     }
+    if (c.blk + 1 == c.nblk) {
+      // split epilogue: sum the four warps' partial outputs, normalise, write
+      if (g < G) {
 #pragma unroll
-    for (int h = 0; h < G; ++h)
-      if (!key_ok) s[h] = -INFINITY;
-    // ---- block max per head -------------------------------------------------
-    float* redm = red + (i & 1) * 4 * G;
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float v = s[h];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-      if (lane == 0) redm[warp * G + h] = v;
-    }
-    __syncthreads();  // K stage fully read; block maxima visible
-    float mb[G];
-    int keepmask = 0;
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      mb[h] = fmaxf(fmaxf(redm[h], redm[G + h]), fmaxf(redm[2 * G + h], redm[3 * G + h]));
-      const bool skip = (i > 0) && thresholding && (mb[h] - m[h] < p.log2_lambda);
-      if (!skip) keepmask |= 1 << h;
-    }
-    if (*abort_flag) {
-      ok = false;
-      break;
-    }
-    if (t == 0) {
-      if (keepmask) load_tile(&tmV, sb + C::OFF_V, key0, bar(C::NK));
-      if (i + C::NK < nblk) load_tile(&tmK, sb + C::OFF_K + stage * C::KV_BYTES, key0 + C::NK * BC, bar(stage));
-      st_vis += G;
-      st_skip += G - __popc(keepmask);
-      st_vload += keepmask ? 1 : 0;
-      st_flops += 2ull * G * BC * D + 2ull * __popc(keepmask) * BC * D;
-    }
-    if (p.mask && t < G) {
-      const int hq = hk * G + t;
-      p.mask[(static_cast<size_t>(b) * p.Hq + hq) * p.nKt + key0 / BC] = ((keepmask >> t) & 1) ? 0 : 1;
-    }
-    if (!keepmask) continue;  // skipped by every head: no V bytes, no P.V
-
-    // ---- online softmax for the heads that keep the block -------------------
-    float alpha[G];
-    float* reds = red + 8 * G;  // second reduction area (sums)
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const bool kh = (keepmask >> h) & 1;
-      const float m_new = kh ? fmaxf(m[h], mb[h]) : m[h];
-      alpha[h] = (kh && m[h] != m_new) ? ptx::ex2(m[h] - m_new) : 1.0f;
-      const float pv = kh ? ptx::ex2(s[h] - m_new) : 0.0f;
-      if (t < BC) ps[h * BC + t] = pv;
-      float v = pv;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) reds[warp * G + h] = v;
-      m[h] = m_new;
-    }
-    bool vw = true;
-    if (lane == 0) vw = ptx::mbar_wait(bar(C::NK), vphase & 1, abort_flag, p.timeout_ns);
-    vw = __shfl_sync(0xffffffffu, vw ? 1 : 0, 0) != 0;
-    ++vphase;
-    if (!vw) *abort_flag = 1;
-    __syncthreads();  // P weights and partial sums visible, V landed
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      l[h] = l[h] * alpha[h] + (reds[h] + reds[G + h] + reds[2 * G + h] + reds[3 * G + h]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[h][e] *= alpha[h];
-    }
-    // ---- O += P V: rows kg, kg+KG, ... ; dims [8c, 8c+8) -----------------
-    {
-      const uint8_t* vst = smem + C::OFF_V;
-      const int bx = (c * 8) / 64;
-      const int chk = c & 7;
-#pragma unroll 4
-      for (int r = 0; r < C::RPT; ++r) {
-        const int j = kg + r * C::KG;
-        const uint4 raw = *reinterpret_cast<const uint4*>(vst + bx * C::KV_BOX + j * 128 + ((chk ^ (j & 7)) << 4));
-        const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-        float vf[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          vf[2 * e] = __uint_as_float(wds[e] << 16);
-          vf[2 * e + 1] = __uint_as_float(wds[e] & 0xffff0000u);
+        for (int i = 0; i < C::NTO; ++i) {
+          oacc[(warp * G + g) * D + 8 * i + 2 * c4] = oa[i][0];
+          oacc[(warp * G + g) * D + 8 * i + 2 * c4 + 1] = oa[i][1];
         }
+      }
+      compute_barrier();
+      const float* fin = split_fin + (pv_seq % C::NFIN) * 2 * G;  // [m[G], l[G]]
+      const int sp = c.split_id % p.S, bhk = c.split_id / p.S;
+      const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
+      for (int i = t; i < G * D; i += C::NC) {
+        const int h = i / D, x = i % D;
+        const float v = (oacc[(0 * G + h) * D + x] + oacc[(1 * G + h) * D + x]) +
+                        (oacc[(2 * G + h) * D + x] + oacc[(3 * G + h) * D + x]);
+        const float lf = fin[G + h];
+        const size_t prow = (static_cast<size_t>(b) * p.Hq + hk * G + h) * p.S + sp;
+        p.o_parts[prow * D + x] = lf > 0.0f ? v / lf : 0.0f;
+        if (x == 0)
+          p.lse_parts[prow] = lf > 0.0f ? (fin[h] + log2f(lf)) * 0.6931471805599453f : -INFINITY;
+      }
+      compute_barrier();  // oacc free again
+      ++pv_seq;
+    }
+  };
+
+  TaskCursor cur = advance_split(blockIdx.x, true);
+  int n = 0;
+  while (cur.split_id < nsplits || npend > 0) {
+    if (cur.split_id < nsplits) {
+      // ---- score and vote task n -------------------------------------------
+      const int bhk = cur.split_id / p.S;
+      const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
+      if (cur.split_id != q_split) {
+        // q fragments of head g (rows g >= G of the padded tile are zero)
+        const __nv_bfloat16* qrow = p.q + (static_cast<size_t>(b) * p.Hq + hk * G + g) * D;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          qa[kk][0] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * c4) : 0u;
+          qa[kk][1] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 8 + 2 * c4) : 0u;
+        }
+        q_split = cur.split_id;
+      }
+      if (cur.blk == 0) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float pw = ps[h * BC + j];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(pw, vf[e], acc[h][e]);
+          m[h] = -INFINITY;
+          l[h] = 0.0f;
         }
       }
+      const int ks = n % C::NK;
+      bool w = true;
+      if (lane == 0) w = ptx::mbar_wait(bar(B_KF + ks), (n / C::NK) & 1, abort_flag, p.timeout_ns);
+      w = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+      if (!w) *abort_flag = 1;
+      const int key0 = task_key0(cur);
+      const int k1 = min((cur.split_id % p.S) * p.Ls + p.Ls, p.Lkv);
+      // S = q K^T for this warp's keys: n-tile j covers keys warp*KW + 8j + [0, 8)
+      float sc[C::NTQ][2];
+      const uint32_t kst = sb + C::OFF_K + ks * C::KV_BYTES;
+#pragma unroll
+      for (int j = 0; j < C::NTQ; ++j) {
+        sc[j][0] = sc[j][1] = 0.0f;
+        const int key = warp * C::KW + 8 * j + (lane & 7);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; kk += 2) {
+          uint32_t b0, b1, b2, b3;
+          dmma::ldsm_x4(kst + dmma::sw_chunk(key, 2 * kk + (lane >> 3), C::KV_BOX), b0, b1, b2, b3);
+          dmma::mma16816(sc[j][0], sc[j][1], qa[kk][0], qa[kk][1], b0, b1, sc[j][0], sc[j][1]);
+          dmma::mma16816(sc[j][0], sc[j][1], qa[kk + 1][0], qa[kk + 1][1], b2, b3, sc[j][0],
+                         sc[j][1]);
+        }
+      }
+      // scale to log2 units, mask keys outside the split, row max of head g
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < C::NTQ; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int kk = key0 + warp * C::KW + 8 * j + 2 * c4 + e;
+          sc[j][e] = (kk < k1 && g < G) ? sc[j][e] * p.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sc[j][e]);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      if (c4 == 0 && g < G) red[warp * G + g] = mx;
+      if (t == 0) abort_seen[n & 1] = *abort_flag;  // one reading, shared by all below
+      compute_barrier();  // K stage read; maxima visible
+      if (abort_seen[n & 1]) {
+        aborted = true;
+        break;
+      }
+      if (t == 0) ptx::mbar_arrive(bar(B_KE + ks));
+      const int slot = n % C::NP;
+      float mb[G];
+      int keepmask = 0;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        mb[h] = fmaxf(fmaxf(red[h], red[G + h]), fmaxf(red[2 * G + h], red[3 * G + h]));
+        const bool skip = (cur.blk > 0) && thresholding && (mb[h] - m[h] < p.log2_lambda);
+        if (!skip) keepmask |= 1 << h;
+      }
+      if (t == 0) {
+        if (keepmask) {
+          // the stage's previous tile belongs to a task at least LA + 1 back,
+          // whose P.V is done and was followed by the barrier above
+          const int vs = vcount % C::NV;
+          load_tile(&tmV, sb + C::OFF_V + vs * C::KV_BYTES, key0, bhk, bar(B_VF + vs));
+          ++vcount;
+        }
+        st_vis += G;
+        st_skip += G - __popc(keepmask);
+        st_flops += 2ull * G * BC * D + 2ull * __popc(keepmask) * BC * D;
+        st_bytes += static_cast<unsigned long long>(BC) * D * 2ull * (keepmask ? 2ull : 1ull);
+      }
+      if (p.mask && t < G) {
+        const size_t hq = static_cast<size_t>(b) * p.Hq + hk * G + t;
+        p.mask[hq * p.nKt + key0 / BC] = ((keepmask >> t) & 1) ? 0 : 1;
+      }
+      // online softmax on the vote side; P of head g into bf16 fragments
+      float alpha[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const bool kh = (keepmask >> h) & 1;
+        const float m_new = kh ? fmaxf(m[h], mb[h]) : m[h];
+        alpha[h] = (kh && m[h] != m_new) ? ptx::ex2(m[h] - m_new) : 1.0f;
+        if (t == 0) {
+          task_alpha[slot * G + h] = alpha[h];
+          task_keep[slot * G + h] = kh ? 1 : 0;
+        }
+        m[h] = m_new;
+      }
+      const bool gk = g < G && ((keepmask >> g) & 1);
+      const float mg = g < G ? m[g] : 0.0f;
+      float sum = 0.0f;
+      uint32_t pr[C::PREGS];
+#pragma unroll
+      for (int j = 0; j < C::NTQ; ++j) {
+        const float p0 = gk ? ptx::ex2(sc[j][0] - mg) : 0.0f;
+        const float p1 = gk ? ptx::ex2(sc[j][1] - mg) : 0.0f;
+        sum += p0 + p1;
+        pr[j] = ptx::pack_bf16x2(p0, p1);  // n-tile j = (k-step j/2, half j%2)
+      }
+#pragma unroll
+      for (int i = 0; i < C::PREGS; ++i) pfrag[(slot * C::NC + t) * C::PREGS + i] = pr[i];
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      float* reds = red + 4 * G;
+      if (c4 == 0 && g < G) reds[warp * G + g] = sum;
+      compute_barrier();  // sums and the task record visible
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        l[h] = l[h] * alpha[h] + ((reds[h] + reds[G + h]) + (reds[2 * G + h] + reds[3 * G + h]));
+      if (cur.blk + 1 == cur.nblk) {
+        if (t == 0) {
+          float* fin = split_fin + (vote_seq % C::NFIN) * 2 * G;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            fin[h] = m[h];
+            fin[G + h] = l[h];
+          }
+        }
+        ++vote_seq;
+      }
+      pend[npend++] = cur;
+      cur = next_task(cur, true);
+      ++n;
     }
-    __syncthreads();  // V stage and weights free for the next block
+    // ---- P.V of the oldest voted task once LA newer ones are voted (or at the end)
+    if (npend > C::LA || (cur.split_id >= nsplits && npend > 0)) {
+      const int done_n = n - npend;  // task index of pend[0]
+      do_pv(pend[0], done_n % C::NP);
+      for (int i = 1; i < npend; ++i) pend[i - 1] = pend[i];
+      --npend;
+    }
   }
 
-  // ---- reduce the KG partial accumulators, write the split's partials -----
-  __syncthreads();
-  float* oacc = reinterpret_cast<float*>(smem + C::OFF_K);  // K/V ring is idle now
-  if (ok && !*abort_flag) {
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) oacc[(kg * G + h) * D + c * 8 + e] = acc[h][e];
-  }
-  __syncthreads();
-  if (ok && !*abort_flag) {
-    for (int i = t; i < G * D; i += C::NT) {
-      const int h = i / D, x = i % D;
-      float v = 0.0f;
-      for (int k = 0; k < C::KG; ++k) v += oacc[(k * G + h) * D + x];
-      const int hq = hk * G + h;
-      const size_t prow = (static_cast<size_t>(b) * p.Hq + hq) * p.S + split;
-      const bool has = l[h] > 0.0f;
-      p.o_parts[prow * D + x] = has ? v / l[h] : 0.0f;
-      if (x == 0) p.lse_parts[prow] = has ? (m[h] + log2f(l[h])) * 0.6931471805599453f : -INFINITY;
+  if (aborted) {
+    if (t == 0) {
+      if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
+      // V copies issued but not consumed land before the CTA exits
+      for (int v = vconsumed; v < vcount; ++v)
+        ptx::mbar_wait(bar(B_VF + v % C::NV), (v / C::NV) & 1, abort_flag, p.timeout_ns);
     }
-    if (t == 0 && p.stats) {
-      const unsigned long long kvb = static_cast<unsigned long long>(BC) * D * 2ull;
-      atomicAdd(&p.stats->tiles_visited, st_vis);
-      atomicAdd(&p.stats->tiles_skipped, st_skip);
-      atomicAdd(&p.stats->v_blocks_loaded, st_vload);
-      atomicAdd(&p.stats->mma_flops, st_flops);
-      atomicAdd(&p.stats->bytes_loaded, kvb * (nblk + st_vload));
-    }
-  } else if (t == 0) {
-    if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
+  } else if (t == 0 && p.stats) {
+    atomicAdd(&p.stats->tiles_visited, st_vis);
+    atomicAdd(&p.stats->tiles_skipped, st_skip);
+    atomicAdd(&p.stats->v_blocks_loaded, static_cast<unsigned long long>(vcount));
+    atomicAdd(&p.stats->mma_flops, st_flops);
+    atomicAdd(&p.stats->bytes_loaded, st_bytes);
   }
 }
 
