@@ -95,7 +95,9 @@ def profiled_traffic(kernel_key):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """nvidia-smi samples (every 50 ms) of SM clock and throttle reasons while
+    running; entering waits for the first sample so the window covers the
+    timed work."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -110,10 +112,14 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            t0 = time.monotonic()
+            while not self.lines and time.monotonic() - t0 < 10.0 and self.proc.poll() is None:
+                time.sleep(0.01)
+            self.lines.clear()
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -341,6 +347,36 @@ def oracle_sample(w, lam, budget_s, seed=0, inputs=None):
 
 
 # ------------------------------------------------------------------ main
+def run_case(name, lam, calls, overrides=()):
+    """Launch one workload's kernel `calls` times with nothing else on the
+    GPU (the command an ncu capture wraps); exits non-zero on a device error.
+    `overrides` are "field=value" strings applied to the named workload."""
+    import torch
+    import synth
+    import dynamic_block_sparse_tiled_b200 as bl
+    w = synth.CONFIGS[name]
+    for ov in overrides:
+        key, val = ov.split("=", 1)
+        cur = getattr(w, key)
+        w = w.replace(**{key: type(cur)(val) if not isinstance(cur, bool) else val == "1"})
+    inp = synth.generate(w)
+    if w.dtype == "bf16":
+        to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    else:
+        to = lambda a: torch.from_numpy(a).cuda()
+    q, k, v = to(inp.q), to(inp.k), to(inp.v)
+    del inp
+    for _ in range(calls):
+        if w.num_splits:
+            bl.attention_decode(q, k, v, lam=lam, Bc=w.Bc, num_splits=w.num_splits)
+        else:
+            bl.attention_prefill(q, k, v, causal=w.causal, lam=lam, Br=w.Br, Bc=w.Bc)
+    torch.cuda.synchronize()
+    rc = bl.blasst_check()
+    print(json.dumps(dict(case=name, calls=calls, status=bl.blasst_status_string(rc))), flush=True)
+    return 0 if rc == 0 else 1
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -386,11 +422,19 @@ def main():
     ap.add_argument("--impl", default="blasst", choices=["blasst", "reference"])
     ap.add_argument("--quick", action="store_true", help="skip the 128K and decode legs")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--case", default=None,
+                    help="profiling driver: run only this workload's kernel --calls times, untimed")
+    ap.add_argument("--calls", type=int, default=4)
+    ap.add_argument("--lam", type=float, default=LAMBDA)
+    ap.add_argument("--override", action="append", default=[],
+                    help="with --case: replace a workload field, e.g. --override B=4")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     if args.impl == "reference":
         return run_reference(args)
+    if args.case:
+        return run_case(args.case, args.lam, args.calls, args.override)
 
     import torch
     import synth
@@ -425,25 +469,28 @@ def main():
         return float(t.item())
 
     # ---- headline: prefill 32K, lambda 1e-3, literal generator -------------
+    # (the clock record spans the headline steps and the lambda = 0 and
+    # calibrated-variant legs of the same kernel right after them)
     pre = Prefill(w, device)
+    wa = synth.CONFIGS[WORKLOAD + "_a12"]
+    pa = Prefill(wa, device)
     barrier()
     with ClockSampler(local) as clk:
         pre, main_r = measure_prefill(w, LAMBDA, args.steps, args.warmup, device, stream, flush_buf,
                                       pre=pre)
-    barrier()
+        barrier()
+        _, dense_r = measure_prefill(w, 0.0, max(3, args.steps // 2), 3, device, stream, flush_buf,
+                                     pre=pre)
+        pa, a_l = measure_prefill(wa, LAMBDA, max(3, args.steps // 2), 3, device, stream, flush_buf,
+                                  pre=pa)
+        _, a_0 = measure_prefill(wa, 0.0, max(3, args.steps // 2), 3, device, stream, flush_buf,
+                                 pre=pa)
     ms = max_over_ranks(main_r["ms"])
     value = ws * main_r["eff_flops"] / (ms * 1e-3) / 1e12
-    _, dense_r = measure_prefill(w, 0.0, max(3, args.steps // 2), 3, device, stream, flush_buf, pre=pre)
-    del pre
+    del pre, pa
     torch.cuda.empty_cache()
 
     extra = {}
-    wa = synth.CONFIGS[WORKLOAD + "_a12"]
-    pa = Prefill(wa, device)
-    pa, a_l = measure_prefill(wa, LAMBDA, max(3, args.steps // 2), 3, device, stream, flush_buf, pre=pa)
-    _, a_0 = measure_prefill(wa, 0.0, max(3, args.steps // 2), 3, device, stream, flush_buf, pre=pa)
-    del pa
-    torch.cuda.empty_cache()
     extra["structured_a12"] = dict(
         skip_frac=a_l["skip_frac"], ms=a_l["ms"], ms_lambda0=a_0["ms"],
         speedup_vs_lambda0=a_0["ms"] / a_l["ms"],

@@ -15,6 +15,7 @@
 
 #include "../../include/blasst.h"
 #include "decode_sm100.cuh"
+#include "prefill_f32_sm100.cuh"
 #include "prefill_sm100.cuh"
 
 namespace {
@@ -109,6 +110,17 @@ int launch_prefill_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   if (set_smem(kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
   const dim3 grid(static_cast<unsigned>(p.nQblk) * p.B * p.Hq);
   kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int BR>
+int launch_prefill_f32(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const blasst::PrefillParams& p, cudaStream_t stream) {
+  using C = blasst::PrefillF32Cfg<BR>;
+  auto kernel = blasst::blasst_prefill_f32_kernel<BR>;
+  if (set_smem(kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
+  const dim3 grid(static_cast<unsigned>(p.nQblk) * p.B * p.Hq);
+  kernel<<<grid, 128, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -215,7 +227,8 @@ int blasst_fwd_ex(const blasst_fwd_args* a) {
   if (a->d != 64 && a->d != 128) return BLASST_EUNSUPPORTED;
   if ((a->Br != 64 && a->Br != 128) || (a->Bc != 64 && a->Bc != 128)) return BLASST_EUNSUPPORTED;
   if (a->causal && a->Lq > a->Lkv) return BLASST_EUNSUPPORTED;
-  if (a->dtype != BLASST_BF16) return BLASST_EUNSUPPORTED;
+  if (a->dtype != BLASST_BF16 && a->dtype != BLASST_FP32) return BLASST_EUNSUPPORTED;
+  if (a->dtype == BLASST_FP32 && (a->d != 64 || a->Bc != 64)) return BLASST_EUNSUPPORTED;
   if (static_cast<long long>(a->B) * a->Hq > (1ll << 24) ||
       static_cast<long long>(a->B) * a->Hq * ((a->Lq + 127) / 128) > 0x7fffffffll)
     return BLASST_EINVAL;
@@ -247,6 +260,16 @@ int blasst_fwd_ex(const blasst_fwd_args* a) {
   p.timeout_ns = kTimeoutNs;
 
   CUtensorMap mq, mk, mv;
+  if (a->dtype == BLASST_FP32) {
+    const auto dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    if (!make_map(&mq, a->q, dt, 4, a->d, a->Lq, a->B * a->Hq, 128) ||
+        !make_map(&mk, a->k, dt, 4, a->d, a->Lkv, a->B * a->Hkv, a->Bc) ||
+        !make_map(&mv, a->v, dt, 4, a->d, a->Lkv, a->B * a->Hkv, a->Bc))
+      return BLASST_ECUDA;
+    const cudaStream_t s = static_cast<cudaStream_t>(a->stream);
+    return a->Br == 64 ? launch_prefill_f32<64>(mq, mk, mv, p, s)
+                       : launch_prefill_f32<128>(mq, mk, mv, p, s);
+  }
   const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!make_map(&mq, a->q, dt, 2, a->d, a->Lq, a->B * a->Hq, 128) ||
       !make_map(&mk, a->k, dt, 2, a->d, a->Lkv, a->B * a->Hkv, a->Bc) ||

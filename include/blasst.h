@@ -93,8 +93,8 @@ BLASST_API int blasst_fwd(const void* q, const void* k, const void* v, void* o, 
                uint8_t* skip_mask_out);
 
 /* Extended form of blasst_fwd: same operation and arguments plus
- *   dtype      BLASST_BF16 (q, k, v, o bf16) or BLASST_FP32 (fp32; d = 64 only;
- *              scores use an error-compensated three-product tf32 split);
+ *   dtype      BLASST_BF16 (q, k, v, o bf16) or BLASST_FP32 (fp32; d = 64, Bc = 64 only;
+ *              both products use an error-compensated three-product tf32 split);
  *   scale      score scale; <= 0 selects 1/sqrt(d);
  *   stream     cudaStream_t to enqueue on (NULL = legacy default stream);
  *   stats_out  nullable DEVICE pointer; counters are added to it. */

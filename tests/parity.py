@@ -9,6 +9,12 @@ fp64 oracle run with the same Br/Bc/lambda):
         tie band |mu - ln(lambda)| < 1e-3 (mu = the oracle's tile margin).
 Rows of a tile whose decision legitimately differs (tie band) are left out of
 the O/lse comparison: both decisions are correct results of the method.
+
+fp32 inputs (the three-product tf32 split on both contractions, relative
+product error near 2^-20; scores of magnitude <= 30 in log2 units and
+|v| <= 5 give O errors near 1e-4 at worst):
+  O:    max |err| <= 5e-4 and mean |err| <= 5e-5
+  lse:  max |err| <= 2e-4
 """
 from __future__ import annotations
 
@@ -19,6 +25,8 @@ O_MEAN_ABS = 2e-3
 LSE_MAX_ABS = 1e-3
 MASK_AGREE = 0.999
 TIE_BAND = 1e-3
+FP32_TOL = dict(o_max=5e-4, o_mean=5e-5, lse_max=2e-4)
+BF16_TOL = dict(o_max=O_MAX_ABS, o_mean=O_MEAN_ABS, lse_max=LSE_MAX_ABS)
 
 
 def to_device(arr, device="cuda"):
@@ -64,7 +72,8 @@ def compare_outputs(o_gpu, lse_gpu, o_ref, lse_ref, row_ok=None):
                 lse_max=float(lerr.max()) if lerr.size else 0.0)
 
 
-def assert_within(stats: dict, what=""):
-    assert stats["o_max"] <= O_MAX_ABS, f"{what} O max-abs {stats['o_max']:.3e}"
-    assert stats["o_mean"] <= O_MEAN_ABS, f"{what} O mean-abs {stats['o_mean']:.3e}"
-    assert stats["lse_max"] <= LSE_MAX_ABS, f"{what} lse max-abs {stats['lse_max']:.3e}"
+def assert_within(stats: dict, what="", tol=None):
+    tol = BF16_TOL if tol is None else tol
+    assert stats["o_max"] <= tol["o_max"], f"{what} O max-abs {stats['o_max']:.3e}"
+    assert stats["o_mean"] <= tol["o_mean"], f"{what} O mean-abs {stats['o_mean']:.3e}"
+    assert stats["lse_max"] <= tol["lse_max"], f"{what} lse max-abs {stats['lse_max']:.3e}"

@@ -67,6 +67,8 @@ def _fwd(lib, **kw):
     (dict(Bc=256), -2),
     (dict(Lq=300, Lkv=256), -2),    # causal with Lq > Lkv
     (dict(dtype=7), -2),
+    (dict(dtype=1, d=128, Bc=64), -2),   # fp32 is d = 64 only
+    (dict(dtype=1, d=64, Bc=128), -2),   # fp32 is Bc = 64 only
 ])
 def test_fwd_rejects_bad_arguments_without_a_gpu(lib, bad, code):
     assert _fwd(lib, **bad) == code
