@@ -12,7 +12,7 @@
 // output accumulator; the skip test always uses the exact running max.
 //
 // One CTA owns 128 query rows of one (batch, query head) and walks the KV
-// blocks of its KV head. Warp roles (352 threads):
+// blocks of its KV head. Warp roles (384 threads):
 //   warps 0-7  softmax: warps w and w+4 share the 32 rows of TMEM lanes
 //              32*(w%4).. and split the block's columns in halves; each takes
 //              its half-row max, the half-row skip test, exp2, its half of P
@@ -23,12 +23,16 @@
 //              independent of the votes);
 //   warp 9     TMA producer for V: loads V of block j only after the vote on
 //              block j says some row group keeps it;
-//   warp 10    tcgen05 issuer: S = Q K^T into one of two TMEM S buffers,
-//              issued two blocks ahead as soon as the softmax has read the
-//              buffer, then O += P V with P read from one of two TMEM P
-//              buffers. P has TMEM of its own so that the issuer
-//              never waits for an MMA to finish: it waits only for the
-//              softmax (P ready), for K and for V.
+//   warp 10    tcgen05 issuer for S = Q K^T into one of two TMEM S buffers,
+//              two blocks ahead, as soon as the softmax has read the buffer;
+//              it also owns the TMEM allocation;
+//   warp 11    tcgen05 issuer for O += P V, P read from one of two TMEM P
+//              buffers, as soon as P and V are there.
+// The two issuers are separate threads because issuing eight MMAs blocks
+// the issuing thread while the tensor pipe's queue is full: with one
+// thread, P V of block j waited behind the look-ahead Q K^T and vice versa.
+// P has TMEM of its own, so no issuer waits for an MMA to finish; they wait
+// only for the softmax (S read, P ready), for K and for V.
 // With Br = 64 the 128 rows form two independent vote groups that share the
 // MMAs: a group that skips contributes zero rows of P and leaves its running
 // statistics untouched.
@@ -71,9 +75,9 @@ constexpr int pow2_at_least(int x) {
 template <int D, int BC, int BR>
 struct PrefillCfg {
   static constexpr int BM = 128;
-  static constexpr int NTHREADS = 352;
+  static constexpr int NTHREADS = 384;
   static constexpr int NSOFT = 256;      // softmax threads (warps 0-7)
-  static constexpr int WARP_K = 8, WARP_V = 9, WARP_MMA = 10;
+  static constexpr int WARP_K = 8, WARP_V = 9, WARP_MMA = 10, WARP_PV = 11;
   static constexpr int NG = BM / BR;     // vote groups
   static constexpr int WPG = BR / 32;    // TMEM lane quarters per vote group
   static constexpr int HALF = BC / 2;    // S columns per softmax warp
@@ -103,10 +107,11 @@ struct PrefillCfg {
   static constexpr int B_PV = B_SC + NS;   // P.V done, one barrier per P buffer
   static constexpr int B_DEC = B_PV + NP;
   static constexpr int B_P = B_DEC + NSLOT;
-  static constexpr int B_DRAIN = B_P + NSLOT;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_DRAIN = B_P + NSLOT;  // [2]: QK issuer, PV issuer
+  static constexpr int NBAR = B_DRAIN + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // misc words: [0] tmem base, [1] abort, [4..7] decisions, [8..23] votes (2 x 8 warps),
+  // misc words: [0] tmem base, [1] abort, [3] always 0 (for waits only a timeout ends),
+  // [4..7] decisions, [8..23] votes (2 x 8 warps),
   // [24..25] softmax-only abort words (by block parity)
   static constexpr int MISC_BYTES = 128;
   static constexpr int OFF_PMAX = OFF_MISC + MISC_BYTES;  // [2][2 halves][128 rows] floats
@@ -131,7 +136,7 @@ __device__ __forceinline__ void record_error(int* err, int code) {
 }
 
 template <int D, int BC, int BR>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     blasst_prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                                const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -202,6 +207,7 @@ __global__ void __launch_bounds__(352, 1)
       ptx::mbar_init(bar(C::B_P + i), 8);
     }
     ptx::mbar_init(bar(C::B_DRAIN), 1);
+    ptx::mbar_init(bar(C::B_DRAIN + 1), 1);
     for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
     ptx::fence_mbar_init();
   }
@@ -297,22 +303,29 @@ __global__ void __launch_bounds__(352, 1)
       }
     }
   } else if (warp == C::WARP_MMA) {
-    // ======================= tcgen05 issuer ===============================
+    // ======================= tcgen05 issuer: S = Q K^T =====================
     if (lane == 0) {
       bool ok = ptx::mbar_wait(bar(C::B_Q), 0, abort_flag, p.timeout_ns);
       ptx::tc_fence_after();
+      // The few instructions between two tcgen05.mma of one thread are on the
+      // critical path: the descriptors are built once and each k-step adds a
+      // compile-time offset (16-byte units) to the start-address field, which
+      // cannot carry (shared addresses < 256 KB).
+      const uint64_t q_desc = ptx::sw128_desc(sb + C::OFF_Q, 16, 1024);
+      const uint64_t k_desc = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
       auto issue_qk = [&](int j) -> bool {
         const int ks = j % C::NK;
         if (!ptx::mbar_wait(bar(C::B_KF + ks), (j / C::NK) & 1, abort_flag, p.timeout_ns))
           return false;
         ptx::tc_fence_after();
         const uint32_t d_tm = tmem + C::S_COL + (j % C::NS) * BC;
+        const uint64_t kd = k_desc + static_cast<uint64_t>(ks * (C::KV_BYTES >> 4));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = ptx::sw128_desc(sb + C::OFF_Q + (kk >> 2) * C::Q_BOX + (kk & 3) * 32,
-                                             16, 1024);
-          const uint64_t bd = ptx::sw128_desc(
-              sb + C::OFF_K + ks * C::KV_BYTES + (kk >> 2) * C::KV_BOX + (kk & 3) * 32, 16, 1024);
+          const uint64_t a =
+              q_desc + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
+          const uint64_t bd =
+              kd + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
           ptx::mma_ss(d_tm, a, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
         ptx::mma_commit(bar(C::B_KE + ks));
@@ -321,38 +334,47 @@ __global__ void __launch_bounds__(352, 1)
       };
       if (ok) ok = issue_qk(0);
       if (ok && nblk > 1) ok = issue_qk(1);
+      // S = Q K^T of block j+2 goes into the S buffer of block j as soon as
+      // every softmax warp has read S_j (well before block j's exponentials
+      // are done), keeping the tensor pipe busy while V_j lands.
+      for (int j = 0; j + 2 < nblk && ok; ++j) {
+        ok = ptx::mbar_wait(bar(C::B_SC + (j % C::NS)), (j / C::NS) & 1, abort_flag,
+                            p.timeout_ns);
+        if (ok) ok = issue_qk(j + 2);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_error(p.err, BLASST_ETIMEOUT);
+      }
+      // Drain: every MMA issued above has completed before TMEM is freed
+      // (bounded, but not cut short by the abort flag).
+      ptx::mma_commit(bar(C::B_DRAIN));
+      ptx::mbar_wait(bar(C::B_DRAIN), 0, &misc[3], p.timeout_ns);
+    }
+  } else if (warp == C::WARP_PV) {
+    // ======================= tcgen05 issuer: O += P V ======================
+    if (lane == 0) {
+      bool ok = true;
+      const uint64_t v_desc = ptx::sw128_desc(sb + C::OFF_V, C::KV_BOX, 1024);
       int pv_count = 0;
       for (int j = 0; j < nblk && ok; ++j) {
-        // Look-ahead first: S = Q K^T of block j+2 goes into the S buffer of
-        // block j as soon as every softmax warp has read S_j (well before
-        // block j's exponentials are done), keeping the tensor pipe busy
-        // while V_j (requested only after block j's vote) lands.
-        if (j + 2 < nblk) {
-          ok = ptx::mbar_wait(bar(C::B_SC + (j % C::NS)), (j / C::NS) & 1, abort_flag,
-                              p.timeout_ns);
-          if (!ok) break;
-          ok = issue_qk(j + 2);
-          if (!ok) break;
-        }
         const int slot = j % C::NSLOT;
         ok = ptx::mbar_wait(bar(C::B_P + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         ptx::tc_fence_after();
-        const bool keep = dec_val[slot] != 0;
-        if (keep) {
+        if (dec_val[slot] != 0) {
           const int vs = pv_count % C::NV;
           ok = ptx::mbar_wait(bar(C::B_VF + vs), (pv_count / C::NV) & 1, abort_flag,
                               p.timeout_ns);
           if (!ok) break;
           ptx::tc_fence_after();
           const uint32_t p_tm = tmem + C::P_COL + (j % C::NP) * (BC / 2);
+          const uint64_t vd = v_desc + static_cast<uint64_t>(vs * (C::KV_BYTES >> 4));
+          ptx::mma_ts(tmem + C::O_COL, p_tm, vd, C::IDESC_PV, pv_count > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < BC / 16; ++kk) {
-            const uint64_t bd =
-                ptx::sw128_desc(sb + C::OFF_V + vs * C::KV_BYTES + kk * 2048, C::KV_BOX, 1024);
-            ptx::mma_ts(tmem + C::O_COL, p_tm + kk * 8, bd, C::IDESC_PV,
-                        (pv_count > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 1; kk < BC / 16; ++kk)
+            ptx::mma_ts(tmem + C::O_COL, p_tm + kk * 8,
+                        vd + static_cast<uint64_t>(kk * (2048 >> 4)), C::IDESC_PV, 1u);
           ptx::mma_commit(bar(C::B_VE + vs));
           ptx::mma_commit(bar(C::B_PV + (j % C::NP)));
           ++pv_count;
@@ -362,9 +384,8 @@ __global__ void __launch_bounds__(352, 1)
         *abort_flag = 1;
         record_error(p.err, BLASST_ETIMEOUT);
       }
-      // Drain: every MMA issued above has completed before TMEM is freed.
-      ptx::mma_commit(bar(C::B_DRAIN));
-      ptx::mbar_wait(bar(C::B_DRAIN), 0, abort_flag, p.timeout_ns);
+      ptx::mma_commit(bar(C::B_DRAIN + 1));
+      ptx::mbar_wait(bar(C::B_DRAIN + 1), 0, &misc[3], p.timeout_ns);
     }
   } else {
     // ======================= softmax warps 0-7 ===========================

@@ -29,19 +29,20 @@ def run_case(w, lam, items=None, check_stats=True):
     ref = oracle.prefill(inp.q, inp.k, inp.v, causal=w.causal, lam=lam32, Br=w.Br, Bc=w.Bc,
                          items=items)
     nQt, nKt = ref["nQt"], ref["nKt"]
-    o_g = parity.bf16_tensor_to_f64(o)
-    lse_g = lse.cpu().numpy().astype(np.float64)
     mask_g = mask.cpu().numpy()
     items_arr = ref["items"]
     bh = items_arr // nQt
     qt = items_arr % nQt
     b, hq = bh // w.Hq, bh % w.Hq
-    # gather the GPU rows of the listed tiles: [n, Br, d]
+    # gather the GPU rows of the listed tiles on the device: [n, Br, d]
     rows = qt[:, None] * w.Br + np.arange(w.Br)[None, :]
     valid = rows < w.Lq
     rows_c = np.minimum(rows, w.Lq - 1)
-    o_gt = o_g[b[:, None], hq[:, None], rows_c]
-    lse_gt = lse_g[b[:, None], hq[:, None], rows_c]
+    ib, ih, ir = (torch.from_numpy(np.ascontiguousarray(x)).to(o.device)
+                  for x in (np.broadcast_to(b[:, None], rows.shape),
+                            np.broadcast_to(hq[:, None], rows.shape), rows_c))
+    o_gt = parity.bf16_tensor_to_f64(o[ib, ih, ir])
+    lse_gt = lse[ib, ih, ir].cpu().numpy().astype(np.float64)
     mask_gt = mask_g.reshape(w.B * w.Hq, nQt, nKt)[bh, qt]
     n_vis, n_dis, ok, dis = parity.compare_masks(mask_gt, ref["mask"], ref["margin"], lam32)
     assert ok, f"mask: {n_dis} of {n_vis} visited tiles disagree outside the tie band"
@@ -123,6 +124,45 @@ def test_prefill_full_size_sampled(cfg):
     items = sorted(items)[:80]
     for lam in w.lambdas:
         run_case(w, lam, items=items, check_stats=False)
+
+
+def _sampled_items(w, n_heads, n_random, seed=0):
+    """First and last query tile of `n_heads` seeded heads (all heads when
+    there are no more) plus `n_random` seeded random tiles."""
+    nQt = -(-w.Lq // w.Br)
+    nbh = w.B * w.Hq
+    rng = np.random.default_rng(seed)
+    heads = range(nbh) if nbh <= n_heads else rng.choice(nbh, size=n_heads, replace=False)
+    items = set()
+    for bh in heads:
+        items.add(int(bh) * nQt + 0)
+        items.add(int(bh) * nQt + nQt - 1)
+    items.update(int(x) for x in rng.integers(0, nbh * nQt, size=n_random))
+    return sorted(items)
+
+
+@pytest.mark.parametrize("cfg", ["prefill_128k", "prefill_128k_a12"])
+def test_prefill_128k_sampled(cfg):
+    """Full 128K, GQA 32/8, every lambda of the workload, sampled tiles (the
+    last tile of a head sees all 131072 keys)."""
+    w = synth.CONFIGS[cfg]
+    items = _sampled_items(w, 8, 16)
+    lams = w.lambdas if cfg.endswith("_a12") else (0.0, 1e-3)
+    for lam in lams:
+        run_case(w, lam, items=items, check_stats=False)
+
+
+def test_prefill_256k_sampled_with_diffuse_heads():
+    """Full 256K, 8 heads of which 4 carry no structure: sampled tiles of
+    both kinds at lambda = 1e-3 (calibrated amplitude, so the structured
+    heads skip and the diffuse ones keep most blocks)."""
+    w = synth.CONFIGS["prefill_256k_a12"]
+    nQt = -(-w.Lq // w.Br)
+    items = _sampled_items(w, 8, 8)
+    hs = sorted({i // nQt for i in items})
+    assert any(h < 4 for h in hs) and any(h >= 4 for h in hs)
+    r = run_case(w, 1e-3, items=items, check_stats=False)
+    assert 0.0 < r["skip"] < 1.0, r
 
 
 def test_prefill_lambda_monotone_full_size():
