@@ -13,26 +13,24 @@
 //
 // One CTA owns 128 query rows of one (batch, query head) and walks the KV
 // blocks of its KV head. Warp roles (384 threads):
-//   warps 0-7  softmax: warps w and w+4 share the 32 rows of TMEM lanes
-//              32*(w%4).. and split the block's columns in halves; each takes
-//              its half-row max, the half-row skip test, exp2, its half of P
-//              (into TMEM), its half of the lazy O rescale and of the
-//              epilogue. The row skip test is exact on halves:
-//              max(a, b) - m < t  <=>  a - m < t  and  b - m < t;
-//   warp 8     TMA producer for Q and K (K runs ahead through a 3-stage ring,
-//              independent of the votes);
+//   warps 0-3  softmax of the even blocks, warps 4-7 softmax of the odd
+//              blocks; thread t of a set owns row t (TMEM lane t) over all
+//              Bc columns of its blocks. The two sets alternate, so on each
+//              SM sub-partition one warp runs the exponentials of block j
+//              while the other reads S, takes the row max and votes on block
+//              j+1: the latency-bound and the MUFU-bound phases overlap.
+//              The running statistics pass from one set to the other through
+//              shared memory right after each vote (the vote on j+1 needs the
+//              running max after j, nothing else of block j);
+//   warp 8     TMA producer for Q and K (3-stage ring, ahead of the votes);
 //   warp 9     TMA producer for V: loads V of block j only after the vote on
-//              block j says some row group keeps it;
-//   warp 10    tcgen05 issuer for S = Q K^T into one of two TMEM S buffers,
-//              two blocks ahead, as soon as the softmax has read the buffer;
-//              it also owns the TMEM allocation;
-//   warp 11    tcgen05 issuer for O += P V, P read from one of two TMEM P
-//              buffers, as soon as P and V are there.
-// The two issuers are separate threads because issuing eight MMAs blocks
-// the issuing thread while the tensor pipe's queue is full: with one
-// thread, P V of block j waited behind the look-ahead Q K^T and vice versa.
-// P has TMEM of its own, so no issuer waits for an MMA to finish; they wait
-// only for the softmax (S read, P ready), for K and for V.
+//              block j says some row group keeps it; writes the skip mask;
+//   warp 10    tcgen05 issuer for S = Q K^T into one of three TMEM S buffers,
+//              three blocks ahead; owns the TMEM allocation;
+//   warp 11    tcgen05 issuer for O += P V. P (bf16) overwrites the first
+//              Bc/2 columns of its block's S buffer, so an S buffer is reused
+//              once the softmax is done with it and, for a kept block, its
+//              P V has completed.
 // With Br = 64 the 128 rows form two independent vote groups that share the
 // MMAs: a group that skips contributes zero rows of P and leaves its running
 // statistics untouched.
@@ -76,17 +74,16 @@ template <int D, int BC, int BR>
 struct PrefillCfg {
   static constexpr int BM = 128;
   static constexpr int NTHREADS = 384;
-  static constexpr int NSOFT = 256;      // softmax threads (warps 0-7)
+  static constexpr int NSOFT = 256;  // softmax threads (warps 0-7), two sets of 128
   static constexpr int WARP_K = 8, WARP_V = 9, WARP_MMA = 10, WARP_PV = 11;
-  static constexpr int NG = BM / BR;     // vote groups
-  static constexpr int WPG = BR / 32;    // TMEM lane quarters per vote group
-  static constexpr int HALF = BC / 2;    // S columns per softmax warp
-  static constexpr int DHALF = D / 2;    // O columns per softmax warp
+  static constexpr int NG = BM / BR;   // vote groups
+  static constexpr int WPG = BR / 32;  // TMEM lane quarters (warps of a set) per vote group
+  static constexpr int NCH = BC / 32;  // 32-column chunks of a block row
+  static constexpr int KEEPC = NCH < 2 ? NCH : 2;  // chunks kept in registers from the max pass
   static constexpr int NK = 3;
   static constexpr int NV = 2;
-  static constexpr int NS = 2;   // S buffers (fp32, BC columns each)
-  static constexpr int NP = 2;   // P buffers (bf16 pairs, BC/2 columns each)
-  static constexpr int NSLOT = 4;
+  static constexpr int NS = 3;     // S buffers (fp32, BC columns; P aliases the first BC/2)
+  static constexpr int NSLOT = 4;  // decision slots (> NS, see the QK issuer)
   static constexpr int DBOX = D / 64;
   static constexpr int Q_BOX = BM * 128;
   static constexpr int KV_BOX = BC * 128;
@@ -102,24 +99,26 @@ struct PrefillCfg {
   static constexpr int B_KE = B_KF + NK;
   static constexpr int B_VF = B_KE + NK;
   static constexpr int B_VE = B_VF + NV;
-  static constexpr int B_SF = B_VE + NV;   // S written (tcgen05 commit)
-  static constexpr int B_SC = B_SF + NS;   // S read by all softmax warps (buffer reusable)
-  static constexpr int B_PV = B_SC + NS;   // P.V done, one barrier per P buffer
-  static constexpr int B_DEC = B_PV + NP;
-  static constexpr int B_P = B_DEC + NSLOT;
-  static constexpr int B_DRAIN = B_P + NSLOT;  // [2]: QK issuer, PV issuer
+  static constexpr int B_SF = B_VE + NV;   // [NS] S written (tcgen05 commit)
+  static constexpr int B_SC = B_SF + NS;   // [NS] block done with by softmax, PV issuer, V producer
+  static constexpr int B_PV = B_SC + NS;   // [NS] P V of the buffer's block done
+  static constexpr int B_DEC = B_PV + NS;  // [NSLOT] decision (V producer)
+  static constexpr int B_P = B_DEC + NSLOT;  // [NSLOT] P ready or block skipped (PV issuer)
+  static constexpr int B_HS = B_P + NSLOT;   // [2] running statistics handed to set s
+  static constexpr int B_DRAIN = B_HS + 2;   // [2] QK issuer, PV issuer
   static constexpr int NBAR = B_DRAIN + 2;
+  static constexpr int SC_COUNT = 4 + 2;     // a softmax set's 4 warps, PV issuer, V producer
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // misc words: [0] tmem base, [1] abort, [3] always 0 (for waits only a timeout ends),
-  // [4..7] decisions, [8..23] votes (2 x 8 warps),
-  // [24..25] softmax-only abort words (by block parity)
+  // misc words: [0] tmem base, [1] abort, [3] always 0 (for waits only a timeout
+  // ends), [4..7] decisions, [8..15] votes [set][warp of set] (Br = 64),
+  // [16..17] softmax abort word per set, [20..21] last kept block handed to set
+  // s, [24..29] kept blocks per S buffer handed to set s ([s][3])
   static constexpr int MISC_BYTES = 128;
-  static constexpr int OFF_PMAX = OFF_MISC + MISC_BYTES;  // [2][2 halves][128 rows] floats
-  static constexpr int OFF_LSUM = OFF_PMAX + 2 * 2 * 128 * 4;  // [2 halves][128 rows] floats
+  static constexpr int OFF_ST = OFF_MISC + MISC_BYTES;  // [2 sets][2: m, mref][128 rows] floats
+  static constexpr int OFF_LSUM = OFF_ST + 2 * 2 * 128 * 4;  // [2 sets][128 rows] floats
   static constexpr int SMEM_BYTES = OFF_LSUM + 2 * 128 * 4 + 1024;  // + alignment slack
-  static constexpr int S_COL = 0;                   // S buffer b at column b * BC
-  static constexpr int P_COL = NS * BC;             // P buffer b at P_COL + b * BC / 2
-  static constexpr int O_COL = P_COL + NP * BC / 2; // O accumulator
+  static constexpr int S_COL = 0;          // S buffer b at column b * BC (P: first BC/2)
+  static constexpr int O_COL = NS * BC;    // O accumulator
   static constexpr int TMEM_COLS = pow2_at_least(O_COL + D);
   static constexpr uint32_t IDESC_QK = ptx::idesc_f32acc(1, 128, BC, false);
   static constexpr uint32_t IDESC_PV = ptx::idesc_f32acc(1, 128, D, true);
@@ -129,6 +128,7 @@ struct PrefillCfg {
   static_assert(BR == 64 || BR == 128, "query tile");
   static_assert(TMEM_COLS <= 512, "TMEM budget");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(NSLOT > NS, "decision slots must outlive the S look-ahead");
 };
 
 __device__ __forceinline__ void record_error(int* err, int code) {
@@ -149,8 +149,10 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = misc + 1;
   volatile int* dec_val = misc + 4;
   volatile int* votes = misc + 8;
-  volatile int* sm_abort = misc + 24;
-  volatile float* pmax = reinterpret_cast<volatile float*>(smem + C::OFF_PMAX);
+  volatile int* sm_abort = misc + 16;
+  volatile int* st_last = misc + 20;
+  volatile int* st_cnt = misc + 24;
+  volatile float* st_rows = reinterpret_cast<volatile float*>(smem + C::OFF_ST);
   volatile float* lsum = reinterpret_cast<volatile float*>(smem + C::OFF_LSUM);
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
 
@@ -199,15 +201,17 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 0; i < C::NS; ++i) {
       ptx::mbar_init(bar(C::B_SF + i), 1);
-      ptx::mbar_init(bar(C::B_SC + i), 8);
+      ptx::mbar_init(bar(C::B_SC + i), C::SC_COUNT);
+      ptx::mbar_init(bar(C::B_PV + i), 1);
     }
-    for (int i = 0; i < C::NP; ++i) ptx::mbar_init(bar(C::B_PV + i), 1);
     for (int i = 0; i < C::NSLOT; ++i) {
       ptx::mbar_init(bar(C::B_DEC + i), 1);
-      ptx::mbar_init(bar(C::B_P + i), 8);
+      ptx::mbar_init(bar(C::B_P + i), 4);
     }
-    ptx::mbar_init(bar(C::B_DRAIN), 1);
-    ptx::mbar_init(bar(C::B_DRAIN + 1), 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(C::B_HS + i), 4);
+      ptx::mbar_init(bar(C::B_DRAIN + i), 1);
+    }
     for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
     ptx::fence_mbar_init();
   }
@@ -249,7 +253,7 @@ __global__ void __launch_bounds__(384, 1)
         *abort_flag = 1;
         record_error(p.err, BLASST_ETIMEOUT);
         // Let the copies already in flight land before the CTA exits.
-        ptx::mbar_wait(bar(C::B_Q), 0, abort_flag, p.timeout_ns);
+        ptx::mbar_wait(bar(C::B_Q), 0, &misc[3], p.timeout_ns);
       }
     }
   } else if (warp == C::WARP_V) {
@@ -264,6 +268,7 @@ __global__ void __launch_bounds__(384, 1)
         ok = ptx::mbar_wait(bar(C::B_DEC + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         const int keepmask = dec_val[slot];
+        ptx::mbar_arrive(bar(C::B_SC + (j % C::NS)));  // decision slot read
         // skip-mask entries and counters for block j (off the softmax path)
         const unsigned long long tile_flops = 2ull * 128ull * BC * D;
         st_flops += tile_flops + (keepmask ? tile_flops : 0ull);
@@ -332,15 +337,24 @@ __global__ void __launch_bounds__(384, 1)
         ptx::mma_commit(bar(C::B_SF + (j % C::NS)));
         return true;
       };
-      if (ok) ok = issue_qk(0);
-      if (ok && nblk > 1) ok = issue_qk(1);
-      // S = Q K^T of block j+2 goes into the S buffer of block j as soon as
-      // every softmax warp has read S_j (well before block j's exponentials
-      // are done), keeping the tensor pipe busy while V_j lands.
-      for (int j = 0; j + 2 < nblk && ok; ++j) {
-        ok = ptx::mbar_wait(bar(C::B_SC + (j % C::NS)), (j / C::NS) & 1, abort_flag,
-                            p.timeout_ns);
-        if (ok) ok = issue_qk(j + 2);
+      for (int j = 0; j < C::NS && j < nblk && ok; ++j) ok = issue_qk(j);
+      // S buffer j % NS takes block j+NS once block j is done with: the
+      // softmax has read S_j (and written P_j), the PV issuer and the V
+      // producer have read decision j (so decision slots and the P / DEC
+      // barriers are never more than NS blocks ahead of their readers), and,
+      // when block j was kept, its P V has completed.
+      int kept[C::NS] = {};
+      for (int j = 0; j + C::NS < nblk && ok; ++j) {
+        const int bsl = j % C::NS;
+        ok = ptx::mbar_wait(bar(C::B_SC + bsl), (j / C::NS) & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        if (dec_val[j % C::NSLOT] != 0) {
+          ++kept[bsl];
+          ok = ptx::mbar_wait(bar(C::B_PV + bsl), (kept[bsl] - 1) & 1, abort_flag,
+                              p.timeout_ns);
+          if (!ok) break;
+        }
+        ok = issue_qk(j + C::NS);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -362,13 +376,15 @@ __global__ void __launch_bounds__(384, 1)
         ok = ptx::mbar_wait(bar(C::B_P + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         ptx::tc_fence_after();
-        if (dec_val[slot] != 0) {
+        const bool keep = dec_val[slot] != 0;
+        ptx::mbar_arrive(bar(C::B_SC + (j % C::NS)));  // decision slot read
+        if (keep) {
           const int vs = pv_count % C::NV;
           ok = ptx::mbar_wait(bar(C::B_VF + vs), (pv_count / C::NV) & 1, abort_flag,
                               p.timeout_ns);
           if (!ok) break;
           ptx::tc_fence_after();
-          const uint32_t p_tm = tmem + C::P_COL + (j % C::NP) * (BC / 2);
+          const uint32_t p_tm = tmem + C::S_COL + (j % C::NS) * BC;
           const uint64_t vd = v_desc + static_cast<uint64_t>(vs * (C::KV_BYTES >> 4));
           ptx::mma_ts(tmem + C::O_COL, p_tm, vd, C::IDESC_PV, pv_count > 0 ? 1u : 0u);
 #pragma unroll
@@ -376,7 +392,7 @@ __global__ void __launch_bounds__(384, 1)
             ptx::mma_ts(tmem + C::O_COL, p_tm + kk * 8,
                         vd + static_cast<uint64_t>(kk * (2048 >> 4)), C::IDESC_PV, 1u);
           ptx::mma_commit(bar(C::B_VE + vs));
-          ptx::mma_commit(bar(C::B_PV + (j % C::NP)));
+          ptx::mma_commit(bar(C::B_PV + (j % C::NS)));
           ++pv_count;
         }
       }
@@ -389,8 +405,8 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else {
     // ======================= softmax warps 0-7 ===========================
+    const int set = warp >> 2;        // 0: even blocks, 1: odd blocks
     const int quad = warp & 3;        // TMEM lane quarter
-    const int half = warp >> 2;       // column half
     const int t = quad * 32 + lane;   // row within the CTA tile
     const int row = r0 + t;
     const bool row_exists = row < p.Lq;
@@ -400,245 +416,271 @@ __global__ void __launch_bounds__(384, 1)
     const int last_col = p.causal ? min(row + p.off, p.Lkv - 1) : p.Lkv - 1;
     const float sl2 = p.scale_log2;
     const bool thresholding = p.log2_lambda > -INFINITY;
-    const bool leader = threadIdx.x == 0;
+    const bool leader = lane == 0 && quad == 0;  // one per set
+    volatile float* st_out = st_rows + (1 - set) * 256;  // handed to the other set
+    volatile float* st_in = st_rows + set * 256;
 
-    float m = -INFINITY, mref = -INFINITY, l = 0.0f;  // l: this half's partial sum
-    int pvn0 = 0, pvn1 = 0;  // P.V products issued on P buffer 0 / 1
-    int last_buf = -1, ncomp = 0;
+    // l: this set's partial row sum, relative to the reference lref
+    float l = 0.0f, lref = -INFINITY;
     bool aborted = false;
 
-    for (int j = 0; j < nblk; ++j) {
-      const int sbuf = j % C::NS;
-      const int pbuf = j % C::NP;
+    auto lane0_wait = [&](uint32_t bar_addr, uint32_t parity) -> bool {
       bool ok = true;
-      if (lane == 0)
-        ok = ptx::mbar_wait(bar(C::B_SF + sbuf), (j / C::NS) & 1, abort_flag, p.timeout_ns);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (lane == 0) ok = ptx::mbar_wait(bar_addr, parity, abort_flag, p.timeout_ns);
+      return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    };
+
+    for (int j = set; j < nblk; j += 2) {
+      const int sbuf = j % C::NS;
+      const uint32_t s_tm = tmem + lane_base + C::S_COL + sbuf * BC;
+      bool ok = lane0_wait(bar(C::B_SF + sbuf), (j / C::NS) & 1);
       ptx::tc_fence_after();
 
-      float s[C::HALF];
-      float mbh = -INFINITY;  // this half-row's max (log2 units)
-      bool rowskip = true;
-      const int col0 = j * BC + half * C::HALF;
+      // ---- row max of block j (masked), first chunks kept in registers ---
+      uint32_t sk[C::KEEPC * 32];
+      float mbh = -INFINITY;
+      const int col0 = j * BC;
+      const bool need_mask = (col0 + BC > p.Lkv) || (p.causal && col0 + BC - 1 > r0 + p.off);
       if (ok) {
-        uint32_t sr[C::HALF];
+        float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < C::HALF / 32; ++c)
-          ptx::tmem_ld32p(tmem + lane_base + C::S_COL + sbuf * BC + half * C::HALF + 32 * c,
-                          sr + 32 * c);
-        ptx::tmem_wait_ld();
-        // S_j is in registers: its TMEM buffer may take block j+2's scores.
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(C::B_SC + sbuf));
+        for (int c = 0; c < C::NCH; ++c) {
+          uint32_t tmp[32];
+          uint32_t* sr = c < C::KEEPC ? sk + 32 * c : tmp;
+          ptx::tmem_ld32p(s_tm + 32 * c, sr);
+          ptx::tmem_wait_ld();
+          if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < C::HALF; ++c) s[c] = __uint_as_float(sr[c]);
-        const bool need_mask =
-            (j * BC + BC > p.Lkv) || (p.causal && j * BC + BC - 1 > r0 + p.off);
-        if (need_mask) {
+            for (int i = 0; i < 32; ++i)
+              if (col0 + 32 * c + i > last_col) sr[i] = __float_as_uint(-INFINITY);
+          }
 #pragma unroll
-          for (int c = 0; c < C::HALF; ++c)
-            if (col0 + c > last_col) s[c] = -INFINITY;
+          for (int i = 0; i < 32; i += 8) {
+            mc[0] = ptx::fmax3(mc[0], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+            mc[1] = ptx::fmax3(mc[1], __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+            mc[2] = ptx::fmax3(mc[2], __uint_as_float(sr[i + 4]), __uint_as_float(sr[i + 5]));
+            mc[3] = ptx::fmax3(mc[3], __uint_as_float(sr[i + 6]), __uint_as_float(sr[i + 7]));
+          }
         }
-        // half-row max: 8 independent chains of three-input max, then a tree
-        float mc[8];
+        mbh = fmaxf(ptx::fmax3(mc[0], mc[1], mc[2]), mc[3]) * sl2;
+      }
+
+      // ---- running statistics after block j-1 (from the other set) -------
+      float m = -INFINITY, mref = -INFINITY;
+      int last_kept = -1;
+      int cnt[C::NS];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          constexpr int W = C::HALF / 8;
-          float a = s[i * W];
+      for (int i = 0; i < C::NS; ++i) cnt[i] = 0;
+      if (j > 0) {
+        const bool ok2 = lane0_wait(bar(C::B_HS + set), ((j - 1) >> 1) & 1);
+        ok = ok && ok2;
+        m = st_in[t];
+        mref = st_in[128 + t];
+        last_kept = st_last[set];
 #pragma unroll
-          for (int c = 1; c + 1 < W; c += 2) a = ptx::fmax3(a, s[i * W + c], s[i * W + c + 1]);
-          if ((W - 1) % 2) a = fmaxf(a, s[i * W + W - 1]);
-          mc[i] = a;
-        }
-        mbh = ptx::fmax3(ptx::fmax3(mc[0], mc[1], mc[2]), ptx::fmax3(mc[3], mc[4], mc[5]),
-                         fmaxf(mc[6], mc[7])) * sl2;
+        for (int i = 0; i < C::NS; ++i) cnt[i] = st_cnt[set * 4 + i];
+      }
+
+      // ---- the vote: every row of the tile (group) must find block j
+      //      negligible; a block beyond a row's causal range votes skip -----
+      bool rowskip = true;
+      if (ok) {
         const bool visited = j <= my_kt_last;
         if (!row_exists || !visited) rowskip = true;
         else if (j == 0 || !thresholding) rowskip = false;
         else rowskip = (mbh - m) < p.log2_lambda;
       }
-      pmax[((j & 1) * 2 + half) * 128 + t] = mbh;
       int keepmask = 0;
       bool any_abort = false;
       if constexpr (C::NG == 1) {
-        // One vote group: the barrier itself ANDs the half-row tests of all
-        // 256 softmax threads. A warp whose wait gave up marks the
-        // softmax-private abort word of this block parity before the barrier.
-        if (!ok && lane == 0) sm_abort[j & 1] = 1;
-        const bool all_skip = ptx::named_bar_and(1, C::NSOFT, rowskip);
-        any_abort = sm_abort[j & 1] != 0;
+        if (!ok && lane == 0) sm_abort[set] = 1;
+        const bool all_skip = ptx::named_bar_and(1 + set, 128, rowskip);
+        any_abort = sm_abort[set] != 0;
         if (j <= kt_last[0] && !all_skip) keepmask = 1;
       } else {
         const unsigned all_skip = __all_sync(0xffffffffu, rowskip) ? 1u : 0u;
-        if (lane == 0) votes[(j & 1) * 8 + warp] = ok ? static_cast<int>(all_skip) : 2;
-        ptx::named_bar_sync(1, C::NSOFT);
+        volatile int* vw = votes + set * 4;  // one word per warp of the set
+        if (lane == 0) vw[quad] = ok ? static_cast<int>(all_skip) : 2;
+        ptx::named_bar_sync(1 + set, 128);
 #pragma unroll
         for (int gg = 0; gg < C::NG; ++gg) {
           bool gskip = true;
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-            for (int w = 0; w < C::WPG; ++w) {
-              const int v = votes[(j & 1) * 8 + hh * 4 + gg * C::WPG + w];
-              if (v == 2) any_abort = true;
-              gskip = gskip && (v != 0);
-            }
+          for (int w = 0; w < C::WPG; ++w) {
+            const int v = vw[gg * C::WPG + w];
+            if (v == 2) any_abort = true;
+            gskip = gskip && (v != 0);
+          }
           if (j <= kt_last[gg] && !gskip) keepmask |= 1 << gg;
         }
+        if (sm_abort[set] != 0) any_abort = true;
+        // the words are rewritten only after this set's next barrier below
+        ptx::named_bar_sync(1 + set, 128);
       }
-      const float mb = fmaxf(mbh, pmax[((j & 1) * 2 + (half ^ 1)) * 128 + t]);
       if (any_abort) {
         aborted = true;
         break;
       }
+
+      // ---- new running statistics, handed to the other set ---------------
+      const bool my_keep = (keepmask >> gi) & 1;
+      const float m_new = my_keep ? fmaxf(m, mbh) : m;
+      const bool need = my_keep && (m_new > mref + C::TAU);
+      const float mref_new = need ? m_new : mref;
+      st_out[t] = m_new;
+      st_out[128 + t] = mref_new;
       if (leader) {
+        st_last[1 - set] = keepmask ? j : last_kept;
+#pragma unroll
+        for (int i = 0; i < C::NS; ++i)
+          st_cnt[(1 - set) * 4 + i] = cnt[i] + ((keepmask && i == sbuf) ? 1 : 0);
         dec_val[j % C::NSLOT] = keepmask;
         ptx::mbar_arrive(bar(C::B_DEC + (j % C::NSLOT)));
       }
-      if (keepmask) {
-        const bool my_keep = (keepmask >> gi) & 1;
-        const float m_new = my_keep ? fmaxf(m, mb) : m;
-        const bool need = my_keep && (m_new > mref + C::TAU);
-        if (__any_sync(0xffffffffu, need)) {
-          const float mref_new = need ? m_new : mref;
-          if (ncomp > 0) {
-            // O must be quiescent: wait for the last issued P.V.
-            bool ok2 = true;
-            if (lane == 0)
-              ok2 = ptx::mbar_wait(bar(C::B_PV + last_buf),
-                                   ((last_buf ? pvn1 : pvn0) - 1) & 1, abort_flag, p.timeout_ns);
-            ok2 = __shfl_sync(0xffffffffu, ok2 ? 1 : 0, 0) != 0;
-            if (!ok2) {
-              *abort_flag = 1;
-              record_error(p.err, BLASST_ETIMEOUT);
-            }
-            ptx::tc_fence_after();
-            const float alpha = need ? ptx::ex2(mref - mref_new) : 1.0f;
-            l *= alpha;
-#pragma unroll
-            for (int c = 0; c < C::DHALF / 32; ++c) {
-              uint32_t r[32];
-              const uint32_t ta = tmem + lane_base + C::O_COL + half * C::DHALF + 32 * c;
-              ptx::tmem_ld32(ta, r);
-              ptx::tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-              ptx::tmem_st32(ta, r);
-            }
-            ptx::tmem_wait_st();
-          }
-          mref = mref_new;
-        }
-        if (my_keep) m = m_new;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::B_HS + (1 - set)));
 
-        uint32_t pk[C::HALF / 2];
-        if (my_keep) {
-          const float neg = -mref;
-          float rs[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) rs[i] = 0.0f;
-#pragma unroll
-          for (int c = 0; c < C::HALF; c += 2) {
-            float x0, x1, p0, p1;
-            ptx::fma2(x0, x1, s[c], s[c + 1], sl2, sl2, neg, neg);
-            // every eighth pair of columns takes the FMA-pipe exp2
-            if (((c >> 1) & 7) == 7) {
-              ptx::exp2_poly2(p0, p1, x0, x1);
-            } else {
-              p0 = ptx::ex2(x0);
-              p1 = ptx::ex2(x1);
-            }
-            const int a = ((c >> 1) & 3) * 2;
-            ptx::add2(rs[a], rs[a + 1], rs[a], rs[a + 1], p0, p1);
-            pk[c / 2] = ptx::pack_bf16x2(p0, p1);
-          }
-          l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < C::HALF / 2; ++c) pk[c] = 0u;
+      if (keepmask) {
+        // l and O follow the reference mref_new
+        if (mref_new != lref) {
+          l = (lref == -INFINITY) ? 0.0f : l * ptx::ex2(lref - mref_new);
+          lref = mref_new;
         }
-        // P buffer pbuf was last read by the P.V of block j-2 (if computed).
-        const int pv_here = pbuf ? pvn1 : pvn0;
-        if (pv_here > 0) {
-          bool ok3 = true;
-          if (lane == 0)
-            ok3 = ptx::mbar_wait(bar(C::B_PV + pbuf), (pv_here - 1) & 1, abort_flag,
-                                 p.timeout_ns);
-          ok3 = __shfl_sync(0xffffffffu, ok3 ? 1 : 0, 0) != 0;
+        if (__any_sync(0xffffffffu, need) && last_kept >= 0) {
+          // O must be quiescent: wait for the last issued P V.
+          const int lb = last_kept % C::NS;
+          const bool ok3 = lane0_wait(bar(C::B_PV + lb), (cnt[lb] - 1) & 1);
           if (!ok3) {
             *abort_flag = 1;
+            if (lane == 0) sm_abort[set] = 1;
             record_error(p.err, BLASST_ETIMEOUT);
           }
           ptx::tc_fence_after();
-        }
+          const float alpha = need ? ptx::ex2(mref - mref_new) : 1.0f;
 #pragma unroll
-        for (int c = 0; c < C::HALF / 32; ++c)
-          ptx::tmem_st16(tmem + lane_base + C::P_COL + pbuf * (BC / 2) + half * (C::HALF / 2) +
-                             16 * c,
-                         pk + 16 * c);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            const uint32_t ta = tmem + lane_base + C::O_COL + 32 * c;
+            ptx::tmem_ld32(ta, r);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            ptx::tmem_st32(ta, r);
+          }
+          ptx::tmem_wait_st();
+        }
+
+        // ---- P = exp2(s * scale*log2e - mref) as bf16 over S's first half -
+        const float neg = -mref_new;
+        float rs[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rs[i] = 0.0f;
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          uint32_t tmp[32];
+          uint32_t* sr = c < C::KEEPC ? sk + 32 * c : tmp;
+          if (c >= C::KEEPC) {
+            ptx::tmem_ld32p(s_tm + 32 * c, sr);
+            ptx::tmem_wait_ld();
+            if (need_mask) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (col0 + 32 * c + i > last_col) sr[i] = __float_as_uint(-INFINITY);
+            }
+          }
+          uint32_t pk[16];
+          if (my_keep) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              float x0, x1, p0, p1;
+              ptx::fma2(x0, x1, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]), sl2, sl2,
+                        neg, neg);
+              // every eighth pair of columns takes the FMA-pipe exp2
+              if (((i >> 1) & 7) == 7) {
+                ptx::exp2_poly2(p0, p1, x0, x1);
+              } else {
+                p0 = ptx::ex2(x0);
+                p1 = ptx::ex2(x1);
+              }
+              const int a = ((i >> 1) & 3) * 2;
+              ptx::add2(rs[a], rs[a + 1], rs[a], rs[a + 1], p0, p1);
+              pk[i / 2] = ptx::pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+          }
+          // P columns [16c, 16c+16) overwrite S columns already in registers
+          ptx::tmem_st16(s_tm + 16 * c, pk);
+        }
+        l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ++ncomp;
-        last_buf = pbuf;
-        if (pbuf) ++pvn1;
-        else ++pvn0;
       }
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(C::B_P + (j % C::NSLOT)));
+      if (lane == 0) {
+        ptx::mbar_arrive(bar(C::B_P + (j % C::NSLOT)));
+        ptx::mbar_arrive(bar(C::B_SC + sbuf));
+      }
     }
 
-    if (aborted) {
-      if (leader) {
-        *abort_flag = 1;
-        record_error(p.err, BLASST_ETIMEOUT);
-      }
+    // ---- epilogue ----------------------------------------------------------
+    if (aborted && leader) {
+      *abort_flag = 1;
+      record_error(p.err, BLASST_ETIMEOUT);
+    }
+    ptx::named_bar_sync(3, C::NSOFT);
+    // final statistics: the state after block nblk-1, handed to set nblk & 1
+    const int fin = nblk & 1;
+    const float mref_fin = st_rows[fin * 256 + 128 + t];
+    const int last_fin = st_last[fin];
+    const float l_mine =
+        (lref == -INFINITY || mref_fin == -INFINITY) ? 0.0f : l * ptx::ex2(lref - mref_fin);
+    lsum[set * 128 + t] = l_mine;
+    bool ok = __shfl_sync(0xffffffffu, (lane == 0 && *abort_flag == 0) ? 1 : 0, 0) != 0;
+    if (ok && last_fin >= 0) {
+      const int lb = last_fin % C::NS;
+      ok = lane0_wait(bar(C::B_PV + lb), (st_cnt[fin * 4 + lb] - 1) & 1);
+    }
+    ptx::tc_fence_after();
+    ptx::named_bar_sync(3, C::NSOFT);
+    const float ltot = lsum[t] + lsum[128 + t];
+    if (!ok || *abort_flag) {
+      if (lane == 0) *abort_flag = 1;
+      record_error(p.err, BLASST_ETIMEOUT);
     } else {
-      // ---- epilogue: O / l -> bf16, lse, masks of unvisited blocks ------
-      bool ok = true;
-      if (ncomp > 0 && lane == 0)
-        ok = ptx::mbar_wait(bar(C::B_PV + last_buf), ((last_buf ? pvn1 : pvn0) - 1) & 1,
-                            abort_flag, p.timeout_ns);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      ptx::tc_fence_after();
-      lsum[half * 128 + t] = l;
-      ptx::named_bar_sync(1, C::NSOFT);
-      const float ltot = l + lsum[(half ^ 1) * 128 + t];
-      if (!ok) {
-        *abort_flag = 1;
-        record_error(p.err, BLASST_ETIMEOUT);
-      } else {
-        const float inv_l = (ltot > 0.0f) ? 1.0f / ltot : 0.0f;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                              (static_cast<size_t>(bh) * p.Lq + row) * D + half * C::DHALF;
+      // warp w writes columns [half*D/2, (half+1)*D/2) of its quarter's rows
+      const int half = set;
+      const float inv_l = (ltot > 0.0f) ? 1.0f / ltot : 0.0f;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
+                            (static_cast<size_t>(bh) * p.Lq + row) * D + half * (D / 2);
 #pragma unroll
-        for (int c = 0; c < C::DHALF / 32; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tmem + lane_base + C::O_COL + half * C::DHALF + 32 * c, r);
-          ptx::tmem_wait_ld();
-          uint32_t w[16];
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tmem + lane_base + C::O_COL + half * (D / 2) + 32 * c, r);
+        ptx::tmem_wait_ld();
+        uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            w[i] = ptx::pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
-                                    __uint_as_float(r[2 * i + 1]) * inv_l);
-          if (row_exists) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+        for (int i = 0; i < 16; ++i)
+          w[i] = ptx::pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
+                                  __uint_as_float(r[2 * i + 1]) * inv_l);
+        if (row_exists) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-          }
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
-        if (row_exists && half == 0)
-          p.lse[static_cast<size_t>(bh) * p.Lq + row] = (mref + log2f(ltot)) * 0.6931471805599453f;
-        if (p.mask) {
+      }
+      if (row_exists && half == 0)
+        p.lse[static_cast<size_t>(bh) * p.Lq + row] = (mref_fin + log2f(ltot)) * 0.6931471805599453f;
+      if (p.mask) {
 #pragma unroll
-          for (int gg = 0; gg < C::NG; ++gg) {
-            if (kt_last[gg] < 0) continue;
-            const int qt = r0 / BR + gg;
-            uint8_t* mrow = p.mask + (static_cast<size_t>(bh) * p.nQt + qt) * p.nKt;
-            for (int jj = nblk + static_cast<int>(threadIdx.x); jj < p.nKt; jj += C::NSOFT)
-              mrow[jj] = 2;
-          }
+        for (int gg = 0; gg < C::NG; ++gg) {
+          if (kt_last[gg] < 0) continue;
+          const int qt = r0 / BR + gg;
+          uint8_t* mrow = p.mask + (static_cast<size_t>(bh) * p.nQt + qt) * p.nKt;
+          for (int jj = nblk + static_cast<int>(threadIdx.x); jj < p.nKt; jj += C::NSOFT)
+            mrow[jj] = 2;
         }
       }
     }
