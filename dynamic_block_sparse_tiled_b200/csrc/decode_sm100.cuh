@@ -17,7 +17,10 @@
 //     (a task = one KV block of one split of one (sequence, KV head)), so the
 //     K prefetch runs across split boundaries without pipeline drains;
 //   - a producer warp streams K through a TMA ring (128-byte swizzled tiles:
-//     a thread reading one key row is bank-conflict free);
+//     a thread reading one key row is bank-conflict free); a second one
+//     loads V when a vote keeps the block and writes the skip mask and the
+//     counters, so no TMA issue or bookkeeping sits on the compute warps'
+//     critical path;
 //   - the votes run LA = 2 tasks ahead of the P.V accumulation. A vote needs
 //     only K and the running max, so the arithmetic is unchanged: task n is
 //     scored and voted (its V load issued at once if some head keeps it)
@@ -57,7 +60,7 @@ struct DecodeParams {
 template <int D, int BC, int G>
 struct DecodeCfg {
   static constexpr int NC = 128;        // compute threads (warps 0-3)
-  static constexpr int NT = NC + 32;    // + producer warp 4
+  static constexpr int NT = NC + 64;    // + K producer warp 4 and V producer warp 5
   static constexpr int LA = 2;          // votes run LA tasks ahead of P.V
   static constexpr int DBOX = D / 64;
   static constexpr int KV_BOX = BC * 128;
@@ -66,6 +69,7 @@ struct DecodeCfg {
   static constexpr int NV = LA + 1;     // V ring stages
   static constexpr int NP = LA + 1;     // task records (P fragments, alpha, keep)
   static constexpr int NFIN = 4;        // split finals ring (> LA + 1 open splits)
+  static constexpr int NDEC = 8;        // decision ring between compute and the V warp
   static constexpr int KW = BC / 4;     // keys per warp
   static constexpr int NTQ = KW / 8;    // q K^T n-tiles (8 keys) per warp
   static constexpr int KSP = KW / 16;   // P V k-steps (16 keys) per warp
@@ -77,10 +81,12 @@ struct DecodeCfg {
   static constexpr int OFF_TASK = OFF_PF + NP * NC * PREGS * 4;      // NP x (G alpha, G keep)
   static constexpr int OFF_RED = OFF_TASK + NP * 2 * G * 4;          // 4 warps x G max, x G sums
   static constexpr int OFF_FIN = OFF_RED + 2 * 4 * G * 4;            // NFIN x (G m, G l)
-  static constexpr int OFF_FLAG = OFF_FIN + NFIN * 2 * G * 4;        // abort words
+  static constexpr int OFF_DEC = OFF_FIN + NFIN * 2 * G * 4;         // NDEC keep masks
+  static constexpr int OFF_FLAG = OFF_DEC + NDEC * 4;                // abort words
   static constexpr int OFF_OACC = (OFF_FLAG + 64 + 15) & ~15;        // 4 warps x G x D fp32
   static constexpr int OFF_BAR = (OFF_OACC + 4 * G * D * 4 + 7) & ~7;
-  static constexpr int NBAR = 2 * NK + NV;                           // K full/empty, V full
+  // K full/empty, V full/empty, decision written / read
+  static constexpr int NBAR = 2 * NK + 2 * NV + 2 * NDEC;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
   static_assert(G <= 8, "rows of the padded tile");
   static_assert(KW % 16 == 0 && (D / 16) % 2 == 0 && NTO % 2 == 0, "tile shapes");
@@ -130,7 +136,7 @@ __device__ __forceinline__ uint32_t sw_chunk(int row, int chunk, int box_bytes) 
 }  // namespace dmma
 
 template <int D, int BC, int G>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(192, 1)
     blasst_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   using C = DecodeCfg<D, BC, G>;
@@ -147,7 +153,9 @@ __global__ void __launch_bounds__(160, 1)
   volatile int* abort_seen = abort_flag + 2;  // [2], decided by thread 0 per task parity
   float* oacc = reinterpret_cast<float*>(smem + C::OFF_OACC);               // [4][G][D]
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
-  const int B_KF = 0, B_KE = C::NK, B_VF = 2 * C::NK;
+  volatile int* dec_ring = reinterpret_cast<volatile int*>(smem + C::OFF_DEC);  // [NDEC]
+  const int B_KF = 0, B_KE = C::NK, B_VF = 2 * C::NK, B_VE = B_VF + C::NV;
+  const int B_DEC = B_VE + C::NV, B_DR = B_DEC + C::NDEC;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int g = lane >> 2, c4 = lane & 3;  // mma fragment row (head) and column pair
@@ -189,10 +197,12 @@ __global__ void __launch_bounds__(160, 1)
   };
 
   if (t == 0) {
-    for (int i = 0; i < C::NBAR; ++i) ptx::mbar_init(bar(i), 1);
+    for (int i = 0; i < C::NBAR; ++i)
+      ptx::mbar_init(bar(i), (i >= B_VE && i < B_VE + C::NV) ? 4 : 1);
     abort_flag[0] = 0;
     abort_seen[0] = 0;
     abort_seen[1] = 0;
+    abort_flag[4] = 0;  // never set: for waits that only a timeout ends
     ptx::fence_mbar_init();
   }
   __syncthreads();
@@ -227,6 +237,61 @@ __global__ void __launch_bounds__(160, 1)
     }
     return;  // the producer warp takes no part in the compute barriers
   }
+  if (warp == 5) {
+    // ======================= V producer, skip mask, counters =============
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmV);
+      TaskCursor c = advance_split(blockIdx.x, false);
+      unsigned long long st_vis = 0, st_skip = 0, st_flops = 0, st_bytes = 0;
+      int n = 0, vcount = 0;
+      bool ok = true;
+      for (; c.split_id < nsplits; ++n) {
+        const int ds = n % C::NDEC;
+        ok = ptx::mbar_wait(bar(B_DEC + ds), (n / C::NDEC) & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        const int keepmask = dec_ring[ds];
+        ptx::mbar_arrive(bar(B_DR + ds));
+        const int bhk = c.split_id / p.S;
+        const int key0 = task_key0(c);
+        if (keepmask) {
+          const int vs = vcount % C::NV;
+          if (vcount >= C::NV) {
+            ok = ptx::mbar_wait(bar(B_VE + vs), ((vcount / C::NV) - 1) & 1, abort_flag,
+                                p.timeout_ns);
+            if (!ok) break;
+          }
+          load_tile(&tmV, sb + C::OFF_V + vs * C::KV_BYTES, key0, bhk, bar(B_VF + vs));
+          ++vcount;
+        }
+        if (p.mask) {
+          const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
+          for (int h = 0; h < G; ++h) {
+            const size_t hq = static_cast<size_t>(b) * p.Hq + hk * G + h;
+            p.mask[hq * p.nKt + key0 / BC] = ((keepmask >> h) & 1) ? 0 : 1;
+          }
+        }
+        st_vis += G;
+        st_skip += G - __popc(keepmask);
+        st_flops += 2ull * G * BC * D + 2ull * __popc(keepmask) * BC * D;
+        st_bytes += static_cast<unsigned long long>(BC) * D * 2ull * (keepmask ? 2ull : 1ull);
+        c = next_task(c, false);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
+      } else if (p.stats) {
+        atomicAdd(&p.stats->tiles_visited, st_vis);
+        atomicAdd(&p.stats->tiles_skipped, st_skip);
+        atomicAdd(&p.stats->v_blocks_loaded, static_cast<unsigned long long>(vcount));
+        atomicAdd(&p.stats->mma_flops, st_flops);
+        atomicAdd(&p.stats->bytes_loaded, st_bytes);
+      }
+      // V copies in flight land before this warp leaves (they normally have).
+      for (int v = (vcount > C::NV ? vcount - C::NV : 0); v < vcount; ++v)
+        ptx::mbar_wait(bar(B_VF + v % C::NV), (v / C::NV) & 1, &abort_flag[4], p.timeout_ns);
+    }
+    return;
+  }
 
   // ======================= compute warps 0-3 ================================
   // Warp w owns keys [w*KW, w*KW + KW) of every block; thread (g, c4) holds,
@@ -242,8 +307,6 @@ __global__ void __launch_bounds__(160, 1)
     m[h] = -INFINITY;
     l[h] = 0.0f;
   }
-  unsigned long long st_vis = 0, st_skip = 0, st_flops = 0, st_bytes = 0;
-  int vcount = 0;     // V tiles issued (thread 0)
   int vconsumed = 0;  // V tiles consumed by the P.V side
   bool aborted = false;
 
@@ -297,6 +360,8 @@ __global__ void __launch_bounds__(160, 1)
                          oa[nn + 1][0], oa[nn + 1][1]);
         }
       }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(B_VE + vs));  // this warp is done reading V
     }
     if (c.blk + 1 == c.nblk) {
       // split epilogue: sum the four warps' partial outputs, normalise, write
@@ -403,21 +468,13 @@ __global__ void __launch_bounds__(160, 1)
         if (!skip) keepmask |= 1 << h;
       }
       if (t == 0) {
-        if (keepmask) {
-          // the stage's previous tile belongs to a task at least LA + 1 back,
-          // whose P.V is done and was followed by the barrier above
-          const int vs = vcount % C::NV;
-          load_tile(&tmV, sb + C::OFF_V + vs * C::KV_BYTES, key0, bhk, bar(B_VF + vs));
-          ++vcount;
-        }
-        st_vis += G;
-        st_skip += G - __popc(keepmask);
-        st_flops += 2ull * G * BC * D + 2ull * __popc(keepmask) * BC * D;
-        st_bytes += static_cast<unsigned long long>(BC) * D * 2ull * (keepmask ? 2ull : 1ull);
-      }
-      if (p.mask && t < G) {
-        const size_t hq = static_cast<size_t>(b) * p.Hq + hk * G + t;
-        p.mask[hq * p.nKt + key0 / BC] = ((keepmask >> t) & 1) ? 0 : 1;
+        // hand the decision to the V warp; its slot was read NDEC tasks ago
+        const int ds = n % C::NDEC;
+        if (n >= C::NDEC &&
+            !ptx::mbar_wait(bar(B_DR + ds), ((n / C::NDEC) - 1) & 1, abort_flag, p.timeout_ns))
+          *abort_flag = 1;
+        dec_ring[ds] = keepmask;
+        ptx::mbar_arrive(bar(B_DEC + ds));
       }
       // online softmax on the vote side; P of head g into bf16 fragments
       float alpha[G];
@@ -477,19 +534,9 @@ __global__ void __launch_bounds__(160, 1)
     }
   }
 
-  if (aborted) {
-    if (t == 0) {
-      if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
-      // V copies issued but not consumed land before the CTA exits
-      for (int v = vconsumed; v < vcount; ++v)
-        ptx::mbar_wait(bar(B_VF + v % C::NV), (v / C::NV) & 1, abort_flag, p.timeout_ns);
-    }
-  } else if (t == 0 && p.stats) {
-    atomicAdd(&p.stats->tiles_visited, st_vis);
-    atomicAdd(&p.stats->tiles_skipped, st_skip);
-    atomicAdd(&p.stats->v_blocks_loaded, static_cast<unsigned long long>(vcount));
-    atomicAdd(&p.stats->mma_flops, st_flops);
-    atomicAdd(&p.stats->bytes_loaded, st_bytes);
+  if (aborted && t == 0) {
+    *abort_flag = 1;
+    if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
   }
 }
 
