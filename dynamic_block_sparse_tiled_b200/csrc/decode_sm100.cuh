@@ -12,25 +12,24 @@
 // the GQA group keeps the block.
 //
 // The kernel is bound by HBM bytes (K always, V of kept blocks), so it is
-// built to keep loads in flight:
+// built to keep loads in flight and the per-block arithmetic off one chain:
 //   - persistent CTAs, one per SM, each streaming a fixed sequence of tasks
 //     (a task = one KV block of one split of one (sequence, KV head)), so the
 //     K prefetch runs across split boundaries without pipeline drains;
-//   - a producer warp streams K through a TMA ring (128-byte swizzled tiles:
-//     a thread reading one key row is bank-conflict free); a second one
-//     loads V when a vote keeps the block and writes the skip mask and the
-//     counters, so no TMA issue or bookkeeping sits on the compute warps'
-//     critical path;
-//   - the votes run LA = 2 tasks ahead of the P.V accumulation. A vote needs
-//     only K and the running max, so the arithmetic is unchanged: task n is
-//     scored and voted (its V load issued at once if some head keeps it)
-//     while the P.V of task n-2 is accumulated from a V tile that had two
-//     scoring steps to arrive.
-// The two contractions of a task (q K^T with G = Hq/Hkv rows, and P V) run as
-// warp-level bf16 mma.sync tiles with the G rows padded to 16: far too thin
-// for tcgen05, but one tile instruction replaces hundreds of dependent FMAs
-// and shared-memory loads, which keeps four warps ahead of the HBM stream.
-// Each of the four compute warps owns a quarter of the block's keys; P stays
+//   - warp 8 streams K through a TMA ring (128-byte swizzled tiles: a thread
+//     reading one key row is bank-conflict free); warp 9 loads V when a vote
+//     keeps the block and writes the skip mask and the counters;
+//   - warps 0-3 score and vote: q K^T, the per-head block max, the vote
+//     against the running max, P = exp2(s - m) and the running sums; a task
+//     record (P fragments, rescale factors, keep flags) goes to shared memory;
+//   - warps 4-7 accumulate O += P V from those records, up to NP tasks
+//     behind, and write each split's normalised output. The two groups run
+//     concurrently (one warp of each per SM sub-partition), so the vote chain
+//     of one block overlaps the P V of an earlier one.
+// Both contractions run as warp-level bf16 mma.sync tiles with the G =
+// Hq/Hkv rows padded to 16: far too thin for tcgen05, but one tile
+// instruction replaces hundreds of dependent FMAs and shared-memory loads.
+// Warp w of each group owns keys [w*Bc/4, (w+1)*Bc/4) of every block; P stays
 // in the accumulator layout of q K^T, which is the operand layout of P V.
 #pragma once
 #include <cuda.h>
@@ -59,17 +58,16 @@ struct DecodeParams {
 
 template <int D, int BC, int G>
 struct DecodeCfg {
-  static constexpr int NC = 128;        // compute threads (warps 0-3)
-  static constexpr int NT = NC + 64;    // + K producer warp 4 and V producer warp 5
-  static constexpr int LA = 2;          // votes run LA tasks ahead of P.V
+  static constexpr int NC = 128;        // vote threads (warps 0-3); P V threads are warps 4-7
+  static constexpr int NT = 320;        // + P V warps 4-7, K producer 8, V producer 9
   static constexpr int DBOX = D / 64;
   static constexpr int KV_BOX = BC * 128;
   static constexpr int KV_BYTES = KV_BOX * DBOX;
   static constexpr int NK = 3;          // K ring stages
-  static constexpr int NV = LA + 1;     // V ring stages
-  static constexpr int NP = LA + 1;     // task records (P fragments, alpha, keep)
-  static constexpr int NFIN = 4;        // split finals ring (> LA + 1 open splits)
-  static constexpr int NDEC = 8;        // decision ring between compute and the V warp
+  static constexpr int NV = 3;          // V ring stages
+  static constexpr int NP = 4;          // task records (P fragments, alpha, keep)
+  static constexpr int NFIN = 8;        // split finals ring (> NP + 1 open splits)
+  static constexpr int NDEC = 8;        // decision ring between the vote warps and the V warp
   static constexpr int KW = BC / 4;     // keys per warp
   static constexpr int NTQ = KW / 8;    // q K^T n-tiles (8 keys) per warp
   static constexpr int KSP = KW / 16;   // P V k-steps (16 keys) per warp
@@ -85,8 +83,8 @@ struct DecodeCfg {
   static constexpr int OFF_FLAG = OFF_DEC + NDEC * 4;                // abort words
   static constexpr int OFF_OACC = (OFF_FLAG + 64 + 15) & ~15;        // 4 warps x G x D fp32
   static constexpr int OFF_BAR = (OFF_OACC + 4 * G * D * 4 + 7) & ~7;
-  // K full/empty, V full/empty, decision written / read
-  static constexpr int NBAR = 2 * NK + 2 * NV + 2 * NDEC;
+  // K full/empty, V full/empty, decision written/read, task record ready/free
+  static constexpr int NBAR = 2 * NK + 2 * NV + 2 * NDEC + 2 * NP;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
   static_assert(G <= 8, "rows of the padded tile");
   static_assert(KW % 16 == 0 && (D / 16) % 2 == 0 && NTO % 2 == 0, "tile shapes");
@@ -136,7 +134,9 @@ __device__ __forceinline__ uint32_t sw_chunk(int row, int chunk, int box_bytes) 
 }  // namespace dmma
 
 template <int D, int BC, int G>
-__global__ void __launch_bounds__(192, 1)
+// 320 threads: at most 3 warps on one SM sub-partition, so up to 168
+// registers per thread.
+__global__ void __launch_bounds__(320, 1)
     blasst_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   using C = DecodeCfg<D, BC, G>;
@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* dec_ring = reinterpret_cast<volatile int*>(smem + C::OFF_DEC);  // [NDEC]
   const int B_KF = 0, B_KE = C::NK, B_VF = 2 * C::NK, B_VE = B_VF + C::NV;
   const int B_DEC = B_VE + C::NV, B_DR = B_DEC + C::NDEC;
+  const int B_TR = B_DR + C::NDEC, B_TF = B_TR + C::NP;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int g = lane >> 2, c4 = lane & 3;  // mma fragment row (head) and column pair
@@ -198,7 +199,8 @@ __global__ void __launch_bounds__(192, 1)
 
   if (t == 0) {
     for (int i = 0; i < C::NBAR; ++i)
-      ptx::mbar_init(bar(i), (i >= B_VE && i < B_VE + C::NV) ? 4 : 1);
+      ptx::mbar_init(bar(i), ((i >= B_VE && i < B_VE + C::NV) || (i >= B_TF && i < B_TF + C::NP))
+                                 ? 4 : 1);
     abort_flag[0] = 0;
     abort_seen[0] = 0;
     abort_seen[1] = 0;
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(192, 1)
       ptx::tma_load_3d(dst + bx * C::KV_BOX, tm, bx * 64, key0, bhk, fb);
   };
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ======================= K producer ====================================
     if (lane == 0) {
       ptx::prefetch_tmap(&tmK);
@@ -237,7 +239,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     return;  // the producer warp takes no part in the compute barriers
   }
-  if (warp == 5) {
+  if (warp == 9) {
     // ======================= V producer, skip mask, counters =============
     if (lane == 0) {
       ptx::prefetch_tmap(&tmV);
@@ -293,13 +295,111 @@ __global__ void __launch_bounds__(192, 1)
     return;
   }
 
-  // ======================= compute warps 0-3 ================================
-  // Warp w owns keys [w*KW, w*KW + KW) of every block; thread (g, c4) holds,
-  // for head g < G, the scores of keys 8j + 2c4, 8j + 2c4 + 1 of each n-tile j
-  // and the outputs of dims 8nn + 2c4, 8nn + 2c4 + 1 of each n-tile nn.
-  float oa[C::NTO][2];
+  if (warp >= 4) {
+    // ======================= P V warps 4-7 =================================
+    // Warp pw owns keys [pw*KW, pw*KW + KW) of every block; thread (g, c4)
+    // accumulates, for head g < G, dims 8nn + 2c4, 8nn + 2c4 + 1 of each
+    // n-tile nn. Tasks come in the order of the vote side's records.
+    const int pw = warp - 4;
+    float oa[C::NTO][2];
 #pragma unroll
-  for (int i = 0; i < C::NTO; ++i) oa[i][0] = oa[i][1] = 0.0f;
+    for (int i = 0; i < C::NTO; ++i) oa[i][0] = oa[i][1] = 0.0f;
+    int vconsumed = 0;  // V tiles consumed
+    int pv_seq = 0;     // splits finished
+    bool failed = false;
+    auto pv_barrier = [&]() { ptx::named_bar_sync(2, 128); };
+    TaskCursor c = advance_split(blockIdx.x, false);
+    for (int n = 0; c.split_id < nsplits; ++n) {
+      const int slot = n % C::NP;
+      bool w = true;
+      if (lane == 0) w = ptx::mbar_wait(bar(B_TR + slot), (n / C::NP) & 1, abort_flag, p.timeout_ns);
+      w = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+      if (!w) failed = true;  // keep going (waits now return at once) so the
+                              // four warps take the same barriers
+      const int* keep = task_keep + slot * G;
+      int any = 0;
+#pragma unroll
+      for (int h = 0; h < G; ++h) any |= keep[h];
+      if (c.blk == 0) {
+#pragma unroll
+        for (int i = 0; i < C::NTO; ++i) oa[i][0] = oa[i][1] = 0.0f;
+      }
+      if (any) {
+        const int vs = vconsumed % C::NV;
+        bool wv = true;
+        if (lane == 0)
+          wv = ptx::mbar_wait(bar(B_VF + vs), (vconsumed / C::NV) & 1, abort_flag, p.timeout_ns);
+        wv = __shfl_sync(0xffffffffu, wv ? 1 : 0, 0) != 0;
+        if (!wv) failed = true;
+        ++vconsumed;
+        const float alpha = g < G ? task_alpha[slot * G + g] : 1.0f;
+#pragma unroll
+        for (int i = 0; i < C::NTO; ++i) {
+          oa[i][0] *= alpha;
+          oa[i][1] *= alpha;
+        }
+        uint32_t pr[C::PREGS];
+#pragma unroll
+        for (int i = 0; i < C::PREGS; ++i)
+          pr[i] = pfrag[(slot * C::NC + pw * 32 + lane) * C::PREGS + i];
+        const uint32_t vst = sb + C::OFF_V + vs * C::KV_BYTES;
+#pragma unroll
+        for (int k2 = 0; k2 < C::KSP; ++k2) {
+          // keys of this k-step: pw*KW + 16*k2 + [0, 16)
+          const int key = pw * C::KW + 16 * k2 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+          for (int nn = 0; nn < C::NTO; nn += 2) {
+            uint32_t b0, b1, b2, b3;
+            dmma::ldsm_x4_t(vst + dmma::sw_chunk(key, nn + (lane >> 4), C::KV_BOX), b0, b1, b2, b3);
+            dmma::mma16816(oa[nn][0], oa[nn][1], pr[2 * k2], pr[2 * k2 + 1], b0, b1, oa[nn][0],
+                           oa[nn][1]);
+            dmma::mma16816(oa[nn + 1][0], oa[nn + 1][1], pr[2 * k2], pr[2 * k2 + 1], b2, b3,
+                           oa[nn + 1][0], oa[nn + 1][1]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(B_VE + vs));  // this warp is done reading V
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(B_TF + slot));  // task record read
+      if (c.blk + 1 == c.nblk) {
+        // split epilogue: sum the four warps' partial outputs, normalise, write
+        if (g < G) {
+#pragma unroll
+          for (int i = 0; i < C::NTO; ++i) {
+            oacc[(pw * G + g) * D + 8 * i + 2 * c4] = oa[i][0];
+            oacc[(pw * G + g) * D + 8 * i + 2 * c4 + 1] = oa[i][1];
+          }
+        }
+        pv_barrier();
+        const float* fin = split_fin + (pv_seq % C::NFIN) * 2 * G;  // [m[G], l[G]]
+        const int sp = c.split_id % p.S, bhk = c.split_id / p.S;
+        const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
+        for (int i = t - 128; i < G * D; i += 128) {
+          const int h = i / D, x = i % D;
+          const float v = (oacc[(0 * G + h) * D + x] + oacc[(1 * G + h) * D + x]) +
+                          (oacc[(2 * G + h) * D + x] + oacc[(3 * G + h) * D + x]);
+          const float lf = fin[G + h];
+          const size_t prow = (static_cast<size_t>(b) * p.Hq + hk * G + h) * p.S + sp;
+          p.o_parts[prow * D + x] = lf > 0.0f ? v / lf : 0.0f;
+          if (x == 0)
+            p.lse_parts[prow] = lf > 0.0f ? (fin[h] + log2f(lf)) * 0.6931471805599453f : -INFINITY;
+        }
+        pv_barrier();  // oacc free again
+        ++pv_seq;
+      }
+      c = next_task(c, false);
+    }
+    if (failed && t == 128) {
+      *abort_flag = 1;
+      if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
+    }
+    return;
+  }
+
+  // ======================= vote warps 0-3 ===================================
+  // Warp w owns keys [w*KW, w*KW + KW) of every block; thread (g, c4) holds,
+  // for head g < G, the scores of keys 8j + 2c4, 8j + 2c4 + 1 of each n-tile j.
   uint32_t qa[D / 16][2];  // q fragments (bf16 pairs) of head g for each k-step
   float m[G], l[G];        // running statistics of the split being voted
 #pragma unroll
@@ -307,94 +407,16 @@ __global__ void __launch_bounds__(192, 1)
     m[h] = -INFINITY;
     l[h] = 0.0f;
   }
-  int vconsumed = 0;  // V tiles consumed by the P.V side
   bool aborted = false;
-
-  TaskCursor pend[C::LA + 1];  // voted tasks awaiting their P.V, oldest first
-  int npend = 0;
   int q_split = -1;  // split whose q rows are in qa
   int vote_seq = 0;  // splits finished on the vote side
-  int pv_seq = 0;    // splits finished on the P.V side
 
   auto compute_barrier = [&]() { ptx::named_bar_sync(1, C::NC); };
 
-  // P.V of one voted task, then the split's epilogue if it was its last block.
-  auto do_pv = [&](const TaskCursor& c, int slot) {
-    const int* keep = task_keep + slot * G;
-    int any = 0;
-#pragma unroll
-    for (int h = 0; h < G; ++h) any |= keep[h];
-    if (c.blk == 0) {
-#pragma unroll
-      for (int i = 0; i < C::NTO; ++i) oa[i][0] = oa[i][1] = 0.0f;
-    }
-    if (any) {
-      const int vs = vconsumed % C::NV;
-      bool w = true;
-      if (lane == 0)
-        w = ptx::mbar_wait(bar(B_VF + vs), (vconsumed / C::NV) & 1, abort_flag, p.timeout_ns);
-      w = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
-      if (!w) *abort_flag = 1;
-      ++vconsumed;
-      const float alpha = g < G ? task_alpha[slot * G + g] : 1.0f;
-#pragma unroll
-      for (int i = 0; i < C::NTO; ++i) {
-        oa[i][0] *= alpha;
-        oa[i][1] *= alpha;
-      }
-      uint32_t pr[C::PREGS];
-#pragma unroll
-      for (int i = 0; i < C::PREGS; ++i) pr[i] = pfrag[(slot * C::NC + t) * C::PREGS + i];
-      const uint32_t vst = sb + C::OFF_V + vs * C::KV_BYTES;
-#pragma unroll
-      for (int k2 = 0; k2 < C::KSP; ++k2) {
-        // keys of this k-step: warp*KW + 16*k2 + [0, 16)
-        const int key = warp * C::KW + 16 * k2 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int nn = 0; nn < C::NTO; nn += 2) {
-          uint32_t b0, b1, b2, b3;
-          dmma::ldsm_x4_t(vst + dmma::sw_chunk(key, nn + (lane >> 4), C::KV_BOX), b0, b1, b2, b3);
-          dmma::mma16816(oa[nn][0], oa[nn][1], pr[2 * k2], pr[2 * k2 + 1], b0, b1, oa[nn][0],
-                         oa[nn][1]);
-          dmma::mma16816(oa[nn + 1][0], oa[nn + 1][1], pr[2 * k2], pr[2 * k2 + 1], b2, b3,
-                         oa[nn + 1][0], oa[nn + 1][1]);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(B_VE + vs));  // this warp is done reading V
-    }
-    if (c.blk + 1 == c.nblk) {
-      // split epilogue: sum the four warps' partial outputs, normalise, write
-      if (g < G) {
-#pragma unroll
-        for (int i = 0; i < C::NTO; ++i) {
-          oacc[(warp * G + g) * D + 8 * i + 2 * c4] = oa[i][0];
-          oacc[(warp * G + g) * D + 8 * i + 2 * c4 + 1] = oa[i][1];
-        }
-      }
-      compute_barrier();
-      const float* fin = split_fin + (pv_seq % C::NFIN) * 2 * G;  // [m[G], l[G]]
-      const int sp = c.split_id % p.S, bhk = c.split_id / p.S;
-      const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
-      for (int i = t; i < G * D; i += C::NC) {
-        const int h = i / D, x = i % D;
-        const float v = (oacc[(0 * G + h) * D + x] + oacc[(1 * G + h) * D + x]) +
-                        (oacc[(2 * G + h) * D + x] + oacc[(3 * G + h) * D + x]);
-        const float lf = fin[G + h];
-        const size_t prow = (static_cast<size_t>(b) * p.Hq + hk * G + h) * p.S + sp;
-        p.o_parts[prow * D + x] = lf > 0.0f ? v / lf : 0.0f;
-        if (x == 0)
-          p.lse_parts[prow] = lf > 0.0f ? (fin[h] + log2f(lf)) * 0.6931471805599453f : -INFINITY;
-      }
-      compute_barrier();  // oacc free again
-      ++pv_seq;
-    }
-  };
-
   TaskCursor cur = advance_split(blockIdx.x, true);
   int n = 0;
-  while (cur.split_id < nsplits || npend > 0) {
-    if (cur.split_id < nsplits) {
+  while (cur.split_id < nsplits) {
+    {
       // ---- score and vote task n -------------------------------------------
       const int bhk = cur.split_id / p.S;
       const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
@@ -476,6 +498,14 @@ __global__ void __launch_bounds__(192, 1)
         dec_ring[ds] = keepmask;
         ptx::mbar_arrive(bar(B_DEC + ds));
       }
+      // the task record slot was last read by the P V warps NP tasks ago
+      if (n >= C::NP) {
+        bool wf = true;
+        if (lane == 0)
+          wf = ptx::mbar_wait(bar(B_TF + slot), ((n / C::NP) - 1) & 1, abort_flag, p.timeout_ns);
+        wf = __shfl_sync(0xffffffffu, wf ? 1 : 0, 0) != 0;
+        if (!wf) *abort_flag = 1;  // seen by every warp at the next task's check
+      }
       // online softmax on the vote side; P of head g into bf16 fragments
       float alpha[G];
 #pragma unroll
@@ -521,16 +551,9 @@ __global__ void __launch_bounds__(192, 1)
         }
         ++vote_seq;
       }
-      pend[npend++] = cur;
+      if (t == 0) ptx::mbar_arrive(bar(B_TR + slot));  // record (and finals) published
       cur = next_task(cur, true);
       ++n;
-    }
-    // ---- P.V of the oldest voted task once LA newer ones are voted (or at the end)
-    if (npend > C::LA || (cur.split_id >= nsplits && npend > 0)) {
-      const int done_n = n - npend;  // task index of pend[0]
-      do_pv(pend[0], done_n % C::NP);
-      for (int i = 1; i < npend; ++i) pend[i - 1] = pend[i];
-      --npend;
     }
   }
 
