@@ -69,10 +69,17 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {
+    "prefill_32k": ("prefill_sm100.cuh", "ptx_sm100.cuh"),
+    "decode_64k": ("decode_sm100.cuh", "ptx_sm100.cuh"),
+}
+
+
+def kernel_source_hash(kernel_key):
+    """Hash of the source files that make up one kernel."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dynamic_block_sparse_tiled_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel_key]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -85,7 +92,7 @@ def profiled_traffic(kernel_key):
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    cur = kernel_source_hash()
+    cur = kernel_source_hash(kernel_key)
     with open(p) as f:
         for line in f:
             parts = line.split()
