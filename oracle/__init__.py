@@ -50,7 +50,7 @@ class _PrefillArgs(C.Structure):
         ("causal", C.c_int), ("lam", C.c_double),
         ("Br", C.c_int64), ("Bc", C.c_int64), ("scale", C.c_double),
         ("ref_mode", C.c_int), ("ref_param", C.c_double),
-        ("items", C.c_void_p), ("n_items", C.c_int64),
+        ("items", C.c_void_p), ("n_items", C.c_int64), ("static_mask", C.c_void_p),
         ("o", C.c_void_p), ("lse", C.c_void_p), ("mask", C.c_void_p),
         ("margin", C.c_void_p), ("nthreads", C.c_int),
     ]
@@ -124,12 +124,14 @@ def _ptr(a):
 
 def prefill(q, k, v, *, causal: bool, lam: float, Br: int, Bc: int, scale: float | None = None,
             items=None, ref_mode: int = 0, ref_param: float = 0.0, nthreads: int = 0,
-            _lib=None) -> dict:
+            static_mask=None, _lib=None) -> dict:
     """Blocked attention with the threshold skip, per query tile.
 
     q: [B, Hq, Lq, d]; k, v: [B, Hkv, Lkv, d]; all the same dtype (uint16 bf16
     bits, float32 or float64), C-contiguous. ``items`` selects flat tile ids
-    ``(b*Hq + hq)*nQt + qt`` (default: every tile). Returns per-item arrays:
+    ``(b*Hq + hq)*nQt + qt`` (default: every tile). ``static_mask``: optional
+    uint8 [B, Hq, nQt, nKt], nonzero = the (query tile, KV block) pair is
+    excluded before any computation. Returns per-item arrays:
     o [n, Br, d], lse [n, Br], mask [n, nKt] (0 computed, 1 skipped, 2 not
     visited), margin [n, nKt] (mu in natural units, NaN where not visited),
     plus the geometry.
@@ -150,6 +152,10 @@ def prefill(q, k, v, *, causal: bool, lam: float, Br: int, Bc: int, scale: float
     else:
         items_arr = np.ascontiguousarray(np.asarray(items, dtype=np.int64))
         n = int(items_arr.size)
+    smask = None
+    if static_mask is not None:
+        smask = np.ascontiguousarray(np.asarray(static_mask, dtype=np.uint8))
+        assert smask.shape == (B, Hq, nQt, nKt), smask.shape
     o = np.zeros((n, Br, d), np.float64)
     lse = np.zeros((n, Br), np.float64)
     mask = np.zeros((n, nKt), np.uint8)
@@ -157,7 +163,7 @@ def prefill(q, k, v, *, causal: bool, lam: float, Br: int, Bc: int, scale: float
     args = _PrefillArgs(
         q.ctypes.data, k.ctypes.data, v.ctypes.data, code, B, Hq, Hkv, Lq, Lkv, d,
         int(bool(causal)), float(lam), Br, Bc, float(scale), int(ref_mode), float(ref_param),
-        _ptr(items_arr), n, o.ctypes.data, lse.ctypes.data, mask.ctypes.data,
+        _ptr(items_arr), n, _ptr(smask), o.ctypes.data, lse.ctypes.data, mask.ctypes.data,
         margin.ctypes.data, int(nthreads))
     rc = (_lib or _load()).oracle_prefill(C.byref(args))
     if rc != 0:

@@ -34,8 +34,13 @@
  *   - scores are s = scale * q.k (natural units); the test is strict;
  *   - a row with no valid key in the block votes "negligible";
  *   - a skipped block adds nothing at all: not to m, not to l, not to O;
- *   - blocks are visited in ascending order; block 0 of every query tile
- *     (and of every decode split) is always computed;
+ *   - blocks are visited in ascending order; the first visited block of
+ *     every query tile (block 0 unless a caller-supplied static block mask
+ *     excludes it) and the first block of every decode split are always
+ *     computed;
+ *   - a block excluded by the static block mask is not visited at all: no
+ *     scores, no vote, nothing added (the static block-sparse attention that
+ *     a pre-pass selector would feed);
  *   - causal masking is bottom-right aligned: key j is visible from query
  *     row i when j <= i + (Lkv - Lq);
  *   - GQA maps query head hq to KV head hq / (Hq / Hkv);
@@ -94,6 +99,9 @@ typedef struct {
   double ref_param;
   const int64_t *items; /* flat tile ids (b*Hq + hq)*nQt + qt, or NULL = all */
   int64_t n_items;
+  /* Optional static block mask [B, Hq, nQt, nKt]: nonzero = the (query tile,
+   * KV block) pair is excluded before any computation; NULL = none. */
+  const uint8_t *static_mask;
   /* Outputs, one slot per listed item (item order):
    *   o      [n_items, Br, d]
    *   lse    [n_items, Br]       natural log; -inf for rows without keys
@@ -151,10 +159,12 @@ static void prefill_tile(const oracle_prefill_args *a, int64_t slot,
 
   uint8_t *mask = a->mask ? a->mask + slot * nKt : NULL;
   double *margin = a->margin ? a->margin + slot * nKt : NULL;
+  const uint8_t *smask = a->static_mask ? a->static_mask + item * nKt : NULL;
+  int visited_before = 0;
 
   /* [T] para 2: KV blocks are walked left to right. */
   for (int64_t kt = 0; kt < nKt; ++kt) {
-    if (kt > kt_last) {
+    if (kt > kt_last || (smask && smask[kt])) {
       if (mask) mask[kt] = MASK_NOT_VISITED;
       if (margin) margin[kt] = NAN;
       continue;
@@ -195,8 +205,10 @@ static void prefill_tile(const oracle_prefill_args *a, int64_t slot,
     }
 
     /* [T] para 5 + [D]: skip when exp(m_blk - m_run) < lambda on every row,
-     * i.e. max_r (m_blk - m_run) < ln(lambda). [T] para 6: never block 0. */
-    int skip = (kt > 0) && (a->lambda > 0.0) && (mu < log_lambda);
+     * i.e. max_r (m_blk - m_run) < ln(lambda). [T] para 6: never the first
+     * visited block. */
+    int skip = visited_before && (a->lambda > 0.0) && (mu < log_lambda);
+    visited_before = 1;
     if (mask) mask[kt] = skip ? MASK_SKIPPED : MASK_COMPUTED;
     if (margin) margin[kt] = mu;
     if (skip) continue; /* no V, no exp, no update of m, l or O */

@@ -339,6 +339,113 @@ def pin_worked_example(orc):
         assert abs(res["lse"][0, 0] - lse_ref) < 1e-14
 
 
+# --------------------------------------------------------------------------
+# Static block-sparse input: a caller-supplied mask excludes (query tile, KV
+# block) pairs before anything is computed.
+# --------------------------------------------------------------------------
+def _static_mask(seed, B, Hq, nQt, nKt, frac):
+    rng = np.random.default_rng(seed)
+    return (rng.random((B, Hq, nQt, nKt)) < frac).astype(np.uint8)
+
+
+def _allowed_from_static(smask, Br, Bc, Lq, Lkv):
+    B, Hq, nQt, nKt = smask.shape
+    allowed = np.ones((B, Hq, Lq, Lkv), bool)
+    for qt in range(nQt):
+        for kt in range(nKt):
+            allowed[:, :, qt * Br:(qt + 1) * Br, kt * Bc:(kt + 1) * Bc] = \
+                (smask[:, :, qt, kt] == 0)[:, :, None, None]
+    return allowed
+
+
+def _compare_with_empty_rows(o, lse, o_ref, lse_ref, any_key):
+    """Rows with no allowed key must give O = 0 and lse = -inf; the rest
+    must match the dense reference."""
+    assert np.all(o[~any_key] == 0.0) and np.all(np.isneginf(lse[~any_key]))
+    np.testing.assert_allclose(o[any_key], o_ref[any_key], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[any_key], lse_ref[any_key], rtol=0, atol=1e-12)
+
+
+def _row_has_key(allowed, causal, Lq, Lkv):
+    if causal:
+        i = np.arange(Lq)[:, None]
+        j = np.arange(Lkv)[None, :]
+        allowed = allowed & (j <= i + (Lkv - Lq))
+    return allowed.any(-1)
+
+
+def pin_static_mask_is_restriction(orc):
+    """With a static block mask and lambda = 0 the result is dense softmax
+    attention over the allowed blocks only (the excluded pairs contribute
+    nothing, as a skipped block does, para 5); an all-zero mask changes
+    nothing; a tile with every block excluded gives O = 0 and lse = -inf;
+    excluded pairs are reported as not visited."""
+    geos = [(1, 4, 2, 200, 200, 16, True, 16, 16), (1, 2, 2, 96, 150, 8, False, 32, 16),
+            (2, 2, 1, 130, 130, 8, True, 32, 32)]
+    for n, (B, Hq, Hkv, Lq, Lkv, d, causal, Br, Bc) in enumerate(geos):
+        q, k, v = rand_qkv(300 + n, B, Hq, Hkv, Lq, Lkv, d, planted=2.0, planted_blocks=(0, 3), Bc=Bc)
+        nQt, nKt = -(-Lq // Br), -(-Lkv // Bc)
+        smask = _static_mask(400 + n, B, Hq, nQt, nKt, 0.35)
+        smask[0, 0, 0, 0] = 1          # the first visited block is not block 0
+        smask[0, -1, nQt // 2, :] = 1  # a tile with every block excluded
+        res = orc.prefill(q, k, v, causal=causal, lam=0.0, Br=Br, Bc=Bc, static_mask=smask)
+        o, lse, mask, _ = _dense_from(res)
+        allowed = _allowed_from_static(smask, Br, Bc, Lq, Lkv)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            o_ref, lse_ref = dense_attention(q, k, v, causal, keep=allowed)
+        _compare_with_empty_rows(o, lse, o_ref, lse_ref, _row_has_key(allowed, causal, Lq, Lkv))
+        m4 = mask.reshape(B, Hq, nQt, nKt)
+        assert np.all(m4[smask != 0] == 2), "an excluded pair was visited"
+        assert not np.any(m4 == 1), "lambda = 0 skipped a block"
+        zero = orc.prefill(q, k, v, causal=causal, lam=0.0, Br=Br, Bc=Bc,
+                           static_mask=np.zeros_like(smask))
+        none = orc.prefill(q, k, v, causal=causal, lam=0.0, Br=Br, Bc=Bc)
+        assert np.array_equal(zero["o"], none["o"]) and np.array_equal(zero["lse"], none["lse"])
+        assert np.array_equal(zero["mask"], none["mask"])
+
+
+def pin_static_mask_with_threshold(orc):
+    """Static mask and lambda > 0 together: the first visited block of every
+    tile is computed (para 6, read as the first block the mask leaves), and
+    the output is dense attention over the blocks that are both allowed and
+    kept, exactly."""
+    q, k, v, kw = _skipping_case()
+    B, Hq, L = q.shape[0], q.shape[1], q.shape[2]
+    Br, Bc = kw["Br"], kw["Bc"]
+    nQt, nKt = -(-L // Br), -(-L // Bc)
+    smask = _static_mask(17, B, Hq, nQt, nKt, 0.3)
+    smask[:, :, 3:6, 0] = 1  # some tiles lose block 0
+    for lam in (1e-3, 0.2):
+        res = orc.prefill(q, k, v, lam=lam, static_mask=smask, **kw)
+        o, lse, mask, _ = _dense_from(res)
+        m4 = mask.reshape(B, Hq, nQt, nKt)
+        assert np.any(m4 == 1), "case did not skip anything"
+        for b in range(B):
+            for h in range(Hq):
+                for qt in range(nQt):
+                    vis = np.nonzero(m4[b, h, qt] != 2)[0]
+                    if vis.size:
+                        assert m4[b, h, qt, vis[0]] == 0, "first visited block was skipped"
+        keep = _kept_keys(res, L, L)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            o_ref, lse_ref = dense_attention(q, k, v, kw["causal"], keep=keep)
+        _compare_with_empty_rows(o, lse, o_ref, lse_ref, _row_has_key(keep, kw["causal"], L, L))
+    # Worked by hand (d = 1, one query, three one-key blocks, scale 1): the
+    # excluded block 0 holds the largest score, 10, which must not enter the
+    # running max. Block 1 (score 0) is the first visited block, computed;
+    # block 2 (score -1) has exp(-1 - 0) = 0.37 >= lambda = 0.1, computed.
+    # Had block 0 raised the running max, block 2 would be dropped.
+    qh = np.ones((1, 1, 1, 1))
+    kh = np.array([10.0, 0.0, -1.0]).reshape(1, 1, 3, 1)
+    vh = np.array([100.0, 1.0, 2.0]).reshape(1, 1, 3, 1)
+    sm = np.array([1, 0, 0], np.uint8).reshape(1, 1, 1, 3)
+    res = orc.prefill(qh, kh, vh, causal=False, lam=0.1, Br=1, Bc=1, scale=1.0, static_mask=sm)
+    assert list(res["mask"][0]) == [2, 0, 0], res["mask"]
+    w1, w2 = 1.0, np.exp(-1.0)
+    assert abs(res["o"][0, 0, 0] - (w1 * 1.0 + w2 * 2.0) / (w1 + w2)) < 1e-14
+    assert abs(res["lse"][0, 0] - np.log(w1 + w2)) < 1e-14
+
+
 ALL_PINS = [
     pin_lambda0_is_dense,
     pin_first_block_always_computed,
@@ -351,6 +458,8 @@ ALL_PINS = [
     pin_decode_split_merge,
     pin_lse_merge,
     pin_worked_example,
+    pin_static_mask_is_restriction,
+    pin_static_mask_with_threshold,
 ]
 
 

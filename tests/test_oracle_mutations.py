@@ -24,7 +24,7 @@ MUTATIONS = [
     ("vote_on_any_row_instead_of_all", "      if (dr > mu) mu = dr;", "      if (dr < mu || mu == -INFINITY) mu = dr;"),
     ("gqa_modulo_mapping", "hk = hq / g;\n  const int64_t r0", "hk = hq % a->Hkv;\n  const int64_t r0"),
     ("lse_without_log", "a->lse[slot * Br + r] = mref[r] + log(l[r]);", "a->lse[slot * Br + r] = mref[r] + l[r];"),
-    ("non_strict_threshold", "(mu < log_lambda);\n    if (mask)", "(mu <= log_lambda);\n    if (mask)"),
+    ("non_strict_threshold", "(mu < log_lambda);\n    visited_before", "(mu <= log_lambda);\n    visited_before"),
     ("vote_without_scale", "        if (sv > mb[r]) mb[r] = sv;",
      "        if (sv / a->scale > mb[r]) mb[r] = sv / a->scale;"),
     ("blocks_right_to_left", "for (int64_t kt = 0; kt < nKt; ++kt) {", "for (int64_t kt = nKt - 1; kt >= 0; --kt) {"),
@@ -32,6 +32,15 @@ MUTATIONS = [
      "const int64_t k1 = (k0 + Ls < a->Lkv ? k0 + Ls : a->Lkv) - 1;"),
     ("merge_weight_sign", "double w = (ls == -INFINITY) ? 0.0 : exp(ls - M);",
      "double w = (ls == -INFINITY) ? 0.0 : exp(M - ls);"),
+    ("static_mask_ignored", "if (kt > kt_last || (smask && smask[kt])) {", "if (kt > kt_last) {"),
+    ("static_masked_block_still_raises_max",
+     "    if (kt > kt_last || (smask && smask[kt])) {\n      if (mask) mask[kt] = MASK_NOT_VISITED;",
+     "    if (smask && smask[kt] && kt <= kt_last) {\n      for (int64_t r = 0; r < nr; ++r) {\n"
+     "        for (int64_t j = 0; j < Bc && kt * Bc + j < a->Lkv; ++j) {\n"
+     "          double dot = 0.0;\n"
+     "          for (int64_t x = 0; x < d; ++x) dot += qrow[r * d + x] * widen(a->k, a->dtype, kvbase + (kt * Bc + j) * d + x);\n"
+     "          if (a->scale * dot > m[r]) m[r] = a->scale * dot;\n        }\n      }\n    }\n"
+     "    if (kt > kt_last || (smask && smask[kt])) {\n      if (mask) mask[kt] = MASK_NOT_VISITED;"),
     ("decode_skipped_block_still_used", "    if (skip) continue;\n    for (int64_t j = 0; j < nc; ++j)\n      for (int64_t x = 0; x < d; ++x)\n        kv_v",
      "    for (int64_t j = 0; j < nc; ++j)\n      for (int64_t x = 0; x < d; ++x)\n        kv_v"),
 ]
