@@ -182,11 +182,11 @@ class Prefill:
         self.mask = torch.empty((w.B, w.Hq, -(-w.Lq // w.Br), -(-w.Lkv // w.Bc)), dtype=torch.uint8,
                                 device=device)
 
-    def run(self, lam, stats=None, stream=None):
+    def run(self, lam, stats=None, stream=None, block_mask=None):
         import dynamic_block_sparse_tiled_b200 as bl
         bl.blasst_fwd_ex(self.q, self.k, self.v, self.o, self.lse, causal=self.w.causal, lam=lam,
                          Br=self.w.Br, Bc=self.w.Bc, skip_mask_out=self.mask, stats_out=stats,
-                         stream=stream)
+                         stream=stream, block_mask_in=block_mask)
 
 
 def flush_l2(buf):
@@ -212,17 +212,18 @@ def time_calls(fn, steps, warmup, stream, flush_buf):
     return times
 
 
-def measure_prefill(w, lam, steps, warmup, device, stream, flush_buf, pre=None):
+def measure_prefill(w, lam, steps, warmup, device, stream, flush_buf, pre=None, block_mask=None):
     import dynamic_block_sparse_tiled_b200 as bl
     pre = pre or Prefill(w, device)
     st = bl.new_stats(device)
-    pre.run(lam, stats=st, stream=stream)
+    pre.run(lam, stats=st, stream=stream, block_mask=block_mask)
     stream.synchronize()
     rc = bl.blasst_check(stream)
     if rc != 0:
         raise RuntimeError(bl.blasst_status_string(rc))
     sd = bl.stats_dict(st)
-    times = time_calls(lambda: pre.run(lam, stream=stream), steps, warmup, stream, flush_buf)
+    times = time_calls(lambda: pre.run(lam, stream=stream, block_mask=block_mask), steps, warmup,
+                       stream, flush_buf)
     mask = pre.mask.cpu().numpy()
     vis = int((mask != 2).sum())
     skip = int((mask == 1).sum())
@@ -314,6 +315,22 @@ def measure_e2e(w, lam, steps, warmup, device, stream):
     ms = statistics.mean(times)
     return dict(value=effective_flops(w) / (ms * 1e-3) / 1e12, unit=UNIT, ms=ms,
                 h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h))
+
+
+def block_sparse_pattern(w, sink_blocks=1, band_blocks=8, random_frac=0.1, seed=0):
+    """A static block mask shaped like a pre-pass selector's output: every
+    query tile keeps the first `sink_blocks` KV blocks, a band of
+    `band_blocks` blocks ending at its diagonal, and a seeded random fraction
+    of the rest; everything else is excluded (mask 1)."""
+    nQt, nKt = -(-w.Lq // w.Br), -(-w.Lkv // w.Bc)
+    rng = np.random.default_rng(seed)
+    keep = rng.random((w.B, w.Hq, nQt, nKt)) < random_frac
+    keep[..., :sink_blocks] = True
+    off = w.Lkv - w.Lq
+    for qt in range(nQt):
+        diag = min(nKt - 1, (min(qt * w.Br + w.Br, w.Lq) - 1 + off) // w.Bc)
+        keep[:, :, qt, max(0, diag - band_blocks + 1):diag + 1] = True
+    return (~keep).astype(np.uint8)
 
 
 # ------------------------------------------------------------- CPU oracle
@@ -520,6 +537,24 @@ def main():
             v["speedup_vs_lambda0"] = base / v["ms"]
         extra["prefill_128k_a12_lambda_curve"] = curve
         del p3
+        torch.cuda.empty_cache()
+
+        # static block-sparse input (a selector's mask) on the 32K workload
+        import torch as _t
+        sm = block_sparse_pattern(w)
+        sm_dev = _t.from_numpy(sm).to(device)
+        ps = Prefill(w, device)
+        ps, s_r = measure_prefill(w, LAMBDA, max(3, args.steps // 2), 3, device, stream, flush_buf,
+                                  pre=ps, block_mask=sm_dev)
+        _, s0_r = measure_prefill(w, LAMBDA, max(3, args.steps // 2), 3, device, stream, flush_buf,
+                                  pre=ps)
+        nvis = s_r["tiles_visited"]
+        extra["static_block_sparse_32k"] = dict(
+            pattern="first block + 8-block diagonal band + 10 % seeded random blocks per query tile",
+            visited_tiles=nvis, visited_frac_of_causal=nvis / max(1, s0_r["tiles_visited"]),
+            ms=s_r["ms"], ms_no_mask=s0_r["ms"], speedup_vs_no_mask=s0_r["ms"] / s_r["ms"],
+            executed_tflops=s_r["exec_flops"] / (s_r["ms"] * 1e-3) / 1e12)
+        del ps, sm_dev
         torch.cuda.empty_cache()
 
         wd = synth.CONFIGS["decode_64k"]

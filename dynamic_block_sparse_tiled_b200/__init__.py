@@ -64,7 +64,7 @@ class _FwdArgs(C.Structure):
         ("B", C.c_int), ("Hq", C.c_int), ("Hkv", C.c_int), ("Lq", C.c_int), ("Lkv", C.c_int),
         ("d", C.c_int), ("causal", C.c_int), ("lam", C.c_float), ("Br", C.c_int), ("Bc", C.c_int),
         ("skip_mask_out", C.c_void_p), ("dtype", C.c_int), ("scale", C.c_float),
-        ("stream", C.c_void_p), ("stats_out", C.c_void_p),
+        ("stream", C.c_void_p), ("stats_out", C.c_void_p), ("block_mask_in", C.c_void_p),
     ]
 
 
@@ -158,10 +158,12 @@ def blasst_fwd(q, k, v, o, lse, B, Hq, Hkv, Lq, Lkv, d, causal, lam, Br, Bc, ski
 
 
 def blasst_fwd_ex(q, k, v, o, lse, *, causal: bool, lam: float, Br: int, Bc: int,
-                  skip_mask_out=None, scale: float = 0.0, stream=None, stats_out=None, dtype=None):
+                  skip_mask_out=None, scale: float = 0.0, stream=None, stats_out=None, dtype=None,
+                  block_mask_in=None):
     """The C entry point of the same name. q [B,Hq,Lq,d], k/v [B,Hkv,Lkv,d], o like q,
     lse [B,Hq,Lq] fp32, skip_mask_out uint8 [B,Hq,ceil(Lq/Br),ceil(Lkv/Bc)] or None,
-    stats_out a ``new_stats()`` tensor or None."""
+    stats_out a ``new_stats()`` tensor or None, block_mask_in an optional uint8
+    [B,Hq,ceil(Lq/Br),ceil(Lkv/Bc)] static block mask (nonzero = excluded)."""
     import torch
     B, Hq, Lq, d = q.shape
     _, Hkv, Lkv, _ = k.shape
@@ -169,7 +171,7 @@ def blasst_fwd_ex(q, k, v, o, lse, *, causal: bool, lam: float, Br: int, Bc: int
         dtype = BLASST_BF16 if q.dtype == torch.bfloat16 else BLASST_FP32
     args = _FwdArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lkv, d,
                     int(bool(causal)), float(lam), Br, Bc, _ptr(skip_mask_out), int(dtype),
-                    float(scale), _stream(stream), _ptr(stats_out))
+                    float(scale), _stream(stream), _ptr(stats_out), _ptr(block_mask_in))
     _check(load_library().blasst_fwd_ex(C.byref(args)), "blasst_fwd_ex")
 
 
@@ -239,7 +241,7 @@ def stats_dict(st) -> dict:
 
 
 def attention_prefill(q, k, v, *, causal=True, lam=0.0, Br=128, Bc=128, scale=0.0,
-                      with_mask=False, stats=None, stream=None):
+                      with_mask=False, stats=None, stream=None, block_mask=None):
     """Allocate outputs with torch and run blasst_fwd_ex. Returns (o, lse, mask)."""
     import torch
     B, Hq, Lq, d = q.shape
@@ -250,7 +252,7 @@ def attention_prefill(q, k, v, *, causal=True, lam=0.0, Br=128, Bc=128, scale=0.
     if with_mask:
         mask = torch.empty((B, Hq, -(-Lq // Br), -(-Lkv // Bc)), dtype=torch.uint8, device=q.device)
     blasst_fwd_ex(q, k, v, o, lse, causal=causal, lam=lam, Br=Br, Bc=Bc, skip_mask_out=mask,
-                  scale=scale, stream=stream, stats_out=stats)
+                  scale=scale, stream=stream, stats_out=stats, block_mask_in=block_mask)
     return o, lse, mask
 
 

@@ -106,10 +106,13 @@ template <int D, int BC, int BR>
 int launch_prefill_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const blasst::PrefillParams& p, cudaStream_t stream) {
   using C = blasst::PrefillCfg<D, BC, BR>;
-  auto kernel = blasst::blasst_prefill_bf16_kernel<D, BC, BR>;
-  if (set_smem(kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
+  const bool listed = p.smask != nullptr;
+  auto kernel = listed ? blasst::blasst_prefill_bf16_kernel<D, BC, BR, true>
+                       : blasst::blasst_prefill_bf16_kernel<D, BC, BR, false>;
+  const int smem = listed ? C::SMEM_BYTES_LISTED : C::SMEM_BYTES;
+  if (set_smem(kernel, smem) != cudaSuccess) return BLASST_ECUDA;
   const dim3 grid(static_cast<unsigned>(p.nQblk) * p.B * p.Hq);
-  kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  kernel<<<grid, C::NTHREADS, smem, stream>>>(mq, mk, mv, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -229,6 +232,7 @@ int blasst_fwd_ex(const blasst_fwd_args* a) {
   if (a->causal && a->Lq > a->Lkv) return BLASST_EUNSUPPORTED;
   if (a->dtype != BLASST_BF16 && a->dtype != BLASST_FP32) return BLASST_EUNSUPPORTED;
   if (a->dtype == BLASST_FP32 && (a->d != 64 || a->Bc != 64)) return BLASST_EUNSUPPORTED;
+  if (a->block_mask_in && (a->Lkv + a->Bc - 1) / a->Bc > 4096) return BLASST_EUNSUPPORTED;
   if (static_cast<long long>(a->B) * a->Hq > (1ll << 24) ||
       static_cast<long long>(a->B) * a->Hq * ((a->Lq + 127) / 128) > 0x7fffffffll)
     return BLASST_EINVAL;
@@ -240,6 +244,7 @@ int blasst_fwd_ex(const blasst_fwd_args* a) {
   p.o = a->o;
   p.lse = a->lse;
   p.mask = a->skip_mask_out;
+  p.smask = a->block_mask_in;
   p.stats = a->stats_out;
   p.err = err;
   p.B = a->B;
@@ -304,6 +309,7 @@ int blasst_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.scale = 0.0f;
   a.stream = nullptr;
   a.stats_out = nullptr;
+  a.block_mask_in = nullptr;
   return blasst_fwd_ex(&a);
 }
 

@@ -152,15 +152,32 @@ __global__ void __launch_bounds__(128, 1)
   const int row = r0 + t;
   const bool row_exists = row < p.Lq;
   const int gi = t / BR;
-  const int my_kt_last = kt_last[gi];
   const int last_col = p.causal ? min(row + p.off, p.Lkv - 1) : p.Lkv - 1;
   const float sl2 = p.scale_log2;
   const bool thresholding = p.log2_lambda > -INFINITY;
   float m = -INFINITY, l = 0.0f;
-  int ncomp = 0, mma_phase = 0, v_phase = 0;
+  int ncomp = 0, mma_phase = 0, v_phase = 0, kload = 0;
+  int nvis[C::NG] = {};  // blocks visited so far per row group (first-block rule)
   unsigned long long st_vis = 0, st_skip = 0, st_vload = 0, st_flops = 0;
 
   for (int j = 0; j < nblk; ++j) {
+    // row groups that visit block j (causal range, optional static mask)
+    uint32_t gvis = 0;
+#pragma unroll
+    for (int gg = 0; gg < C::NG; ++gg)
+      if (j <= kt_last[gg] &&
+          (!p.smask ||
+           p.smask[(static_cast<size_t>(bh) * p.nQt + (r0 / BR + gg)) * p.nKt + j] == 0))
+        gvis |= 1u << gg;
+    if (!gvis) {  // excluded before anything is computed
+      if (t == 0 && p.mask) {
+#pragma unroll
+        for (int gg = 0; gg < C::NG; ++gg)
+          if (kt_last[gg] >= 0)
+            p.mask[(static_cast<size_t>(bh) * p.nQt + (r0 / BR + gg)) * p.nKt + j] = 2;
+      }
+      continue;
+    }
     // ---- K_j, split, S = Qh Kh + Qh Kl + Ql Kh ------------------------------
     __syncthreads();  // previous block's K/V tiles and MMAs are done with
     if (t == 0) {
@@ -168,7 +185,8 @@ __global__ void __launch_bounds__(128, 1)
       ptx::tma_load_3d(sb + C::OFF_KH, &tmK, 0, j * C::BC, bhk, bar(1));
       ptx::tma_load_3d(sb + C::OFF_KH + C::KV_BOX, &tmK, 32, j * C::BC, bhk, bar(1));
     }
-    wait_all(1, j & 1);
+    wait_all(1, kload & 1);
+    ++kload;
     split(C::OFF_KH, C::OFF_KL, C::KV_BYTES);
     ptx::tc_fence_before();
     if (__syncthreads_or(bad ? 1 : 0)) break;
@@ -212,11 +230,14 @@ __global__ void __launch_bounds__(128, 1)
       mx = fmaxf(mx, s[c]);
     }
     const float mb = mx * sl2;
-    const bool visited = j <= my_kt_last;
+    const bool visited = (gvis >> gi) & 1;
     bool rowskip;
     if (!row_exists || !visited) rowskip = true;
-    else if (j == 0 || !thresholding) rowskip = false;
+    else if (nvis[gi] == 0 || !thresholding) rowskip = false;  // first visited block
+    else if (mb == -INFINITY) rowskip = true;                    // no visible key here
     else rowskip = (mb - m) < p.log2_lambda;
+#pragma unroll
+    for (int gg = 0; gg < C::NG; ++gg) nvis[gg] += (gvis >> gg) & 1;
     const unsigned all = __all_sync(0xffffffffu, rowskip) ? 1u : 0u;
     if (lane == 0) votes[warp] = static_cast<int>(all);
     __syncthreads();
@@ -226,7 +247,7 @@ __global__ void __launch_bounds__(128, 1)
       bool gskip = true;
 #pragma unroll
       for (int w = 0; w < C::WPG; ++w) gskip = gskip && votes[gg * C::WPG + w] != 0;
-      if (j <= kt_last[gg] && !gskip) keepmask |= 1 << gg;
+      if (((gvis >> gg) & 1) && !gskip) keepmask |= 1 << gg;
     }
     if (t == 0) {
       const unsigned long long tile_flops = 2ull * 128ull * C::BC * C::D;
@@ -236,7 +257,7 @@ __global__ void __launch_bounds__(128, 1)
       for (int gg = 0; gg < C::NG; ++gg) {
         if (kt_last[gg] < 0) continue;
         uint8_t code = 2;
-        if (j <= kt_last[gg]) {
+        if ((gvis >> gg) & 1) {
           ++st_vis;
           code = ((keepmask >> gg) & 1) ? 0 : 1;
           if (code == 1) ++st_skip;
@@ -274,7 +295,7 @@ __global__ void __launch_bounds__(128, 1)
       for (int c = 0; c < C::BC / 32; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float pv = my_keep ? ptx::ex2(fmaf(s[32 * c + i], sl2, -m)) : 0.0f;
+          const float pv = (my_keep && m > -INFINITY) ? ptx::ex2(fmaf(s[32 * c + i], sl2, -m)) : 0.0f;
           l += pv;
           s[32 * c + i] = pv;
           r[i] = __float_as_uint(tf32_trunc(pv));
@@ -362,7 +383,7 @@ __global__ void __launch_bounds__(128, 1)
       atomicAdd(&p.stats->v_blocks_loaded, st_vload);
       atomicAdd(&p.stats->mma_flops, st_flops);
       atomicAdd(&p.stats->bytes_loaded, static_cast<unsigned long long>(C::Q_BYTES) +
-                                            kvb * (nblk + st_vload));
+                                            kvb * (kload + st_vload));
     }
   } else if (t == 0) {
     record_error(p.err, BLASST_ETIMEOUT);

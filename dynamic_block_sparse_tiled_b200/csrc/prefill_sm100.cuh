@@ -34,6 +34,12 @@
 // With Br = 64 the 128 rows form two independent vote groups that share the
 // MMAs: a group that skips contributes zero rows of P and leaves its running
 // statistics untouched.
+// An optional static block mask (block-sparse input) excludes (query tile,
+// KV block) pairs before anything is computed: the CTA then walks a list of
+// the blocks some row group still visits, built in shared memory at start;
+// every role iterates over list positions (pipeline slots and parities) and
+// reads the block index from the list. The first-block rule applies to the
+// first listed block.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -50,6 +56,7 @@ struct PrefillParams {
   void* o;
   float* lse;
   uint8_t* mask;
+  const uint8_t* smask;  // optional static block mask [B, Hq, nQt, nKt], nonzero = excluded
   blasst_stats* stats;
   int* err;
   int B, Hq, Hkv, Lq, Lkv;
@@ -116,7 +123,11 @@ struct PrefillCfg {
   static constexpr int MISC_BYTES = 128;
   static constexpr int OFF_ST = OFF_MISC + MISC_BYTES;  // [2 sets][2: m, mref][128 rows] floats
   static constexpr int OFF_LSUM = OFF_ST + 2 * 2 * 128 * 4;  // [2 sets][128 rows] floats
-  static constexpr int SMEM_BYTES = OFF_LSUM + 2 * 128 * 4 + 1024;  // + alignment slack
+  static constexpr int MAX_LIST = 4096;  // listed blocks with a static mask (Lkv <= 4096 Bc)
+  static constexpr int OFF_LIST = OFF_LSUM + 2 * 128 * 4;     // [MAX_LIST] kt | groups << 16
+  static constexpr int OFF_SCAN = OFF_LIST + MAX_LIST * 4;    // [NTHREADS] counts
+  static constexpr int SMEM_BYTES = OFF_LIST + 1024;                   // + alignment slack
+  static constexpr int SMEM_BYTES_LISTED = OFF_SCAN + NTHREADS * 4 + 1024;
   static constexpr int S_COL = 0;          // S buffer b at column b * BC (P: first BC/2)
   static constexpr int O_COL = NS * BC;    // O accumulator
   static constexpr int TMEM_COLS = pow2_at_least(O_COL + D);
@@ -127,7 +138,7 @@ struct PrefillCfg {
   static_assert(BC == 64 || BC == 128, "KV block");
   static_assert(BR == 64 || BR == 128, "query tile");
   static_assert(TMEM_COLS <= 512, "TMEM budget");
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(SMEM_BYTES_LISTED <= 227 * 1024, "shared memory budget");
   static_assert(NSLOT > NS, "decision slots must outlive the S look-ahead");
 };
 
@@ -135,7 +146,9 @@ __device__ __forceinline__ void record_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
-template <int D, int BC, int BR>
+// LISTED: compiled for a static block mask (p.smask != null) or without one;
+// the version without keeps no list and none of its bookkeeping.
+template <int D, int BC, int BR, bool LISTED>
 __global__ void __launch_bounds__(384, 1)
     blasst_prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                                const __grid_constant__ CUtensorMap tmK,
@@ -188,6 +201,71 @@ __global__ void __launch_bounds__(384, 1)
     nblk = max(nblk, kt_last[gg] + 1);
   }
 
+  // ---- static block mask: list of the blocks some row group visits --------
+  constexpr bool listed = LISTED;
+  uint32_t* vlist = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
+  if constexpr (LISTED) {
+    // every thread takes a contiguous strip of blocks; counts, an exclusive
+    // scan over the CTA, then the strips are written in order
+    int* scan = reinterpret_cast<int*>(smem + C::OFF_SCAN);
+    const int strip = (nblk + C::NTHREADS - 1) / C::NTHREADS;
+    const int k0 = static_cast<int>(threadIdx.x) * strip;
+    const int k1 = min(k0 + strip, nblk);
+    auto groups_of = [&](int kt) -> uint32_t {
+      uint32_t gm = 0;
+#pragma unroll
+      for (int gg = 0; gg < C::NG; ++gg)
+        if (kt <= kt_last[gg] &&
+            p.smask[(static_cast<size_t>(bh) * p.nQt + (r0 / BR + gg)) * p.nKt + kt] == 0)
+          gm |= 1u << gg;
+      return gm;
+    };
+    int cnt = 0;
+    for (int kt = k0; kt < k1; ++kt) cnt += groups_of(kt) ? 1 : 0;
+    scan[threadIdx.x] = cnt;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int acc = 0;
+      for (int i = 0; i < C::NTHREADS; ++i) {
+        const int c = scan[i];
+        scan[i] = acc;
+        acc += c;
+      }
+      misc[2] = acc;
+    }
+    __syncthreads();
+    int pos = scan[threadIdx.x];
+    for (int kt = k0; kt < k1; ++kt) {
+      const uint32_t gm = groups_of(kt);
+      if (gm) vlist[pos++] = static_cast<uint32_t>(kt) | (gm << 16);
+    }
+    // every (tile, block) pair starts as "not visited"; the V warp writes the
+    // visited ones after the barrier below
+    if (p.mask) {
+#pragma unroll
+      for (int gg = 0; gg < C::NG; ++gg) {
+        if (kt_last[gg] < 0) continue;
+        uint8_t* mrow = p.mask + (static_cast<size_t>(bh) * p.nQt + (r0 / BR + gg)) * p.nKt;
+        for (int kt = static_cast<int>(threadIdx.x); kt < p.nKt; kt += C::NTHREADS) mrow[kt] = 2;
+      }
+    }
+    __syncthreads();
+    nblk = misc[2];  // from here on: number of listed blocks
+  }
+  // block index and visiting row groups of list position j
+  auto kt_of = [&](int j) -> int {
+    if constexpr (LISTED) return static_cast<int>(vlist[j] & 0xFFFFu);
+    else return j;
+  };
+  auto groups_at = [&](int j) -> uint32_t {
+    if constexpr (LISTED) return vlist[j] >> 16;
+    uint32_t gm = 0;
+#pragma unroll
+    for (int gg = 0; gg < C::NG; ++gg)
+      if (j <= kt_last[gg]) gm |= 1u << gg;
+    return gm;
+  };
+
   // ---- set-up -------------------------------------------------------------
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(C::B_Q), 1);
@@ -212,7 +290,8 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_init(bar(C::B_HS + i), 4);
       ptx::mbar_init(bar(C::B_DRAIN + i), 1);
     }
-    for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
+    for (int i = 1; i < C::MISC_BYTES / 4; ++i)
+      if (i != 2) misc[i] = 0;
     ptx::fence_mbar_init();
   }
   if (warp == C::WARP_MMA) {
@@ -247,7 +326,7 @@ __global__ void __launch_bounds__(384, 1)
           ok = ptx::mbar_wait(bar(C::B_KE + ks), ((j / C::NK) - 1) & 1, abort_flag,
                               p.timeout_ns);
         if (!ok) break;
-        load_kv(&tmK, sb + C::OFF_K + ks * C::KV_BYTES, j, bar(C::B_KF + ks));
+        load_kv(&tmK, sb + C::OFF_K + ks * C::KV_BYTES, kt_of(j), bar(C::B_KF + ks));
       }
       if (!ok) {
         *abort_flag = 1;
@@ -272,17 +351,19 @@ __global__ void __launch_bounds__(384, 1)
         // skip-mask entries and counters for block j (off the softmax path)
         const unsigned long long tile_flops = 2ull * 128ull * BC * D;
         st_flops += tile_flops + (keepmask ? tile_flops : 0ull);
+        const int kt = kt_of(j);
+        const uint32_t gvis = groups_at(j);
 #pragma unroll
         for (int gg = 0; gg < C::NG; ++gg) {
           if (kt_last[gg] < 0) continue;
           uint8_t code = 2;
-          if (j <= kt_last[gg]) {
+          if ((gvis >> gg) & 1) {
             ++st_vis;
             code = ((keepmask >> gg) & 1) ? 0 : 1;
             if (code == 1) ++st_skip;
           }
           if (p.mask)
-            p.mask[(static_cast<size_t>(bh) * p.nQt + (r0 / BR + gg)) * p.nKt + j] = code;
+            p.mask[(static_cast<size_t>(bh) * p.nQt + (r0 / BR + gg)) * p.nKt + kt] = code;
         }
         if (keepmask != 0) {
           const int vs = vcount % C::NV;
@@ -290,7 +371,7 @@ __global__ void __launch_bounds__(384, 1)
             ok = ptx::mbar_wait(bar(C::B_VE + vs), ((vcount / C::NV) - 1) & 1, abort_flag,
                                 p.timeout_ns);
           if (!ok) break;
-          load_kv(&tmV, sb + C::OFF_V + vs * C::KV_BYTES, j, bar(C::B_VF + vs));
+          load_kv(&tmV, sb + C::OFF_V + vs * C::KV_BYTES, kt, bar(C::B_VF + vs));
           ++vcount;
         }
       }
@@ -411,7 +492,6 @@ __global__ void __launch_bounds__(384, 1)
     const int row = r0 + t;
     const bool row_exists = row < p.Lq;
     const int gi = t / BR;
-    const int my_kt_last = kt_last[gi];
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int last_col = p.causal ? min(row + p.off, p.Lkv - 1) : p.Lkv - 1;
     const float sl2 = p.scale_log2;
@@ -439,7 +519,9 @@ __global__ void __launch_bounds__(384, 1)
       // ---- row max of block j (masked), first chunks kept in registers ---
       uint32_t sk[C::KEEPC * 32];
       float mbh = -INFINITY;
-      const int col0 = j * BC;
+      const int kt = kt_of(j);
+      const uint32_t gvis = groups_at(j);
+      const int col0 = kt * BC;
       const bool need_mask = (col0 + BC > p.Lkv) || (p.causal && col0 + BC - 1 > r0 + p.off);
       if (ok) {
         float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -485,9 +567,10 @@ __global__ void __launch_bounds__(384, 1)
       //      negligible; a block beyond a row's causal range votes skip -----
       bool rowskip = true;
       if (ok) {
-        const bool visited = j <= my_kt_last;
+        const bool visited = (gvis >> gi) & 1;
         if (!row_exists || !visited) rowskip = true;
         else if (j == 0 || !thresholding) rowskip = false;
+        else if (LISTED && mbh == -INFINITY) rowskip = true;  // no visible key here
         else rowskip = (mbh - m) < p.log2_lambda;
       }
       int keepmask = 0;
@@ -496,7 +579,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok && lane == 0) sm_abort[set] = 1;
         const bool all_skip = ptx::named_bar_and(1 + set, 128, rowskip);
         any_abort = sm_abort[set] != 0;
-        if (j <= kt_last[0] && !all_skip) keepmask = 1;
+        if ((gvis & 1u) && !all_skip) keepmask = 1;
       } else {
         const unsigned all_skip = __all_sync(0xffffffffu, rowskip) ? 1u : 0u;
         volatile int* vw = votes + set * 4;  // one word per warp of the set
@@ -511,7 +594,7 @@ __global__ void __launch_bounds__(384, 1)
             if (v == 2) any_abort = true;
             gskip = gskip && (v != 0);
           }
-          if (j <= kt_last[gg] && !gskip) keepmask |= 1 << gg;
+          if (((gvis >> gg) & 1) && !gskip) keepmask |= 1 << gg;
         }
         if (sm_abort[set] != 0) any_abort = true;
         // the words are rewritten only after this set's next barrier below
@@ -589,7 +672,8 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
           uint32_t pk[16];
-          if (my_keep) {
+          // (with a static mask a row may have no key yet: it adds nothing)
+          if (my_keep && (!LISTED || mref_new > -INFINITY)) {
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
               float x0, x1, p0, p1;
@@ -632,8 +716,9 @@ __global__ void __launch_bounds__(384, 1)
     ptx::named_bar_sync(3, C::NSOFT);
     // final statistics: the state after block nblk-1, handed to set nblk & 1
     const int fin = nblk & 1;
-    const float mref_fin = st_rows[fin * 256 + 128 + t];
-    const int last_fin = st_last[fin];
+    // (a static mask can leave no block at all: then O = 0, lse = -inf)
+    const float mref_fin = nblk > 0 ? st_rows[fin * 256 + 128 + t] : -INFINITY;
+    const int last_fin = nblk > 0 ? st_last[fin] : -1;
     const float l_mine =
         (lref == -INFINITY || mref_fin == -INFINITY) ? 0.0f : l * ptx::ex2(lref - mref_fin);
     lsum[set * 128 + t] = l_mine;
@@ -673,7 +758,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (row_exists && half == 0)
         p.lse[static_cast<size_t>(bh) * p.Lq + row] = (mref_fin + log2f(ltot)) * 0.6931471805599453f;
-      if (p.mask) {
+      if (p.mask && !listed) {  // with a static mask every entry was preset
 #pragma unroll
         for (int gg = 0; gg < C::NG; ++gg) {
           if (kt_last[gg] < 0) continue;

@@ -97,7 +97,20 @@ BLASST_API int blasst_fwd(const void* q, const void* k, const void* v, void* o, 
  *              both products use an error-compensated three-product tf32 split);
  *   scale      score scale; <= 0 selects 1/sqrt(d);
  *   stream     cudaStream_t to enqueue on (NULL = legacy default stream);
- *   stats_out  nullable DEVICE pointer; counters are added to it. */
+ *   stats_out  nullable DEVICE pointer; counters are added to it;
+ *   block_mask_in  nullable DEVICE pointer, uint8 [B, Hq, ceil(Lq/Br), ceil(Lkv/Bc)]:
+ *              a static block-sparse mask. A nonzero entry excludes that
+ *              (query tile, KV block) pair before anything is computed: no
+ *              scores, no vote, nothing added, reported as 2 (not visited) in
+ *              skip_mask_out. The threshold skip then runs over the blocks
+ *              left, and the first of them is always computed (the
+ *              first-block rule of "BLASST: Dynamic BLocked Attention
+ *              Sparsity via Softmax Thresholding", the post's figure, read
+ *              for the blocks the mask leaves). Rows left with no key get
+ *              O = 0 and lse = -inf. This is the block-sparse input that a
+ *              pre-pass selector feeds; the pages describe such selectors
+ *              (CRISP, FlashPrefill) but give no interface for it. Requires
+ *              ceil(Lkv/Bc) <= 4096, else BLASST_EUNSUPPORTED. */
 typedef struct blasst_fwd_args {
   const void* q;
   const void* k;
@@ -113,6 +126,7 @@ typedef struct blasst_fwd_args {
   float scale;
   void* stream;
   blasst_stats* stats_out;
+  const uint8_t* block_mask_in;
 } blasst_fwd_args;
 BLASST_API int blasst_fwd_ex(const blasst_fwd_args* args);
 

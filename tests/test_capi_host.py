@@ -47,7 +47,7 @@ def _fwd(lib, **kw):
     import dynamic_block_sparse_tiled_b200 as bl
     base = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0x50000, B=1, Hq=4, Hkv=2,
                 Lq=256, Lkv=256, d=128, causal=1, lam=1e-3, Br=128, Bc=128, skip_mask_out=None,
-                dtype=0, scale=0.0, stream=None, stats_out=None)
+                dtype=0, scale=0.0, stream=None, stats_out=None, block_mask_in=None)
     base.update(kw)
     args = bl._FwdArgs(*[base[f[0]] for f in bl._FwdArgs._fields_])
     return lib.blasst_fwd_ex(C.byref(args))
@@ -69,6 +69,7 @@ def _fwd(lib, **kw):
     (dict(dtype=7), -2),
     (dict(dtype=1, d=128, Bc=64), -2),   # fp32 is d = 64 only
     (dict(dtype=1, d=64, Bc=128), -2),   # fp32 is Bc = 64 only
+    (dict(Lq=4096 * 128 + 1, Lkv=4096 * 128 + 1, block_mask_in=0x60000), -2),  # list too long
 ])
 def test_fwd_rejects_bad_arguments_without_a_gpu(lib, bad, code):
     assert _fwd(lib, **bad) == code

@@ -14,20 +14,22 @@ def _lib():
     return bl
 
 
-def run_case(w, lam, items=None, check_stats=True):
-    """Run GPU and oracle on workload ``w`` at threshold ``lam`` and compare."""
+def run_case(w, lam, items=None, check_stats=True, static_mask=None):
+    """Run GPU and oracle on workload ``w`` at threshold ``lam`` and compare
+    (optionally with a static block mask, uint8 [B, Hq, nQt, nKt])."""
     import torch
     bl = _lib()
     inp = synth.generate(w)
     q, k, v = (parity.to_device(a) for a in (inp.q, inp.k, inp.v))
     st = bl.new_stats()
     lam32 = float(np.float32(lam))
+    sm_dev = None if static_mask is None else torch.from_numpy(static_mask).cuda()
     o, lse, mask = bl.attention_prefill(q, k, v, causal=w.causal, lam=lam32, Br=w.Br, Bc=w.Bc,
-                                        with_mask=True, stats=st)
+                                        with_mask=True, stats=st, block_mask=sm_dev)
     assert bl.blasst_check() == 0
     torch.cuda.synchronize()
     ref = oracle.prefill(inp.q, inp.k, inp.v, causal=w.causal, lam=lam32, Br=w.Br, Bc=w.Bc,
-                         items=items)
+                         items=items, static_mask=static_mask)
     nQt, nKt = ref["nQt"], ref["nKt"]
     mask_g = mask.cpu().numpy()
     items_arr = ref["items"]
@@ -47,6 +49,10 @@ def run_case(w, lam, items=None, check_stats=True):
     n_vis, n_dis, ok, dis = parity.compare_masks(mask_gt, ref["mask"], ref["margin"], lam32)
     assert ok, f"mask: {n_dis} of {n_vis} visited tiles disagree outside the tie band"
     row_ok = valid & ~dis.any(axis=1)[:, None]
+    # rows left with no key at all (a static mask can do that): O = 0, lse = -inf
+    empty = row_ok & np.isneginf(ref["lse"])
+    assert np.all(np.isneginf(lse_gt[empty])) and np.all(o_gt[empty] == 0.0)
+    row_ok = row_ok & ~empty
     stats = parity.compare_outputs(o_gt, lse_gt, ref["o"], ref["lse"], row_ok)
     parity.assert_within(stats, w.name, parity.FP32_TOL if w.dtype == "fp32" else None)
     if check_stats and items is None:
@@ -107,6 +113,55 @@ def test_prefill_fp32_parity(name, over, lam):
     r = run_case(w, lam)
     if lam >= 1e-3 and w.amp > 3 and w.causal:
         assert r["skip"] > 0.05, f"skip path not exercised: {r}"
+
+
+def _static_mask_for(w, seed, frac=0.4):
+    """Seeded static block mask with the awkward cases forced in: tiles that
+    lose block 0, and one tile that loses every block."""
+    nQt, nKt = -(-w.Lq // w.Br), -(-w.Lkv // w.Bc)
+    rng = np.random.default_rng(seed)
+    sm = (rng.random((w.B, w.Hq, nQt, nKt)) < frac).astype(np.uint8)
+    sm[:, :, 1::3, 0] = 1
+    sm[0, -1, nQt // 2, :] = 1
+    return sm
+
+
+STATIC = [
+    ("gqa_2k_a12", BASE.replace(name="s1", Hq=4, Hkv=2, Lq=2048, Lkv=2048, amp=12.0, window=256,
+                                n_needles=2)),
+    ("br64_ragged", BASE.replace(name="s2", Hq=2, Hkv=1, Lq=777, Lkv=777, Br=64, amp=12.0,
+                                 window=256, n_needles=2)),
+    ("d64_bc64", BASE.replace(name="s3", Hq=2, Hkv=2, Lq=640, Lkv=640, d=64, Br=64, Bc=64,
+                              amp=12.0, window=256, n_needles=2)),
+    ("noncausal", BASE.replace(name="s4", Hq=2, Hkv=2, Lq=512, Lkv=900, causal=False, amp=12.0,
+                               window=256, n_needles=2)),
+    ("fp32_tiny", synth.CONFIGS["tiny_fp32_1k"].replace(name="s5", amp=12.0, window=128,
+                                                         n_needles=2)),
+]
+
+
+@pytest.mark.parametrize("name,w", STATIC, ids=[s[0] for s in STATIC])
+@pytest.mark.parametrize("lam", [0.0, 1e-3])
+def test_prefill_static_block_mask(name, w, lam):
+    """Caller-supplied static block mask: excluded pairs are not visited, the
+    first block left is computed, the rest against the oracle as usual."""
+    sm = _static_mask_for(w, 11)
+    r = run_case(w, lam, static_mask=sm)
+    assert r["n_vis"] > 0
+
+
+def test_prefill_static_mask_all_zero_is_no_mask():
+    """An all-zero static mask gives the same bits as no mask."""
+    import torch
+    bl = _lib()
+    w = BASE.replace(name="z", Hq=2, Hkv=1, Lq=1024, Lkv=1024, amp=12.0, window=256, n_needles=2)
+    inp = synth.generate(w)
+    q, k, v = (parity.to_device(a) for a in (inp.q, inp.k, inp.v))
+    zero = torch.zeros((1, 2, 8, 8), dtype=torch.uint8, device="cuda")
+    a = bl.attention_prefill(q, k, v, causal=True, lam=1e-3, with_mask=True)
+    b = bl.attention_prefill(q, k, v, causal=True, lam=1e-3, with_mask=True, block_mask=zero)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
 
 
 @pytest.mark.parametrize("cfg", ["prefill_32k", "prefill_32k_a12"])
