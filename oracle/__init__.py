@@ -69,6 +69,18 @@ class _DecodeArgs(C.Structure):
     ]
 
 
+class _BackwardArgs(C.Structure):
+    _fields_ = [
+        ("q", C.c_void_p), ("k", C.c_void_p), ("v", C.c_void_p), ("dout", C.c_void_p),
+        ("dtype", C.c_int),
+        ("B", C.c_int64), ("Hq", C.c_int64), ("Hkv", C.c_int64),
+        ("Lq", C.c_int64), ("Lkv", C.c_int64), ("d", C.c_int64),
+        ("causal", C.c_int), ("Br", C.c_int64), ("Bc", C.c_int64), ("scale", C.c_double),
+        ("tile_mask", C.c_void_p),
+        ("dq", C.c_void_p), ("dk", C.c_void_p), ("dv", C.c_void_p), ("nthreads", C.c_int),
+    ]
+
+
 class Oracle:
     """Handle on one compiled copy of the oracle (``path`` defaults to the
     library built from ``blasst_oracle.c``; the tests also load copies with a
@@ -85,6 +97,8 @@ class Oracle:
         lib.oracle_lse_merge.restype = None
         lib.oracle_split_len.argtypes = [C.c_int64, C.c_int64, C.c_int64]
         lib.oracle_split_len.restype = C.c_int64
+        lib.oracle_backward.argtypes = [C.POINTER(_BackwardArgs)]
+        lib.oracle_backward.restype = C.c_int
         self.lib = lib
 
     def prefill(self, *a, **kw):
@@ -98,6 +112,9 @@ class Oracle:
 
     def split_len(self, *a, **kw):
         return split_len(*a, _lib=self.lib, **kw)
+
+    def backward(self, *a, **kw):
+        return backward(*a, _lib=self.lib, **kw)
 
 
 def _load():
@@ -235,3 +252,33 @@ def lse_merge(o_parts, lse_parts, _lib=None):
     (_lib or _load()).oracle_lse_merge(o_parts.ctypes.data, lse_parts.ctypes.data, n, S, d, o.ctypes.data,
                              lse.ctypes.data)
     return o, lse
+
+
+def backward(q, k, v, dout, *, causal: bool, Br: int, Bc: int, scale: float | None = None,
+             tile_mask=None, nthreads: int = 0, _lib=None):
+    """Gradients (dq, dk, dv) of softmax attention over the kept keys, the
+    forward's decisions held fixed. ``tile_mask``: uint8 [B, Hq, nQt, nKt] in
+    the layout of the forward's skip mask (0 = the pair was computed and is
+    kept); None keeps every causally visible key. Inputs as for ``prefill``;
+    ``dout`` is dL/dO in the same dtype. Returns float64 arrays."""
+    q, k, v, dout = (np.ascontiguousarray(t) for t in (q, k, v, dout))
+    code = _dtype_code(q)
+    assert all(_dtype_code(t) == code for t in (k, v, dout))
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    tm = None
+    if tile_mask is not None:
+        tm = np.ascontiguousarray(np.asarray(tile_mask, dtype=np.uint8))
+        assert tm.shape == (B, Hq, -(-Lq // Br), -(-Lkv // Bc)), tm.shape
+    dq = np.zeros((B, Hq, Lq, d), np.float64)
+    dk = np.zeros((B, Hkv, Lkv, d), np.float64)
+    dv = np.zeros((B, Hkv, Lkv, d), np.float64)
+    args = _BackwardArgs(q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, code,
+                         B, Hq, Hkv, Lq, Lkv, d, int(bool(causal)), Br, Bc, float(scale),
+                         _ptr(tm), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, int(nthreads))
+    rc = (_lib or _load()).oracle_backward(C.byref(args))
+    if rc != 0:
+        raise ValueError("oracle_backward rejected its arguments")
+    return dq, dk, dv

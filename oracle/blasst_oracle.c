@@ -471,3 +471,147 @@ int oracle_decode(oracle_decode_args *a) {
                      a->o, a->lse);
   return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward pass with the forward's decisions held fixed.                    */
+/* ------------------------------------------------------------------------ */
+/*
+ * With the skip decisions of a forward pass held constant, its output is
+ * softmax attention over the kept keys of each row ([T] para 5: a dropped
+ * block contributes nothing), so the gradient of a loss L(O) is the one of
+ * that restricted attention. Written out from the definitions, per query
+ * row i with kept key set K_i and s_ij = scale * q_i . k_j:
+ *   P_ij  = exp(s_ij - lse_i) for j in K_i, else 0, lse_i = ln sum_K_i exp(s_ij)
+ *   O_i   = sum_j P_ij v_j
+ *   dP_ij = dO_i . v_j,   D_i = sum_j P_ij dP_ij  (= dO_i . O_i)
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j  = scale * sum_i dS_ij q_i,   dV_j = sum_i P_ij dO_i
+ * (summed over the query heads that share a KV head). The kept set comes
+ * from a tile mask in the layout of the forward's skip mask: a (query tile,
+ * KV block) pair is kept when its entry is 0; NULL keeps every causally
+ * visible key. Everything in double.
+ */
+typedef struct {
+  const void *q, *k, *v, *dout;
+  int dtype;
+  int64_t B, Hq, Hkv, Lq, Lkv, d;
+  int causal;
+  int64_t Br, Bc;
+  double scale;
+  const uint8_t *tile_mask; /* [B, Hq, nQt, nKt], 0 = kept; NULL = all visible kept */
+  double *dq;               /* [B, Hq, Lq, d] */
+  double *dk, *dv;          /* [B, Hkv, Lkv, d] */
+  int nthreads;
+} oracle_backward_args;
+
+typedef struct {
+  const oracle_backward_args *a;
+  int64_t next;
+  pthread_mutex_t mu;
+} backward_ctx;
+
+/* One (b, hk) unit: every query head of the group, every row. */
+static void backward_unit(const oracle_backward_args *a, int64_t unit, double *qi,
+                          double *doi, double *s, double *p, double *ds) {
+  const int64_t d = a->d, Lq = a->Lq, Lkv = a->Lkv, g = a->Hq / a->Hkv;
+  const int64_t nQt = (Lq + a->Br - 1) / a->Br, nKt = (Lkv + a->Bc - 1) / a->Bc;
+  const int64_t b = unit / a->Hkv, hk = unit % a->Hkv;
+  const int64_t off = Lkv - Lq;
+  const int64_t kvbase = ((b * a->Hkv + hk) * Lkv) * d;
+  for (int64_t hh = 0; hh < g; ++hh) {
+    const int64_t hq = hk * g + hh;
+    const int64_t qbase = ((b * a->Hq + hq) * Lq) * d;
+    for (int64_t i = 0; i < Lq; ++i) {
+      for (int64_t x = 0; x < d; ++x) {
+        qi[x] = widen(a->q, a->dtype, qbase + i * d + x);
+        doi[x] = widen(a->dout, a->dtype, qbase + i * d + x);
+      }
+      const int64_t qt = i / a->Br;
+      double mx = -INFINITY;
+      for (int64_t j = 0; j < Lkv; ++j) {
+        int kept = !a->causal || j <= i + off;
+        if (kept && a->tile_mask)
+          kept = a->tile_mask[((b * a->Hq + hq) * nQt + qt) * nKt + j / a->Bc] == 0;
+        double sv = -INFINITY;
+        if (kept) {
+          double dot = 0.0;
+          for (int64_t x = 0; x < d; ++x) dot += qi[x] * widen(a->k, a->dtype, kvbase + j * d + x);
+          sv = a->scale * dot;
+        }
+        s[j] = sv;
+        if (sv > mx) mx = sv;
+      }
+      double *dqi = a->dq + qbase + i * d;
+      for (int64_t x = 0; x < d; ++x) dqi[x] = 0.0;
+      if (mx == -INFINITY) continue; /* no kept key: O = 0, no gradient */
+      double sum = 0.0;
+      for (int64_t j = 0; j < Lkv; ++j) sum += s[j] == -INFINITY ? 0.0 : exp(s[j] - mx);
+      const double lse = mx + log(sum);
+      double D = 0.0;
+      for (int64_t j = 0; j < Lkv; ++j) {
+        p[j] = s[j] == -INFINITY ? 0.0 : exp(s[j] - lse);
+        double dp = 0.0;
+        if (p[j] != 0.0)
+          for (int64_t x = 0; x < d; ++x) dp += doi[x] * widen(a->v, a->dtype, kvbase + j * d + x);
+        ds[j] = dp; /* dP for now */
+        D += p[j] * dp;
+      }
+      for (int64_t j = 0; j < Lkv; ++j) {
+        if (p[j] == 0.0) continue;
+        const double dsj = p[j] * (ds[j] - D);
+        double *dkj = a->dk + kvbase + j * d;
+        double *dvj = a->dv + kvbase + j * d;
+        for (int64_t x = 0; x < d; ++x) {
+          dqi[x] += a->scale * dsj * widen(a->k, a->dtype, kvbase + j * d + x);
+          dkj[x] += a->scale * dsj * qi[x];
+          dvj[x] += p[j] * doi[x];
+        }
+      }
+    }
+  }
+}
+
+static void *backward_worker(void *vp) {
+  backward_ctx *ctx = (backward_ctx *)vp;
+  const oracle_backward_args *a = ctx->a;
+  double *qi = malloc(sizeof(double) * a->d);
+  double *doi = malloc(sizeof(double) * a->d);
+  double *s = malloc(sizeof(double) * a->Lkv);
+  double *p = malloc(sizeof(double) * a->Lkv);
+  double *ds = malloc(sizeof(double) * a->Lkv);
+  if (!qi || !doi || !s || !p || !ds) goto out;
+  for (;;) {
+    pthread_mutex_lock(&ctx->mu);
+    int64_t unit = ctx->next++;
+    pthread_mutex_unlock(&ctx->mu);
+    if (unit >= a->B * a->Hkv) break;
+    backward_unit(a, unit, qi, doi, s, p, ds);
+  }
+out:
+  free(qi); free(doi); free(s); free(p); free(ds);
+  return NULL;
+}
+
+int oracle_backward(oracle_backward_args *a) {
+  if (!a || a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Hq % a->Hkv || a->Lq <= 0 ||
+      a->Lkv <= 0 || a->d <= 0 || a->Br <= 0 || a->Bc <= 0 || !a->dq || !a->dk || !a->dv)
+    return -1;
+  memset(a->dk, 0, sizeof(double) * (size_t)(a->B * a->Hkv * a->Lkv * a->d));
+  memset(a->dv, 0, sizeof(double) * (size_t)(a->B * a->Hkv * a->Lkv * a->d));
+  backward_ctx ctx;
+  ctx.a = a;
+  ctx.next = 0;
+  pthread_mutex_init(&ctx.mu, NULL);
+  int64_t total = a->B * a->Hkv;
+  int nt = resolve_threads(a->nthreads);
+  if (nt > total) nt = (int)total;
+  if (nt > 512) nt = 512;
+  pthread_t th[512];
+  int ok[512], any = 0;
+  for (int t = 0; t < nt; ++t) { ok[t] = pthread_create(&th[t], NULL, backward_worker, &ctx) == 0; any |= ok[t]; }
+  for (int t = 0; t < nt; ++t) if (ok[t]) pthread_join(th[t], NULL);
+  if (!any) backward_worker(&ctx);
+  pthread_mutex_destroy(&ctx.mu);
+  return 0;
+}

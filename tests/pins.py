@@ -446,6 +446,76 @@ def pin_static_mask_with_threshold(orc):
     assert abs(res["lse"][0, 0] - np.log(w1 + w2)) < 1e-14
 
 
+# --------------------------------------------------------------------------
+# Backward pass with the forward's decisions held fixed: checked against
+# central finite differences of the independent dense brute force.
+# --------------------------------------------------------------------------
+def _fd_grads(q, k, v, dout, causal, keep, h=1e-6):
+    """dL/dq, dL/dk, dL/dv of L = sum(dout * O) by central differences."""
+    def loss(qq, kk, vv):
+        o, _ = dense_attention(qq, kk, vv, causal, keep=keep)
+        return float(np.nansum(dout * np.nan_to_num(o)))
+    grads = []
+    for t_idx in range(3):
+        base = [q.copy(), k.copy(), v.copy()]
+        gr = np.zeros_like(base[t_idx])
+        it = np.nditer(base[t_idx], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            plus = [x.copy() for x in base]
+            minus = [x.copy() for x in base]
+            plus[t_idx][idx] += h
+            minus[t_idx][idx] -= h
+            gr[idx] = (loss(*plus) - loss(*minus)) / (2 * h)
+        grads.append(gr)
+    return grads
+
+
+def pin_backward_matches_finite_differences(orc):
+    """The gradient of softmax attention over the kept keys (a dropped block
+    contributes nothing, para 5, and the decisions are held fixed) agrees with
+    central differences of the dense brute force: dense, causal and
+    non-causal, and with a tile mask removing some (query tile, KV block)
+    pairs, including a whole tile."""
+    B, Hq, Hkv, L, d, Br, Bc = 1, 2, 1, 20, 4, 4, 4
+    for causal in (True, False):
+        for masked in (False, True):
+            rng = np.random.default_rng(21 + 2 * causal + masked)
+            q, k, v = (rng.standard_normal(sh) for sh in
+                       ((B, Hq, L, d), (B, Hkv, L, d), (B, Hkv, L, d)))
+            dout = rng.standard_normal((B, Hq, L, d))
+            nT = -(-L // Br)
+            tm = None
+            keep = None
+            if masked:
+                tm = (rng.random((B, Hq, nT, nT)) < 0.3).astype(np.uint8)
+                tm[..., 0] = 0
+                tm[0, 1, 2, :] = 2  # a tile with nothing kept
+                keep = _allowed_from_static(tm, Br, Bc, L, L)
+            dq, dk, dv = orc.backward(q, k, v, dout, causal=causal, Br=Br, Bc=Bc, tile_mask=tm)
+            with np.errstate(invalid="ignore", divide="ignore"):
+                fq, fk, fv = _fd_grads(q, k, v, dout, causal, keep)
+            for got, ref in ((dq, fq), (dk, fk), (dv, fv)):
+                np.testing.assert_allclose(got, ref, rtol=0, atol=2e-7)
+
+
+def pin_backward_gqa_replication(orc):
+    """Query heads sharing a KV head: dq equals the run with the KV heads
+    replicated, and dk, dv are the sums over the replicas."""
+    rng = np.random.default_rng(5)
+    B, Hq, Hkv, L, d = 1, 4, 2, 24, 8
+    q = rng.standard_normal((B, Hq, L, d))
+    k = rng.standard_normal((B, Hkv, L, d))
+    v = rng.standard_normal((B, Hkv, L, d))
+    dout = rng.standard_normal((B, Hq, L, d))
+    dq, dk, dv = orc.backward(q, k, v, dout, causal=True, Br=8, Bc=8)
+    kr, vr = np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1)
+    dq2, dk2, dv2 = orc.backward(q, kr, vr, dout, causal=True, Br=8, Bc=8)
+    np.testing.assert_allclose(dq, dq2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk, dk2.reshape(B, Hkv, 2, L, d).sum(2), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv, dv2.reshape(B, Hkv, 2, L, d).sum(2), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [
     pin_lambda0_is_dense,
     pin_first_block_always_computed,
@@ -460,6 +530,8 @@ ALL_PINS = [
     pin_worked_example,
     pin_static_mask_is_restriction,
     pin_static_mask_with_threshold,
+    pin_backward_matches_finite_differences,
+    pin_backward_gqa_replication,
 ]
 
 

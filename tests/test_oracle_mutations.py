@@ -41,6 +41,11 @@ MUTATIONS = [
      "          for (int64_t x = 0; x < d; ++x) dot += qrow[r * d + x] * widen(a->k, a->dtype, kvbase + (kt * Bc + j) * d + x);\n"
      "          if (a->scale * dot > m[r]) m[r] = a->scale * dot;\n        }\n      }\n    }\n"
      "    if (kt > kt_last || (smask && smask[kt])) {\n      if (mask) mask[kt] = MASK_NOT_VISITED;"),
+    ("backward_drops_D", "const double dsj = p[j] * (ds[j] - D);", "const double dsj = p[j] * ds[j];"),
+    ("backward_dk_from_k", "dkj[x] += a->scale * dsj * qi[x];",
+     "dkj[x] += a->scale * dsj * widen(a->k, a->dtype, kvbase + j * d + x);"),
+    ("backward_dv_without_p", "dvj[x] += p[j] * doi[x];", "dvj[x] += doi[x];"),
+    ("backward_ignores_tile_mask", "if (kept && a->tile_mask)", "if (0 && kept && a->tile_mask)"),
     ("decode_skipped_block_still_used", "    if (skip) continue;\n    for (int64_t j = 0; j < nc; ++j)\n      for (int64_t x = 0; x < d; ++x)\n        kv_v",
      "    for (int64_t j = 0; j < nc; ++j)\n      for (int64_t x = 0; x < d; ++x)\n        kv_v"),
 ]
