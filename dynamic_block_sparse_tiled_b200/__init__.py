@@ -25,7 +25,8 @@ __all__ = [
     "blasst_fwd", "blasst_fwd_ex", "blasst_decode", "blasst_decode_workspace_bytes",
     "blasst_lse_merge", "blasst_check", "blasst_selftest_exp2",
     "blasst_decode_noalloc", "blasst_decode_noalloc_max_bytes", "blasst_status_string", "blasst_version",
-    "attention_prefill", "attention_decode", "new_stats", "stats_dict",
+    "blasst_bwd", "blasst_bwd_workspace_bytes",
+    "attention_prefill", "attention_backward", "attention_decode", "new_stats", "stats_dict",
     "BLASST_OK", "BLASST_EINVAL", "BLASST_EUNSUPPORTED", "BLASST_ECUDA", "BLASST_ETIMEOUT",
     "BLASST_EWORKSPACE", "BLASST_BF16", "BLASST_FP32",
 ]
@@ -68,6 +69,18 @@ class _FwdArgs(C.Structure):
     ]
 
 
+class _BwdArgs(C.Structure):
+    _fields_ = [
+        ("q", C.c_void_p), ("k", C.c_void_p), ("v", C.c_void_p), ("o", C.c_void_p),
+        ("dout", C.c_void_p), ("lse", C.c_void_p),
+        ("dq", C.c_void_p), ("dk", C.c_void_p), ("dv", C.c_void_p),
+        ("B", C.c_int), ("Hq", C.c_int), ("Hkv", C.c_int), ("Lq", C.c_int), ("Lkv", C.c_int),
+        ("d", C.c_int), ("causal", C.c_int), ("Br", C.c_int), ("Bc", C.c_int),
+        ("skip_mask", C.c_void_p), ("scale", C.c_float),
+        ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t), ("stream", C.c_void_p),
+    ]
+
+
 def load_library(path: str | None = None):
     """Load ``libblasst.so`` (raises if it has not been built)."""
     global _lib
@@ -85,6 +98,10 @@ def load_library(path: str | None = None):
         lib.blasst_fwd.restype = i
         lib.blasst_fwd_ex.argtypes = [C.POINTER(_FwdArgs)]
         lib.blasst_fwd_ex.restype = i
+        lib.blasst_bwd.argtypes = [C.POINTER(_BwdArgs)]
+        lib.blasst_bwd.restype = i
+        lib.blasst_bwd_workspace_bytes.argtypes = [i, i, i]
+        lib.blasst_bwd_workspace_bytes.restype = sz
         lib.blasst_decode_workspace_bytes.argtypes = [i, i, i, i]
         lib.blasst_decode_workspace_bytes.restype = sz
         lib.blasst_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp, vp, vp]
@@ -175,6 +192,25 @@ def blasst_fwd_ex(q, k, v, o, lse, *, causal: bool, lam: float, Br: int, Bc: int
     _check(load_library().blasst_fwd_ex(C.byref(args)), "blasst_fwd_ex")
 
 
+def blasst_bwd_workspace_bytes(B: int, Hq: int, Lq: int) -> int:
+    return int(load_library().blasst_bwd_workspace_bytes(B, Hq, Lq))
+
+
+def blasst_bwd(q, k, v, o, dout, lse, dq, dk, dv, *, causal: bool, Br: int, Bc: int,
+               workspace, skip_mask=None, scale: float = 0.0, stream=None):
+    """The C entry point of the same name. q, o, dout [B,Hq,Lq,d] bf16; k, v
+    [B,Hkv,Lkv,d] bf16; lse [B,Hq,Lq] fp32; dq [B,Hq,Lq,d], dk/dv [B,Hkv,Lkv,d]
+    fp32 outputs; skip_mask the forward's uint8 decisions or None; workspace a
+    uint8 CUDA tensor of blasst_bwd_workspace_bytes() bytes."""
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    args = _BwdArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                    _ptr(dv), B, Hq, Hkv, Lq, Lkv, d, int(bool(causal)), Br, Bc, _ptr(skip_mask),
+                    float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                    _stream(stream))
+    _check(load_library().blasst_bwd(C.byref(args)), "blasst_bwd")
+
+
 def blasst_decode_workspace_bytes(B: int, Hq: int, d: int, num_splits: int) -> int:
     return int(load_library().blasst_decode_workspace_bytes(B, Hq, d, num_splits))
 
@@ -254,6 +290,23 @@ def attention_prefill(q, k, v, *, causal=True, lam=0.0, Br=128, Bc=128, scale=0.
     blasst_fwd_ex(q, k, v, o, lse, causal=causal, lam=lam, Br=Br, Bc=Bc, skip_mask_out=mask,
                   scale=scale, stream=stream, stats_out=stats, block_mask_in=block_mask)
     return o, lse, mask
+
+
+def attention_backward(q, k, v, o, lse, dout, *, causal=True, Br=128, Bc=128, skip_mask=None,
+                       scale=0.0, stream=None, workspace=None):
+    """Allocate fp32 gradients (and the workspace) with torch and run
+    blasst_bwd with the forward's decisions ``skip_mask``. Returns (dq, dk, dv)."""
+    import torch
+    B, Hq, Lq, d = q.shape
+    dq = torch.empty((B, Hq, Lq, d), dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(blasst_bwd_workspace_bytes(B, Hq, Lq), dtype=torch.uint8,
+                                device=q.device)
+    blasst_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal=causal, Br=Br, Bc=Bc, workspace=workspace,
+               skip_mask=skip_mask, scale=scale, stream=stream)
+    return dq, dk, dv
 
 
 def attention_decode(q, k_cache, v_cache, *, lam=0.0, Bc=128, num_splits=64, with_mask=False,

@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "../../include/blasst.h"
+#include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "prefill_f32_sm100.cuh"
 #include "prefill_sm100.cuh"
@@ -311,6 +312,87 @@ int blasst_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.stats_out = nullptr;
   a.block_mask_in = nullptr;
   return blasst_fwd_ex(&a);
+}
+
+size_t blasst_bwd_workspace_bytes(int B, int Hq, int Lq) {
+  if (B <= 0 || Hq <= 0 || Lq <= 0) return 0;
+  const size_t lqp = (static_cast<size_t>(Lq) + 63) / 64 * 64;
+  return 2 * static_cast<size_t>(B) * Hq * lqp * sizeof(float);
+}
+
+int blasst_bwd(const blasst_bwd_args* a) {
+  if (!a) return BLASST_EINVAL;
+  if (!a->q || !a->k || !a->v || !a->o || !a->dout || !a->lse || !a->dq || !a->dk || !a->dv)
+    return BLASST_EINVAL;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o) ||
+      !aligned16(a->dout) || !aligned16(a->lse) || !aligned16(a->dq) || !aligned16(a->dk) ||
+      !aligned16(a->dv))
+    return BLASST_EINVAL;
+  if (a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Lq <= 0 || a->Lkv <= 0) return BLASST_EINVAL;
+  if (a->Hq % a->Hkv != 0) return BLASST_EINVAL;
+  if (a->d != 128) return BLASST_EUNSUPPORTED;
+  if ((a->Br != 64 && a->Br != 128) || (a->Bc != 64 && a->Bc != 128)) return BLASST_EUNSUPPORTED;
+  if (a->causal && a->Lq > a->Lkv) return BLASST_EUNSUPPORTED;
+  if (static_cast<long long>(a->B) * a->Hq > (1ll << 24) ||
+      static_cast<long long>(a->B) * a->Hkv * ((a->Lkv + 127) / 128) > 0x7fffffffll ||
+      static_cast<long long>(a->B) * a->Hq * (((a->Lq + 63) / 64) * 64) / 8 > 0x7fffffffll)
+    return BLASST_EINVAL;
+  const size_t need = blasst_bwd_workspace_bytes(a->B, a->Hq, a->Lq);
+  if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
+    return BLASST_EWORKSPACE;
+
+  int* err = error_word();
+  if (!err) return BLASST_ECUDA;
+
+  const int LqP = (a->Lq + 63) / 64 * 64;
+  const long long n_rows = static_cast<long long>(a->B) * a->Hq * LqP;
+  blasst::BwdParams p{};
+  p.dq = a->dq;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.nl2 = static_cast<const float*>(a->workspace);
+  p.drow = static_cast<const float*>(a->workspace) + n_rows;
+  p.fmask = a->skip_mask;
+  p.err = err;
+  p.B = a->B;
+  p.Hq = a->Hq;
+  p.Hkv = a->Hkv;
+  p.Lq = a->Lq;
+  p.Lkv = a->Lkv;
+  p.g = a->Hq / a->Hkv;
+  p.LqP = LqP;
+  p.nT = LqP / 64;
+  p.nKb = (a->Lkv + 127) / 128;
+  p.Brf = a->Br;
+  p.Bcf = a->Bc;
+  p.nQf = (a->Lq + a->Br - 1) / a->Br;
+  p.nKf = (a->Lkv + a->Bc - 1) / a->Bc;
+  p.causal = a->causal ? 1 : 0;
+  p.off = a->Lkv - a->Lq;
+  const double scale = a->scale > 0.0f ? static_cast<double>(a->scale)
+                                       : 1.0 / std::sqrt(static_cast<double>(a->d));
+  p.scale = static_cast<float>(scale);
+  p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+  p.timeout_ns = kTimeoutNs;
+
+  CUtensorMap mq, mdo, mk, mv;
+  const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&mq, a->q, dt, 2, a->d, a->Lq, a->B * a->Hq, 64) ||
+      !make_map(&mdo, a->dout, dt, 2, a->d, a->Lq, a->B * a->Hq, 64) ||
+      !make_map(&mk, a->k, dt, 2, a->d, a->Lkv, a->B * a->Hkv, 128) ||
+      !make_map(&mv, a->v, dt, 2, a->d, a->Lkv, a->B * a->Hkv, 128))
+    return BLASST_ECUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(a->stream);
+  blasst::blasst_bwd_rows_kernel<<<static_cast<unsigned>((n_rows + 7) / 8), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(a->o), static_cast<const __nv_bfloat16*>(a->dout), a->lse,
+      const_cast<float*>(p.nl2), const_cast<float*>(p.drow), a->dq, n_rows, a->Lq, LqP);
+  int rc = cuda_status(cudaGetLastError());
+  if (rc != BLASST_OK) return rc;
+  using C = blasst::BwdCfg;
+  if (set_smem(blasst::blasst_bwd_kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
+  const dim3 grid(static_cast<unsigned>(p.nKb) * p.B * p.Hkv);
+  blasst::blasst_bwd_kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(mq, mdo, mk, mv, p);
+  return cuda_status(cudaGetLastError());
 }
 
 size_t blasst_decode_workspace_bytes(int B, int Hq, int d, int num_splits) {

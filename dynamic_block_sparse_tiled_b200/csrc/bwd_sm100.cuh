@@ -1,0 +1,687 @@
+// bwd_sm100.cuh - backward pass of blocked attention with softmax
+// thresholding on sm_100a (tcgen05 + TMEM + TMA), with the forward's
+// decisions held fixed.
+//
+// What is differentiated ("BLASST: Dynamic BLocked Attention Sparsity via
+// Softmax Thresholding", Telegram channel seeallochnaya, post 3655,
+// paragraphs 2-6 after the headline): the forward's output is softmax
+// attention over the keys it kept; a dropped (query tile, KV block) pair adds
+// nothing, its V is never used. The skip decisions are a step function of the
+// scores, so with them held fixed the gradient is the gradient of attention
+// restricted to the kept pairs:
+//   P  = exp(scale q.k - lse)   on kept (row, key) pairs, 0 elsewhere,
+//   Dr = rowsum(dO * O),
+//   dS = P * (dO.v - Dr),
+//   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO,
+// summed over the query heads of a GQA group for dK and dV. The pages give
+// no backward pass; this is the plain reading that the forward's definition
+// fixes.
+//
+// Layout of the work: one CTA per (batch, KV head, 128-key block j). K_j and
+// V_j stay in shared memory; the CTA walks the 64-row query tiles of the g
+// query heads whose pair with block j the forward kept, in order. Per pair
+// (all products on the tensor cores, 128 x 64 or 128 x 128 tiles):
+//   S^T  = K Q^T          (TMEM, lanes = keys)       bf16 SS
+//   dP^T = V dO^T         (TMEM, lanes = keys)       bf16 SS
+//   P^T, dS^T by the compute warps, one key row per thread;
+//   P^T (bf16) overwrites S^T in TMEM, dS^T (bf16) goes to shared memory;
+//   dV  += P^T dO         (TMEM accumulator)         bf16 TS
+//   dK  += dS^T Q         (TMEM accumulator)         bf16 SS
+//   dQ^T = K^T dS^T       (TMEM, lanes = head dims)  bf16 SS, then added to
+//                          the fp32 dQ in global memory with red.add, one
+//                          warp instruction per query row and 32 dims.
+// Computing the transposed S and dP puts the keys on TMEM lanes, so P^T can
+// feed dV straight from TMEM and every product keeps M = 128; dQ^T keeps the
+// head dims on lanes so that each red.add of a warp covers 128 contiguous
+// bytes of one dQ row.
+//
+// Warp roles (320 threads):
+//   warps 0-3  compute: P^T and dS^T, then the dV epilogue;
+//   warps 4-7  dQ writers: drain dQ^T from TMEM and add it to global dQ,
+//              then the dK epilogue;
+//   warp 8     producer: K and V once, then per pair Q, dO (TMA, 3-stage
+//              ring) and the pair's row statistics (bulk copies); builds the
+//              pair list by scanning the forward's decisions;
+//   warp 9     tcgen05 issuer; owns the TMEM allocation.
+// TMEM (512 columns): S^T/P^T x2 [0,128), dP^T/dQ^T x2 [128,256),
+// dV [256,384), dK [384,512).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/blasst.h"
+#include "ptx_sm100.cuh"
+
+namespace blasst {
+
+struct BwdParams {
+  float* dq;                // [B, Hq, Lq, 128] fp32, zeroed by the row pass, accumulated here
+  float* dk;                // [B, Hkv, Lkv, 128] fp32
+  float* dv;                // [B, Hkv, Lkv, 128] fp32
+  const float* nl2;         // [B*Hq, LqP]: -lse * log2(e), -inf for rows without keys / padding
+  const float* drow;        // [B*Hq, LqP]: rowsum(dO * O), 0 on padding
+  const uint8_t* fmask;     // forward decisions [B, Hq, nQf, nKf], 0 = computed; null = all
+  int* err;
+  int B, Hq, Hkv, Lq, Lkv, g;
+  int LqP;    // Lq rounded up to 64
+  int nT;     // ceil(Lq / 64) query tiles of the backward
+  int nKb;    // ceil(Lkv / 128) key blocks of the backward
+  int Brf, Bcf;  // the forward's tile sizes (decisions are per Brf x Bcf pair)
+  int nQf, nKf;  // ceil(Lq / Brf), ceil(Lkv / Bcf)
+  int causal;
+  int off;       // Lkv - Lq
+  float scale;       // score scale
+  float scale_log2;  // scale * log2(e)
+  uint64_t timeout_ns;
+};
+
+struct BwdCfg {
+  static constexpr int D = 128;
+  static constexpr int BK = 128;  // keys per CTA
+  static constexpr int BQ = 64;   // query rows per pair
+  static constexpr int NTHREADS = 320;
+  static constexpr int WARP_LOAD = 8, WARP_MMA = 9;
+  static constexpr int NST = 3;  // Q / dO stages
+  static constexpr int KV_BOX = BK * 128;      // [128 keys][64 dims] bf16, 16 KB
+  static constexpr int KV_BYTES = 2 * KV_BOX;  // 32 KB
+  static constexpr int Q_BOX = BQ * 128;       // [64 rows][64 dims] bf16, 8 KB
+  static constexpr int Q_BYTES = 2 * Q_BOX;    // 16 KB
+  static constexpr int DS_BYTES = BK * 128;    // [128 keys][64 q] bf16, 16 KB
+  static constexpr int ROWST_BYTES = 2 * BQ * 4;  // nl2[64], drow[64]
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;
+  static constexpr int OFF_DO = OFF_Q + NST * Q_BYTES;
+  static constexpr int OFF_DS = OFF_DO + NST * Q_BYTES;
+  static constexpr int OFF_RS = OFF_DS + 2 * DS_BYTES;
+  static constexpr int OFF_REC = OFF_RS + NST * ROWST_BYTES;  // [NST] int4 {hq, t, keep bits, end}
+  static constexpr int OFF_BAR = OFF_REC + NST * 16;
+  // barriers
+  static constexpr int B_KV = 0;
+  static constexpr int B_QF = 1;               // [NST] stage loaded (+ record)
+  static constexpr int B_QE = B_QF + NST;      // [NST] stage free: issuer commit + 4 writer warps
+  static constexpr int B_SF = B_QE + NST;      // [2] S^T ready
+  static constexpr int B_PR = B_SF + 2;        // [2] P^T in TMEM (4 compute warps)
+  static constexpr int B_DPF = B_PR + 2;       // [2] dP^T ready
+  static constexpr int B_DSR = B_DPF + 2;      // [2] dS^T in shared memory (4 compute warps)
+  static constexpr int B_DSE = B_DSR + 2;      // [2] dS^T buffer free (issuer commit)
+  static constexpr int B_DQF = B_DSE + 2;      // [2] dQ^T ready
+  static constexpr int B_DQE = B_DQF + 2;      // [2] dQ^T drained (4 writer warps)
+  static constexpr int B_ACC = B_DQE + 2;      // dV, dK final
+  static constexpr int B_DRAIN = B_ACC + 1;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int QE_COUNT = 1 + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  // misc words: [0] tmem base, [1] abort, [3] always 0 (waits only a timeout
+  // ends), [4] pairs processed (issuer)
+  static constexpr int MISC_BYTES = 64;
+  static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+  static constexpr int S_COL = 0;      // S^T buffer b at b * 64 (P^T: first 32 columns)
+  static constexpr int DP_COL = 128;   // dP^T / dQ^T buffer b at 128 + b * 64
+  static constexpr int DV_COL = 256;
+  static constexpr int DK_COL = 384;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32acc(128, BQ, false, false);
+  static constexpr uint32_t IDESC_DV = ptx::idesc_bf16_f32acc(128, D, false, true);
+  static constexpr uint32_t IDESC_DK = ptx::idesc_bf16_f32acc(128, D, false, true);
+  static constexpr uint32_t IDESC_DQ = ptx::idesc_bf16_f32acc(128, BQ, true, true);
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(OFF_DS % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_DO % 1024 == 0, "1 KB aligned tiles");
+};
+
+// Row pass before the pair kernel, one warp per (batch, query head, row) of
+// the 64-padded query range: drow = rowsum(dO * O) (fp32 accumulation of the
+// bf16 operands), nl2 = -lse * log2(e) (-inf where the forward kept no key,
+// so that P = 0 there, and on padding rows), and the fp32 dQ row cleared for
+// the pair kernel's additions.
+__global__ void __launch_bounds__(256)
+    blasst_bwd_rows_kernel(const __nv_bfloat16* __restrict__ o,
+                           const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
+                           float* __restrict__ nl2, float* __restrict__ drow,
+                           float* __restrict__ dq, long long n_rows, int Lq, int LqP) {
+  const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= n_rows) return;
+  const long long bh = r / LqP;
+  const int q = static_cast<int>(r % LqP);
+  if (q >= Lq) {
+    if (lane == 0) {
+      nl2[r] = -INFINITY;
+      drow[r] = 0.0f;
+    }
+    return;
+  }
+  const size_t row = static_cast<size_t>(bh) * Lq + q;
+  const uint2 ov = reinterpret_cast<const uint2*>(o + row * 128)[lane];
+  const uint2 dv = reinterpret_cast<const uint2*>(dout + row * 128)[lane];
+  const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+  const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+  float acc = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float2 a = __bfloat1622float2(o2[i]);
+    const float2 c = __bfloat1622float2(d2[i]);
+    acc = fmaf(a.x, c.x, acc);
+    acc = fmaf(a.y, c.y, acc);
+  }
+#pragma unroll
+  for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+  reinterpret_cast<float4*>(dq + row * 128)[lane] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  if (lane == 0) {
+    const float l = lse[row];
+    nl2[r] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
+    drow[r] = acc;
+  }
+}
+
+__device__ __forceinline__ void bwd_record_error(int* err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+// Which 64-key halves of the CTA's key block j the forward kept for query
+// tile t (64 rows) of head bh: bit h set = keys [128 j + 64 h, +64) kept.
+__device__ __forceinline__ uint32_t bwd_keep_bits(const BwdParams& p, int bh, int t, int j) {
+  if (p.causal && j * BwdCfg::BK > t * BwdCfg::BQ + (BwdCfg::BQ - 1) + p.off) return 0u;
+  if (!p.fmask) return 3u;
+  const int qf = (t * BwdCfg::BQ) / p.Brf;
+  const uint8_t* row = p.fmask + (static_cast<size_t>(bh) * p.nQf + qf) * p.nKf;
+  if (p.Bcf == BwdCfg::BK) return row[j] == 0 ? 3u : 0u;
+  uint32_t r = row[2 * j] == 0 ? 1u : 0u;
+  if (2 * j + 1 < p.nKf && row[2 * j + 1] == 0) r |= 2u;
+  return r;
+}
+
+__global__ void __launch_bounds__(320, 1)
+    blasst_bwd_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmDO,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const BwdParams p) {
+  using C = BwdCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = ptx::smem_u32(smem);
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = misc + 1;
+  volatile int* recw = reinterpret_cast<volatile int*>(smem + C::OFF_REC);
+  auto put_rec = [&](int s, int hq, int t, int keep, int end) {
+    recw[4 * s] = hq;
+    recw[4 * s + 1] = t;
+    recw[4 * s + 2] = keep;
+    recw[4 * s + 3] = end;
+  };
+  auto get_rec = [&](int s) -> int4 {
+    return make_int4(recw[4 * s], recw[4 * s + 1], recw[4 * s + 2], recw[4 * s + 3]);
+  };
+  auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: key block j of KV head (b, hk). Under a causal mask block
+  // 0 meets the most query tiles, so ascending j runs the longest CTAs first.
+  const int nbhk = p.B * p.Hkv;
+  const int j = static_cast<int>(blockIdx.x) / nbhk;
+  const int bhk = static_cast<int>(blockIdx.x) % nbhk;
+  const int b = bhk / p.Hkv;
+  const int hk = bhk % p.Hkv;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar(C::B_KV), 1);
+    for (int i = 0; i < C::NST; ++i) {
+      ptx::mbar_init(bar(C::B_QF + i), 1);
+      ptx::mbar_init(bar(C::B_QE + i), C::QE_COUNT);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(C::B_SF + i), 1);
+      ptx::mbar_init(bar(C::B_PR + i), 4);
+      ptx::mbar_init(bar(C::B_DPF + i), 1);
+      ptx::mbar_init(bar(C::B_DSR + i), 4);
+      ptx::mbar_init(bar(C::B_DSE + i), 1);
+      ptx::mbar_init(bar(C::B_DQF + i), 1);
+      ptx::mbar_init(bar(C::B_DQE + i), 4);
+    }
+    ptx::mbar_init(bar(C::B_ACC), 1);
+    ptx::mbar_init(bar(C::B_DRAIN), 1);
+    for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == C::WARP_MMA) {
+    ptx::tmem_alloc(ptx::smem_u32(const_cast<int*>(misc)), C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+
+  // every lane of the warp waits (the data behind the barrier is read by all)
+  auto warp_wait = [&](uint32_t bar_addr, uint32_t parity) -> bool {
+    const bool ok = ptx::mbar_wait(bar_addr, parity, abort_flag, p.timeout_ns);
+    return __all_sync(0xffffffffu, ok) != 0;
+  };
+  auto fail = [&]() {
+    *abort_flag = 1;
+    bwd_record_error(p.err, BLASST_ETIMEOUT);
+  };
+
+  if (warp == C::WARP_LOAD) {
+    // ======================= producer ====================================
+    bool ok = true;
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmQ);
+      ptx::prefetch_tmap(&tmDO);
+      ptx::prefetch_tmap(&tmK);
+      ptx::prefetch_tmap(&tmV);
+      ptx::mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_BYTES);
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx) {
+        ptx::tma_load_3d(sb + C::OFF_K + bx * C::KV_BOX, &tmK, bx * 64, j * C::BK, bhk, bar(C::B_KV));
+        ptx::tma_load_3d(sb + C::OFF_V + bx * C::KV_BOX, &tmV, bx * 64, j * C::BK, bhk, bar(C::B_KV));
+      }
+    }
+    // first query tile that can see block j
+    int t_lo = 0;
+    if (p.causal) {
+      const int num = j * C::BK - p.off - (C::BQ - 1);
+      t_lo = num <= 0 ? 0 : (num + C::BQ - 1) / C::BQ;
+    }
+    int i = 0;  // pairs issued
+    for (int hh = 0; hh < p.g && ok; ++hh) {
+      const int hq = hk * p.g + hh;
+      const int bh = b * p.Hq + hq;
+      for (int t0 = t_lo; t0 < p.nT && ok; t0 += 32) {
+        const int t = t0 + lane;
+        const uint32_t km = t < p.nT ? bwd_keep_bits(p, bh, t, j) : 0u;
+        uint32_t bal = __ballot_sync(0xffffffffu, km != 0u);
+        while (bal != 0u) {
+          const int l = __ffs(bal) - 1;
+          bal &= bal - 1u;
+          const int tt = t0 + l;
+          const uint32_t kmv = __shfl_sync(0xffffffffu, km, l);
+          bool okl = true;
+          if (lane == 0) {
+            const int s = i % C::NST;
+            if (i >= C::NST)
+              okl = ptx::mbar_wait(bar(C::B_QE + s), ((i / C::NST) - 1) & 1, abort_flag,
+                                   p.timeout_ns);
+            if (okl) {
+              put_rec(s, hq, tt, static_cast<int>(kmv), 0);
+              const uint32_t fb = bar(C::B_QF + s);
+              ptx::mbar_arrive_expect_tx(fb, 2 * C::Q_BYTES + C::ROWST_BYTES);
+#pragma unroll
+              for (int bx = 0; bx < 2; ++bx) {
+                ptx::tma_load_3d(sb + C::OFF_Q + s * C::Q_BYTES + bx * C::Q_BOX, &tmQ, bx * 64,
+                                 tt * C::BQ, bh, fb);
+                ptx::tma_load_3d(sb + C::OFF_DO + s * C::Q_BYTES + bx * C::Q_BOX, &tmDO, bx * 64,
+                                 tt * C::BQ, bh, fb);
+              }
+              const size_t ro = static_cast<size_t>(bh) * p.LqP + static_cast<size_t>(tt) * C::BQ;
+              const uint32_t rs = sb + C::OFF_RS + s * C::ROWST_BYTES;
+              ptx::bulk_load(rs, p.nl2 + ro, C::BQ * 4, fb);
+              ptx::bulk_load(rs + C::BQ * 4, p.drow + ro, C::BQ * 4, fb);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, okl ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          ++i;
+        }
+      }
+    }
+    if (lane == 0) {
+      if (ok) {
+        // end record: every consumer stops at pair index i
+        const int s = i % C::NST;
+        if (i >= C::NST)
+          ok = ptx::mbar_wait(bar(C::B_QE + s), ((i / C::NST) - 1) & 1, abort_flag, p.timeout_ns);
+        if (ok) {
+          put_rec(s, -1, 0, 0, 1);
+          ptx::mbar_arrive(bar(C::B_QF + s));
+        }
+      }
+      if (!ok) {
+        fail();
+        // let the copies already in flight land before the CTA exits
+        for (int k = i - C::NST < 0 ? 0 : i - C::NST; k < i; ++k)
+          ptx::mbar_wait(bar(C::B_QF + k % C::NST), (k / C::NST) & 1, &misc[3], p.timeout_ns);
+        ptx::mbar_wait(bar(C::B_KV), 0, &misc[3], p.timeout_ns);
+      }
+    }
+  } else if (warp == C::WARP_MMA) {
+    // ======================= tcgen05 issuer ==============================
+    if (lane == 0) {
+      bool ok = ptx::mbar_wait(bar(C::B_KV), 0, abort_flag, p.timeout_ns);
+      ptx::tc_fence_after();
+      // descriptors (k-steps add 16-byte units to the start-address field)
+      const uint64_t dK_kmaj = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
+      const uint64_t dV_kmaj = ptx::sw128_desc(sb + C::OFF_V, 16, 1024);
+      const uint64_t dK_mn = ptx::sw128_desc(sb + C::OFF_K, C::KV_BOX, 1024);
+      const uint64_t dQ_kmaj = ptx::sw128_desc(sb + C::OFF_Q, 16, 1024);
+      const uint64_t dDO_kmaj = ptx::sw128_desc(sb + C::OFF_DO, 16, 1024);
+      const uint64_t dQ_mn = ptx::sw128_desc(sb + C::OFF_Q, C::Q_BOX, 1024);
+      const uint64_t dDO_mn = ptx::sw128_desc(sb + C::OFF_DO, C::Q_BOX, 1024);
+      const uint64_t dDS_kmaj = ptx::sw128_desc(sb + C::OFF_DS, 16, 1024);
+      const uint64_t dDS_mn = ptx::sw128_desc(sb + C::OFF_DS, C::DS_BYTES, 1024);
+      constexpr uint64_t QST = C::Q_BYTES >> 4;   // stage stride, 16-byte units
+      constexpr uint64_t DSB = C::DS_BYTES >> 4;  // dS buffer stride
+      int n = 0x7fffffff;  // pairs; known once the end record is seen
+
+      // 1: pair ready, 0: end record, -1: the wait gave up
+      auto stage_ready = [&](int i) -> int {
+        const int s = i % C::NST;
+        if (!ptx::mbar_wait(bar(C::B_QF + s), (i / C::NST) & 1, abort_flag, p.timeout_ns))
+          return -1;
+        return recw[4 * s + 3] != 0 ? 0 : 1;
+      };
+      // S^T = K Q^T and dP^T = V dO^T: M = 128 keys, N = 64 rows, K = 128 dims
+      auto issue_s = [&](int i) {
+        const uint64_t st = static_cast<uint64_t>(i % C::NST) * QST;
+        const uint32_t d_tm = tmem + C::S_COL + (i & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = dK_kmaj + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
+          const uint64_t bq = dQ_kmaj + st + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
+          ptx::mma_ss(d_tm, a, bq, C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar(C::B_SF + (i & 1)));
+      };
+      auto issue_dp = [&](int i) {
+        const uint64_t st = static_cast<uint64_t>(i % C::NST) * QST;
+        const uint32_t d_tm = tmem + C::DP_COL + (i & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = dV_kmaj + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
+          const uint64_t bo = dDO_kmaj + st + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
+          ptx::mma_ss(d_tm, a, bo, C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar(C::B_DPF + (i & 1)));
+      };
+
+      if (ok) {
+        const int r0 = stage_ready(0);
+        if (r0 < 0) ok = false;
+        else if (r0 == 0) n = 0;
+        else {
+          ptx::tc_fence_after();
+          issue_s(0);
+          issue_dp(0);
+          const int r1 = stage_ready(1);
+          if (r1 < 0) ok = false;
+          else if (r1 == 0) n = 1;
+          else {
+            ptx::tc_fence_after();
+            issue_s(1);
+          }
+        }
+      }
+      for (int i = 0; ok && i < n; ++i) {
+        const int bs = i & 1;
+        const uint64_t st = static_cast<uint64_t>(i % C::NST) * QST;
+        // dV += P^T dO: M = 128 keys, N = 128 dims, K = 64 rows (P^T from TMEM)
+        if (!ptx::mbar_wait(bar(C::B_PR + bs), (i >> 1) & 1, abort_flag, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t p_tm = tmem + C::S_COL + bs * 64;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::mma_ts(tmem + C::DV_COL, p_tm + kk * 8,
+                      dDO_mn + st + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DV,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+        // dP^T of the next pair, once the dQ^T that shares its buffer is drained
+        if (i + 1 < n) {
+          if (i >= 1 && !ptx::mbar_wait(bar(C::B_DQE + ((i + 1) & 1)), ((i - 1) >> 1) & 1,
+                                        abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          issue_dp(i + 1);
+        }
+        // dK += dS^T Q (M = 128 keys, N = 128 dims, K = 64 rows) and
+        // dQ^T = K^T dS^T (M = 128 dims, N = 64 rows, K = 128 keys)
+        if (!ptx::mbar_wait(bar(C::B_DSR + bs), (i >> 1) & 1, abort_flag, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint64_t dsk = dDS_kmaj + static_cast<uint64_t>(bs) * DSB;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::mma_ss(tmem + C::DK_COL, dsk + static_cast<uint64_t>((kk * 32) >> 4),
+                      dQ_mn + st + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DK,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t dsm = dDS_mn + static_cast<uint64_t>(bs) * DSB;
+        const uint32_t dq_tm = tmem + C::DP_COL + bs * 64;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::mma_ss(dq_tm, dK_mn + static_cast<uint64_t>((kk * 2048) >> 4),
+                      dsm + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DQ,
+                      kk > 0 ? 1u : 0u);
+        ptx::mma_commit(bar(C::B_DQF + bs));
+        ptx::mma_commit(bar(C::B_QE + i % C::NST));
+        ptx::mma_commit(bar(C::B_DSE + bs));
+        // S^T two pairs ahead (its buffer's P^T was read by the dV above)
+        if (i + 2 < n) {
+          const int r = stage_ready(i + 2);
+          if (r < 0) {
+            ok = false;
+            break;
+          }
+          if (r == 0) {
+            n = i + 2;
+          } else {
+            ptx::tc_fence_after();
+            issue_s(i + 2);
+          }
+        }
+      }
+      ptx::mma_commit(bar(C::B_ACC));
+      if (!ok) fail();
+      // drain: every MMA issued above has completed before TMEM is freed
+      // (bounded, not cut short by the abort flag)
+      ptx::mma_commit(bar(C::B_DRAIN));
+      ptx::mbar_wait(bar(C::B_DRAIN), 0, &misc[3], p.timeout_ns);
+    }
+  } else if (warp < 4) {
+    // ======================= compute: P^T, dS^T, then dV ===================
+    const int kl = warp * 32 + lane;  // key row of the block (TMEM lane)
+    const int kg = j * C::BK + kl;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const bool key_ok = kg < p.Lkv;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    int npairs = 0;
+    for (int i = 0;; ++i) {
+      const int s = i % C::NST;
+      const int bs = i & 1;
+      ok = warp_wait(bar(C::B_QF + s), (i / C::NST) & 1);
+      if (!ok) break;
+      const int4 rc = get_rec(s);
+      if (rc.w != 0) break;
+      ok = warp_wait(bar(C::B_SF + bs), (i >> 1) & 1);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      // column c (query row 64 t + c) is kept for this key iff c >= lim
+      int lim;
+      if (!key_ok || ((static_cast<uint32_t>(rc.z) >> (kl >> 6)) & 1u) == 0u) lim = C::BQ;
+      else if (p.causal) lim = kg - p.off - rc.y * C::BQ;
+      else lim = 0;
+      const float* rs = reinterpret_cast<const float*>(smem + C::OFF_RS + s * C::ROWST_BYTES);
+      float pv[64];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tmem + lane_base + C::S_COL + bs * 64 + 32 * h, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 nl = reinterpret_cast<const float4*>(rs)[8 * h + c4];
+          const float nla[4] = {nl.x, nl.y, nl.z, nl.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = 32 * h + 4 * c4 + u;
+            const float x = fmaf(__uint_as_float(r[4 * c4 + u]), sl2, nla[u]);
+            pv[c] = (c >= lim) ? ptx::ex2(x) : 0.0f;
+          }
+        }
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = ptx::pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+        ptx::tmem_st32(tmem + lane_base + C::S_COL + bs * 64, pk);
+        ptx::tmem_wait_st();
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::B_PR + bs));
+
+      ok = warp_wait(bar(C::B_DPF + bs), (i >> 1) & 1);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (i >= 2) {
+        ok = warp_wait(bar(C::B_DSE + bs), ((i - 2) >> 1) & 1);
+        if (!ok) break;
+      }
+      uint8_t* dsrow = smem + C::OFF_DS + bs * C::DS_BYTES + kl * 128;
+      const float* dr = rs + C::BQ;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tmem + lane_base + C::DP_COL + bs * 64 + 32 * h, r);
+        ptx::tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 dd = reinterpret_cast<const float4*>(dr)[8 * h + c4];
+          const int c = 32 * h + 4 * c4;
+          const float d0 = pv[c] * (__uint_as_float(r[4 * c4]) - dd.x);
+          const float d1 = pv[c + 1] * (__uint_as_float(r[4 * c4 + 1]) - dd.y);
+          const float d2 = pv[c + 2] * (__uint_as_float(r[4 * c4 + 2]) - dd.z);
+          const float d3 = pv[c + 3] * (__uint_as_float(r[4 * c4 + 3]) - dd.w);
+          w[2 * c4] = ptx::pack_bf16x2(d0, d1);
+          w[2 * c4 + 1] = ptx::pack_bf16x2(d2, d3);
+        }
+        // row kl of the 128-byte-swizzled tile: 16-byte chunk c8 at c8 ^ (kl % 8)
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int c8 = 4 * h + ch;
+          *reinterpret_cast<uint4*>(dsrow + ((c8 ^ (kl & 7)) << 4)) =
+              make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::B_DSR + bs));
+      ++npairs;
+    }
+    if (!ok) fail();
+    // ---- dV epilogue: row kl of dV = TMEM lane kl, 128 fp32 columns
+    if (ok) ok = warp_wait(bar(C::B_ACC), 0);
+    ptx::tc_fence_after();
+    if (ok && *abort_flag == 0) {
+      float* dst = p.dv + (static_cast<size_t>(bhk) * p.Lkv + (key_ok ? kg : 0)) * C::D;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        if (npairs > 0) {
+          ptx::tmem_ld32(tmem + lane_base + C::DV_COL + 32 * c, r);
+          ptx::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) r[u] = 0u;
+        }
+        if (key_ok) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            reinterpret_cast<uint4*>(dst + 32 * c)[u] =
+                make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+        }
+      }
+    }
+  } else {
+    // ======================= dQ writers (warps 4-7), then dK ==============
+    const int qd = warp - 4;
+    const int x = qd * 32 + lane;  // head dim of dQ^T (TMEM lane)
+    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+    const float scale = p.scale;
+    bool ok = true;
+    int npairs = 0;
+    for (int i = 0;; ++i) {
+      const int s = i % C::NST;
+      const int bs = i & 1;
+      ok = warp_wait(bar(C::B_QF + s), (i / C::NST) & 1);
+      if (!ok) break;
+      const int4 rc = get_rec(s);
+      if (rc.w != 0) break;
+      ok = warp_wait(bar(C::B_DQF + bs), (i >> 1) & 1);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      uint32_t r0[32], r1[32];
+      ptx::tmem_ld32(tmem + lane_base + C::DP_COL + bs * 64, r0);
+      ptx::tmem_ld32(tmem + lane_base + C::DP_COL + bs * 64 + 32, r1);
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(bar(C::B_DQE + bs));
+        ptx::mbar_arrive(bar(C::B_QE + s));
+      }
+      const int q0 = rc.y * C::BQ;
+      const int nrows = min(C::BQ, p.Lq - q0);
+      float* base = p.dq + (static_cast<size_t>(b * p.Hq + rc.x) * p.Lq + q0) * C::D + x;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (c < nrows) atomicAdd(base + static_cast<size_t>(c) * C::D, __uint_as_float(r0[c]) * scale);
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (32 + c < nrows)
+          atomicAdd(base + static_cast<size_t>(32 + c) * C::D, __uint_as_float(r1[c]) * scale);
+      ++npairs;
+    }
+    if (!ok) fail();
+    // ---- dK epilogue: row (32 qd + lane) of dK = TMEM lane, scaled
+    const int kl = qd * 32 + lane;
+    const int kg = j * C::BK + kl;
+    const bool key_ok = kg < p.Lkv;
+    if (ok) ok = warp_wait(bar(C::B_ACC), 0);
+    ptx::tc_fence_after();
+    if (ok && *abort_flag == 0) {
+      float* dst = p.dk + (static_cast<size_t>(bhk) * p.Lkv + (key_ok ? kg : 0)) * C::D;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        if (npairs > 0) {
+          ptx::tmem_ld32(tmem + lane_base + C::DK_COL + 32 * c, r);
+          ptx::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) r[u] = 0u;
+        }
+        if (key_ok) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            reinterpret_cast<float4*>(dst + 32 * c)[u] =
+                make_float4(__uint_as_float(r[4 * u]) * scale, __uint_as_float(r[4 * u + 1]) * scale,
+                            __uint_as_float(r[4 * u + 2]) * scale, __uint_as_float(r[4 * u + 3]) * scale);
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == C::WARP_MMA) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace blasst

@@ -259,6 +259,16 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t ab_format, int M, i
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// kind::f16 with bf16 A and B, fp32 accumulation, either operand stored
+// K-contiguous (false) or M/N-contiguous (true; a_major at bit 15, b_major
+// at bit 16). An A operand read from TMEM is always K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32acc(int M, int N, bool a_mn_major,
+                                                         bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // ------------------------------------------------------------------- math
 // Three-input max (sm_100 form of max.f32).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

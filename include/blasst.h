@@ -130,6 +130,56 @@ typedef struct blasst_fwd_args {
 } blasst_fwd_args;
 BLASST_API int blasst_fwd_ex(const blasst_fwd_args* args);
 
+/* Backward pass of the prefill with the forward's skip decisions held fixed.
+ * The decisions are a step function of the scores, so the gradient is that
+ * of softmax attention restricted to the (row, key) pairs the forward kept
+ * (a dropped block adds nothing to O: "BLASST: Dynamic BLocked Attention
+ * Sparsity via Softmax Thresholding", paragraph 5 after the headline, the
+ * skip rule). With P = exp(scale q.k - lse) on kept pairs (0 elsewhere),
+ * Dr = rowsum(dO * O) and dS = P * (dO.v - Dr):
+ *     dq = scale dS K,   dk = scale dS^T Q,   dv = P^T dO,
+ * dk and dv summed over the query heads of each GQA group. The pages give no
+ * backward pass; this is the reading the forward's definition fixes.
+ *   q, o, dout [B, Hq, Lq, d] bf16; k, v [B, Hkv, Lkv, d] bf16; lse [B, Hq, Lq]
+ *              fp32 (natural log), the forward's outputs for these inputs.
+ *   dq         [B, Hq, Lq, d] fp32, overwritten.
+ *   dk, dv     [B, Hkv, Lkv, d] fp32, overwritten.
+ *   causal     as in the forward (bottom-right aligned; Lq <= Lkv).
+ *   Br, Bc     the forward's tile sizes (64 or 128): skip_mask is read per
+ *              (Br-row tile, Bc-key block).
+ *   skip_mask  the forward's skip_mask_out, uint8 [B, Hq, ceil(Lq/Br),
+ *              ceil(Lkv/Bc)]: only pairs with entry 0 take part. NULL: every
+ *              causally visible pair does (a forward with lambda = 0 and no
+ *              static mask).
+ *   scale      score scale; <= 0 selects 1/sqrt(d).
+ *   workspace  device buffer of at least blasst_bwd_workspace_bytes(B, Hq, Lq)
+ *              bytes, 16-byte aligned (per-row statistics).
+ * d must be 128 (else BLASST_EUNSUPPORTED). Rows whose lse is -inf (no key
+ * kept) get dq = 0 and add nothing to dk, dv. */
+typedef struct blasst_bwd_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;
+  float* dq;
+  float* dk;
+  float* dv;
+  int B, Hq, Hkv, Lq, Lkv, d;
+  int causal;
+  int Br, Bc;
+  const uint8_t* skip_mask;
+  float scale;
+  void* workspace;
+  size_t workspace_bytes;
+  void* stream;
+} blasst_bwd_args;
+BLASST_API int blasst_bwd(const blasst_bwd_args* args);
+
+/* Bytes of workspace blasst_bwd needs: two fp32 [B, Hq, ceil(Lq/64)*64]. */
+BLASST_API size_t blasst_bwd_workspace_bytes(int B, int Hq, int Lq);
+
 /* Bytes of caller workspace that blasst_decode needs: fp32 partial outputs
  * [B, Hq, num_splits, d] plus fp32 partial lse [B, Hq, num_splits]. */
 BLASST_API size_t blasst_decode_workspace_bytes(int B, int Hq, int d, int num_splits);

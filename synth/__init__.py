@@ -42,6 +42,7 @@ _lib = None
 
 # stream ids of the counter-based generator
 STREAM_Q, STREAM_K, STREAM_V, STREAM_U, STREAM_W, STREAM_BLOCKS = 1, 2, 3, 4, 5, 6
+STREAM_DO = 7
 
 
 def build(force: bool = False) -> str:
@@ -262,6 +263,24 @@ def generate(w: Workload, out_q=None, out_k=None, out_v=None, nthreads: int = 0)
     _fill(w, w.Hkv, w.Lkv, STREAM_K, amp_k, u, wd, w.window_k_amp, 0, k, nthreads)
     _fill(w, w.Hkv, w.Lkv, STREAM_V, None, None, None, 0.0, 0, v, nthreads)
     return Inputs(w, q, k, v, u, planted)
+
+
+def grad_output(w: Workload, out=None) -> np.ndarray:
+    """dL/dO for the backward pass: i.i.d. N(0, 1) entries of shape
+    [B, Hq, Lq, d] (the gradient of a random linear loss), as bf16 bit
+    patterns (round to nearest even) or float32, like ``generate``."""
+    shp = (w.B, w.Hq, w.Lq, w.d)
+    x = normals(w.seed, STREAM_DO, 0, int(np.prod(shp))).astype(np.float32).reshape(shp)
+    if w.dtype == "fp32":
+        res = x
+    else:
+        bits = x.view(np.uint32)
+        res = ((bits + np.uint32(0x7FFF) + ((bits >> np.uint32(16)) & np.uint32(1)))
+               >> np.uint32(16)).astype(np.uint16)
+    if out is None:
+        return res
+    out[...] = res
+    return out
 
 
 def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:

@@ -75,6 +75,44 @@ def test_fwd_rejects_bad_arguments_without_a_gpu(lib, bad, code):
     assert _fwd(lib, **bad) == code
 
 
+def _bwd(lib, **kw):
+    import dynamic_block_sparse_tiled_b200 as bl
+    base = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, dout=0x50000, lse=0x60000,
+                dq=0x70000, dk=0x80000, dv=0x90000, B=1, Hq=4, Hkv=2, Lq=256, Lkv=256, d=128,
+                causal=1, Br=128, Bc=128, skip_mask=None, scale=0.0, workspace=0xA0000,
+                workspace_bytes=1 << 20, stream=None)
+    base.update(kw)
+    args = bl._BwdArgs(*[base[f[0]] for f in bl._BwdArgs._fields_])
+    return lib.blasst_bwd(C.byref(args))
+
+
+def test_bwd_workspace_bytes(lib):
+    assert lib.blasst_bwd_workspace_bytes(2, 4, 100) == 2 * 2 * 4 * 128 * 4
+    assert lib.blasst_bwd_workspace_bytes(1, 32, 32768) == 2 * 32 * 32768 * 4
+    assert lib.blasst_bwd_workspace_bytes(0, 4, 100) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (None, -1),
+    (dict(dout=None), -1),
+    (dict(dq=0x70004), -1),         # misaligned
+    (dict(Hq=3, Hkv=2), -1),
+    (dict(Lq=0), -1),
+    (dict(d=64), -2),               # the backward is d = 128 only
+    (dict(Br=32), -2),
+    (dict(Bc=256), -2),
+    (dict(Lq=300, Lkv=256), -2),    # causal with Lq > Lkv
+    (dict(workspace=None), -5),
+    (dict(workspace_bytes=2 * 4 * 256 * 4 - 16), -5),
+    (dict(workspace=0xA0008), -5),  # misaligned workspace
+])
+def test_bwd_rejects_bad_arguments_without_a_gpu(lib, bad, code):
+    if bad is None:
+        assert lib.blasst_bwd(None) == code
+    else:
+        assert _bwd(lib, **bad) == code
+
+
 def test_decode_workspace_and_rejections(lib):
     ws = lib.blasst_decode_workspace_bytes(16, 32, 128, 64)
     assert ws == 16 * 32 * 64 * (128 + 1) * 4

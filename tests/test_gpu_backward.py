@@ -1,0 +1,162 @@
+"""GPU parity of the backward pass (blasst_bwd) against the fp64 oracle.
+
+The forward's decisions are held fixed. To give both sides the same decision
+set without feeding anything from the CUDA path into the oracle, the decisions
+come from the oracle's forward (its skip mask at the case's lambda, or a
+seeded static mask); the GPU forward then runs with lambda = 0 and those
+decisions as its static block mask, so its O and lse cover exactly the pairs
+the oracle kept, and the GPU backward reads the same mask. One case runs the
+GPU forward with the threshold itself and checks that its mask equals the
+oracle's before comparing gradients.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import parity
+import synth
+
+BASE = synth.CONFIGS["prefill_32k"]
+
+
+def _lib():
+    from dynamic_block_sparse_tiled_b200 import build
+    build.build()
+    import dynamic_block_sparse_tiled_b200 as bl
+    return bl
+
+
+def _static_mask(w, seed, p_excl, empty_tiles=()):
+    """Seeded static mask: each (tile, block) pair excluded with probability
+    p_excl; the listed (b, hq, qt) tiles lose every block."""
+    nQt, nKt = -(-w.Lq // w.Br), -(-w.Lkv // w.Bc)
+    r = synth.draws_u64(seed, 11, 0, w.B * w.Hq * nQt * nKt).astype(np.float64) / 2.0 ** 64
+    m = (r < p_excl).astype(np.uint8).reshape(w.B, w.Hq, nQt, nKt)
+    for (b, hq, qt) in empty_tiles:
+        m[b, hq, qt, :] = 1
+    return m
+
+
+def _structural_zeros(w, fmask):
+    """Rows no kept pair reaches: query rows with no kept key (their dq is
+    exactly 0) and keys that no query row of their GQA group keeps (their dk
+    and dv are exactly 0). Returns bool [B, Hq, Lq], bool [B, Hkv, Lkv]."""
+    B, Hq, Hkv, Lq, Lkv, Br, Bc = w.B, w.Hq, w.Hkv, w.Lq, w.Lkv, w.Br, w.Bc
+    nQt, nKt = -(-Lq // Br), -(-Lkv // Bc)
+    keep_t = np.ones((B, Hq, nQt, nKt), bool) if fmask is None else (fmask == 0)
+    off = Lkv - Lq
+    rows = np.arange(Lq)
+    keys = np.arange(Lkv)
+    q_zero = np.ones((B, Hq, Lq), bool)
+    k_zero = np.ones((B, Hkv, Lkv), bool)
+    for b in range(B):
+        for hq in range(Hq):
+            kt_of_key = keys // Bc
+            for qt in range(nQt):
+                r = rows[qt * Br:(qt + 1) * Br]
+                kept_blocks = keep_t[b, hq, qt]
+                vis = kept_blocks[kt_of_key][None, :] & (
+                    (keys[None, :] <= r[:, None] + off) if w.causal else True)
+                q_zero[b, hq, r] &= ~vis.any(axis=1)
+                k_zero[b, hq // (Hq // Hkv)] &= ~vis.any(axis=0)
+    return q_zero, k_zero
+
+
+def run_bwd_case(w, lam, static=None, gpu_decisions=False):
+    import torch
+    bl = _lib()
+    inp = synth.generate(w)
+    dout = synth.grad_output(w)
+    q, k, v, do = (parity.to_device(a) for a in (inp.q, inp.k, inp.v, dout))
+    if lam > 0 or static is not None:
+        ref_f = oracle.prefill(inp.q, inp.k, inp.v, causal=w.causal, lam=float(np.float32(lam)),
+                               Br=w.Br, Bc=w.Bc, static_mask=static)
+        _, _, fmask, _ = oracle.prefill_dense(ref_f)
+        fmask = np.ascontiguousarray(fmask)
+    else:
+        fmask = None
+    if gpu_decisions:
+        o, lse, gmask = bl.attention_prefill(q, k, v, causal=w.causal, lam=float(np.float32(lam)),
+                                             Br=w.Br, Bc=w.Bc, with_mask=True)
+        assert np.array_equal(gmask.cpu().numpy(), fmask), "GPU and oracle decisions differ"
+        mask_dev = gmask
+    else:
+        excl = None if fmask is None else torch.from_numpy((fmask != 0).astype(np.uint8)).cuda()
+        o, lse, _ = bl.attention_prefill(q, k, v, causal=w.causal, lam=0.0, Br=w.Br, Bc=w.Bc,
+                                         block_mask=excl)
+        mask_dev = None if fmask is None else torch.from_numpy(fmask).cuda()
+    dq, dk, dv = bl.attention_backward(q, k, v, o, lse, do, causal=w.causal, Br=w.Br, Bc=w.Bc,
+                                       skip_mask=mask_dev)
+    assert bl.blasst_check() == 0
+    rq, rk, rv = oracle.backward(inp.q, inp.k, inp.v, dout, causal=w.causal, Br=w.Br, Bc=w.Bc,
+                                 tile_mask=fmask)
+    gq, gk, gv = (t.cpu().numpy().astype(np.float64) for t in (dq, dk, dv))
+    q_zero, k_zero = _structural_zeros(w, fmask)
+    errs = {}
+    for name, g, r, z in (("dq", gq, rq, q_zero), ("dk", gk, rk, k_zero), ("dv", gv, rv, k_zero)):
+        assert np.all(np.isfinite(g)), f"{w.name} {name} not finite"
+        errs[name] = parity.assert_grad_within(g, r, f"{w.name} {name}")
+        # rows that no kept pair reaches are exact zeros on both sides
+        assert np.all(r[z] == 0.0)
+        assert np.all(g[z] == 0.0), f"{w.name} {name}: nonzero rows that no kept pair reaches"
+    print(w.name, {k: {m: f"{x:.2e}" for m, x in e.items()} for k, e in errs.items()},
+          "empty rows", int(q_zero.sum()), "unreached keys", int(k_zero.sum()))
+    return errs
+
+
+CASES = [
+    # name, overrides, lambda, static-mask spec
+    ("dense_gqa_1k", dict(Hq=4, Hkv=2, Lq=1024, Lkv=1024, window=256, n_needles=2), 0.0, None),
+    ("a12_gqa_2k_lam", dict(Hq=4, Hkv=2, Lq=2048, Lkv=2048, amp=12.0, window=256, n_needles=2),
+     1e-3, None),
+    ("ragged_1000_br64_bc64", dict(Hq=2, Hkv=1, Lq=1000, Lkv=1000, Br=64, Bc=64, amp=12.0,
+                                   window=256, n_needles=2), 1e-2, None),
+    ("br64_bc128", dict(Hq=2, Hkv=2, Lq=1024, Lkv=1024, Br=64, amp=12.0, window=256, n_needles=2),
+     1e-3, None),
+    ("br128_bc64", dict(Hq=2, Hkv=2, Lq=1024, Lkv=1024, Bc=64, amp=12.0, window=256, n_needles=2),
+     1e-3, None),
+    ("noncausal_512x900", dict(Hq=2, Hkv=2, Lq=512, Lkv=900, causal=False, amp=12.0, window=256,
+                               n_needles=2), 1e-3, None),
+    ("causal_300x1000", dict(Hq=2, Hkv=1, Lq=300, Lkv=1000, amp=12.0, window=256, n_needles=2),
+     1e-3, None),
+    ("g8_512", dict(Hq=8, Hkv=1, Lq=512, Lkv=512, amp=12.0, window=128, n_needles=2), 1e-3, None),
+    ("static_with_empty_rows", dict(Hq=2, Hkv=2, Lq=768, Lkv=768, amp=12.0, window=256,
+                                    n_needles=2), 1e-3, (5, 0.3, ((0, 1, 2), (0, 0, 5)))),
+    ("all_excluded", dict(Hq=2, Hkv=1, Lq=384, Lkv=384), 0.0, (6, 1.1, ())),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,over,lam,spec", CASES, ids=[c[0] for c in CASES])
+def test_backward_matches_oracle(name, over, lam, spec):
+    w = BASE.replace(name=name, **over)
+    static = None
+    if spec is not None:
+        seed, p_excl, empty = spec
+        static = _static_mask(w, seed, p_excl, empty)
+    run_bwd_case(w, lam, static=static)
+
+
+@pytest.mark.gpu
+def test_backward_with_the_gpu_forward_decisions():
+    """End to end as a caller runs it: the GPU forward's own skip mask feeds
+    the GPU backward (the seeded case has no decision in the tie band)."""
+    w = BASE.replace(name="e2e_gqa_1k", Hq=4, Hkv=2, Lq=1024, Lkv=1024, amp=12.0, window=256,
+                     n_needles=2)
+    run_bwd_case(w, 1e-3, gpu_decisions=True)
+
+
+@pytest.mark.gpu
+def test_backward_all_excluded_gives_zeros():
+    import torch
+    bl = _lib()
+    w = BASE.replace(name="zeros", Hq=2, Hkv=1, Lq=256, Lkv=256)
+    inp = synth.generate(w)
+    q, k, v = (parity.to_device(a) for a in (inp.q, inp.k, inp.v))
+    do = parity.to_device(synth.grad_output(w))
+    mask = torch.ones((1, 2, 2, 2), dtype=torch.uint8, device="cuda")
+    o, lse, _ = bl.attention_prefill(q, k, v, causal=True, block_mask=mask)
+    dq, dk, dv = bl.attention_backward(q, k, v, o, lse, do, causal=True, skip_mask=mask)
+    assert bl.blasst_check() == 0
+    for t in (dq, dk, dv):
+        assert int(torch.count_nonzero(t)) == 0
