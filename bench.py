@@ -72,6 +72,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "prefill_32k": ("prefill_sm100.cuh", "ptx_sm100.cuh"),
     "decode_64k": ("decode_sm100.cuh", "ptx_sm100.cuh"),
+    "backward_32k": ("bwd_sm100.cuh", "ptx_sm100.cuh"),
 }
 
 
@@ -233,6 +234,78 @@ def measure_prefill(w, lam, steps, warmup, device, stream, flush_buf, pre=None, 
                      v_blocks=sd["v_blocks_loaded"], bytes_loaded=sd["bytes_loaded"])
 
 
+def backward_pairs(w, mask):
+    """(64-row query tile, 128-key block) pairs the backward computes, from
+    the forward's decisions (uint8 [B, Hq, nQt, nKt], 0 = computed)."""
+    nT = -(-w.Lq // 64)
+    nKb = -(-w.Lkv // 128)
+    t = np.arange(nT)
+    j = np.arange(nKb)
+    qf = (t * 64) // w.Br
+    keep = mask == 0                                      # [B, Hq, nQt, nKt]
+    if w.Bc == 128:
+        kb = keep[:, :, qf][:, :, :, j]
+    else:
+        k0 = keep[:, :, qf][:, :, :, 2 * j]
+        j1 = np.minimum(2 * j + 1, keep.shape[-1] - 1)
+        k1 = keep[:, :, qf][:, :, :, j1] & ((2 * j + 1) < keep.shape[-1])[None, None, None, :]
+        kb = k0 | k1
+    if w.causal:
+        vis = (j[None, :] * 128) <= (t[:, None] * 64 + 63 + (w.Lkv - w.Lq))
+        kb = kb & vis[None, None]
+    return int(kb.sum())
+
+
+BWD_FLOPS_PER_PAIR = 5 * 2 * 128 * 64 * 128  # S^T, dP^T, dV, dK, dQ^T products
+
+
+class Backward:
+    """Device-resident dO, gradients and workspace for the backward of a
+    prefill workload (the forward's outputs come from ``pre``)."""
+
+    def __init__(self, pre, device):
+        import torch
+        import synth
+        import dynamic_block_sparse_tiled_b200 as bl
+        w = pre.w
+        self.pre = pre
+        self.do = torch.from_numpy(synth.grad_output(w).view(np.int16)).view(torch.bfloat16).to(device)
+        self.dq = torch.empty((w.B, w.Hq, w.Lq, w.d), dtype=torch.float32, device=device)
+        self.dk = torch.empty((w.B, w.Hkv, w.Lkv, w.d), dtype=torch.float32, device=device)
+        self.dv = torch.empty_like(self.dk)
+        self.ws = torch.empty(bl.blasst_bwd_workspace_bytes(w.B, w.Hq, w.Lq), dtype=torch.uint8,
+                              device=device)
+
+    def run(self, stream=None):
+        import dynamic_block_sparse_tiled_b200 as bl
+        p, w = self.pre, self.pre.w
+        bl.blasst_bwd(p.q, p.k, p.v, p.o, self.do, p.lse, self.dq, self.dk, self.dv,
+                      causal=w.causal, Br=w.Br, Bc=w.Bc, workspace=self.ws, skip_mask=p.mask,
+                      stream=stream)
+
+
+def measure_backward(w, lam, steps, warmup, device, stream, flush_buf, pre=None, bwd=None):
+    """Forward once at ``lam`` (its O, lse and decisions), then time the
+    backward with those decisions."""
+    import dynamic_block_sparse_tiled_b200 as bl
+    pre = pre or Prefill(w, device)
+    pre.run(lam, stream=stream)
+    bwd = bwd or Backward(pre, device)
+    bwd.run(stream=stream)
+    stream.synchronize()
+    rc = bl.blasst_check(stream)
+    if rc != 0:
+        raise RuntimeError(bl.blasst_status_string(rc))
+    times = time_calls(lambda: bwd.run(stream=stream), steps, warmup, stream, flush_buf)
+    mask = pre.mask.cpu().numpy()
+    pairs = backward_pairs(w, mask)
+    ms = statistics.mean(times)
+    flops = pairs * BWD_FLOPS_PER_PAIR
+    return pre, bwd, dict(ms=ms, times=times, pairs=pairs, exec_flops=float(flops),
+                          executed_tflops=flops / (ms * 1e-3) / 1e12,
+                          skip_frac=float((mask == 1).sum()) / max(int((mask != 2).sum()), 1))
+
+
 def measure_decode(w, lam, steps, warmup, device, stream, flush_buf):
     import torch
     import dynamic_block_sparse_tiled_b200 as bl
@@ -378,6 +451,10 @@ def run_case(name, lam, calls, overrides=()):
     import torch
     import synth
     import dynamic_block_sparse_tiled_b200 as bl
+    ncalls = calls
+    backward = name.startswith("backward:")
+    if backward:
+        name = name.split(":", 1)[1]
     w = synth.CONFIGS[name]
     for ov in overrides:
         key, val = ov.split("=", 1)
@@ -390,6 +467,14 @@ def run_case(name, lam, calls, overrides=()):
         to = lambda a: torch.from_numpy(a).cuda()
     q, k, v = to(inp.q), to(inp.k), to(inp.v)
     del inp
+    if backward:
+        o, lse, mask = bl.attention_prefill(q, k, v, causal=w.causal, lam=lam, Br=w.Br, Bc=w.Bc,
+                                            with_mask=True)
+        do = torch.from_numpy(synth.grad_output(w).view(np.int16)).view(torch.bfloat16).cuda()
+        for _ in range(calls):
+            bl.attention_backward(q, k, v, o, lse, do, causal=w.causal, Br=w.Br, Bc=w.Bc,
+                                  skip_mask=mask)
+        calls = 0
     for _ in range(calls):
         if w.num_splits:
             bl.attention_decode(q, k, v, lam=lam, Bc=w.Bc, num_splits=w.num_splits)
@@ -397,7 +482,8 @@ def run_case(name, lam, calls, overrides=()):
             bl.attention_prefill(q, k, v, causal=w.causal, lam=lam, Br=w.Br, Bc=w.Bc)
     torch.cuda.synchronize()
     rc = bl.blasst_check()
-    print(json.dumps(dict(case=name, calls=calls, status=bl.blasst_status_string(rc))), flush=True)
+    print(json.dumps(dict(case=("backward:" if backward else "") + name, calls=ncalls,
+                          status=bl.blasst_status_string(rc))), flush=True)
     return 0 if rc == 0 else 1
 
 
@@ -447,7 +533,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip the 128K and decode legs")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--case", default=None,
-                    help="profiling driver: run only this workload's kernel --calls times, untimed")
+                    help="profiling driver: run only this workload's kernel --calls times, untimed "
+                         "(backward:<workload> runs one forward, then the backward --calls times)")
     ap.add_argument("--calls", type=int, default=4)
     ap.add_argument("--lam", type=float, default=LAMBDA)
     ap.add_argument("--override", action="append", default=[],
@@ -556,6 +643,33 @@ def main():
             executed_tflops=s_r["exec_flops"] / (s_r["ms"] * 1e-3) / 1e12)
         del ps, sm_dev
         torch.cuda.empty_cache()
+
+        # backward with the forward's decisions held fixed, 32K workload
+        pb = Prefill(w, device)
+        pb, bb, b_l = measure_backward(w, LAMBDA, max(3, args.steps // 2), 3, device, stream,
+                                       flush_buf, pre=pb)
+        del pb, bb
+        torch.cuda.empty_cache()
+        pb = Prefill(wa, device)
+        pb, bb, ba_l = measure_backward(wa, LAMBDA, max(3, args.steps // 2), 3, device, stream,
+                                        flush_buf, pre=pb)
+        _, _, ba_0 = measure_backward(wa, 0.0, max(3, args.steps // 2), 3, device, stream,
+                                      flush_buf, pre=pb, bwd=bb)
+        del pb, bb
+        torch.cuda.empty_cache()
+        extra["backward_32k"] = dict(
+            ms=b_l["ms"], pairs=b_l["pairs"], skip_frac=b_l["skip_frac"],
+            executed_tflops=b_l["executed_tflops"],
+            roofline=dict(bound="tensor", achieved=b_l["executed_tflops"],
+                          peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                          frac=b_l["executed_tflops"] / peaks["bf16_tflops"],
+                          traffic=profiled_traffic("backward_32k"),
+                          algorithmic="per computed (64-row tile, 128-key block) pair: 5 products "
+                                      "of 2*128*64*128 flops (S^T, dP^T, dV, dK, dQ^T)"),
+            a12=dict(ms=ba_l["ms"], ms_lambda0=ba_0["ms"], speedup_vs_lambda0=ba_0["ms"] / ba_l["ms"],
+                     skip_frac=ba_l["skip_frac"], executed_tflops=ba_l["executed_tflops"]),
+            note="dq, dk, dv in fp32; one call = the row pass (rowsum(dO*O), dq cleared) and the "
+                 "pair kernel")
 
         wd = synth.CONFIGS["decode_64k"]
         dres = measure_decode(wd, LAMBDA, max(5, args.steps), 3, device, stream, flush_buf)

@@ -95,6 +95,22 @@ bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int el
   return r == CUDA_SUCCESS;
 }
 
+// 3-D map over a dense fp32 [heads, L, d] tensor without swizzle, box
+// (32 columns, rows, 1): the target of TMA reduce-adds.
+bool make_map_f32_plain(CUtensorMap* map, void* base, int d, int L, int heads, int box_rows) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(d) * 4 * L};
+  cuuint32_t box[3] = {32, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
   const cudaError_t e =
@@ -375,9 +391,10 @@ int blasst_bwd(const blasst_bwd_args* a) {
   p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
   p.timeout_ns = kTimeoutNs;
 
-  CUtensorMap mq, mdo, mk, mv;
+  CUtensorMap mq, mdo, mk, mv, mdq;
   const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!make_map(&mq, a->q, dt, 2, a->d, a->Lq, a->B * a->Hq, 64) ||
+  if (!make_map_f32_plain(&mdq, a->dq, a->d, a->Lq, a->B * a->Hq, 64) ||
+      !make_map(&mq, a->q, dt, 2, a->d, a->Lq, a->B * a->Hq, 64) ||
       !make_map(&mdo, a->dout, dt, 2, a->d, a->Lq, a->B * a->Hq, 64) ||
       !make_map(&mk, a->k, dt, 2, a->d, a->Lkv, a->B * a->Hkv, 128) ||
       !make_map(&mv, a->v, dt, 2, a->d, a->Lkv, a->B * a->Hkv, 128))
@@ -391,7 +408,7 @@ int blasst_bwd(const blasst_bwd_args* a) {
   using C = blasst::BwdCfg;
   if (set_smem(blasst::blasst_bwd_kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
   const dim3 grid(static_cast<unsigned>(p.nKb) * p.B * p.Hkv);
-  blasst::blasst_bwd_kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(mq, mdo, mk, mv, p);
+  blasst::blasst_bwd_kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(mq, mdo, mk, mv, mdq, p);
   return cuda_status(cudaGetLastError());
 }
 

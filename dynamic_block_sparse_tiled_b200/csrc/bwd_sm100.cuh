@@ -27,18 +27,22 @@
 //   P^T (bf16) overwrites S^T in TMEM, dS^T (bf16) goes to shared memory;
 //   dV  += P^T dO         (TMEM accumulator)         bf16 TS
 //   dK  += dS^T Q         (TMEM accumulator)         bf16 SS
-//   dQ^T = K^T dS^T       (TMEM, lanes = head dims)  bf16 SS, then added to
-//                          the fp32 dQ in global memory with red.add, one
-//                          warp instruction per query row and 32 dims.
+//   dQ^T = K^T dS^T       (TMEM, lanes = head dims)  bf16 SS, then staged in
+//                          shared memory as a [64 rows][128 dims] fp32 tile
+//                          and added to the fp32 dQ in global memory by two
+//                          TMA reduce-adds (the add happens in L2).
 // Computing the transposed S and dP puts the keys on TMEM lanes, so P^T can
 // feed dV straight from TMEM and every product keeps M = 128; dQ^T keeps the
-// head dims on lanes so that each red.add of a warp covers 128 contiguous
-// bytes of one dQ row.
+// head dims on lanes, so a warp's store of one staged dQ row covers 32
+// consecutive dims (128 contiguous bytes, no bank conflicts). The staging
+// tile reuses the pair's Q and dO stage: both are dead once dQ^T is done
+// (every product that reads them was issued before it and the tensor core
+// completes them in order).
 //
 // Warp roles (320 threads):
 //   warps 0-3  compute: P^T and dS^T, then the dV epilogue;
-//   warps 4-7  dQ writers: drain dQ^T from TMEM and add it to global dQ,
-//              then the dK epilogue;
+//   warps 4-7  dQ writers: drain dQ^T from TMEM, stage it, add it to global
+//              dQ with TMA reduce-adds, then the dK epilogue;
 //   warp 8     producer: K and V once, then per pair Q, dO (TMA, 3-stage
 //              ring) and the pair's row statistics (bulk copies); builds the
 //              pair list by scanning the forward's decisions;
@@ -82,14 +86,15 @@ struct BwdCfg {
   static constexpr int D = 128;
   static constexpr int BK = 128;  // keys per CTA
   static constexpr int BQ = 64;   // query rows per pair
-  static constexpr int NTHREADS = 320;
-  static constexpr int WARP_LOAD = 8, WARP_MMA = 9;
-  static constexpr int NST = 3;  // Q / dO stages
+  static constexpr int NTHREADS = 352;
+  static constexpr int WARP_LOAD = 8, WARP_MMA = 9, WARP_SP = 10;
+  static constexpr int NST = 4;  // Q / dO stages
   static constexpr int KV_BOX = BK * 128;      // [128 keys][64 dims] bf16, 16 KB
   static constexpr int KV_BYTES = 2 * KV_BOX;  // 32 KB
   static constexpr int Q_BOX = BQ * 128;       // [64 rows][64 dims] bf16, 8 KB
   static constexpr int Q_BYTES = 2 * Q_BOX;    // 16 KB
   static constexpr int DS_BYTES = BK * 128;    // [128 keys][64 q] bf16, 16 KB
+  static constexpr int DQS_BYTES = BQ * 32 * 4;  // one warp's staged [64 rows][32 dims] fp32, 8 KB
   static constexpr int ROWST_BYTES = 2 * BQ * 4;  // nl2[64], drow[64]
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_BYTES;
@@ -97,28 +102,32 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + NST * Q_BYTES;
   static constexpr int OFF_DS = OFF_DO + NST * Q_BYTES;
   static constexpr int OFF_RS = OFF_DS + 2 * DS_BYTES;
-  static constexpr int OFF_REC = OFF_RS + NST * ROWST_BYTES;  // [NST] int4 {hq, t, keep bits, end}
+  static constexpr int OFF_REC = OFF_RS + NST * ROWST_BYTES;  // [NST] {hq, t, keep bits, end}
   static constexpr int OFF_BAR = OFF_REC + NST * 16;
   // barriers
   static constexpr int B_KV = 0;
   static constexpr int B_QF = 1;               // [NST] stage loaded (+ record)
-  static constexpr int B_QE = B_QF + NST;      // [NST] stage free: issuer commit + 4 writer warps
+  static constexpr int B_QE = B_QF + NST;      // [NST] stage free: issuer commit + the set's 4 dQ adds read
   static constexpr int B_SF = B_QE + NST;      // [2] S^T ready
-  static constexpr int B_PR = B_SF + 2;        // [2] P^T in TMEM (4 compute warps)
+  static constexpr int B_PR = B_SF + 2;        // [2] P^T in TMEM (4 warps of a compute set)
   static constexpr int B_DPF = B_PR + 2;       // [2] dP^T ready
-  static constexpr int B_DSR = B_DPF + 2;      // [2] dS^T in shared memory (4 compute warps)
+  static constexpr int B_DSR = B_DPF + 2;      // [2] dS^T in shared memory (4 warps of a set)
   static constexpr int B_DSE = B_DSR + 2;      // [2] dS^T buffer free (issuer commit)
   static constexpr int B_DQF = B_DSE + 2;      // [2] dQ^T ready
-  static constexpr int B_DQE = B_DQF + 2;      // [2] dQ^T drained (4 writer warps)
-  static constexpr int B_ACC = B_DQE + 2;      // dV, dK final
-  static constexpr int B_DRAIN = B_ACC + 1;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_DQE = B_DQF + 2;      // [2] dQ^T drained (4 warps of a set)
+  static constexpr int B_ZERO = B_DQE + 2;     // dV, dK accumulators cleared (8 compute warps)
+  static constexpr int B_SFREE = B_ZERO + 1;   // [2] dV of the buffer's pair done (P^T read)
+  static constexpr int B_ACC = B_SFREE + 2;    // dV, dK final
+  static constexpr int B_DRAIN = B_ACC + 1;    // [2] the two issuers' drains
+  static constexpr int NBAR = B_DRAIN + 2;
   static constexpr int QE_COUNT = 1 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // misc words: [0] tmem base, [1] abort, [3] always 0 (waits only a timeout
-  // ends), [4] pairs processed (issuer)
+  // misc words: [0] tmem base, [1] abort, [3] always 0 (waits only a timeout ends)
   static constexpr int MISC_BYTES = 64;
-  static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+  // no alignment slack: the kernel checks that the dynamic shared memory
+  // base is 1024-byte aligned (it is when the kernel has no static shared
+  // memory) and reports BLASST_EUNSUPPORTED otherwise
+  static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES;
   static constexpr int S_COL = 0;      // S^T buffer b at b * 64 (P^T: first 32 columns)
   static constexpr int DP_COL = 128;   // dP^T / dQ^T buffer b at 128 + b * 64
   static constexpr int DV_COL = 256;
@@ -194,16 +203,21 @@ __device__ __forceinline__ uint32_t bwd_keep_bits(const BwdParams& p, int bh, in
   return r;
 }
 
-__global__ void __launch_bounds__(320, 1)
+
+__global__ void __launch_bounds__(352, 1)
     blasst_bwd_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmDO,
                       const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const BwdParams p) {
+                      const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdCfg;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sb = ptx::smem_u32(smem);
+  if ((sb & 1023u) != 0u) {  // uniform over the CTA; nothing set up yet
+    if (threadIdx.x == 0) bwd_record_error(p.err, BLASST_EUNSUPPORTED);
+    return;
+  }
   volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* abort_flag = misc + 1;
   volatile int* recw = reinterpret_cast<volatile int*>(smem + C::OFF_REC);
@@ -244,8 +258,12 @@ __global__ void __launch_bounds__(320, 1)
       ptx::mbar_init(bar(C::B_DQF + i), 1);
       ptx::mbar_init(bar(C::B_DQE + i), 4);
     }
+    ptx::mbar_init(bar(C::B_ZERO), 8);
     ptx::mbar_init(bar(C::B_ACC), 1);
-    ptx::mbar_init(bar(C::B_DRAIN), 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(C::B_SFREE + i), 1);
+      ptx::mbar_init(bar(C::B_DRAIN + i), 1);
+    }
     for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
     ptx::fence_mbar_init();
   }
@@ -332,11 +350,13 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     if (lane == 0) {
-      if (ok) {
-        // end record: every consumer stops at pair index i
-        const int s = i % C::NST;
-        if (i >= C::NST)
-          ok = ptx::mbar_wait(bar(C::B_QE + s), ((i / C::NST) - 1) & 1, abort_flag, p.timeout_ns);
+      // two end records (pair indices i and i + 1): the issuer and the writers
+      // stop at the first, each compute set at the first of its parity
+      for (int e = 0; e < 2 && ok; ++e) {
+        const int ie = i + e;
+        const int s = ie % C::NST;
+        if (ie >= C::NST)
+          ok = ptx::mbar_wait(bar(C::B_QE + s), ((ie / C::NST) - 1) & 1, abort_flag, p.timeout_ns);
         if (ok) {
           put_rec(s, -1, 0, 0, 1);
           ptx::mbar_arrive(bar(C::B_QF + s));
@@ -350,10 +370,19 @@ __global__ void __launch_bounds__(320, 1)
         ptx::mbar_wait(bar(C::B_KV), 0, &misc[3], p.timeout_ns);
       }
     }
-  } else if (warp == C::WARP_MMA) {
-    // ======================= tcgen05 issuer ==============================
+  } else if (warp == C::WARP_SP || warp == C::WARP_MMA) {
+    // ======================= tcgen05 issuers =============================
+    // Two threads issue MMAs, each in its own order; what one reads of the
+    // other's results is ordered through the compute sets' barriers or an
+    // explicit commit:
+    //   warp 10: S^T(i) (into S buffer i%2 once dV(i-2) has read P^T(i-2))
+    //            and dP^T(i) (into dP buffer i%2 once dQ^T(i-2) is drained);
+    //   warp 9:  dV(i) (after P^T(i)), dK(i) and dQ^T(i) (after dS^T(i)).
+    //            S^T(i) and dP^T(i) are complete by then (the compute set has
+    //            read them), so the commit after dQ^T(i) also frees the stage.
     if (lane == 0) {
       bool ok = ptx::mbar_wait(bar(C::B_KV), 0, abort_flag, p.timeout_ns);
+      if (warp == C::WARP_MMA && ok) ok = ptx::mbar_wait(bar(C::B_ZERO), 0, abort_flag, p.timeout_ns);
       ptx::tc_fence_after();
       // descriptors (k-steps add 16-byte units to the start-address field)
       const uint64_t dK_kmaj = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
@@ -367,138 +396,135 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t dDS_mn = ptx::sw128_desc(sb + C::OFF_DS, C::DS_BYTES, 1024);
       constexpr uint64_t QST = C::Q_BYTES >> 4;   // stage stride, 16-byte units
       constexpr uint64_t DSB = C::DS_BYTES >> 4;  // dS buffer stride
-      int n = 0x7fffffff;  // pairs; known once the end record is seen
-
-      // 1: pair ready, 0: end record, -1: the wait gave up
+      // 1: pair ready, 0: end record, -1: the wait gave up. Neither issuer
+      // can fall a full stage cycle behind: a stage is reloaded only after
+      // warp 9's commit for its pair.
       auto stage_ready = [&](int i) -> int {
         const int s = i % C::NST;
         if (!ptx::mbar_wait(bar(C::B_QF + s), (i / C::NST) & 1, abort_flag, p.timeout_ns))
           return -1;
         return recw[4 * s + 3] != 0 ? 0 : 1;
       };
-      // S^T = K Q^T and dP^T = V dO^T: M = 128 keys, N = 64 rows, K = 128 dims
-      auto issue_s = [&](int i) {
-        const uint64_t st = static_cast<uint64_t>(i % C::NST) * QST;
-        const uint32_t d_tm = tmem + C::S_COL + (i & 1) * 64;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = dK_kmaj + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
-          const uint64_t bq = dQ_kmaj + st + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
-          ptx::mma_ss(d_tm, a, bq, C::IDESC_S, kk > 0 ? 1u : 0u);
+      for (int i = 0; ok; ++i) {
+        const int r = stage_ready(i);
+        if (r < 0) {
+          ok = false;
+          break;
         }
-        ptx::mma_commit(bar(C::B_SF + (i & 1)));
-      };
-      auto issue_dp = [&](int i) {
-        const uint64_t st = static_cast<uint64_t>(i % C::NST) * QST;
-        const uint32_t d_tm = tmem + C::DP_COL + (i & 1) * 64;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = dV_kmaj + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
-          const uint64_t bo = dDO_kmaj + st + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
-          ptx::mma_ss(d_tm, a, bo, C::IDESC_S, kk > 0 ? 1u : 0u);
-        }
-        ptx::mma_commit(bar(C::B_DPF + (i & 1)));
-      };
-
-      if (ok) {
-        const int r0 = stage_ready(0);
-        if (r0 < 0) ok = false;
-        else if (r0 == 0) n = 0;
-        else {
-          ptx::tc_fence_after();
-          issue_s(0);
-          issue_dp(0);
-          const int r1 = stage_ready(1);
-          if (r1 < 0) ok = false;
-          else if (r1 == 0) n = 1;
-          else {
-            ptx::tc_fence_after();
-            issue_s(1);
-          }
-        }
-      }
-      for (int i = 0; ok && i < n; ++i) {
+        if (r == 0) break;
         const int bs = i & 1;
         const uint64_t st = static_cast<uint64_t>(i % C::NST) * QST;
-        // dV += P^T dO: M = 128 keys, N = 128 dims, K = 64 rows (P^T from TMEM)
-        if (!ptx::mbar_wait(bar(C::B_PR + bs), (i >> 1) & 1, abort_flag, p.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
-        const uint32_t p_tm = tmem + C::S_COL + bs * 64;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_ts(tmem + C::DV_COL, p_tm + kk * 8,
-                      dDO_mn + st + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DV,
-                      (i > 0 || kk > 0) ? 1u : 0u);
-        // dP^T of the next pair, once the dQ^T that shares its buffer is drained
-        if (i + 1 < n) {
-          if (i >= 1 && !ptx::mbar_wait(bar(C::B_DQE + ((i + 1) & 1)), ((i - 1) >> 1) & 1,
-                                        abort_flag, p.timeout_ns)) {
+        if (warp == C::WARP_SP) {
+          // S^T = K Q^T and dP^T = V dO^T: M = 128 keys, N = 64 rows, K = 128 dims
+          if (i >= 2 && !ptx::mbar_wait(bar(C::B_SFREE + bs), ((i - 2) >> 1) & 1, abort_flag,
+                                        p.timeout_ns)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          issue_dp(i + 1);
-        }
-        // dK += dS^T Q (M = 128 keys, N = 128 dims, K = 64 rows) and
-        // dQ^T = K^T dS^T (M = 128 dims, N = 64 rows, K = 128 keys)
-        if (!ptx::mbar_wait(bar(C::B_DSR + bs), (i >> 1) & 1, abort_flag, p.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
-        const uint64_t dsk = dDS_kmaj + static_cast<uint64_t>(bs) * DSB;
+          const uint32_t s_tm = tmem + C::S_COL + bs * 64;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_ss(tmem + C::DK_COL, dsk + static_cast<uint64_t>((kk * 32) >> 4),
-                      dQ_mn + st + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DK,
-                      (i > 0 || kk > 0) ? 1u : 0u);
-        const uint64_t dsm = dDS_mn + static_cast<uint64_t>(bs) * DSB;
-        const uint32_t dq_tm = tmem + C::DP_COL + bs * 64;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          ptx::mma_ss(dq_tm, dK_mn + static_cast<uint64_t>((kk * 2048) >> 4),
-                      dsm + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DQ,
-                      kk > 0 ? 1u : 0u);
-        ptx::mma_commit(bar(C::B_DQF + bs));
-        ptx::mma_commit(bar(C::B_QE + i % C::NST));
-        ptx::mma_commit(bar(C::B_DSE + bs));
-        // S^T two pairs ahead (its buffer's P^T was read by the dV above)
-        if (i + 2 < n) {
-          const int r = stage_ready(i + 2);
-          if (r < 0) {
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = dK_kmaj + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
+            const uint64_t bq = dQ_kmaj + st + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
+            ptx::mma_ss(s_tm, a, bq, C::IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          ptx::mma_commit(bar(C::B_SF + bs));
+          if (i >= 2 && !ptx::mbar_wait(bar(C::B_DQE + bs), ((i - 2) >> 1) & 1, abort_flag,
+                                        p.timeout_ns)) {
             ok = false;
             break;
           }
-          if (r == 0) {
-            n = i + 2;
-          } else {
-            ptx::tc_fence_after();
-            issue_s(i + 2);
+          ptx::tc_fence_after();
+          const uint32_t dp_tm = tmem + C::DP_COL + bs * 64;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = dV_kmaj + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
+            const uint64_t bo = dDO_kmaj + st + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
+            ptx::mma_ss(dp_tm, a, bo, C::IDESC_S, kk > 0 ? 1u : 0u);
           }
+          ptx::mma_commit(bar(C::B_DPF + bs));
+        } else {
+          // dV += P^T dO: M = 128 keys, N = 128 dims, K = 64 rows (P^T from TMEM)
+          if (!ptx::mbar_wait(bar(C::B_PR + bs), (i >> 1) & 1, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t p_tm = tmem + C::S_COL + bs * 64;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_ts(tmem + C::DV_COL, p_tm + kk * 8,
+                        dDO_mn + st + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DV, 1u);
+          ptx::mma_commit(bar(C::B_SFREE + bs));
+          // dK += dS^T Q (M = 128 keys, N = 128 dims, K = 64 rows) and
+          // dQ^T = K^T dS^T (M = 128 dims, N = 64 rows, K = 128 keys)
+          if (!ptx::mbar_wait(bar(C::B_DSR + bs), (i >> 1) & 1, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t dsk = dDS_kmaj + static_cast<uint64_t>(bs) * DSB;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_ss(tmem + C::DK_COL, dsk + static_cast<uint64_t>((kk * 32) >> 4),
+                        dQ_mn + st + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DK, 1u);
+          const uint64_t dsm = dDS_mn + static_cast<uint64_t>(bs) * DSB;
+          const uint32_t dq_tm = tmem + C::DP_COL + bs * 64;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            ptx::mma_ss(dq_tm, dK_mn + static_cast<uint64_t>((kk * 2048) >> 4),
+                        dsm + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DQ,
+                        kk > 0 ? 1u : 0u);
+          ptx::mma_commit(bar(C::B_DQF + bs));
+          ptx::mma_commit(bar(C::B_QE + i % C::NST));
+          ptx::mma_commit(bar(C::B_DSE + bs));
         }
       }
-      ptx::mma_commit(bar(C::B_ACC));
+      if (warp == C::WARP_MMA) ptx::mma_commit(bar(C::B_ACC));
       if (!ok) fail();
-      // drain: every MMA issued above has completed before TMEM is freed
-      // (bounded, not cut short by the abort flag)
-      ptx::mma_commit(bar(C::B_DRAIN));
-      ptx::mbar_wait(bar(C::B_DRAIN), 0, &misc[3], p.timeout_ns);
+      // drain: every MMA this thread issued has completed before TMEM is
+      // freed (bounded, not cut short by the abort flag)
+      const int dr = warp == C::WARP_MMA ? 0 : 1;
+      ptx::mma_commit(bar(C::B_DRAIN + dr));
+      ptx::mbar_wait(bar(C::B_DRAIN + dr), 0, &misc[3], p.timeout_ns);
     }
-  } else if (warp < 4) {
-    // ======================= compute: P^T, dS^T, then dV ===================
-    const int kl = warp * 32 + lane;  // key row of the block (TMEM lane)
+  } else {
+    // ======================= compute sets: P^T, dS^T, dQ ==================
+    // set 0 takes the even pairs, set 1 the odd ones (S^T, dP^T, P^T and dS^T
+    // buffer = set), so one set's exponentials overlap the other set's TMEM
+    // reads and waits on the same SM sub-partition. After dS^T a set drains
+    // its pair's dQ^T: TMEM lanes are head dims there, warp quad takes dims
+    // [32 quad, 32 quad + 32), stages them as a [64 rows][32 dims] fp32 tile
+    // in the pair's Q / dO stage (dead once dQ^T is done: every product that
+    // reads the stage was issued before it and the tensor core completes them
+    // in order) and adds the tile to global dQ with one TMA reduce-add.
+    const int set = warp >> 2;
+    const int quad = warp & 3;
+    const int kl = quad * 32 + lane;  // key row of the block (TMEM lane)
     const int kg = j * C::BK + kl;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const bool key_ok = kg < p.Lkv;
     const float sl2 = p.scale_log2;
+    const uint32_t acc_col = set == 0 ? C::DV_COL : C::DK_COL;
+    {
+      // clear this set's accumulator rows (set 0: dV, set 1: dK); every dV and
+      // dK product then accumulates
+      uint32_t z[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) z[u] = 0u;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ptx::tmem_st32(tmem + lane_base + acc_col + 32 * c, z);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::B_ZERO));
+    }
     bool ok = true;
-    int npairs = 0;
-    for (int i = 0;; ++i) {
+    const int bs = set;
+    int pend_stage = -1;  // stage whose dQ add this warp has issued but not yet released
+    for (int i = set;; i += 2) {
       const int s = i % C::NST;
-      const int bs = i & 1;
       ok = warp_wait(bar(C::B_QF + s), (i / C::NST) & 1);
       if (!ok) break;
       const int4 rc = get_rec(s);
@@ -539,7 +565,16 @@ __global__ void __launch_bounds__(320, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(C::B_PR + bs));
+      if (lane == 0) {
+        ptx::mbar_arrive(bar(C::B_PR + bs));
+        if (pend_stage >= 0) {
+          // the previous pair's dQ add has long been issued: once it has read
+          // its staged tile, that pair's stage may be reloaded
+          ptx::bulk_wait_group_read0();
+          ptx::mbar_arrive(bar(C::B_QE + pend_stage));
+        }
+      }
+      pend_stage = -1;
 
       ok = warp_wait(bar(C::B_DPF + bs), (i >> 1) & 1);
       if (!ok) break;
@@ -579,97 +614,58 @@ __global__ void __launch_bounds__(320, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(C::B_DSR + bs));
-      ++npairs;
-    }
-    if (!ok) fail();
-    // ---- dV epilogue: row kl of dV = TMEM lane kl, 128 fp32 columns
-    if (ok) ok = warp_wait(bar(C::B_ACC), 0);
-    ptx::tc_fence_after();
-    if (ok && *abort_flag == 0) {
-      float* dst = p.dv + (static_cast<size_t>(bhk) * p.Lkv + (key_ok ? kg : 0)) * C::D;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        if (npairs > 0) {
-          ptx::tmem_ld32(tmem + lane_base + C::DV_COL + 32 * c, r);
-          ptx::tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) r[u] = 0u;
-        }
-        if (key_ok) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            reinterpret_cast<uint4*>(dst + 32 * c)[u] =
-                make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
-        }
-      }
-    }
-  } else {
-    // ======================= dQ writers (warps 4-7), then dK ==============
-    const int qd = warp - 4;
-    const int x = qd * 32 + lane;  // head dim of dQ^T (TMEM lane)
-    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
-    const float scale = p.scale;
-    bool ok = true;
-    int npairs = 0;
-    for (int i = 0;; ++i) {
-      const int s = i % C::NST;
-      const int bs = i & 1;
-      ok = warp_wait(bar(C::B_QF + s), (i / C::NST) & 1);
-      if (!ok) break;
-      const int4 rc = get_rec(s);
-      if (rc.w != 0) break;
+
       ok = warp_wait(bar(C::B_DQF + bs), (i >> 1) & 1);
       if (!ok) break;
       ptx::tc_fence_after();
-      uint32_t r0[32], r1[32];
-      ptx::tmem_ld32(tmem + lane_base + C::DP_COL + bs * 64, r0);
-      ptx::tmem_ld32(tmem + lane_base + C::DP_COL + bs * 64 + 32, r1);
-      ptx::tmem_wait_ld();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        ptx::mbar_arrive(bar(C::B_DQE + bs));
-        ptx::mbar_arrive(bar(C::B_QE + s));
+      {
+        uint32_t r0[32], r1[32];
+        ptx::tmem_ld32(tmem + lane_base + C::DP_COL + bs * 64, r0);
+        ptx::tmem_ld32(tmem + lane_base + C::DP_COL + bs * 64 + 32, r1);
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_DQE + bs));
+        const int slot = (quad < 2 ? C::OFF_Q + quad * C::DQS_BYTES
+                                   : C::OFF_DO + (quad - 2) * C::DQS_BYTES) + s * C::Q_BYTES;
+        float* tile = reinterpret_cast<float*>(smem + slot);
+        const float scale = p.scale;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) tile[c * 32 + lane] = __uint_as_float(r0[c]) * scale;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) tile[(32 + c) * 32 + lane] = __uint_as_float(r1[c]) * scale;
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::tma_reduce_add_3d(&tmDQ, sb + slot, 32 * quad, rc.y * C::BQ, b * p.Hq + rc.x);
+          ptx::bulk_commit_group();
+        }
+        pend_stage = s;  // released once the add has read it (after the next P^T)
       }
-      const int q0 = rc.y * C::BQ;
-      const int nrows = min(C::BQ, p.Lq - q0);
-      float* base = p.dq + (static_cast<size_t>(b * p.Hq + rc.x) * p.Lq + q0) * C::D + x;
-#pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if (c < nrows) atomicAdd(base + static_cast<size_t>(c) * C::D, __uint_as_float(r0[c]) * scale);
-#pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if (32 + c < nrows)
-          atomicAdd(base + static_cast<size_t>(32 + c) * C::D, __uint_as_float(r1[c]) * scale);
-      ++npairs;
+    }
+    if (lane == 0) {
+      ptx::bulk_wait_group0();  // every dQ add of this warp has completed
+      if (pend_stage >= 0) ptx::mbar_arrive(bar(C::B_QE + pend_stage));
     }
     if (!ok) fail();
-    // ---- dK epilogue: row (32 qd + lane) of dK = TMEM lane, scaled
-    const int kl = qd * 32 + lane;
-    const int kg = j * C::BK + kl;
-    const bool key_ok = kg < p.Lkv;
+    // ---- epilogue: set 0 writes dV, set 1 writes dK (scaled); row kl = TMEM lane
     if (ok) ok = warp_wait(bar(C::B_ACC), 0);
     ptx::tc_fence_after();
     if (ok && *abort_flag == 0) {
-      float* dst = p.dk + (static_cast<size_t>(bhk) * p.Lkv + (key_ok ? kg : 0)) * C::D;
+      const float f = set == 0 ? 1.0f : p.scale;
+      float* dst = (set == 0 ? p.dv : p.dk) +
+                   (static_cast<size_t>(bhk) * p.Lkv + (key_ok ? kg : 0)) * C::D;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        if (npairs > 0) {
-          ptx::tmem_ld32(tmem + lane_base + C::DK_COL + 32 * c, r);
-          ptx::tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) r[u] = 0u;
-        }
+        ptx::tmem_ld32(tmem + lane_base + acc_col + 32 * c, r);
+        ptx::tmem_wait_ld();
         if (key_ok) {
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             reinterpret_cast<float4*>(dst + 32 * c)[u] =
-                make_float4(__uint_as_float(r[4 * u]) * scale, __uint_as_float(r[4 * u + 1]) * scale,
-                            __uint_as_float(r[4 * u + 2]) * scale, __uint_as_float(r[4 * u + 3]) * scale);
+                make_float4(__uint_as_float(r[4 * u]) * f, __uint_as_float(r[4 * u + 1]) * f,
+                            __uint_as_float(r[4 * u + 2]) * f, __uint_as_float(r[4 * u + 3]) * f);
         }
       }
     }
