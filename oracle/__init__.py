@@ -81,6 +81,15 @@ class _BackwardArgs(C.Structure):
     ]
 
 
+class _BackwardRowsArgs(C.Structure):
+    _fields_ = [
+        ("base", _BackwardArgs),
+        ("n_rows", C.c_int64), ("rows", C.c_void_p), ("dq_rows", C.c_void_p),
+        ("kv_b", C.c_int64), ("kv_h", C.c_int64), ("key_lo", C.c_int64), ("key_hi", C.c_int64),
+        ("dk_part", C.c_void_p), ("dv_part", C.c_void_p), ("nthreads", C.c_int),
+    ]
+
+
 class Oracle:
     """Handle on one compiled copy of the oracle (``path`` defaults to the
     library built from ``blasst_oracle.c``; the tests also load copies with a
@@ -97,6 +106,8 @@ class Oracle:
         lib.oracle_lse_merge.restype = None
         lib.oracle_split_len.argtypes = [C.c_int64, C.c_int64, C.c_int64]
         lib.oracle_split_len.restype = C.c_int64
+        lib.oracle_backward_rows.argtypes = [C.POINTER(_BackwardRowsArgs)]
+        lib.oracle_backward_rows.restype = C.c_int
         lib.oracle_backward.argtypes = [C.POINTER(_BackwardArgs)]
         lib.oracle_backward.restype = C.c_int
         self.lib = lib
@@ -115,6 +126,9 @@ class Oracle:
 
     def backward(self, *a, **kw):
         return backward(*a, _lib=self.lib, **kw)
+
+    def backward_rows(self, *a, **kw):
+        return backward_rows(*a, _lib=self.lib, **kw)
 
 
 def _load():
@@ -282,3 +296,38 @@ def backward(q, k, v, dout, *, causal: bool, Br: int, Bc: int, scale: float | No
     if rc != 0:
         raise ValueError("oracle_backward rejected its arguments")
     return dq, dk, dv
+
+
+def backward_rows(q, k, v, dout, *, causal: bool, Br: int, Bc: int, rows, scale: float | None = None,
+                  tile_mask=None, kv_keys=None, nthreads: int = 0, _lib=None):
+    """Sampled rows of ``backward``: dq of the query rows ``rows`` (flat ids
+    ``(b*Hq + hq)*Lq + i``) as [n, d], and, with ``kv_keys = (b, hk, lo, hi)``,
+    the terms those rows add to dk and dv of keys [lo, hi) of KV head (b, hk)
+    as two [hi - lo, d] arrays (complete when ``rows`` holds every row that
+    keeps one of those keys). Returns (dq_rows, dk_part, dv_part), float64."""
+    q, k, v, dout = (np.ascontiguousarray(t) for t in (q, k, v, dout))
+    code = _dtype_code(q)
+    assert all(_dtype_code(t) == code for t in (k, v, dout))
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    tm = None
+    if tile_mask is not None:
+        tm = np.ascontiguousarray(np.asarray(tile_mask, dtype=np.uint8))
+        assert tm.shape == (B, Hq, -(-Lq // Br), -(-Lkv // Bc)), tm.shape
+    rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    dq_rows = np.zeros((rows_arr.size, d), np.float64)
+    kb, kh, lo, hi = kv_keys if kv_keys is not None else (0, 0, 0, 0)
+    dk_part = np.zeros((hi - lo, d), np.float64)
+    dv_part = np.zeros((hi - lo, d), np.float64)
+    base = _BackwardArgs(q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, code,
+                         B, Hq, Hkv, Lq, Lkv, d, int(bool(causal)), Br, Bc, float(scale),
+                         _ptr(tm), None, None, None, 0)
+    args = _BackwardRowsArgs(base, rows_arr.size, _ptr(rows_arr), dq_rows.ctypes.data,
+                             kb, kh, lo, hi, dk_part.ctypes.data if hi > lo else None,
+                             dv_part.ctypes.data if hi > lo else None, int(nthreads))
+    rc = (_lib or _load()).oracle_backward_rows(C.byref(args))
+    if rc != 0:
+        raise ValueError("oracle_backward_rows rejected its arguments")
+    return dq_rows, dk_part, dv_part

@@ -511,64 +511,80 @@ typedef struct {
   pthread_mutex_t mu;
 } backward_ctx;
 
+/* One query row i of head (b, hq): writes dq_i (d values) and adds the
+ * row's terms to dk and dv for the keys in [key_lo, key_hi) (dk_acc[j -
+ * key_lo], dv_acc[j - key_lo]; NULL adds nothing). Scratch: qi, doi [d];
+ * s, p, ds [Lkv]. */
+static void backward_row(const oracle_backward_args *a, int64_t b, int64_t hq, int64_t i,
+                         double *qi, double *doi, double *s, double *p, double *ds, double *dqi,
+                         double *dk_acc, double *dv_acc, int64_t key_lo, int64_t key_hi) {
+  const int64_t d = a->d, Lq = a->Lq, Lkv = a->Lkv, g = a->Hq / a->Hkv;
+  const int64_t nQt = (Lq + a->Br - 1) / a->Br, nKt = (Lkv + a->Bc - 1) / a->Bc;
+  const int64_t off = Lkv - Lq;
+  const int64_t hk = hq / g;
+  const int64_t kvbase = ((b * a->Hkv + hk) * Lkv) * d;
+  const int64_t qbase = ((b * a->Hq + hq) * Lq) * d;
+  for (int64_t x = 0; x < d; ++x) {
+    qi[x] = widen(a->q, a->dtype, qbase + i * d + x);
+    doi[x] = widen(a->dout, a->dtype, qbase + i * d + x);
+  }
+  const int64_t qt = i / a->Br;
+  double mx = -INFINITY;
+  for (int64_t j = 0; j < Lkv; ++j) {
+    int kept = !a->causal || j <= i + off;
+    if (kept && a->tile_mask)
+      kept = a->tile_mask[((b * a->Hq + hq) * nQt + qt) * nKt + j / a->Bc] == 0;
+    double sv = -INFINITY;
+    if (kept) {
+      double dot = 0.0;
+      for (int64_t x = 0; x < d; ++x) dot += qi[x] * widen(a->k, a->dtype, kvbase + j * d + x);
+      sv = a->scale * dot;
+    }
+    s[j] = sv;
+    if (sv > mx) mx = sv;
+  }
+  for (int64_t x = 0; x < d; ++x) dqi[x] = 0.0;
+  if (mx == -INFINITY) return; /* no kept key: O = 0, no gradient */
+  double sum = 0.0;
+  for (int64_t j = 0; j < Lkv; ++j) sum += s[j] == -INFINITY ? 0.0 : exp(s[j] - mx);
+  const double lse = mx + log(sum);
+  double D = 0.0;
+  for (int64_t j = 0; j < Lkv; ++j) {
+    p[j] = s[j] == -INFINITY ? 0.0 : exp(s[j] - lse);
+    double dp = 0.0;
+    if (p[j] != 0.0)
+      for (int64_t x = 0; x < d; ++x) dp += doi[x] * widen(a->v, a->dtype, kvbase + j * d + x);
+    ds[j] = dp; /* dP for now */
+    D += p[j] * dp;
+  }
+  for (int64_t j = 0; j < Lkv; ++j) {
+    if (p[j] == 0.0) continue;
+    const double dsj = p[j] * (ds[j] - D);
+    const int in_range = dk_acc && j >= key_lo && j < key_hi;
+    double *dkj = in_range ? dk_acc + (j - key_lo) * d : NULL;
+    double *dvj = in_range ? dv_acc + (j - key_lo) * d : NULL;
+    for (int64_t x = 0; x < d; ++x) {
+      dqi[x] += a->scale * dsj * widen(a->k, a->dtype, kvbase + j * d + x);
+      if (in_range) {
+        dkj[x] += a->scale * dsj * qi[x];
+        dvj[x] += p[j] * doi[x];
+      }
+    }
+  }
+}
+
 /* One (b, hk) unit: every query head of the group, every row. */
 static void backward_unit(const oracle_backward_args *a, int64_t unit, double *qi,
                           double *doi, double *s, double *p, double *ds) {
   const int64_t d = a->d, Lq = a->Lq, Lkv = a->Lkv, g = a->Hq / a->Hkv;
-  const int64_t nQt = (Lq + a->Br - 1) / a->Br, nKt = (Lkv + a->Bc - 1) / a->Bc;
   const int64_t b = unit / a->Hkv, hk = unit % a->Hkv;
-  const int64_t off = Lkv - Lq;
   const int64_t kvbase = ((b * a->Hkv + hk) * Lkv) * d;
   for (int64_t hh = 0; hh < g; ++hh) {
     const int64_t hq = hk * g + hh;
     const int64_t qbase = ((b * a->Hq + hq) * Lq) * d;
-    for (int64_t i = 0; i < Lq; ++i) {
-      for (int64_t x = 0; x < d; ++x) {
-        qi[x] = widen(a->q, a->dtype, qbase + i * d + x);
-        doi[x] = widen(a->dout, a->dtype, qbase + i * d + x);
-      }
-      const int64_t qt = i / a->Br;
-      double mx = -INFINITY;
-      for (int64_t j = 0; j < Lkv; ++j) {
-        int kept = !a->causal || j <= i + off;
-        if (kept && a->tile_mask)
-          kept = a->tile_mask[((b * a->Hq + hq) * nQt + qt) * nKt + j / a->Bc] == 0;
-        double sv = -INFINITY;
-        if (kept) {
-          double dot = 0.0;
-          for (int64_t x = 0; x < d; ++x) dot += qi[x] * widen(a->k, a->dtype, kvbase + j * d + x);
-          sv = a->scale * dot;
-        }
-        s[j] = sv;
-        if (sv > mx) mx = sv;
-      }
-      double *dqi = a->dq + qbase + i * d;
-      for (int64_t x = 0; x < d; ++x) dqi[x] = 0.0;
-      if (mx == -INFINITY) continue; /* no kept key: O = 0, no gradient */
-      double sum = 0.0;
-      for (int64_t j = 0; j < Lkv; ++j) sum += s[j] == -INFINITY ? 0.0 : exp(s[j] - mx);
-      const double lse = mx + log(sum);
-      double D = 0.0;
-      for (int64_t j = 0; j < Lkv; ++j) {
-        p[j] = s[j] == -INFINITY ? 0.0 : exp(s[j] - lse);
-        double dp = 0.0;
-        if (p[j] != 0.0)
-          for (int64_t x = 0; x < d; ++x) dp += doi[x] * widen(a->v, a->dtype, kvbase + j * d + x);
-        ds[j] = dp; /* dP for now */
-        D += p[j] * dp;
-      }
-      for (int64_t j = 0; j < Lkv; ++j) {
-        if (p[j] == 0.0) continue;
-        const double dsj = p[j] * (ds[j] - D);
-        double *dkj = a->dk + kvbase + j * d;
-        double *dvj = a->dv + kvbase + j * d;
-        for (int64_t x = 0; x < d; ++x) {
-          dqi[x] += a->scale * dsj * widen(a->k, a->dtype, kvbase + j * d + x);
-          dkj[x] += a->scale * dsj * qi[x];
-          dvj[x] += p[j] * doi[x];
-        }
-      }
-    }
+    for (int64_t i = 0; i < Lq; ++i)
+      backward_row(a, b, hq, i, qi, doi, s, p, ds, a->dq + qbase + i * d, a->dk + kvbase,
+                   a->dv + kvbase, 0, Lkv);
   }
 }
 
@@ -612,6 +628,119 @@ int oracle_backward(oracle_backward_args *a) {
   for (int t = 0; t < nt; ++t) { ok[t] = pthread_create(&th[t], NULL, backward_worker, &ctx) == 0; any |= ok[t]; }
   for (int t = 0; t < nt; ++t) if (ok[t]) pthread_join(th[t], NULL);
   if (!any) backward_worker(&ctx);
+  pthread_mutex_destroy(&ctx.mu);
+  return 0;
+}
+
+/* Sampled rows of the backward pass (for problems too large for the full
+ * one): dq of the listed query rows (flat ids (b*Hq + hq)*Lq + i), and the
+ * terms those rows add to dk and dv of the keys [key_lo, key_hi) of KV head
+ * (kv_b, kv_h). When the listed rows include every row that keeps one of
+ * those keys (e.g. the last rows of every head of the group for the last
+ * keys under a causal mask), those dk and dv rows are complete. */
+typedef struct {
+  oracle_backward_args base; /* dq, dk, dv, nthreads of base unused */
+  int64_t n_rows;
+  const int64_t *rows;
+  double *dq_rows;        /* [n_rows, d] */
+  int64_t kv_b, kv_h, key_lo, key_hi;
+  double *dk_part, *dv_part; /* [key_hi - key_lo, d], overwritten */
+  int nthreads;
+} oracle_backward_rows_args;
+
+typedef struct {
+  const oracle_backward_rows_args *a;
+  int64_t next;
+  pthread_mutex_t mu;
+  double *acc; /* per-thread dk/dv partials: [nt][2][nk * d] */
+  int64_t nk;
+} rows_ctx;
+
+typedef struct {
+  rows_ctx *ctx;
+  int t;
+} rows_worker_arg;
+
+static void *backward_rows_worker(void *vp) {
+  rows_worker_arg *wa = (rows_worker_arg *)vp;
+  rows_ctx *ctx = wa->ctx;
+  const oracle_backward_rows_args *a = ctx->a;
+  const oracle_backward_args *ba = &a->base;
+  const int64_t d = ba->d, g = ba->Hq / ba->Hkv;
+  double *dk_acc = ctx->acc + (int64_t)wa->t * 2 * ctx->nk * d;
+  double *dv_acc = dk_acc + ctx->nk * d;
+  double *qi = malloc(sizeof(double) * d);
+  double *doi = malloc(sizeof(double) * d);
+  double *s = malloc(sizeof(double) * ba->Lkv);
+  double *p = malloc(sizeof(double) * ba->Lkv);
+  double *ds = malloc(sizeof(double) * ba->Lkv);
+  if (!qi || !doi || !s || !p || !ds) goto out;
+  for (;;) {
+    pthread_mutex_lock(&ctx->mu);
+    int64_t r = ctx->next++;
+    pthread_mutex_unlock(&ctx->mu);
+    if (r >= a->n_rows) break;
+    const int64_t id = a->rows[r];
+    const int64_t bh = id / ba->Lq, i = id % ba->Lq;
+    const int64_t b = bh / ba->Hq, hq = bh % ba->Hq;
+    const int mine = ctx->nk > 0 && b == a->kv_b && hq / g == a->kv_h;
+    backward_row(ba, b, hq, i, qi, doi, s, p, ds, a->dq_rows + r * d, mine ? dk_acc : NULL,
+                 mine ? dv_acc : NULL, a->key_lo, a->key_hi);
+  }
+out:
+  free(qi); free(doi); free(s); free(p); free(ds);
+  return NULL;
+}
+
+int oracle_backward_rows(oracle_backward_rows_args *a) {
+  const oracle_backward_args *ba = a ? &a->base : NULL;
+  if (!a || ba->B <= 0 || ba->Hq <= 0 || ba->Hkv <= 0 || ba->Hq % ba->Hkv || ba->Lq <= 0 ||
+      ba->Lkv <= 0 || ba->d <= 0 || ba->Br <= 0 || ba->Bc <= 0 || a->n_rows < 0 ||
+      (a->n_rows > 0 && (!a->rows || !a->dq_rows)))
+    return -1;
+  for (int64_t r = 0; r < a->n_rows; ++r)
+    if (a->rows[r] < 0 || a->rows[r] >= ba->B * ba->Hq * ba->Lq) return -1;
+  int64_t nk = a->key_hi - a->key_lo;
+  if (nk < 0 || a->key_lo < 0 || a->key_hi > ba->Lkv) return -1;
+  if (nk > 0 && (!a->dk_part || !a->dv_part)) return -1;
+  int nt = resolve_threads(a->nthreads);
+  if (nt > 512) nt = 512;
+  if (a->n_rows > 0 && nt > a->n_rows) nt = (int)a->n_rows;
+  if (nt < 1) nt = 1;
+  rows_ctx ctx;
+  ctx.a = a;
+  ctx.next = 0;
+  ctx.nk = nk;
+  pthread_mutex_init(&ctx.mu, NULL);
+  ctx.acc = calloc((size_t)nt * 2 * (size_t)(nk > 0 ? nk : 1) * (size_t)ba->d, sizeof(double));
+  if (!ctx.acc) {
+    pthread_mutex_destroy(&ctx.mu);
+    return -2;
+  }
+  pthread_t th[512];
+  rows_worker_arg wa[512];
+  int ok[512], any = 0;
+  for (int t = 0; t < nt; ++t) {
+    wa[t].ctx = &ctx;
+    wa[t].t = t;
+    ok[t] = pthread_create(&th[t], NULL, backward_rows_worker, &wa[t]) == 0;
+    any |= ok[t];
+  }
+  for (int t = 0; t < nt; ++t) if (ok[t]) pthread_join(th[t], NULL);
+  if (!any) backward_rows_worker(&wa[0]);
+  if (nk > 0) {
+    const int64_t n = nk * ba->d;
+    for (int64_t e = 0; e < n; ++e) {
+      double sk = 0.0, sv = 0.0;
+      for (int t = 0; t < nt; ++t) {
+        sk += ctx.acc[(int64_t)t * 2 * n + e];
+        sv += ctx.acc[(int64_t)t * 2 * n + n + e];
+      }
+      a->dk_part[e] = sk;
+      a->dv_part[e] = sv;
+    }
+  }
+  free(ctx.acc);
   pthread_mutex_destroy(&ctx.mu);
   return 0;
 }

@@ -516,6 +516,28 @@ def pin_backward_gqa_replication(orc):
     np.testing.assert_allclose(dv, dv2.reshape(B, Hkv, 2, L, d).sum(2), rtol=0, atol=1e-12)
 
 
+def pin_backward_rows_agree_with_full(orc):
+    """The sampled-rows entry (used at sizes the full backward cannot reach)
+    returns the full backward's dq rows, and its dk, dv of a key range are
+    the full ones once every row that keeps those keys is listed."""
+    rng = np.random.default_rng(8)
+    B, Hq, Hkv, L, d = 2, 4, 2, 48, 8
+    q = rng.standard_normal((B, Hq, L, d))
+    k = rng.standard_normal((B, Hkv, L, d))
+    v = rng.standard_normal((B, Hkv, L, d))
+    dout = rng.standard_normal((B, Hq, L, d))
+    tm = (rng.random((B, Hq, 6, 6)) < 0.3).astype(np.uint8)
+    tm[..., 0] = 0
+    dq, dk, dv = orc.backward(q, k, v, dout, causal=True, Br=8, Bc=8, tile_mask=tm)
+    b, hk, lo, hi = 1, 1, 20, 35
+    rows = [(b * Hq + hq) * L + i for hq in (2, 3) for i in range(L)]
+    rq, rk, rv = orc.backward_rows(q, k, v, dout, causal=True, Br=8, Bc=8, tile_mask=tm,
+                                   rows=rows, kv_keys=(b, hk, lo, hi))
+    np.testing.assert_allclose(rq, dq[b, 2:4].reshape(-1, d), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(rk, dk[b, hk, lo:hi], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(rv, dv[b, hk, lo:hi], rtol=0, atol=1e-12)
+
+
 ALL_PINS = [
     pin_lambda0_is_dense,
     pin_first_block_always_computed,
@@ -532,6 +554,7 @@ ALL_PINS = [
     pin_static_mask_with_threshold,
     pin_backward_matches_finite_differences,
     pin_backward_gqa_replication,
+    pin_backward_rows_agree_with_full,
 ]
 
 

@@ -160,3 +160,49 @@ def test_backward_all_excluded_gives_zeros():
     assert bl.blasst_check() == 0
     for t in (dq, dk, dv):
         assert int(torch.count_nonzero(t)) == 0
+
+
+@pytest.mark.gpu
+def test_backward_full_size_sampled():
+    """The 32K prefill workload as the benchmark runs it (GPU forward at
+    lambda = 1e-3, its decisions into the GPU backward), checked on outputs
+    the oracle computes one by one: dq of seeded rows plus the last rows of
+    one GQA group, and dk, dv of the last key block of that group's KV head
+    (under the causal mask only those last rows keep those keys, so the
+    oracle's dk, dv rows there are complete). Decisions of the sampled tiles
+    come from the oracle's own forward and must match the GPU's."""
+    bl = _lib()
+    w = BASE
+    lam = float(np.float32(1e-3))
+    inp = synth.generate(w)
+    dout = synth.grad_output(w)
+    q, k, v, do = (parity.to_device(a) for a in (inp.q, inp.k, inp.v, dout))
+    o, lse, gmask = bl.attention_prefill(q, k, v, causal=True, lam=lam, Br=w.Br, Bc=w.Bc,
+                                         with_mask=True)
+    dq, dk, dv = bl.attention_backward(q, k, v, o, lse, do, causal=True, Br=w.Br, Bc=w.Bc,
+                                       skip_mask=gmask)
+    assert bl.blasst_check() == 0
+    nQt, nKt = -(-w.Lq // w.Br), -(-w.Lkv // w.Bc)
+    g = w.Hq // w.Hkv
+    hk = 3
+    r = synth.draws_u64(17, 12, 0, 32)
+    rows = [(int(r[2 * n]) % w.Hq) * w.Lq + int(r[2 * n + 1]) % w.Lq for n in range(16)]
+    rows += [(hk * g + hh) * w.Lq + i for hh in range(g) for i in range(w.Lq - w.Bc, w.Lq)]
+    rows = np.array(rows, np.int64)
+    tiles = np.unique((rows // w.Lq) * nQt + (rows % w.Lq) // w.Br)
+    ref_f = oracle.prefill(inp.q, inp.k, inp.v, causal=True, lam=lam, Br=w.Br, Bc=w.Bc,
+                           items=tiles)
+    gm = gmask.cpu().numpy().reshape(w.Hq * nQt, nKt)[tiles]
+    n_vis, n_dis, ok, dis = parity.compare_masks(gm, ref_f["mask"], ref_f["margin"], lam)
+    assert ok and n_dis == 0, f"{n_dis} sampled tiles decided differently"
+    tm = np.full((w.B, w.Hq, nQt, nKt), 2, np.uint8)
+    tm.reshape(w.Hq * nQt, nKt)[tiles] = ref_f["mask"]
+    rq, rk, rv = oracle.backward_rows(inp.q, inp.k, inp.v, dout, causal=True, Br=w.Br, Bc=w.Bc,
+                                      tile_mask=tm, rows=rows,
+                                      kv_keys=(0, hk, w.Lkv - w.Bc, w.Lkv))
+    gq = dq.reshape(-1, w.d)[rows].cpu().numpy().astype(np.float64)
+    gk = dk[0, hk, w.Lkv - w.Bc:].cpu().numpy().astype(np.float64)
+    gv = dv[0, hk, w.Lkv - w.Bc:].cpu().numpy().astype(np.float64)
+    e = {n: parity.assert_grad_within(a, b_, f"32K {n}")
+         for n, a, b_ in (("dq", gq, rq), ("dk", gk, rk), ("dv", gv, rv))}
+    print("32K sampled", {k_: {m: f"{x:.2e}" for m, x in v_.items()} for k_, v_ in e.items()})
