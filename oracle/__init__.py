@@ -90,6 +90,18 @@ class _BackwardRowsArgs(C.Structure):
     ]
 
 
+class _SelectArgs(C.Structure):
+    _fields_ = [
+        ("q", C.c_void_p), ("k", C.c_void_p), ("dtype", C.c_int),
+        ("B", C.c_int64), ("Hq", C.c_int64), ("Hkv", C.c_int64),
+        ("Lq", C.c_int64), ("Lkv", C.c_int64), ("d", C.c_int64),
+        ("causal", C.c_int), ("Br", C.c_int64), ("Bc", C.c_int64),
+        ("scale", C.c_double), ("tau", C.c_double), ("gamma", C.c_double),
+        ("mask_out", C.c_void_p), ("cstruct_out", C.c_void_p), ("amap_out", C.c_void_p),
+        ("nthreads", C.c_int),
+    ]
+
+
 class Oracle:
     """Handle on one compiled copy of the oracle (``path`` defaults to the
     library built from ``blasst_oracle.c``; the tests also load copies with a
@@ -106,6 +118,8 @@ class Oracle:
         lib.oracle_lse_merge.restype = None
         lib.oracle_split_len.argtypes = [C.c_int64, C.c_int64, C.c_int64]
         lib.oracle_split_len.restype = C.c_int64
+        lib.oracle_select.argtypes = [C.POINTER(_SelectArgs)]
+        lib.oracle_select.restype = C.c_int
         lib.oracle_backward_rows.argtypes = [C.POINTER(_BackwardRowsArgs)]
         lib.oracle_backward_rows.restype = C.c_int
         lib.oracle_backward.argtypes = [C.POINTER(_BackwardArgs)]
@@ -129,6 +143,9 @@ class Oracle:
 
     def backward_rows(self, *a, **kw):
         return backward_rows(*a, _lib=self.lib, **kw)
+
+    def select(self, *a, **kw):
+        return select(*a, _lib=self.lib, **kw)
 
 
 def _load():
@@ -331,3 +348,30 @@ def backward_rows(q, k, v, dout, *, causal: bool, Br: int, Bc: int, rows, scale:
     if rc != 0:
         raise ValueError("oracle_backward_rows rejected its arguments")
     return dq_rows, dk_part, dv_part
+
+
+def select(q, k, *, causal: bool, Br: int, Bc: int, tau: float, gamma: float,
+           scale: float | None = None, with_map: bool = True, nthreads: int = 0, _lib=None) -> dict:
+    """Pre-pass block selector (CRISP-style, on the block-pooled attention
+    estimate). Returns mask uint8 [B, Hq, nQt, nKt] (0 = selected, 1 = not;
+    the forward's static-mask convention), cstruct [B, Hq] and, with
+    ``with_map``, the estimated map amap [B, Hq, nQt, nKt] (NaN where not
+    visible)."""
+    q, k = (np.ascontiguousarray(t) for t in (q, k))
+    code = _dtype_code(q)
+    assert _dtype_code(k) == code
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    nQt, nKt = -(-Lq // Br), -(-Lkv // Bc)
+    mask = np.zeros((B, Hq, nQt, nKt), np.uint8)
+    cs = np.zeros((B, Hq), np.float64)
+    amap = np.zeros((B, Hq, nQt, nKt), np.float64) if with_map else None
+    args = _SelectArgs(q.ctypes.data, k.ctypes.data, code, B, Hq, Hkv, Lq, Lkv, d,
+                       int(bool(causal)), Br, Bc, float(scale), float(tau), float(gamma),
+                       mask.ctypes.data, cs.ctypes.data, _ptr(amap), int(nthreads))
+    rc = (_lib or _load()).oracle_select(C.byref(args))
+    if rc != 0:
+        raise ValueError("oracle_select rejected its arguments")
+    return dict(mask=mask, cstruct=cs, amap=amap, nQt=nQt, nKt=nKt)

@@ -744,3 +744,199 @@ int oracle_backward_rows(oracle_backward_rows_args *a) {
   pthread_mutex_destroy(&ctx.mu);
   return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Pre-pass block selector (the block-sparse input the forward can take).    */
+/* ------------------------------------------------------------------------ */
+/*
+ * [C] the CRISP review (rit.work, blog/crisp-sparse-attention-long-prefill),
+ *     section "What was done" (Что сделали), paragraphs 3-5:
+ *       - the selector works from an approximate attention map that is
+ *         already computed (FlexPrefill's pooled estimate);
+ *       - C_struct is the share of that map on the initial positions and
+ *         the local window; it routes each head to the structured
+ *         (Vertical-Slash) path or to the pooled path;
+ *       - on the structured path the first and the last block are always
+ *         kept, the mean background mass is taken over the other blocks and
+ *         the blocks above it are selected;
+ *       - on the pooled path the cumulative rule stays: blocks are added
+ *         until together they cover a given share of the attention.
+ * Readings (the page gives no formulas or constants):
+ *   - the map is the block-pooled estimate: per head, q_t = mean of the
+ *     query rows of tile t, k_j = mean of the keys of block j, and
+ *     A[t][j] = softmax over the blocks j visible from tile t of
+ *     scale * q_t . k_j (visible: under a causal mask, j up to the block of
+ *     the tile's last row, bottom-right aligned);
+ *   - "last block" and "local window" = the tile's last visible block;
+ *     "initial positions" = block 0;
+ *   - C_struct = the mean over the head's tiles of A[t][0] + A[t][last(t)]
+ *     (A[t][0] once when the two coincide); structured when C_struct >= tau;
+ *   - structured: keep 0 and last(t); background = mean of A[t][j] over the
+ *     other visible blocks; keep those with A[t][j] > background (strict);
+ *   - pooled: order the visible blocks by A descending (ties by index),
+ *     take the shortest prefix whose sum reaches gamma, theta = the last
+ *     value taken, keep every visible block with A[t][j] >= theta;
+ *   - output: uint8 mask [B, Hq, nQt, nKt], 0 = selected, 1 = not selected
+ *     (causally invisible blocks are 1), the static-mask convention.
+ */
+typedef struct {
+  const void *q, *k;
+  int dtype;
+  int64_t B, Hq, Hkv, Lq, Lkv, d;
+  int causal;
+  int64_t Br, Bc;
+  double scale, tau, gamma;
+  uint8_t *mask_out;    /* [B, Hq, nQt, nKt] */
+  double *cstruct_out;  /* [B, Hq] or NULL */
+  double *amap_out;     /* [B, Hq, nQt, nKt] or NULL; NaN where not visible */
+  int nthreads;
+} oracle_select_args;
+
+typedef struct {
+  const oracle_select_args *a;
+  int64_t next;
+  pthread_mutex_t mu;
+} select_ctx;
+
+static int64_t select_last_block(const oracle_select_args *a, int64_t t) {
+  const int64_t nKt = (a->Lkv + a->Bc - 1) / a->Bc;
+  if (!a->causal) return nKt - 1;
+  int64_t r1 = (t + 1) * a->Br;
+  if (r1 > a->Lq) r1 = a->Lq;
+  int64_t jl = (r1 - 1 + (a->Lkv - a->Lq)) / a->Bc;
+  return jl < nKt - 1 ? jl : nKt - 1;
+}
+
+/* One (b, hq): the pooled map, C_struct, the route and every tile's blocks. */
+static void select_head(const oracle_select_args *a, int64_t bh, double *qbar, double *kbar,
+                        double *amap, int64_t *order) {
+  const int64_t d = a->d, Lq = a->Lq, Lkv = a->Lkv;
+  const int64_t nQt = (Lq + a->Br - 1) / a->Br, nKt = (Lkv + a->Bc - 1) / a->Bc;
+  const int64_t b = bh / a->Hq, hq = bh % a->Hq, hk = hq / (a->Hq / a->Hkv);
+  const int64_t qbase = bh * Lq * d, kbase = (b * a->Hkv + hk) * Lkv * d;
+  /* pooled rows */
+  for (int64_t t = 0; t < nQt; ++t) {
+    const int64_t r0 = t * a->Br, r1 = (t + 1) * a->Br < Lq ? (t + 1) * a->Br : Lq;
+    for (int64_t x = 0; x < d; ++x) {
+      double acc = 0.0;
+      for (int64_t i = r0; i < r1; ++i) acc += widen(a->q, a->dtype, qbase + i * d + x);
+      qbar[t * d + x] = acc / (double)(r1 - r0);
+    }
+  }
+  for (int64_t j = 0; j < nKt; ++j) {
+    const int64_t c0 = j * a->Bc, c1 = (j + 1) * a->Bc < Lkv ? (j + 1) * a->Bc : Lkv;
+    for (int64_t x = 0; x < d; ++x) {
+      double acc = 0.0;
+      for (int64_t i = c0; i < c1; ++i) acc += widen(a->k, a->dtype, kbase + i * d + x);
+      kbar[j * d + x] = acc / (double)(c1 - c0);
+    }
+  }
+  /* the map: softmax over visible blocks of scale * q_t . k_j */
+  double cs = 0.0;
+  for (int64_t t = 0; t < nQt; ++t) {
+    const int64_t jl = select_last_block(a, t);
+    double *row = amap + t * nKt;
+    double mx = -INFINITY;
+    for (int64_t j = 0; j < nKt; ++j) {
+      if (j > jl) {
+        row[j] = NAN;
+        continue;
+      }
+      double dot = 0.0;
+      for (int64_t x = 0; x < d; ++x) dot += qbar[t * d + x] * kbar[j * d + x];
+      row[j] = a->scale * dot;
+      if (row[j] > mx) mx = row[j];
+    }
+    double sum = 0.0;
+    for (int64_t j = 0; j <= jl; ++j) {
+      row[j] = exp(row[j] - mx);
+      sum += row[j];
+    }
+    for (int64_t j = 0; j <= jl; ++j) row[j] /= sum;
+    cs += row[0] + (jl > 0 ? row[jl] : 0.0);
+  }
+  cs /= (double)nQt;
+  const int structured = cs >= a->tau;
+  if (a->cstruct_out) a->cstruct_out[bh] = cs;
+  /* per tile */
+  for (int64_t t = 0; t < nQt; ++t) {
+    const int64_t jl = select_last_block(a, t);
+    const double *row = amap + t * nKt;
+    uint8_t *m = a->mask_out + (bh * nQt + t) * nKt;
+    for (int64_t j = 0; j < nKt; ++j) m[j] = 1;
+    if (structured) {
+      m[0] = 0;
+      m[jl] = 0;
+      if (jl >= 2) {
+        double bg = 0.0;
+        for (int64_t j = 1; j < jl; ++j) bg += row[j];
+        bg /= (double)(jl - 1);
+        for (int64_t j = 1; j < jl; ++j)
+          if (row[j] > bg) m[j] = 0;
+      }
+    } else {
+      /* descending by value, ties by index (insertion sort: small rows) */
+      int64_t n = jl + 1;
+      for (int64_t j = 0; j < n; ++j) {
+        int64_t p = j;
+        while (p > 0 && row[order[p - 1]] < row[j]) {
+          order[p] = order[p - 1];
+          --p;
+        }
+        order[p] = j;
+      }
+      double cum = 0.0, theta = row[order[0]];
+      for (int64_t r = 0; r < n; ++r) {
+        cum += row[order[r]];
+        theta = row[order[r]];
+        if (cum >= a->gamma) break;
+      }
+      for (int64_t j = 0; j < n; ++j)
+        if (row[j] >= theta) m[j] = 0;
+    }
+  }
+  if (a->amap_out) memcpy(a->amap_out + bh * nQt * nKt, amap, sizeof(double) * nQt * nKt);
+}
+
+static void *select_worker(void *vp) {
+  select_ctx *ctx = (select_ctx *)vp;
+  const oracle_select_args *a = ctx->a;
+  const int64_t nQt = (a->Lq + a->Br - 1) / a->Br, nKt = (a->Lkv + a->Bc - 1) / a->Bc;
+  double *qbar = malloc(sizeof(double) * nQt * a->d);
+  double *kbar = malloc(sizeof(double) * nKt * a->d);
+  double *amap = malloc(sizeof(double) * nQt * nKt);
+  int64_t *order = malloc(sizeof(int64_t) * nKt);
+  if (!qbar || !kbar || !amap || !order) goto out;
+  for (;;) {
+    pthread_mutex_lock(&ctx->mu);
+    int64_t bh = ctx->next++;
+    pthread_mutex_unlock(&ctx->mu);
+    if (bh >= a->B * a->Hq) break;
+    select_head(a, bh, qbar, kbar, amap, order);
+  }
+out:
+  free(qbar); free(kbar); free(amap); free(order);
+  return NULL;
+}
+
+int oracle_select(oracle_select_args *a) {
+  if (!a || a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Hq % a->Hkv || a->Lq <= 0 ||
+      a->Lkv <= 0 || a->d <= 0 || a->Br <= 0 || a->Bc <= 0 || !a->mask_out ||
+      (a->causal && a->Lq > a->Lkv) || !(a->gamma > 0.0 && a->gamma <= 1.0))
+    return -1;
+  select_ctx ctx;
+  ctx.a = a;
+  ctx.next = 0;
+  pthread_mutex_init(&ctx.mu, NULL);
+  int64_t total = a->B * a->Hq;
+  int nt = resolve_threads(a->nthreads);
+  if (nt > total) nt = (int)total;
+  if (nt > 512) nt = 512;
+  pthread_t th[512];
+  int ok[512], any = 0;
+  for (int t = 0; t < nt; ++t) { ok[t] = pthread_create(&th[t], NULL, select_worker, &ctx) == 0; any |= ok[t]; }
+  for (int t = 0; t < nt; ++t) if (ok[t]) pthread_join(th[t], NULL);
+  if (!any) select_worker(&ctx);
+  pthread_mutex_destroy(&ctx.mu);
+  return 0;
+}

@@ -538,6 +538,106 @@ def pin_backward_rows_agree_with_full(orc):
     np.testing.assert_allclose(rv, dv[b, hk, lo:hi], rtol=0, atol=1e-12)
 
 
+# --------------------------------------------------------------------------
+# Pre-pass block selector (CRISP-style) feeding the static block mask.
+# --------------------------------------------------------------------------
+def pin_select_worked_example(orc):
+    """Hand-worked C_struct, structured-path and pooled-path masks
+    (tests/golden/selector_worked_example.json): d = 1, one row per tile and
+    one key per block, so the pooled map is a normalised weight prefix."""
+    with open(os.path.join(GOLDEN, "selector_worked_example.json")) as f:
+        fx = json.load(f)
+    w = np.array(fx["weights"], np.float64)
+    L = w.size
+    q = np.ones((1, 1, L, 1))
+    k = np.log(w).reshape(1, 1, L, 1)
+    for route in ("structured", "pooled"):
+        c = fx[route]
+        r = orc.select(q, k, causal=True, Br=1, Bc=1, tau=c["tau"], gamma=c.get("gamma", 0.9),
+                       scale=1.0)
+        assert abs(r["cstruct"][0, 0] - fx["cstruct_value"]) < 1e-14
+        assert r["mask"][0, 0].tolist() == c["mask"], (route, r["mask"][0, 0].tolist())
+        for t in range(L):
+            row = w[:t + 1] / w[:t + 1].sum()
+            np.testing.assert_allclose(r["amap"][0, 0, t, :t + 1], row, rtol=0, atol=1e-15)
+            assert np.all(np.isnan(r["amap"][0, 0, t, t + 1:]))
+
+
+def pin_select_map_is_block_mass(orc):
+    """With every query row of a tile equal and every key row of a block
+    equal, the pooled map is exactly the share of dense softmax attention
+    (numpy brute force over all keys) that falls in each block; non-causal,
+    a ragged last tile and a ragged last block, GQA."""
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, Lq, Lkv, d, Br, Bc = 1, 4, 2, 44, 52, 8, 8, 16
+    nQt, nKt = -(-Lq // Br), -(-Lkv // Bc)
+    qt = rng.standard_normal((B, Hq, nQt, d))
+    kb = rng.standard_normal((B, Hkv, nKt, d))
+    q = np.repeat(qt, Br, axis=2)[:, :, :Lq]
+    k = np.repeat(kb, Bc, axis=2)[:, :, :Lkv]
+    r = orc.select(q, k, causal=False, Br=Br, Bc=Bc, tau=0.5, gamma=0.9)
+    scale = 1.0 / np.sqrt(d)
+    g = Hq // Hkv
+    for hq in range(Hq):
+        s = scale * q[0, hq] @ k[0, hq // g].T
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        for t in range(nQt):
+            mass = np.array([p[t * Br, j * Bc:(j + 1) * Bc].sum() for j in range(nKt)])
+            # the pooled map weights a block by its key count only through its
+            # mean: with equal key rows a block's mass is count * exp(s) / Z,
+            # the map's is exp(s) / Z'; compare after dividing out the counts
+            counts = np.array([min(Bc, Lkv - j * Bc) for j in range(nKt)], np.float64)
+            per_key = mass / counts
+            np.testing.assert_allclose(r["amap"][0, hq, t], per_key / per_key.sum(), rtol=1e-13,
+                                       atol=0)
+
+
+def pin_select_extremes(orc):
+    """gamma = 1 keeps every visible block on the pooled path; tau = 0 puts
+    every head on the structured path and tau = 3 none; a uniform map keeps
+    only the first and last block on the structured path; causally invisible
+    blocks are never selected."""
+    rng = np.random.default_rng(9)
+    B, Hq, Hkv, L, d = 1, 2, 1, 96, 8
+    q = rng.standard_normal((B, Hq, L, d))
+    k = rng.standard_normal((B, Hkv, L, d))
+    nT = L // 16
+    vis = np.tril(np.ones((nT, nT), bool))
+    r = orc.select(q, k, causal=True, Br=16, Bc=16, tau=3.0, gamma=1.0)
+    assert np.array_equal(r["mask"][0, 0] == 0, vis) and np.array_equal(r["mask"][0, 1] == 0, vis)
+    r0 = orc.select(q, k, causal=True, Br=16, Bc=16, tau=0.0, gamma=0.5)
+    assert np.all((r0["mask"] == 0) <= vis)
+    for t in range(nT):
+        assert r0["mask"][0, 0, t, 0] == 0 and r0["mask"][0, 0, t, t] == 0
+    kz = np.zeros_like(k)  # every score equal: a uniform map
+    ru = orc.select(q, kz, causal=True, Br=16, Bc=16, tau=0.0, gamma=0.5)
+    for t in range(nT):
+        exp_row = np.ones(nT, np.uint8)
+        exp_row[0] = 0
+        exp_row[t] = 0
+        assert ru["mask"][0, 0, t].tolist() == exp_row.tolist()
+    n = np.arange(1, nT + 1)
+    cs_uniform = np.mean(np.where(n > 1, 2.0 / n, 1.0))
+    assert abs(ru["cstruct"][0, 0] - cs_uniform) < 1e-14
+
+
+def pin_select_permutation(orc):
+    """Non-causal: permuting the key blocks other than the first and the last
+    permutes the selected blocks of every tile the same way, on both paths."""
+    rng = np.random.default_rng(12)
+    B, Hq, Hkv, L, d, Bc = 1, 2, 1, 128, 8, 16
+    q = rng.standard_normal((B, Hq, 64, d))
+    k = rng.standard_normal((B, Hkv, L, d)) * 2.0
+    nKt = L // Bc
+    perm = np.concatenate([[0], rng.permutation(np.arange(1, nKt - 1)), [nKt - 1]])
+    kp = k.reshape(B, Hkv, nKt, Bc, d)[:, :, perm].reshape(B, Hkv, L, d)
+    for tau in (0.0, 3.0):
+        a = orc.select(q, k, causal=False, Br=16, Bc=Bc, tau=tau, gamma=0.8)
+        b = orc.select(q, kp, causal=False, Br=16, Bc=Bc, tau=tau, gamma=0.8)
+        assert np.array_equal(a["mask"][..., perm], b["mask"])
+
+
 ALL_PINS = [
     pin_lambda0_is_dense,
     pin_first_block_always_computed,
@@ -555,6 +655,10 @@ ALL_PINS = [
     pin_backward_matches_finite_differences,
     pin_backward_gqa_replication,
     pin_backward_rows_agree_with_full,
+    pin_select_worked_example,
+    pin_select_map_is_block_mass,
+    pin_select_extremes,
+    pin_select_permutation,
 ]
 
 

@@ -46,6 +46,16 @@ MUTATIONS = [
      "dkj[x] += a->scale * dsj * widen(a->k, a->dtype, kvbase + j * d + x);"),
     ("backward_dv_without_p", "dvj[x] += p[j] * doi[x];", "dvj[x] += doi[x];"),
     ("backward_ignores_tile_mask", "if (kept && a->tile_mask)", "if (0 && kept && a->tile_mask)"),
+    ("select_background_includes_first", "for (int64_t j = 1; j < jl; ++j) bg += row[j];",
+     "for (int64_t j = 0; j < jl; ++j) bg += row[j];"),
+    ("select_background_not_strict", "if (row[j] > bg) m[j] = 0;", "if (row[j] >= bg) m[j] = 0;"),
+    ("select_theta_strict", "if (row[j] >= theta) m[j] = 0;", "if (row[j] > theta) m[j] = 0;"),
+    ("select_cstruct_without_window", "cs += row[0] + (jl > 0 ? row[jl] : 0.0);", "cs += row[0];"),
+    ("select_route_inverted", "const int structured = cs >= a->tau;", "const int structured = cs < a->tau;"),
+    ("select_ragged_block_mean", "kbar[j * d + x] = acc / (double)(c1 - c0);",
+     "kbar[j * d + x] = acc / (double)a->Bc;"),
+    ("select_last_block_off_by_one", "int64_t jl = (r1 - 1 + (a->Lkv - a->Lq)) / a->Bc;",
+     "int64_t jl = (r1 + (a->Lkv - a->Lq)) / a->Bc;"),
     ("decode_skipped_block_still_used", "    if (skip) continue;\n    for (int64_t j = 0; j < nc; ++j)\n      for (int64_t x = 0; x < d; ++x)\n        kv_v",
      "    for (int64_t j = 0; j < nc; ++j)\n      for (int64_t x = 0; x < d; ++x)\n        kv_v"),
 ]
