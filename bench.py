@@ -256,7 +256,8 @@ def backward_pairs(w, mask):
     return int(kb.sum())
 
 
-BWD_FLOPS_PER_PAIR = 5 * 2 * 128 * 64 * 128  # S^T, dP^T, dV, dK, dQ^T products
+BWD_FLOPS_PER_PAIR = 5 * 2 * 128 * 64 * 128
+SEL_TAU, SEL_GAMMA = 0.2, 0.9  # selector route threshold and pooled-path coverage  # S^T, dP^T, dV, dK, dQ^T products
 
 
 class Backward:
@@ -453,7 +454,8 @@ def run_case(name, lam, calls, overrides=()):
     import dynamic_block_sparse_tiled_b200 as bl
     ncalls = calls
     backward = name.startswith("backward:")
-    if backward:
+    select = name.startswith("select:")
+    if backward or select:
         name = name.split(":", 1)[1]
     w = synth.CONFIGS[name]
     for ov in overrides:
@@ -467,6 +469,10 @@ def run_case(name, lam, calls, overrides=()):
         to = lambda a: torch.from_numpy(a).cuda()
     q, k, v = to(inp.q), to(inp.k), to(inp.v)
     del inp
+    if select:
+        for _ in range(calls):
+            bl.select_blocks(q, k, causal=w.causal, Br=w.Br, Bc=w.Bc, tau=SEL_TAU, gamma=SEL_GAMMA)
+        calls = 0
     if backward:
         o, lse, mask = bl.attention_prefill(q, k, v, causal=w.causal, lam=lam, Br=w.Br, Bc=w.Bc,
                                             with_mask=True)
@@ -482,7 +488,8 @@ def run_case(name, lam, calls, overrides=()):
             bl.attention_prefill(q, k, v, causal=w.causal, lam=lam, Br=w.Br, Bc=w.Bc)
     torch.cuda.synchronize()
     rc = bl.blasst_check()
-    print(json.dumps(dict(case=("backward:" if backward else "") + name, calls=ncalls,
+    print(json.dumps(dict(case=("backward:" if backward else "select:" if select else "") + name,
+                          calls=ncalls,
                           status=bl.blasst_status_string(rc))), flush=True)
     return 0 if rc == 0 else 1
 
@@ -534,7 +541,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--case", default=None,
                     help="profiling driver: run only this workload's kernel --calls times, untimed "
-                         "(backward:<workload> runs one forward, then the backward --calls times)")
+                         "(backward:<workload> runs one forward, then the backward --calls times; "
+                         "select:<workload> runs the block selector)")
     ap.add_argument("--calls", type=int, default=4)
     ap.add_argument("--lam", type=float, default=LAMBDA)
     ap.add_argument("--override", action="append", default=[],
@@ -643,6 +651,41 @@ def main():
             executed_tflops=s_r["exec_flops"] / (s_r["ms"] * 1e-3) / 1e12)
         del ps, sm_dev
         torch.cuda.empty_cache()
+
+        # pre-pass block selector (CRISP-style) feeding the static mask
+        sel = {}
+        for wn in (WORKLOAD, WORKLOAD + "_a12"):
+            ws_ = synth.CONFIGS[wn]
+            ps = Prefill(ws_, device)
+            nq, nk = -(-ws_.Lq // ws_.Br), -(-ws_.Lkv // ws_.Bc)
+            smask = torch.empty((ws_.B, ws_.Hq, nq, nk), dtype=torch.uint8, device=device)
+            sws = torch.empty(bl.blasst_select_workspace_bytes(ws_.B, ws_.Hq, ws_.Hkv, ws_.Lq,
+                                                               ws_.Lkv, ws_.d, ws_.Br, ws_.Bc),
+                              dtype=torch.uint8, device=device)
+            run_sel = lambda: bl.blasst_select_blocks(ps.q, ps.k, smask, causal=ws_.causal,
+                                                      Br=ws_.Br, Bc=ws_.Bc, tau=SEL_TAU,
+                                                      gamma=SEL_GAMMA, workspace=sws,
+                                                      stream=stream)
+            run_sel()
+            stream.synchronize()
+            t_sel = statistics.mean(time_calls(run_sel, max(5, args.steps), 3, stream, flush_buf))
+            causal_tiles = causal_pairs(-(-ws_.Lq // ws_.Br), -(-ws_.Lkv // ws_.Bc)) * ws_.B * ws_.Hq
+            nsel = int((smask == 0).sum().item())
+            ps, m_r = measure_prefill(ws_, LAMBDA, max(3, args.steps // 2), 3, device, stream,
+                                      flush_buf, pre=ps, block_mask=smask)
+            _, n_r = measure_prefill(ws_, LAMBDA, max(3, args.steps // 2), 3, device, stream,
+                                     flush_buf, pre=ps)
+            sel_bytes = 2.0 * ws_.d * (ws_.B * ws_.Hq * ws_.Lq + ws_.B * ws_.Hkv * ws_.Lkv)
+            gbs = sel_bytes / (t_sel * 1e-3) / 1e9
+            sel[wn] = dict(selector_ms=t_sel, selected_frac_of_causal=nsel / max(causal_tiles, 1),
+                           fwd_ms_with_mask=m_r["ms"], fwd_ms_without=n_r["ms"],
+                           speedup_selector_plus_fwd=n_r["ms"] / (t_sel + m_r["ms"]),
+                           roofline=dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"],
+                                         unit="GB/s", frac=gbs / peaks["hbm_gbs"],
+                                         algorithmic="Q and K read once (bf16)"))
+            del ps, smask, sws
+            torch.cuda.empty_cache()
+        extra["selector_32k"] = dict(tau=SEL_TAU, gamma=SEL_GAMMA, **sel)
 
         # backward with the forward's decisions held fixed, 32K workload
         pb = Prefill(w, device)

@@ -25,7 +25,8 @@ __all__ = [
     "blasst_fwd", "blasst_fwd_ex", "blasst_decode", "blasst_decode_workspace_bytes",
     "blasst_lse_merge", "blasst_check", "blasst_selftest_exp2",
     "blasst_decode_noalloc", "blasst_decode_noalloc_max_bytes", "blasst_status_string", "blasst_version",
-    "blasst_bwd", "blasst_bwd_workspace_bytes",
+    "blasst_bwd", "blasst_bwd_workspace_bytes", "blasst_select_blocks",
+    "blasst_select_workspace_bytes", "select_blocks",
     "attention_prefill", "attention_backward", "attention_decode", "new_stats", "stats_dict",
     "BLASST_OK", "BLASST_EINVAL", "BLASST_EUNSUPPORTED", "BLASST_ECUDA", "BLASST_ETIMEOUT",
     "BLASST_EWORKSPACE", "BLASST_BF16", "BLASST_FP32",
@@ -81,6 +82,17 @@ class _BwdArgs(C.Structure):
     ]
 
 
+class _SelectArgs(C.Structure):
+    _fields_ = [
+        ("q", C.c_void_p), ("k", C.c_void_p),
+        ("B", C.c_int), ("Hq", C.c_int), ("Hkv", C.c_int), ("Lq", C.c_int), ("Lkv", C.c_int),
+        ("d", C.c_int), ("causal", C.c_int), ("Br", C.c_int), ("Bc", C.c_int),
+        ("scale", C.c_float), ("tau", C.c_float), ("gamma", C.c_float),
+        ("mask_out", C.c_void_p), ("cstruct_out", C.c_void_p),
+        ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t), ("stream", C.c_void_p),
+    ]
+
+
 def load_library(path: str | None = None):
     """Load ``libblasst.so`` (raises if it has not been built)."""
     global _lib
@@ -98,6 +110,10 @@ def load_library(path: str | None = None):
         lib.blasst_fwd.restype = i
         lib.blasst_fwd_ex.argtypes = [C.POINTER(_FwdArgs)]
         lib.blasst_fwd_ex.restype = i
+        lib.blasst_select_blocks.argtypes = [C.POINTER(_SelectArgs)]
+        lib.blasst_select_blocks.restype = i
+        lib.blasst_select_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+        lib.blasst_select_workspace_bytes.restype = sz
         lib.blasst_bwd.argtypes = [C.POINTER(_BwdArgs)]
         lib.blasst_bwd.restype = i
         lib.blasst_bwd_workspace_bytes.argtypes = [i, i, i]
@@ -211,6 +227,25 @@ def blasst_bwd(q, k, v, o, dout, lse, dq, dk, dv, *, causal: bool, Br: int, Bc: 
     _check(load_library().blasst_bwd(C.byref(args)), "blasst_bwd")
 
 
+def blasst_select_workspace_bytes(B, Hq, Hkv, Lq, Lkv, d, Br, Bc) -> int:
+    return int(load_library().blasst_select_workspace_bytes(B, Hq, Hkv, Lq, Lkv, d, Br, Bc))
+
+
+def blasst_select_blocks(q, k, mask_out, *, causal: bool, Br: int, Bc: int, tau: float,
+                         gamma: float, workspace, scale: float = 0.0, cstruct_out=None,
+                         stream=None):
+    """The C entry point of the same name. q [B,Hq,Lq,d], k [B,Hkv,Lkv,d] bf16;
+    mask_out uint8 [B,Hq,ceil(Lq/Br),ceil(Lkv/Bc)]; cstruct_out fp32 [B,Hq] or
+    None; workspace a uint8 CUDA tensor of blasst_select_workspace_bytes()."""
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    args = _SelectArgs(_ptr(q), _ptr(k), B, Hq, Hkv, Lq, Lkv, d, int(bool(causal)), Br, Bc,
+                       float(scale), float(tau), float(gamma), _ptr(mask_out), _ptr(cstruct_out),
+                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                       _stream(stream))
+    _check(load_library().blasst_select_blocks(C.byref(args)), "blasst_select_blocks")
+
+
 def blasst_decode_workspace_bytes(B: int, Hq: int, d: int, num_splits: int) -> int:
     return int(load_library().blasst_decode_workspace_bytes(B, Hq, d, num_splits))
 
@@ -307,6 +342,24 @@ def attention_backward(q, k, v, o, lse, dout, *, causal=True, Br=128, Bc=128, sk
     blasst_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal=causal, Br=Br, Bc=Bc, workspace=workspace,
                skip_mask=skip_mask, scale=scale, stream=stream)
     return dq, dk, dv
+
+
+def select_blocks(q, k, *, causal=True, Br=128, Bc=128, tau=0.2, gamma=0.9, scale=0.0,
+                  stream=None, workspace=None):
+    """Allocate the mask (and the workspace) with torch and run
+    blasst_select_blocks. Returns (mask, cstruct): mask uint8
+    [B,Hq,nQt,nKt] (0 = selected), ready for attention_prefill(block_mask=...)."""
+    import torch
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    mask = torch.empty((B, Hq, -(-Lq // Br), -(-Lkv // Bc)), dtype=torch.uint8, device=q.device)
+    cs = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(blasst_select_workspace_bytes(B, Hq, Hkv, Lq, Lkv, d, Br, Bc),
+                                dtype=torch.uint8, device=q.device)
+    blasst_select_blocks(q, k, mask, causal=causal, Br=Br, Bc=Bc, tau=tau, gamma=gamma,
+                         workspace=workspace, scale=scale, cstruct_out=cs, stream=stream)
+    return mask, cs
 
 
 def attention_decode(q, k_cache, v_cache, *, lam=0.0, Bc=128, num_splits=64, with_mask=False,

@@ -18,6 +18,7 @@
 #include "decode_sm100.cuh"
 #include "prefill_f32_sm100.cuh"
 #include "prefill_sm100.cuh"
+#include "select_sm100.cuh"
 
 namespace {
 
@@ -409,6 +410,72 @@ int blasst_bwd(const blasst_bwd_args* a) {
   if (set_smem(blasst::blasst_bwd_kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
   const dim3 grid(static_cast<unsigned>(p.nKb) * p.B * p.Hkv);
   blasst::blasst_bwd_kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(mq, mdo, mk, mv, mdq, p);
+  return cuda_status(cudaGetLastError());
+}
+
+size_t blasst_select_workspace_bytes(int B, int Hq, int Hkv, int Lq, int Lkv, int d, int Br,
+                                     int Bc) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Lkv <= 0 || d <= 0 || Br <= 0 || Bc <= 0)
+    return 0;
+  const size_t nQt = (static_cast<size_t>(Lq) + Br - 1) / Br;
+  const size_t nKt = (static_cast<size_t>(Lkv) + Bc - 1) / Bc;
+  return (static_cast<size_t>(B) * Hq * nQt * d + static_cast<size_t>(B) * Hkv * nKt * d +
+          static_cast<size_t>(B) * Hq * nQt * 3) * sizeof(float);
+}
+
+int blasst_select_blocks(const blasst_select_args* a) {
+  if (!a) return BLASST_EINVAL;
+  if (!a->q || !a->k || !a->mask_out) return BLASST_EINVAL;
+  if (!aligned16(a->q) || !aligned16(a->k)) return BLASST_EINVAL;
+  if (a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Lq <= 0 || a->Lkv <= 0) return BLASST_EINVAL;
+  if (a->Hq % a->Hkv != 0) return BLASST_EINVAL;
+  if (!(a->gamma > 0.0f && a->gamma <= 1.0f) || !std::isfinite(a->tau)) return BLASST_EINVAL;
+  if (a->d != 64 && a->d != 128) return BLASST_EUNSUPPORTED;
+  if ((a->Br != 64 && a->Br != 128) || (a->Bc != 64 && a->Bc != 128)) return BLASST_EUNSUPPORTED;
+  if (a->causal && a->Lq > a->Lkv) return BLASST_EUNSUPPORTED;
+  const int nQt = (a->Lq + a->Br - 1) / a->Br, nKt = (a->Lkv + a->Bc - 1) / a->Bc;
+  if (nKt > 32 * blasst::SEL_MAXJ) return BLASST_EUNSUPPORTED;
+  const long long rows = static_cast<long long>(a->B) * a->Hq * nQt;
+  if (rows + static_cast<long long>(a->B) * a->Hkv * nKt > 0x7fffffffll) return BLASST_EINVAL;
+  const size_t need = blasst_select_workspace_bytes(a->B, a->Hq, a->Hkv, a->Lq, a->Lkv, a->d,
+                                                    a->Br, a->Bc);
+  if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
+    return BLASST_EWORKSPACE;
+  blasst::SelectParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(a->q);
+  p.k = static_cast<const __nv_bfloat16*>(a->k);
+  p.qbar = static_cast<float*>(a->workspace);
+  p.kbar = p.qbar + static_cast<size_t>(rows) * a->d;
+  p.rowst = p.kbar + static_cast<size_t>(a->B) * a->Hkv * nKt * a->d;
+  p.mask = a->mask_out;
+  p.cstruct = a->cstruct_out;
+  p.B = a->B;
+  p.Hq = a->Hq;
+  p.Hkv = a->Hkv;
+  p.Lq = a->Lq;
+  p.Lkv = a->Lkv;
+  p.d = a->d;
+  p.g = a->Hq / a->Hkv;
+  p.Br = a->Br;
+  p.Bc = a->Bc;
+  p.nQt = nQt;
+  p.nKt = nKt;
+  p.causal = a->causal ? 1 : 0;
+  p.off = a->Lkv - a->Lq;
+  p.scale = a->scale > 0.0f ? a->scale
+                            : static_cast<float>(1.0 / std::sqrt(static_cast<double>(a->d)));
+  p.tau = a->tau;
+  p.gamma = a->gamma;
+  const cudaStream_t s = static_cast<cudaStream_t>(a->stream);
+  const unsigned npool = static_cast<unsigned>(rows + static_cast<long long>(a->B) * a->Hkv * nKt);
+  blasst::blasst_select_pool_kernel<<<npool, 128, 0, s>>>(p);
+  int rc = cuda_status(cudaGetLastError());
+  if (rc != BLASST_OK) return rc;
+  const unsigned nrow_blocks = static_cast<unsigned>((rows + 7) / 8);
+  blasst::blasst_select_rows_kernel<<<nrow_blocks, 256, 0, s>>>(p);
+  rc = cuda_status(cudaGetLastError());
+  if (rc != BLASST_OK) return rc;
+  blasst::blasst_select_mask_kernel<<<nrow_blocks, 256, 0, s>>>(p);
   return cuda_status(cudaGetLastError());
 }
 

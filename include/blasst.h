@@ -180,6 +180,51 @@ BLASST_API int blasst_bwd(const blasst_bwd_args* args);
 /* Bytes of workspace blasst_bwd needs: two fp32 [B, Hq, ceil(Lq/64)*64]. */
 BLASST_API size_t blasst_bwd_workspace_bytes(int B, int Hq, int Lq);
 
+/* Pre-pass block selector producing a static block mask for blasst_fwd_ex
+ * (block_mask_in), after the CRISP review (rit.work, blog/crisp-sparse-
+ * attention-long-prefill, section "What was done", paragraphs 3-5). The page
+ * gives no formulas; the readings:
+ *   - map: per query head, qb_t = mean of the rows of query tile t, kb_j =
+ *     mean of the keys of KV block j, A[t][j] = softmax over the blocks
+ *     visible from tile t (causal: bottom-right) of scale * qb_t . kb_j;
+ *   - C_struct = mean over tiles of A[t][0] + A[t][last(t)], last(t) the
+ *     tile's last visible block; the head is "structured" when C_struct >= tau;
+ *   - structured: keep block 0, block last(t), and the blocks in between
+ *     whose A is strictly above the mean A of those in-between blocks;
+ *   - otherwise: keep the largest-A blocks until they cover gamma of the row,
+ *     plus every block tied with the last one taken.
+ *   q [B, Hq, Lq, d], k [B, Hkv, Lkv, d] bf16 (device).
+ *   Br, Bc     tile sizes of the forward that will read the mask (64 or 128).
+ *   mask_out   uint8 [B, Hq, ceil(Lq/Br), ceil(Lkv/Bc)], fully written:
+ *              0 = selected, 1 = not selected (invisible blocks are 1).
+ *   cstruct_out nullable fp32 [B, Hq].
+ *   tau, gamma route threshold and pooled-path coverage (0 < gamma <= 1).
+ *   scale      <= 0 selects 1/sqrt(d).
+ *   workspace  >= blasst_select_workspace_bytes(...) bytes, 16-byte aligned.
+ * d in {64, 128}; ceil(Lkv/Bc) <= 2048 (else BLASST_EUNSUPPORTED). */
+typedef struct blasst_select_args {
+  const void* q;
+  const void* k;
+  int B, Hq, Hkv, Lq, Lkv, d;
+  int causal;
+  int Br, Bc;
+  float scale;
+  float tau;
+  float gamma;
+  uint8_t* mask_out;
+  float* cstruct_out;
+  void* workspace;
+  size_t workspace_bytes;
+  void* stream;
+} blasst_select_args;
+BLASST_API int blasst_select_blocks(const blasst_select_args* args);
+
+/* Workspace bytes of blasst_select_blocks: the pooled rows (fp32
+ * [B*Hq, nQt, d] and [B*Hkv, nKt, d]) and three fp32 row statistics per
+ * query tile. */
+BLASST_API size_t blasst_select_workspace_bytes(int B, int Hq, int Hkv, int Lq, int Lkv, int d,
+                                                int Br, int Bc);
+
 /* Bytes of caller workspace that blasst_decode needs: fp32 partial outputs
  * [B, Hq, num_splits, d] plus fp32 partial lse [B, Hq, num_splits]. */
 BLASST_API size_t blasst_decode_workspace_bytes(int B, int Hq, int d, int num_splits);

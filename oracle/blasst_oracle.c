@@ -807,9 +807,20 @@ static int64_t select_last_block(const oracle_select_args *a, int64_t t) {
   return jl < nKt - 1 ? jl : nKt - 1;
 }
 
+typedef struct {
+  double v;
+  int64_t j;
+} select_item;
+
+static int select_cmp(const void *x, const void *y) {
+  const select_item *a = (const select_item *)x, *b = (const select_item *)y;
+  if (a->v != b->v) return a->v > b->v ? -1 : 1;
+  return a->j < b->j ? -1 : (a->j > b->j ? 1 : 0);
+}
+
 /* One (b, hq): the pooled map, C_struct, the route and every tile's blocks. */
 static void select_head(const oracle_select_args *a, int64_t bh, double *qbar, double *kbar,
-                        double *amap, int64_t *order) {
+                        double *amap, select_item *order) {
   const int64_t d = a->d, Lq = a->Lq, Lkv = a->Lkv;
   const int64_t nQt = (Lq + a->Br - 1) / a->Br, nKt = (Lkv + a->Bc - 1) / a->Bc;
   const int64_t b = bh / a->Hq, hq = bh % a->Hq, hk = hq / (a->Hq / a->Hkv);
@@ -875,20 +886,17 @@ static void select_head(const oracle_select_args *a, int64_t bh, double *qbar, d
           if (row[j] > bg) m[j] = 0;
       }
     } else {
-      /* descending by value, ties by index (insertion sort: small rows) */
+      /* descending by value, ties by index (library sort) */
       int64_t n = jl + 1;
       for (int64_t j = 0; j < n; ++j) {
-        int64_t p = j;
-        while (p > 0 && row[order[p - 1]] < row[j]) {
-          order[p] = order[p - 1];
-          --p;
-        }
-        order[p] = j;
+        order[j].v = row[j];
+        order[j].j = j;
       }
-      double cum = 0.0, theta = row[order[0]];
+      qsort(order, (size_t)n, sizeof(select_item), select_cmp);
+      double cum = 0.0, theta = order[0].v;
       for (int64_t r = 0; r < n; ++r) {
-        cum += row[order[r]];
-        theta = row[order[r]];
+        cum += order[r].v;
+        theta = order[r].v;
         if (cum >= a->gamma) break;
       }
       for (int64_t j = 0; j < n; ++j)
@@ -905,7 +913,7 @@ static void *select_worker(void *vp) {
   double *qbar = malloc(sizeof(double) * nQt * a->d);
   double *kbar = malloc(sizeof(double) * nKt * a->d);
   double *amap = malloc(sizeof(double) * nQt * nKt);
-  int64_t *order = malloc(sizeof(int64_t) * nKt);
+  select_item *order = malloc(sizeof(select_item) * nKt);
   if (!qbar || !kbar || !amap || !order) goto out;
   for (;;) {
     pthread_mutex_lock(&ctx->mu);

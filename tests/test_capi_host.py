@@ -113,6 +113,42 @@ def test_bwd_rejects_bad_arguments_without_a_gpu(lib, bad, code):
         assert _bwd(lib, **bad) == code
 
 
+def _sel(lib, **kw):
+    import dynamic_block_sparse_tiled_b200 as bl
+    base = dict(q=0x10000, k=0x20000, B=1, Hq=4, Hkv=2, Lq=256, Lkv=256, d=128, causal=1,
+                Br=128, Bc=128, scale=0.0, tau=0.2, gamma=0.9, mask_out=0x30000,
+                cstruct_out=None, workspace=0x40000, workspace_bytes=1 << 20, stream=None)
+    base.update(kw)
+    args = bl._SelectArgs(*[base[f[0]] for f in bl._SelectArgs._fields_])
+    return lib.blasst_select_blocks(C.byref(args))
+
+
+def test_select_workspace_bytes(lib):
+    # qbar 4*2*128 + kbar 2*2*128 + row statistics 4*2*3, fp32
+    assert lib.blasst_select_workspace_bytes(1, 4, 2, 256, 256, 128, 128, 128) == \
+        (4 * 2 * 128 + 2 * 2 * 128 + 4 * 2 * 3) * 4
+    assert lib.blasst_select_workspace_bytes(0, 4, 2, 256, 256, 128, 128, 128) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(q=None), -1),
+    (dict(mask_out=None), -1),
+    (dict(k=0x20008), -1),
+    (dict(Hq=3), -1),
+    (dict(gamma=0.0), -1),
+    (dict(gamma=1.5), -1),
+    (dict(tau=float("nan")), -1),
+    (dict(d=96), -2),
+    (dict(Bc=32), -2),
+    (dict(Lq=300), -2),                               # causal with Lq > Lkv
+    (dict(Lq=2049 * 128, Lkv=2049 * 128), -2),        # more than 2048 KV blocks
+    (dict(workspace=None), -5),
+    (dict(workspace_bytes=64), -5),
+])
+def test_select_rejects_bad_arguments_without_a_gpu(lib, bad, code):
+    assert _sel(lib, **bad) == code
+
+
 def test_decode_workspace_and_rejections(lib):
     ws = lib.blasst_decode_workspace_bytes(16, 32, 128, 64)
     assert ws == 16 * 32 * 64 * (128 + 1) * 4
