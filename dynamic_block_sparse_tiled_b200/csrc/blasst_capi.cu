@@ -420,7 +420,8 @@ size_t blasst_select_workspace_bytes(int B, int Hq, int Hkv, int Lq, int Lkv, in
   const size_t nQt = (static_cast<size_t>(Lq) + Br - 1) / Br;
   const size_t nKt = (static_cast<size_t>(Lkv) + Bc - 1) / Bc;
   return (static_cast<size_t>(B) * Hq * nQt * d + static_cast<size_t>(B) * Hkv * nKt * d +
-          static_cast<size_t>(B) * Hq * nQt * 3) * sizeof(float);
+          static_cast<size_t>(B) * Hq * nQt * 3 + static_cast<size_t>(B) * Hq * nQt * nKt) *
+         sizeof(float);
 }
 
 int blasst_select_blocks(const blasst_select_args* a) {
@@ -447,6 +448,7 @@ int blasst_select_blocks(const blasst_select_args* a) {
   p.qbar = static_cast<float*>(a->workspace);
   p.kbar = p.qbar + static_cast<size_t>(rows) * a->d;
   p.rowst = p.kbar + static_cast<size_t>(a->B) * a->Hkv * nKt * a->d;
+  p.scores = p.rowst + static_cast<size_t>(rows) * 3;
   p.mask = a->mask_out;
   p.cstruct = a->cstruct_out;
   p.B = a->B;
@@ -472,7 +474,9 @@ int blasst_select_blocks(const blasst_select_args* a) {
   int rc = cuda_status(cudaGetLastError());
   if (rc != BLASST_OK) return rc;
   const unsigned nrow_blocks = static_cast<unsigned>((rows + 7) / 8);
-  blasst::blasst_select_rows_kernel<<<nrow_blocks, 256, 0, s>>>(p);
+  const unsigned ntile_blocks = static_cast<unsigned>(static_cast<long long>(a->B) * a->Hq *
+                                                      ((nQt + 7) / 8));
+  blasst::blasst_select_rows_kernel<<<ntile_blocks, 256, 0, s>>>(p);
   rc = cuda_status(cudaGetLastError());
   if (rc != BLASST_OK) return rc;
   blasst::blasst_select_mask_kernel<<<nrow_blocks, 256, 0, s>>>(p);

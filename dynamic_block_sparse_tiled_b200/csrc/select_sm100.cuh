@@ -18,8 +18,9 @@
 // blocks are 1): the prefill's block_mask_in convention.
 //
 // Three small kernels: pooled means (one CTA per tile or block; reads Q and
-// K once, HBM-bound), row statistics (one warp per tile row of the map: max,
-// normaliser and the row's C_struct term), selection (one warp per tile row:
+// K once, HBM-bound), row statistics (one warp per tile row of the map: the
+// scores, kept for the next kernel, their max, normaliser and the row's
+// C_struct term), selection (one warp per tile row, reading the scores back:
 // the head's C_struct summed in a fixed order, the route, then the row's
 // blocks; the cumulative threshold is found by bisection on the float bits of
 // the map values, which picks the same set as sorting and taking a prefix).
@@ -37,6 +38,7 @@ struct SelectParams {
   float* qbar;             // [B*Hq, nQt, d]
   float* kbar;             // [B*Hkv, nKt, d]
   float* rowst;            // [B*Hq, nQt, 3]: max score, normaliser, C_struct term
+  float* scores;           // [B*Hq, nQt, nKt]: scale * qb_t . kb_j of visible blocks
   uint8_t* mask;           // [B, Hq, nQt, nKt]
   float* cstruct;          // [B, Hq] or null
   int B, Hq, Hkv, Lq, Lkv, d, g;
@@ -106,34 +108,6 @@ __global__ void __launch_bounds__(128) blasst_select_pool_kernel(SelectParams p)
   }
 }
 
-// Scores of tile row t against every visible block, lane-strided over blocks.
-// Returns the number of visible blocks; s[m] holds block lane + 32 m.
-__device__ __forceinline__ int sel_row_scores(const SelectParams& p, int bh, int t, int lane,
-                                              const float* qb, float (&s)[SEL_MAXJ]) {
-  const int hk = (bh % p.Hq) / p.g + (bh / p.Hq) * p.Hkv;
-  const int nvis = sel_last_block(p, t) + 1;
-  const float4* q4 = reinterpret_cast<const float4*>(qb);
-#pragma unroll
-  for (int m = 0; m < SEL_MAXJ; ++m) {
-    const int j = lane + 32 * m;
-    s[m] = -INFINITY;
-    if (32 * m < nvis && j < nvis) {
-      const float4* k4 = reinterpret_cast<const float4*>(p.kbar + (static_cast<size_t>(hk) * p.nKt + j) * p.d);
-      float dot = 0.0f;
-      for (int x = 0; x < p.d / 4; ++x) {
-        const float4 a = q4[x];
-        const float4 b = k4[x];
-        dot = fmaf(a.x, b.x, dot);
-        dot = fmaf(a.y, b.y, dot);
-        dot = fmaf(a.z, b.z, dot);
-        dot = fmaf(a.w, b.w, dot);
-      }
-      s[m] = p.scale * dot;
-    }
-  }
-  return nvis;
-}
-
 __device__ __forceinline__ float sel_warp_sum(float v) {
 #pragma unroll
   for (int sh = 16; sh > 0; sh >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sh);
@@ -145,25 +119,65 @@ __device__ __forceinline__ float sel_warp_max(float v) {
   return v;
 }
 
-// Row statistics: one warp per (b, hq, t).
+// Row statistics. One CTA per (b, hq, 8 consecutive tiles), one warp per
+// tile row; the head's pooled keys are staged transposed in shared memory 32
+// blocks at a time, so lane l of every warp reads block (32 c + l) without
+// bank conflicts and each pooled key is read from L2 once per CTA.
 __global__ void __launch_bounds__(256) blasst_select_rows_kernel(SelectParams p) {
   __shared__ __align__(16) float qs[8][128];
+  __shared__ __align__(16) float kT[128][32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + w;
-  if (row >= static_cast<long long>(p.B) * p.Hq * p.nQt) return;
-  const int bh = static_cast<int>(row / p.nQt), t = static_cast<int>(row % p.nQt);
-  for (int x = lane; x < p.d; x += 32) qs[w][x] = p.qbar[static_cast<size_t>(row) * p.d + x];
-  __syncwarp();
+  const int ntg = (p.nQt + 7) / 8;
+  const int bh = static_cast<int>(blockIdx.x) / ntg;
+  const int t0 = (static_cast<int>(blockIdx.x) % ntg) * 8;
+  const int t = t0 + w;
+  const bool active = t < p.nQt;
+  const int hk = (bh % p.Hq) / p.g + (bh / p.Hq) * p.Hkv;
+  const size_t row = static_cast<size_t>(bh) * p.nQt + t;
+  if (active)
+    for (int x = lane; x < p.d; x += 32) qs[w][x] = p.qbar[row * p.d + x];
+  const int nvis = active ? sel_last_block(p, t) + 1 : 0;
+  const int nv_max = sel_last_block(p, min(t0 + 7, p.nQt - 1)) + 1;  // nondecreasing in t
+  const float4* kb4 = reinterpret_cast<const float4*>(p.kbar + static_cast<size_t>(hk) * p.nKt * p.d);
+  const int d4 = p.d / 4;
   float s[SEL_MAXJ];
-  const int nvis = sel_row_scores(p, bh, t, lane, qs[w], s);
+#pragma unroll
+  for (int m = 0; m < SEL_MAXJ; ++m) s[m] = -INFINITY;
+#pragma unroll
+  for (int m = 0; m < SEL_MAXJ; ++m) {
+    if (32 * m >= nv_max) break;
+    __syncthreads();  // the previous chunk has been read (and qs written)
+    for (int e = threadIdx.x; e < 32 * d4; e += 256) {
+      const int jj = e & 31, x4 = e >> 5, j = 32 * m + jj;
+      const float4 v = j < p.nKt ? kb4[static_cast<size_t>(j) * d4 + x4] : make_float4(0, 0, 0, 0);
+      kT[4 * x4][jj] = v.x;
+      kT[4 * x4 + 1][jj] = v.y;
+      kT[4 * x4 + 2][jj] = v.z;
+      kT[4 * x4 + 3][jj] = v.w;
+    }
+    __syncthreads();
+    if (32 * m < nvis) {
+      float dot = 0.0f;
+      for (int x = 0; x < p.d; ++x) dot = fmaf(qs[w][x], kT[x][lane], dot);
+      if (32 * m + lane < nvis) s[m] = p.scale * dot;
+    }
+  }
+  if (!active) return;
+  float* srow = p.scores + row * p.nKt;
   float mx = -INFINITY;
 #pragma unroll
-  for (int m = 0; m < SEL_MAXJ; ++m) mx = fmaxf(mx, s[m]);
+  for (int m = 0; m < SEL_MAXJ; ++m) {
+    if (32 * m >= nvis) break;
+    if (lane + 32 * m < nvis) srow[lane + 32 * m] = s[m];
+    mx = fmaxf(mx, s[m]);
+  }
   mx = sel_warp_max(mx);
   float z = 0.0f;
 #pragma unroll
-  for (int m = 0; m < SEL_MAXJ; ++m)
+  for (int m = 0; m < SEL_MAXJ; ++m) {
+    if (32 * m >= nvis) break;
     if (s[m] > -INFINITY) z += expf(s[m] - mx);
+  }
   z = sel_warp_sum(z);
   // C_struct term: A[t][0] + A[t][last] (A[t][0] once when they coincide)
   const int jl = nvis - 1;
@@ -176,7 +190,7 @@ __global__ void __launch_bounds__(256) blasst_select_rows_kernel(SelectParams p)
   }
   term = sel_warp_sum(term);
   if (lane == 0) {
-    float* st = p.rowst + static_cast<size_t>(row) * 3;
+    float* st = p.rowst + row * 3;
     st[0] = mx;
     st[1] = z;
     st[2] = term;
@@ -185,7 +199,6 @@ __global__ void __launch_bounds__(256) blasst_select_rows_kernel(SelectParams p)
 
 // Selection: one warp per (b, hq, t).
 __global__ void __launch_bounds__(256) blasst_select_mask_kernel(SelectParams p) {
-  __shared__ __align__(16) float qs[8][128];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + w;
   if (row >= static_cast<long long>(p.B) * p.Hq * p.nQt) return;
@@ -197,15 +210,19 @@ __global__ void __launch_bounds__(256) blasst_select_mask_kernel(SelectParams p)
   cs = sel_warp_sum(cs) / static_cast<float>(p.nQt);
   const bool structured = cs >= p.tau;
   if (t == 0 && lane == 0 && p.cstruct) p.cstruct[bh] = cs;
-  for (int x = lane; x < p.d; x += 32) qs[w][x] = p.qbar[static_cast<size_t>(row) * p.d + x];
-  __syncwarp();
-  float s[SEL_MAXJ];
-  const int nvis = sel_row_scores(p, bh, t, lane, qs[w], s);
+  const int nvis = sel_last_block(p, t) + 1;
+  const float* srow = p.scores + static_cast<size_t>(row) * p.nKt;
   const float mx = p.rowst[static_cast<size_t>(row) * 3];
   const float z = p.rowst[static_cast<size_t>(row) * 3 + 1];
   float a[SEL_MAXJ];
 #pragma unroll
-  for (int m = 0; m < SEL_MAXJ; ++m) a[m] = s[m] > -INFINITY ? expf(s[m] - mx) / z : -1.0f;
+  for (int m = 0; m < SEL_MAXJ; ++m) a[m] = -1.0f;
+#pragma unroll
+  for (int m = 0; m < SEL_MAXJ; ++m) {
+    if (32 * m >= nvis) break;
+    const int j = lane + 32 * m;
+    if (j < nvis) a[m] = expf(srow[j] - mx) / z;
+  }
   const int jl = nvis - 1;
   float thr;        // keep A > thr (structured) or A >= thr (pooled)
   bool strict;
@@ -213,6 +230,7 @@ __global__ void __launch_bounds__(256) blasst_select_mask_kernel(SelectParams p)
     float bg = 0.0f;
 #pragma unroll
     for (int m = 0; m < SEL_MAXJ; ++m) {
+      if (32 * m >= nvis) break;
       const int j = lane + 32 * m;
       if (j >= 1 && j < jl) bg += a[m];
     }
@@ -228,8 +246,10 @@ __global__ void __launch_bounds__(256) blasst_select_mask_kernel(SelectParams p)
       const float th = __uint_as_float(mid);
       float mass = 0.0f;
 #pragma unroll
-      for (int m = 0; m < SEL_MAXJ; ++m)
+      for (int m = 0; m < SEL_MAXJ; ++m) {
+        if (32 * m >= nvis) break;
         if (a[m] >= th) mass += a[m];
+      }
       mass = sel_warp_sum(mass);
       if (mass >= p.gamma) lo = mid;
       else hi = mid;
@@ -238,18 +258,17 @@ __global__ void __launch_bounds__(256) blasst_select_mask_kernel(SelectParams p)
     strict = false;
   }
   uint8_t* mrow = p.mask + static_cast<size_t>(row) * p.nKt;
-  for (int j = lane; j < p.nKt; j += 32) {
-    const int m = j >> 5;
-    float v = -1.0f;
 #pragma unroll
-    for (int mm = 0; mm < SEL_MAXJ; ++mm)
-      if (mm == m) v = a[mm];
+  for (int m = 0; m < SEL_MAXJ; ++m) {
+    const int j = lane + 32 * m;
+    if (32 * m >= p.nKt) break;
     bool sel = false;
     if (j <= jl) {
+      const float v = a[m];
       if (structured) sel = (j == 0 || j == jl) || (strict ? v > thr : v >= thr);
       else sel = v >= thr;
     }
-    mrow[j] = sel ? 0 : 1;
+    if (j < p.nKt) mrow[j] = sel ? 0 : 1;
   }
 }
 

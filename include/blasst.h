@@ -220,8 +220,8 @@ typedef struct blasst_select_args {
 BLASST_API int blasst_select_blocks(const blasst_select_args* args);
 
 /* Workspace bytes of blasst_select_blocks: the pooled rows (fp32
- * [B*Hq, nQt, d] and [B*Hkv, nKt, d]) and three fp32 row statistics per
- * query tile. */
+ * [B*Hq, nQt, d] and [B*Hkv, nKt, d]), three fp32 row statistics per query
+ * tile and the fp32 block scores [B*Hq, nQt, nKt]. */
 BLASST_API size_t blasst_select_workspace_bytes(int B, int Hq, int Hkv, int Lq, int Lkv, int d,
                                                 int Br, int Bc);
 

@@ -124,9 +124,9 @@ def _sel(lib, **kw):
 
 
 def test_select_workspace_bytes(lib):
-    # qbar 4*2*128 + kbar 2*2*128 + row statistics 4*2*3, fp32
+    # qbar 4*2*128 + kbar 2*2*128 + row statistics 4*2*3 + scores 4*2*2, fp32
     assert lib.blasst_select_workspace_bytes(1, 4, 2, 256, 256, 128, 128, 128) == \
-        (4 * 2 * 128 + 2 * 2 * 128 + 4 * 2 * 3) * 4
+        (4 * 2 * 128 + 2 * 2 * 128 + 4 * 2 * 3 + 4 * 2 * 2) * 4
     assert lib.blasst_select_workspace_bytes(0, 4, 2, 256, 256, 128, 128, 128) == 0
 
 
