@@ -26,7 +26,8 @@ __all__ = [
     "blasst_lse_merge", "blasst_check", "blasst_selftest_exp2",
     "blasst_decode_noalloc", "blasst_decode_noalloc_max_bytes", "blasst_status_string", "blasst_version",
     "blasst_bwd", "blasst_bwd_workspace_bytes", "blasst_select_blocks",
-    "blasst_select_workspace_bytes", "select_blocks",
+    "blasst_select_workspace_bytes", "select_blocks", "blasst_decode_mla",
+    "blasst_decode_mla_workspace_bytes", "attention_decode_mla",
     "attention_prefill", "attention_backward", "attention_decode", "new_stats", "stats_dict",
     "BLASST_OK", "BLASST_EINVAL", "BLASST_EUNSUPPORTED", "BLASST_ECUDA", "BLASST_ETIMEOUT",
     "BLASST_EWORKSPACE", "BLASST_BF16", "BLASST_FP32",
@@ -110,6 +111,10 @@ def load_library(path: str | None = None):
         lib.blasst_fwd.restype = i
         lib.blasst_fwd_ex.argtypes = [C.POINTER(_FwdArgs)]
         lib.blasst_fwd_ex.restype = i
+        lib.blasst_decode_mla.argtypes = [vp, vp, vp, vp, i, i, i, f, i, f, vp, sz, vp, vp, vp]
+        lib.blasst_decode_mla.restype = i
+        lib.blasst_decode_mla_workspace_bytes.argtypes = [i, i, i]
+        lib.blasst_decode_mla_workspace_bytes.restype = sz
         lib.blasst_select_blocks.argtypes = [C.POINTER(_SelectArgs)]
         lib.blasst_select_blocks.restype = i
         lib.blasst_select_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
@@ -225,6 +230,23 @@ def blasst_bwd(q, k, v, o, dout, lse, dq, dk, dv, *, causal: bool, Br: int, Bc: 
                     float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
                     _stream(stream))
     _check(load_library().blasst_bwd(C.byref(args)), "blasst_bwd")
+
+
+def blasst_decode_mla_workspace_bytes(B: int, H: int, num_splits: int) -> int:
+    return int(load_library().blasst_decode_mla_workspace_bytes(B, H, num_splits))
+
+
+def blasst_decode_mla(q, cache, o, lse, *, lam: float, num_splits: int, workspace, scale: float = 0.0,
+                      skip_mask_out=None, stats_out=None, stream=None):
+    """The C entry point of the same name. q [B,H,576], cache [B,L,576] bf16;
+    o [B,H,512] bf16, lse [B,H] fp32; workspace a uint8 CUDA tensor."""
+    B, H = q.shape[0], q.shape[1]
+    L = cache.shape[1]
+    rc = load_library().blasst_decode_mla(
+        _ptr(q), _ptr(cache), _ptr(o), _ptr(lse), B, H, L, float(lam), num_splits, float(scale),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(skip_mask_out),
+        _ptr(stats_out), _stream(stream))
+    _check(rc, "blasst_decode_mla")
 
 
 def blasst_select_workspace_bytes(B, Hq, Hkv, Lq, Lkv, d, Br, Bc) -> int:
@@ -360,6 +382,27 @@ def select_blocks(q, k, *, causal=True, Br=128, Bc=128, tau=0.2, gamma=0.9, scal
     blasst_select_blocks(q, k, mask, causal=causal, Br=Br, Bc=Bc, tau=tau, gamma=gamma,
                          workspace=workspace, scale=scale, cstruct_out=cs, stream=stream)
     return mask, cs
+
+
+def attention_decode_mla(q, cache, *, lam=0.0, num_splits=32, scale=0.0, with_mask=False,
+                         stats=None, stream=None, workspace=None):
+    """MLA-shaped decode (one latent KV head, 576-wide rows, 512-wide values):
+    allocate outputs and workspace with torch and run blasst_decode_mla.
+    Returns (o [B,H,512] bf16, lse [B,H], mask [B,H,ceil(L/64)] or None)."""
+    import torch
+    B, H = q.shape[0], q.shape[1]
+    L = cache.shape[1]
+    o = torch.empty((B, H, 512), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(blasst_decode_mla_workspace_bytes(B, H, num_splits),
+                                dtype=torch.uint8, device=q.device)
+    mask = None
+    if with_mask:
+        mask = torch.empty((B, H, -(-L // 64)), dtype=torch.uint8, device=q.device)
+    blasst_decode_mla(q, cache, o, lse, lam=lam, num_splits=num_splits, workspace=workspace,
+                      scale=scale, skip_mask_out=mask, stats_out=stats, stream=stream)
+    return o, lse, mask
 
 
 def attention_decode(q, k_cache, v_cache, *, lam=0.0, Bc=128, num_splits=64, with_mask=False,

@@ -15,6 +15,7 @@
 
 #include "../../include/blasst.h"
 #include "bwd_sm100.cuh"
+#include "decode_mla_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "prefill_f32_sm100.cuh"
 #include "prefill_sm100.cuh"
@@ -562,6 +563,64 @@ int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void*
   int rc = dispatch_decode(d, Bc, g, mk, mv, p, s);
   if (rc != BLASST_OK) return rc;
   return blasst_lse_merge(p.o_parts, p.lse_parts, o, lse, B * Hq, d, num_splits, BLASST_BF16,
+                          stream);
+}
+
+size_t blasst_decode_mla_workspace_bytes(int B, int H, int num_splits) {
+  if (B <= 0 || H <= 0 || num_splits <= 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * num_splits;
+  return rows * (blasst::MlaCfg::DV + 1) * sizeof(float);
+}
+
+int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int B, int H, int L,
+                      float lambda, int num_splits, float scale, void* workspace,
+                      size_t workspace_bytes, uint8_t* skip_mask_out, blasst_stats* stats_out,
+                      void* stream) {
+  using C = blasst::MlaCfg;
+  if (!q || !cache || !o || !lse) return BLASST_EINVAL;
+  if (!aligned16(q) || !aligned16(cache) || !aligned16(o) || !aligned16(lse)) return BLASST_EINVAL;
+  if (B <= 0 || H <= 0 || L <= 0 || num_splits <= 0) return BLASST_EINVAL;
+  if (!(lambda >= 0.0f && lambda < 1.0f)) return BLASST_EINVAL;
+  if (H % C::HG != 0) return BLASST_EUNSUPPORTED;
+  if (num_splits > 65535 || B > 65535 || static_cast<long long>(B) * num_splits * (H / C::HG) >
+                                            0x7fffffffll)
+    return BLASST_EINVAL;
+  const size_t need = blasst_decode_mla_workspace_bytes(B, H, num_splits);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return BLASST_EWORKSPACE;
+  int* err = error_word();
+  if (!err) return BLASST_ECUDA;
+  const size_t rows = static_cast<size_t>(B) * H * num_splits;
+  blasst::MlaParams p{};
+  p.o_parts = static_cast<float*>(workspace);
+  p.lse_parts = static_cast<float*>(workspace) + rows * C::DV;
+  p.mask = skip_mask_out;
+  p.stats = stats_out;
+  p.err = err;
+  p.B = B;
+  p.H = H;
+  p.L = L;
+  p.S = num_splits;
+  {
+    const long long per = (static_cast<long long>(L) + num_splits - 1) / num_splits;
+    p.Ls = static_cast<int>(((per + C::BC - 1) / C::BC) * C::BC);
+  }
+  p.nKt = (L + C::BC - 1) / C::BC;
+  const double sc = scale > 0.0f ? static_cast<double>(scale)
+                                 : 1.0 / std::sqrt(static_cast<double>(C::DQK));
+  p.scale_log2 = static_cast<float>(sc * 1.4426950408889634);
+  p.log2_lambda = log2_lambda_of(lambda);
+  p.timeout_ns = kTimeoutNs;
+  CUtensorMap mq, mc;
+  const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&mq, q, dt, 2, C::DQK, H, B, C::HG) || !make_map(&mc, cache, dt, 2, C::DQK, L, B, C::BC))
+    return BLASST_ECUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (set_smem(blasst::blasst_decode_mla_kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
+  const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * num_splits * (H / C::HG));
+  blasst::blasst_decode_mla_kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(mq, mc, p);
+  int rc = cuda_status(cudaGetLastError());
+  if (rc != BLASST_OK) return rc;
+  return blasst_lse_merge(p.o_parts, p.lse_parts, o, lse, B * H, C::DV, num_splits, BLASST_BF16,
                           stream);
 }
 

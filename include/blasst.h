@@ -275,6 +275,35 @@ BLASST_API int blasst_decode_noalloc(const void* q, const void* k_cache, const v
 /* Size in bytes of the fixed array blasst_decode_noalloc uses. */
 BLASST_API size_t blasst_decode_noalloc_max_bytes(void);
 
+/* Split-KV decode with softmax thresholding for multi-head latent attention
+ * (MLA) caches, in the absorbed form: every query head has a 576-wide query
+ * (512 latent + 64 rotary dims); every cached token one 576-wide row c shared
+ * by all heads (latent in dims 0-511, rotary key in 512-575); scores
+ * scale * q_h . c_j; the output o_h = sum_j p_hj c_j[0:512]. That is softmax
+ * attention with one KV head, K = c, V = c[:, 0:512]. The post ("BLASST:
+ * Dynamic BLocked Attention Sparsity via Softmax Thresholding", paragraph 9
+ * after the headline) says only that the method is compatible with MLA; the
+ * skip rule here is the decode one, per (head, 64-key block), the first
+ * block of each split always computed, then the log-sum-exp merge of
+ * blasst_decode. V is part of the cached rows already read for the scores, so
+ * a skip saves no bytes; a block's P V is skipped for a group of 16 heads
+ * when every head of the group drops it.
+ *   q          [B, H, 576] bf16;  cache [B, L, 576] bf16.
+ *   o          [B, H, 512] bf16;  lse [B, H] fp32 (natural log).
+ *   H          a multiple of 16.
+ *   num_splits splits of ceil(ceil(L/S)/64)*64 keys each.
+ *   scale      score scale; <= 0 selects 1/sqrt(576).
+ *   workspace  >= blasst_decode_mla_workspace_bytes(B, H, num_splits).
+ *   skip_mask_out nullable uint8 [B, H, ceil(L/64)] (0 computed, 1 skipped).
+ *   stats_out  nullable device blasst_stats. */
+BLASST_API int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int B, int H,
+                                 int L, float lambda, int num_splits, float scale, void* workspace,
+                                 size_t workspace_bytes, uint8_t* skip_mask_out,
+                                 blasst_stats* stats_out, void* stream);
+
+/* Workspace bytes of blasst_decode_mla: fp32 [B, H, S, 512] + [B, H, S]. */
+BLASST_API size_t blasst_decode_mla_workspace_bytes(int B, int H, int num_splits);
+
 /* Log-sum-exp merge of split partials (the second half of blasst_decode):
  *   o_parts [n_rows, num_splits, d] fp32, normalised per split;
  *   lse_parts [n_rows, num_splits] fp32, -inf marks an empty split;

@@ -149,6 +149,27 @@ def test_select_rejects_bad_arguments_without_a_gpu(lib, bad, code):
     assert _sel(lib, **bad) == code
 
 
+def test_decode_mla_workspace_and_rejections(lib):
+    ws = lib.blasst_decode_mla_workspace_bytes(8, 128, 32)
+    assert ws == 8 * 128 * 32 * (512 + 1) * 4
+    vp = 0x10000
+    f = C.c_float
+    # heads not a multiple of 16
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 24, 4096, f(1e-3), 4, f(0.0), vp, 1 << 30,
+                                 None, None, None) == -2
+    # lambda out of range, bad sizes, misaligned pointers
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 32, 4096, f(1.0), 4, f(0.0), vp, 1 << 30,
+                                 None, None, None) == -1
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 0, 32, 4096, f(1e-3), 4, f(0.0), vp, 1 << 30,
+                                 None, None, None) == -1
+    assert lib.blasst_decode_mla(vp + 8, vp, vp, vp, 2, 32, 4096, f(1e-3), 4, f(0.0), vp, 1 << 30,
+                                 None, None, None) == -1
+    # workspace too small
+    need = lib.blasst_decode_mla_workspace_bytes(2, 32, 4)
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 32, 4096, f(1e-3), 4, f(0.0), vp, need - 16,
+                                 None, None, None) == -5
+
+
 def test_decode_workspace_and_rejections(lib):
     ws = lib.blasst_decode_workspace_bytes(16, 32, 128, 64)
     assert ws == 16 * 32 * 64 * (128 + 1) * 4
