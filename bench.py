@@ -234,6 +234,52 @@ def measure_prefill(w, lam, steps, warmup, device, stream, flush_buf, pre=None, 
                      v_blocks=sd["v_blocks_loaded"], bytes_loaded=sd["bytes_loaded"])
 
 
+def measure_decode_mla(w, steps, device, stream, flush_buf, peaks):
+    """MLA decode at lambda = 0 and at the workload's lambda: time, executed
+    TFLOP/s against the bf16 peak, bytes against the copy bandwidth."""
+    import torch
+    import synth
+    import dynamic_block_sparse_tiled_b200 as bl
+    inp = synth.generate(w)
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    q, c = to(inp.q[:, :, 0, :]), to(inp.k[:, 0])
+    del inp
+    ws = torch.empty(bl.blasst_decode_mla_workspace_bytes(w.B, w.Hq, w.num_splits), dtype=torch.uint8,
+                     device=device)
+    o = torch.empty((w.B, w.Hq, 512), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
+    mask = torch.empty((w.B, w.Hq, -(-w.Lkv // 64)), dtype=torch.uint8, device=device)
+    res = {}
+    for lam in (0.0, w.lambdas[0]):
+        st = bl.new_stats(device)
+        bl.blasst_decode_mla(q, c, o, lse, lam=lam, num_splits=w.num_splits, workspace=ws,
+                             skip_mask_out=mask, stats_out=st, stream=stream)
+        stream.synchronize()
+        rc = bl.blasst_check(stream)
+        if rc != 0:
+            raise RuntimeError(bl.blasst_status_string(rc))
+        sd = bl.stats_dict(st)
+        run = lambda: bl.blasst_decode_mla(q, c, o, lse, lam=lam, num_splits=w.num_splits,
+                                           workspace=ws, stream=stream)
+        ms = statistics.mean(time_calls(run, steps, 3, stream, flush_buf))
+        tf = sd["mma_flops"] / (ms * 1e-3) / 1e12
+        gbs = sd["bytes_loaded"] / (ms * 1e-3) / 1e9
+        res[str(lam)] = dict(ms=ms, executed_tflops=tf, gbs=gbs,
+                             skip_frac=sd["tiles_skipped"] / max(sd["tiles_visited"], 1))
+    base = res["0.0"]["ms"]
+    for v in res.values():
+        v["speedup_vs_lambda0"] = base / v["ms"]
+    top = res[str(w.lambdas[0])]
+    res["roofline"] = dict(bound="tensor", achieved=top["executed_tflops"],
+                           peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                           frac=top["executed_tflops"] / peaks["bf16_tflops"],
+                           hbm_frac=top["gbs"] / peaks["hbm_gbs"],
+                           note="mma.sync m16n8k16 tiles (16 heads per CTA); the cache is read "
+                                "once from HBM, re-read from L2 by each of the 8 head groups")
+    res["config"] = dict(B=w.B, H=w.Hq, L=w.Lkv, num_splits=w.num_splits, amplitude=w.amp)
+    return res
+
+
 def backward_pairs(w, mask):
     """(64-row query tile, 128-key block) pairs the backward computes, from
     the forward's decisions (uint8 [B, Hq, nQt, nKt], 0 = computed)."""
@@ -469,6 +515,12 @@ def run_case(name, lam, calls, overrides=()):
         to = lambda a: torch.from_numpy(a).cuda()
     q, k, v = to(inp.q), to(inp.k), to(inp.v)
     del inp
+    if w.num_splits and w.d == 576:  # MLA-shaped decode: one latent head, values = dims 0-511
+        qm, cm = q[:, :, 0, :].contiguous(), k[:, 0].contiguous()
+        del q, k, v
+        for _ in range(calls):
+            bl.attention_decode_mla(qm, cm, lam=lam, num_splits=w.num_splits)
+        calls = 0
     if select:
         for _ in range(calls):
             bl.select_blocks(q, k, causal=w.causal, Br=w.Br, Bc=w.Bc, tau=SEL_TAU, gamma=SEL_GAMMA)
@@ -686,6 +738,13 @@ def main():
             del ps, smask, sws
             torch.cuda.empty_cache()
         extra["selector_32k"] = dict(tau=SEL_TAU, gamma=SEL_GAMMA, **sel)
+
+        # MLA-shaped decode (latent cache, 128 heads), literal and calibrated
+        mla = {}
+        for wn in ("decode_mla_64k", "decode_mla_64k_a12"):
+            mla[wn] = measure_decode_mla(synth.CONFIGS[wn], max(5, args.steps), device, stream,
+                                         flush_buf, peaks)
+        extra["decode_mla_64k"] = mla
 
         # backward with the forward's decisions held fixed, 32K workload
         pb = Prefill(w, device)
