@@ -234,7 +234,7 @@ def measure_prefill(w, lam, steps, warmup, device, stream, flush_buf, pre=None, 
                      v_blocks=sd["v_blocks_loaded"], bytes_loaded=sd["bytes_loaded"])
 
 
-def measure_decode_mla(w, steps, device, stream, flush_buf, peaks):
+def measure_decode_mla(w, steps, device, stream, flush_buf, peaks, Bc=32):
     """MLA decode at lambda = 0 and at the workload's lambda: time, executed
     TFLOP/s against the bf16 peak, bytes against the copy bandwidth."""
     import torch
@@ -248,18 +248,18 @@ def measure_decode_mla(w, steps, device, stream, flush_buf, peaks):
                      device=device)
     o = torch.empty((w.B, w.Hq, 512), dtype=torch.bfloat16, device=device)
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
-    mask = torch.empty((w.B, w.Hq, -(-w.Lkv // 64)), dtype=torch.uint8, device=device)
+    mask = torch.empty((w.B, w.Hq, -(-w.Lkv // Bc)), dtype=torch.uint8, device=device)
     res = {}
     for lam in (0.0, w.lambdas[0]):
         st = bl.new_stats(device)
-        bl.blasst_decode_mla(q, c, o, lse, lam=lam, num_splits=w.num_splits, workspace=ws,
+        bl.blasst_decode_mla(q, c, o, lse, lam=lam, Bc=Bc, num_splits=w.num_splits, workspace=ws,
                              skip_mask_out=mask, stats_out=st, stream=stream)
         stream.synchronize()
         rc = bl.blasst_check(stream)
         if rc != 0:
             raise RuntimeError(bl.blasst_status_string(rc))
         sd = bl.stats_dict(st)
-        run = lambda: bl.blasst_decode_mla(q, c, o, lse, lam=lam, num_splits=w.num_splits,
+        run = lambda: bl.blasst_decode_mla(q, c, o, lse, lam=lam, Bc=Bc, num_splits=w.num_splits,
                                            workspace=ws, stream=stream)
         ms = statistics.mean(time_calls(run, steps, 3, stream, flush_buf))
         tf = sd["mma_flops"] / (ms * 1e-3) / 1e12
@@ -274,9 +274,11 @@ def measure_decode_mla(w, steps, device, stream, flush_buf, peaks):
                            peak=peaks["bf16_tflops"], unit="TFLOP/s",
                            frac=top["executed_tflops"] / peaks["bf16_tflops"],
                            hbm_frac=top["gbs"] / peaks["hbm_gbs"],
-                           note="mma.sync m16n8k16 tiles (16 heads per CTA); the cache is read "
-                                "once from HBM, re-read from L2 by each of the 8 head groups")
-    res["config"] = dict(B=w.B, H=w.Hq, L=w.Lkv, num_splits=w.num_splits, amplitude=w.amp)
+                           note=("tcgen05, 128 heads per CTA, two CTAs per split (one output half "
+                                 "each, both form the scores)") if Bc == 32 else
+                                ("mma.sync m16n8k16 tiles (16 heads per CTA); the cache is read "
+                                 "once from HBM, re-read from L2 by each of the 8 head groups"))
+    res["config"] = dict(B=w.B, H=w.Hq, L=w.Lkv, num_splits=w.num_splits, amplitude=w.amp, Bc=Bc)
     return res
 
 
@@ -743,7 +745,10 @@ def main():
         mla = {}
         for wn in ("decode_mla_64k", "decode_mla_64k_a12"):
             mla[wn] = measure_decode_mla(synth.CONFIGS[wn], max(5, args.steps), device, stream,
-                                         flush_buf, peaks)
+                                         flush_buf, peaks, Bc=32)
+        mla["decode_mla_64k_mma_sync_bc64"] = measure_decode_mla(
+            synth.CONFIGS["decode_mla_64k"], max(5, args.steps), device, stream, flush_buf, peaks,
+            Bc=64)
         extra["decode_mla_64k"] = mla
 
         # backward with the forward's decisions held fixed, 32K workload

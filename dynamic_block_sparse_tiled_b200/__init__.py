@@ -111,7 +111,7 @@ def load_library(path: str | None = None):
         lib.blasst_fwd.restype = i
         lib.blasst_fwd_ex.argtypes = [C.POINTER(_FwdArgs)]
         lib.blasst_fwd_ex.restype = i
-        lib.blasst_decode_mla.argtypes = [vp, vp, vp, vp, i, i, i, f, i, f, vp, sz, vp, vp, vp]
+        lib.blasst_decode_mla.argtypes = [vp, vp, vp, vp, i, i, i, f, i, i, f, vp, sz, vp, vp, vp]
         lib.blasst_decode_mla.restype = i
         lib.blasst_decode_mla_workspace_bytes.argtypes = [i, i, i]
         lib.blasst_decode_mla_workspace_bytes.restype = sz
@@ -236,14 +236,14 @@ def blasst_decode_mla_workspace_bytes(B: int, H: int, num_splits: int) -> int:
     return int(load_library().blasst_decode_mla_workspace_bytes(B, H, num_splits))
 
 
-def blasst_decode_mla(q, cache, o, lse, *, lam: float, num_splits: int, workspace, scale: float = 0.0,
-                      skip_mask_out=None, stats_out=None, stream=None):
+def blasst_decode_mla(q, cache, o, lse, *, lam: float, Bc: int, num_splits: int, workspace,
+                      scale: float = 0.0, skip_mask_out=None, stats_out=None, stream=None):
     """The C entry point of the same name. q [B,H,576], cache [B,L,576] bf16;
     o [B,H,512] bf16, lse [B,H] fp32; workspace a uint8 CUDA tensor."""
     B, H = q.shape[0], q.shape[1]
     L = cache.shape[1]
     rc = load_library().blasst_decode_mla(
-        _ptr(q), _ptr(cache), _ptr(o), _ptr(lse), B, H, L, float(lam), num_splits, float(scale),
+        _ptr(q), _ptr(cache), _ptr(o), _ptr(lse), B, H, L, float(lam), Bc, num_splits, float(scale),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(skip_mask_out),
         _ptr(stats_out), _stream(stream))
     _check(rc, "blasst_decode_mla")
@@ -384,14 +384,18 @@ def select_blocks(q, k, *, causal=True, Br=128, Bc=128, tau=0.2, gamma=0.9, scal
     return mask, cs
 
 
-def attention_decode_mla(q, cache, *, lam=0.0, num_splits=32, scale=0.0, with_mask=False,
+def attention_decode_mla(q, cache, *, lam=0.0, num_splits=32, Bc=None, scale=0.0, with_mask=False,
                          stats=None, stream=None, workspace=None):
     """MLA-shaped decode (one latent KV head, 576-wide rows, 512-wide values):
-    allocate outputs and workspace with torch and run blasst_decode_mla.
-    Returns (o [B,H,512] bf16, lse [B,H], mask [B,H,ceil(L/64)] or None)."""
+    allocate outputs and workspace with torch and run blasst_decode_mla
+    (Bc: 32 = the tensor-core kernel, the default when H is a multiple of
+    128; 64 = the mma.sync kernel). Returns (o [B,H,512] bf16, lse [B,H],
+    mask [B,H,ceil(L/Bc)] or None)."""
     import torch
     B, H = q.shape[0], q.shape[1]
     L = cache.shape[1]
+    if Bc is None:
+        Bc = 32 if H % 128 == 0 else 64
     o = torch.empty((B, H, 512), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
     if workspace is None:
@@ -399,8 +403,8 @@ def attention_decode_mla(q, cache, *, lam=0.0, num_splits=32, scale=0.0, with_ma
                                 dtype=torch.uint8, device=q.device)
     mask = None
     if with_mask:
-        mask = torch.empty((B, H, -(-L // 64)), dtype=torch.uint8, device=q.device)
-    blasst_decode_mla(q, cache, o, lse, lam=lam, num_splits=num_splits, workspace=workspace,
+        mask = torch.empty((B, H, -(-L // Bc)), dtype=torch.uint8, device=q.device)
+    blasst_decode_mla(q, cache, o, lse, lam=lam, Bc=Bc, num_splits=num_splits, workspace=workspace,
                       scale=scale, skip_mask_out=mask, stats_out=stats, stream=stream)
     return o, lse, mask
 

@@ -573,15 +573,18 @@ size_t blasst_decode_mla_workspace_bytes(int B, int H, int num_splits) {
 }
 
 int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int B, int H, int L,
-                      float lambda, int num_splits, float scale, void* workspace,
+                      float lambda, int Bc, int num_splits, float scale, void* workspace,
                       size_t workspace_bytes, uint8_t* skip_mask_out, blasst_stats* stats_out,
                       void* stream) {
   using C = blasst::MlaCfg;
+  using T = blasst::mla::TcCfg;
   if (!q || !cache || !o || !lse) return BLASST_EINVAL;
   if (!aligned16(q) || !aligned16(cache) || !aligned16(o) || !aligned16(lse)) return BLASST_EINVAL;
   if (B <= 0 || H <= 0 || L <= 0 || num_splits <= 0) return BLASST_EINVAL;
   if (!(lambda >= 0.0f && lambda < 1.0f)) return BLASST_EINVAL;
-  if (H % C::HG != 0) return BLASST_EUNSUPPORTED;
+  if (Bc != T::BC && Bc != C::BC) return BLASST_EUNSUPPORTED;
+  const bool tc = Bc == T::BC;  // tcgen05 kernel: 32-key blocks, groups of 128 heads
+  if (H % (tc ? T::HM : C::HG) != 0) return BLASST_EUNSUPPORTED;
   if (num_splits > 65535 || B > 65535 || static_cast<long long>(B) * num_splits * (H / C::HG) >
                                             0x7fffffffll)
     return BLASST_EINVAL;
@@ -602,9 +605,9 @@ int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int
   p.S = num_splits;
   {
     const long long per = (static_cast<long long>(L) + num_splits - 1) / num_splits;
-    p.Ls = static_cast<int>(((per + C::BC - 1) / C::BC) * C::BC);
+    p.Ls = static_cast<int>(((per + Bc - 1) / Bc) * Bc);
   }
-  p.nKt = (L + C::BC - 1) / C::BC;
+  p.nKt = (L + Bc - 1) / Bc;
   const double sc = scale > 0.0f ? static_cast<double>(scale)
                                  : 1.0 / std::sqrt(static_cast<double>(C::DQK));
   p.scale_log2 = static_cast<float>(sc * 1.4426950408889634);
@@ -612,12 +615,20 @@ int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int
   p.timeout_ns = kTimeoutNs;
   CUtensorMap mq, mc;
   const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!make_map(&mq, q, dt, 2, C::DQK, H, B, C::HG) || !make_map(&mc, cache, dt, 2, C::DQK, L, B, C::BC))
+  if (!make_map(&mq, q, dt, 2, C::DQK, H, B, tc ? T::HM : C::HG) ||
+      !make_map(&mc, cache, dt, 2, C::DQK, L, B, Bc))
     return BLASST_ECUDA;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (set_smem(blasst::blasst_decode_mla_kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
-  const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * num_splits * (H / C::HG));
-  blasst::blasst_decode_mla_kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(mq, mc, p);
+  if (tc) {
+    if (set_smem(blasst::blasst_decode_mla_tc_kernel, T::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
+    const unsigned grid =
+        static_cast<unsigned>(static_cast<long long>(B) * num_splits * (H / T::HM) * 2);
+    blasst::blasst_decode_mla_tc_kernel<<<grid, T::NTHREADS, T::SMEM_BYTES, s>>>(mq, mc, p);
+  } else {
+    if (set_smem(blasst::blasst_decode_mla_kernel, C::SMEM_BYTES) != cudaSuccess) return BLASST_ECUDA;
+    const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * num_splits * (H / C::HG));
+    blasst::blasst_decode_mla_kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(mq, mc, p);
+  }
   int rc = cuda_status(cudaGetLastError());
   if (rc != BLASST_OK) return rc;
   return blasst_lse_merge(p.o_parts, p.lse_parts, o, lse, B * H, C::DV, num_splits, BLASST_BF16,

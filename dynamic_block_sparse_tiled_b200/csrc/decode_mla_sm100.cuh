@@ -320,4 +320,316 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core version for 128 heads per latent KV head (M = 128): tcgen05.mma
+// with the scores and the output in TMEM. The 128 x 512 fp32 output needs all
+// 512 TMEM columns, so two CTAs share a (sequence, split): both compute the
+// same scores and decisions, each accumulates one half of the 512 output
+// columns.
+//   warps 0-3  one head per thread (TMEM lane): the block's scores, the vote,
+//              lazy rescaling (the reference max moves only when it has grown
+//              by more than 8 in log2 units; then the O half in TMEM is scaled
+//              after the previous P V has completed), P (bf16) over S;
+//   warp 4     TMA: Q once (nine [128 heads][64 dims] boxes), 32-key blocks of
+//              the cache through a 2-stage ring;
+//   warp 5     tcgen05 issuer and TMEM owner: S = Q C^T (M 128, N 32, K 576)
+//              into one of two S buffers, O_half += P V_half (M 128, N 256,
+//              K 32, P from TMEM, V MN-major from the stage), skipped when no
+//              head of the 128 keeps the block.
+namespace mla {
+struct TcCfg {
+  static constexpr int DQK = 576, DV = 512, BC = 32, HM = 128;
+  static constexpr int NTHREADS = 192;
+  static constexpr int NBOX = DQK / 64;             // 9
+  static constexpr int Q_BOX = HM * 128;            // 16 KB
+  static constexpr int Q_BYTES = NBOX * Q_BOX;      // 144 KB
+  static constexpr int KV_BOX = BC * 128;           // 4 KB
+  static constexpr int KV_BYTES = NBOX * KV_BOX;    // 36 KB
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_BAR = OFF_K + 2 * KV_BYTES;
+  static constexpr int B_Q = 0, B_KF = 1, B_KE = 3, B_SF = 5, B_PR = 7, B_PVD = 9, B_DRAIN = 11;
+  static constexpr int NBAR = 12;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  // misc words: [0] tmem base, [1] abort, [2] always 0, [4..5] block kept by some head (per S buffer)
+  static constexpr int MISC_BYTES = 64;
+  static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+  static constexpr int S_COL = 0;    // S buffer b at 32 b (P: first 16 columns)
+  static constexpr int O_COL = 256;  // this CTA's 256 output columns
+  static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32acc(128, BC, false, false);
+  static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32acc(128, 256, false, true);
+  static constexpr float TAU = 8.0f;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+}  // namespace mla
+
+__global__ void __launch_bounds__(192, 1)
+    blasst_decode_mla_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                const __grid_constant__ CUtensorMap tmC, const MlaParams p) {
+  using C = mla::TcCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = ptx::smem_u32(smem);
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = misc + 1;
+  auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // (sequence, split, head group of 128, half of the output columns)
+  const int NG = p.H / C::HM;
+  const int half = static_cast<int>(blockIdx.x) & 1;
+  const int rest = static_cast<int>(blockIdx.x) >> 1;
+  const int hgrp = rest % NG;
+  const int bs = rest / NG;
+  const int s = bs % p.S, b = bs / p.S;
+  const int key_lo = s * p.Ls;
+  const int key_hi = min(key_lo + p.Ls, p.L);
+  const int nblk = key_hi > key_lo ? (key_hi - key_lo + C::BC - 1) / C::BC : 0;
+  const size_t head0 = static_cast<size_t>(b) * p.H + hgrp * C::HM;
+
+  if (nblk == 0) {  // an empty split: nothing kept, lse = -inf
+    for (int e = tid; e < C::HM * 256; e += C::NTHREADS)
+      p.o_parts[((head0 + e / 256) * p.S + s) * C::DV + 256 * half + e % 256] = 0.0f;
+    if (half == 0 && tid < C::HM) p.lse_parts[(head0 + tid) * p.S + s] = -INFINITY;
+    return;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < C::NBAR; ++i) ptx::mbar_init(bar(i), (i == C::B_PR || i == C::B_PR + 1) ? 4 : 1);
+    for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(ptx::smem_u32(const_cast<int*>(misc)), C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+
+  if (warp == 4) {
+    // ======================= TMA producer ================================
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmQ);
+      ptx::prefetch_tmap(&tmC);
+      ptx::mbar_arrive_expect_tx(bar(C::B_Q), C::Q_BYTES);
+#pragma unroll
+      for (int bx = 0; bx < C::NBOX; ++bx)
+        ptx::tma_load_3d(sb + C::OFF_Q + bx * C::Q_BOX, &tmQ, bx * 64, hgrp * C::HM, b, bar(C::B_Q));
+      bool ok = true;
+      int n = 0;
+      for (; n < nblk && ok; ++n) {
+        const int st = n & 1;
+        if (n >= 2)
+          ok = ptx::mbar_wait(bar(C::B_KE + st), ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        ptx::mbar_arrive_expect_tx(bar(C::B_KF + st), C::KV_BYTES);
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          ptx::tma_load_3d(sb + C::OFF_K + st * C::KV_BYTES + bx * C::KV_BOX, &tmC, bx * 64,
+                           key_lo + n * C::BC, b, bar(C::B_KF + st));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
+        // let the copies in flight land before the CTA exits
+        ptx::mbar_wait(bar(C::B_Q), 0, &misc[2], p.timeout_ns);
+        for (int k = n - 2 < 0 ? 0 : n - 2; k < n; ++k)
+          ptx::mbar_wait(bar(C::B_KF + (k & 1)), (k >> 1) & 1, &misc[2], p.timeout_ns);
+      }
+    }
+  } else if (warp == 5) {
+    // ======================= tcgen05 issuer ==============================
+    if (lane == 0) {
+      bool ok = ptx::mbar_wait(bar(C::B_Q), 0, abort_flag, p.timeout_ns);
+      ptx::tc_fence_after();
+      const uint64_t q_desc = ptx::sw128_desc(sb + C::OFF_Q, 16, 1024);
+      const uint64_t k_desc = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
+      const uint64_t v_desc = ptx::sw128_desc(sb + C::OFF_K + 4 * half * C::KV_BOX, C::KV_BOX, 1024);
+      auto issue_s = [&](int n) -> bool {
+        const int st = n & 1;
+        if (!ptx::mbar_wait(bar(C::B_KF + st), (n >> 1) & 1, abort_flag, p.timeout_ns)) return false;
+        ptx::tc_fence_after();
+        const uint32_t d_tm = tmem + C::S_COL + st * C::BC;
+        const uint64_t kd = k_desc + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < C::DQK / 16; ++kk) {
+          const uint64_t a = q_desc + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
+          const uint64_t bd = kd + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
+          ptx::mma_ss(d_tm, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar(C::B_SF + st));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok && nblk > 1) ok = issue_s(1);
+      bool any_pv = false;
+      for (int n = 0; n < nblk && ok; ++n) {
+        const int st = n & 1;
+        ok = ptx::mbar_wait(bar(C::B_PR + st), (n >> 1) & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (misc[4 + st] != 0) {
+          // O_half += P V_half: K = the block's 32 keys in two steps of 16
+          const uint32_t p_tm = tmem + C::S_COL + st * C::BC;
+          const uint64_t vd = v_desc + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < C::BC / 16; ++kk)
+            ptx::mma_ts(tmem + C::O_COL, p_tm + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4),
+                        C::IDESC_PV, (any_pv || kk > 0) ? 1u : 0u);
+          any_pv = true;
+        }
+        ptx::mma_commit(bar(C::B_KE + st));   // the stage may be reloaded
+        ptx::mma_commit(bar(C::B_PVD + st));  // O holds every P V up to block n
+        if (n + 2 < nblk) ok = issue_s(n + 2);  // into S buffer st: P(n) was read above
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
+      }
+      ptx::mma_commit(bar(C::B_DRAIN));
+      ptx::mbar_wait(bar(C::B_DRAIN), 0, &misc[2], p.timeout_ns);
+    }
+  } else {
+    // ======================= softmax: one head per thread ===================
+    // Every exit from the loop and every optional wait is agreed by the four
+    // warps through barrier reductions, so no warp is left at a named barrier.
+    const int h = tid;  // TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float m = -INFINITY, mref = -INFINITY, l = 0.0f;
+    bool ok = true;
+    unsigned long long n_skip = 0, n_pv = 0;
+    for (int n = 0; n < nblk; ++n) {
+      const int st = n & 1;
+      ok = ptx::named_bar_and(2, 128, ptx::mbar_wait(bar(C::B_SF + st), (n >> 1) & 1, abort_flag,
+                                                      p.timeout_ns));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      uint32_t r[32];
+      ptx::tmem_ld32(tmem + lane_base + C::S_COL + st * C::BC, r);
+      ptx::tmem_wait_ld();
+      const int kbase = key_lo + n * C::BC;
+      float sv[32];
+      float mb = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        sv[c] = (kbase + c < key_hi) ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
+        mb = fmaxf(mb, sv[c]);
+      }
+      const bool skip = n > 0 && p.log2_lambda > -INFINITY && (mb - m < p.log2_lambda);
+      const float m_new = skip ? m : fmaxf(m, mb);
+      const bool move_ref = !skip && (mref == -INFINITY || m_new - mref > C::TAU);
+      const bool scale_o = move_ref && n > 0;  // O holds P V of earlier blocks
+      // some head must scale O: wait (all threads) for the previous P V
+      if (!ptx::named_bar_and(3, 128, !scale_o)) {
+        ok = ptx::named_bar_and(4, 128, ptx::mbar_wait(bar(C::B_PVD + ((n - 1) & 1)),
+                                                        ((n - 1) >> 1) & 1, abort_flag,
+                                                        p.timeout_ns));
+        if (!ok) break;
+        ptx::tc_fence_after();
+      }
+      // O rescale, warp-uniform: tcgen05.ld/st are warp-wide instructions, so
+      // every lane takes part when any head of the warp moves its reference
+      // (factor 1 for the others)
+      const float f_move = (mref == -INFINITY) ? 0.0f : ptx::ex2(mref - m_new);
+      if (__any_sync(0xffffffffu, scale_o)) {
+        const float fo = scale_o ? f_move : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tmem + lane_base + C::O_COL + 32 * c, o);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * fo);
+          ptx::tmem_st32(tmem + lane_base + C::O_COL + 32 * c, o);
+        }
+      }
+      uint32_t pk[16];
+      if (!skip) {
+        m = m_new;
+        if (move_ref) {
+          l *= f_move;
+          mref = m;
+        }
+        float ps = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float p0 = ptx::ex2(sv[2 * c] - mref), p1 = ptx::ex2(sv[2 * c + 1] - mref);
+          ps += p0 + p1;
+          pk[c] = ptx::pack_bf16x2(p0, p1);
+        }
+        l += ps;
+      } else {
+        ++n_skip;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pk[c] = 0u;
+      }
+      ptx::tmem_st16(tmem + lane_base + C::S_COL + st * C::BC, pk);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      // does any of the 128 heads keep the block? (P V is skipped otherwise)
+      const bool none = ptx::named_bar_and(1, 128, skip);
+      if (tid == 0) {
+        misc[4 + st] = none ? 0 : 1;
+        n_pv += none ? 0 : 1;
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::B_PR + st));
+      if (half == 0 && p.mask) p.mask[(head0 + h) * p.nKt + (key_lo / C::BC + n)] = skip ? 1 : 0;
+    }
+    if (ok) {
+      // the last P V, then this split's O half and lse
+      ok = ptx::named_bar_and(2, 128, ptx::mbar_wait(bar(C::B_PVD + ((nblk - 1) & 1)),
+                                                      ((nblk - 1) >> 1) & 1, abort_flag,
+                                                      p.timeout_ns));
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
+    } else {
+      ptx::tc_fence_after();
+      const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+      float* op = p.o_parts + ((head0 + h) * p.S + s) * C::DV + 256 * half;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t o[32];
+        ptx::tmem_ld32(tmem + lane_base + C::O_COL + 32 * c, o);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          reinterpret_cast<float4*>(op + 32 * c)[u] =
+              make_float4(__uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
+                          __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
+      }
+      if (half == 0)
+        p.lse_parts[(head0 + h) * p.S + s] =
+            l > 0.0f ? (mref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      if (p.stats) {
+        if (half == 0) atomicAdd(&p.stats->tiles_skipped, n_skip);
+        if (h == 0) {
+          const unsigned long long s_fl = 2ull * C::HM * C::BC * C::DQK;
+          const unsigned long long pv_fl = 2ull * C::HM * C::BC * 256;
+          atomicAdd(&p.stats->mma_flops, static_cast<unsigned long long>(nblk) * s_fl + n_pv * pv_fl);
+          atomicAdd(&p.stats->bytes_loaded,
+                    static_cast<unsigned long long>(nblk) * C::KV_BYTES + C::Q_BYTES);
+          if (half == 0) {
+            atomicAdd(&p.stats->tiles_visited, static_cast<unsigned long long>(nblk) * C::HM);
+            atomicAdd(&p.stats->v_blocks_loaded, static_cast<unsigned long long>(nblk));
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
 }  // namespace blasst

@@ -283,21 +283,23 @@ BLASST_API size_t blasst_decode_noalloc_max_bytes(void);
  * attention with one KV head, K = c, V = c[:, 0:512]. The post ("BLASST:
  * Dynamic BLocked Attention Sparsity via Softmax Thresholding", paragraph 9
  * after the headline) says only that the method is compatible with MLA; the
- * skip rule here is the decode one, per (head, 64-key block), the first
+ * skip rule here is the decode one, per (head, Bc-key block), the first
  * block of each split always computed, then the log-sum-exp merge of
  * blasst_decode. V is part of the cached rows already read for the scores, so
- * a skip saves no bytes; a block's P V is skipped for a group of 16 heads
- * when every head of the group drops it.
+ * a skip saves no bytes; a block's P V is skipped for a group of heads (128
+ * with Bc = 32, 16 with Bc = 64) when every head of the group drops it.
  *   q          [B, H, 576] bf16;  cache [B, L, 576] bf16.
  *   o          [B, H, 512] bf16;  lse [B, H] fp32 (natural log).
- *   H          a multiple of 16.
- *   num_splits splits of ceil(ceil(L/S)/64)*64 keys each.
+ *   Bc         decision block: 32 (tensor-core kernel, H a multiple of 128)
+ *              or 64 (mma.sync kernel, H a multiple of 16).
+ *   num_splits splits of ceil(ceil(L/S)/Bc)*Bc keys each.
  *   scale      score scale; <= 0 selects 1/sqrt(576).
  *   workspace  >= blasst_decode_mla_workspace_bytes(B, H, num_splits).
- *   skip_mask_out nullable uint8 [B, H, ceil(L/64)] (0 computed, 1 skipped).
+ *   skip_mask_out nullable uint8 [B, H, ceil(L/Bc)] (0 computed, 1 skipped).
  *   stats_out  nullable device blasst_stats. */
 BLASST_API int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int B, int H,
-                                 int L, float lambda, int num_splits, float scale, void* workspace,
+                                 int L, float lambda, int Bc, int num_splits, float scale,
+                                 void* workspace,
                                  size_t workspace_bytes, uint8_t* skip_mask_out,
                                  blasst_stats* stats_out, void* stream);
 

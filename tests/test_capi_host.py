@@ -154,19 +154,24 @@ def test_decode_mla_workspace_and_rejections(lib):
     assert ws == 8 * 128 * 32 * (512 + 1) * 4
     vp = 0x10000
     f = C.c_float
+    # decision blocks other than 32 / 64, and 32 with heads not a multiple of 128
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 128, 4096, f(1e-3), 128, 4, f(0.0), vp, 1 << 30,
+                                 None, None, None) == -2
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 64, 4096, f(1e-3), 32, 4, f(0.0), vp, 1 << 30,
+                                 None, None, None) == -2
     # heads not a multiple of 16
-    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 24, 4096, f(1e-3), 4, f(0.0), vp, 1 << 30,
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 24, 4096, f(1e-3), 64, 4, f(0.0), vp, 1 << 30,
                                  None, None, None) == -2
     # lambda out of range, bad sizes, misaligned pointers
-    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 32, 4096, f(1.0), 4, f(0.0), vp, 1 << 30,
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 32, 4096, f(1.0), 64, 4, f(0.0), vp, 1 << 30,
                                  None, None, None) == -1
-    assert lib.blasst_decode_mla(vp, vp, vp, vp, 0, 32, 4096, f(1e-3), 4, f(0.0), vp, 1 << 30,
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 0, 32, 4096, f(1e-3), 64, 4, f(0.0), vp, 1 << 30,
                                  None, None, None) == -1
-    assert lib.blasst_decode_mla(vp + 8, vp, vp, vp, 2, 32, 4096, f(1e-3), 4, f(0.0), vp, 1 << 30,
+    assert lib.blasst_decode_mla(vp + 8, vp, vp, vp, 2, 32, 4096, f(1e-3), 64, 4, f(0.0), vp, 1 << 30,
                                  None, None, None) == -1
     # workspace too small
     need = lib.blasst_decode_mla_workspace_bytes(2, 32, 4)
-    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 32, 4096, f(1e-3), 4, f(0.0), vp, need - 16,
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 32, 4096, f(1e-3), 64, 4, f(0.0), vp, need - 16,
                                  None, None, None) == -5
 
 

@@ -31,16 +31,17 @@ def _oracle_v(k):
     return v
 
 
-def run_mla(w, lam, seqs=None, heads=None):
-    """Run the GPU kernel on the whole workload; compare sequences ``seqs``
-    and heads ``heads`` (default all) with the oracle."""
+def run_mla(w, lam, seqs=None, heads=None, Bc=64):
+    """Run the GPU kernel on the whole workload (Bc = 32: the tensor-core
+    kernel, 64: the mma.sync kernel); compare sequences ``seqs`` and heads
+    ``heads`` (default all) with the oracle run with the same block size."""
     bl = _lib()
     inp = synth.generate(w)
     qd = parity.to_device(inp.q[:, :, 0, :].copy())   # [B, H, 576]
     cd = parity.to_device(inp.k[:, 0].copy())         # [B, L, 576]
     lam32 = float(np.float32(lam))
     st = bl.new_stats()
-    o, lse, mask = bl.attention_decode_mla(qd, cd, lam=lam32, num_splits=w.num_splits,
+    o, lse, mask = bl.attention_decode_mla(qd, cd, lam=lam32, num_splits=w.num_splits, Bc=Bc,
                                            with_mask=True, stats=st)
     assert bl.blasst_check() == 0
     seqs = range(w.B) if seqs is None else seqs
@@ -53,7 +54,7 @@ def run_mla(w, lam, seqs=None, heads=None):
     for b in seqs:
         qb = np.ascontiguousarray(inp.q[b:b + 1, heads])
         kb = np.ascontiguousarray(inp.k[b:b + 1])
-        ref = oracle.decode(qb, kb, _oracle_v(kb), lam=lam32, Bc=64, num_splits=w.num_splits)
+        ref = oracle.decode(qb, kb, _oracle_v(kb), lam=lam32, Bc=Bc, num_splits=w.num_splits)
         assert np.all(ref["o"][..., 512:] == 0.0)
         n_vis, n_dis, ok, dis = parity.compare_masks(mask_g[b:b + 1, heads], ref["mask"],
                                                      ref["margin"], lam32)
@@ -67,29 +68,35 @@ def run_mla(w, lam, seqs=None, heads=None):
     sd = bl.stats_dict(st)
     assert sd["tiles_visited"] == mask_g.size
     assert sd["tiles_skipped"] == int((mask_g == 1).sum())
-    print(w.name, lam, {k_: f"{v_:.2e}" for k_, v_ in worst.items()}, "skip", np.round(skip, 3))
+    print(w.name, f"Bc={Bc}", lam, {k_: f"{v_:.2e}" for k_, v_ in worst.items()}, "skip", np.round(skip, 3))
     return worst
 
 
 SMALL = [
-    ("mla_4k_a12", dict(B=2, Hq=32, Lkv=4096, num_splits=4, amp=12.0, n_needles=2)),
-    ("mla_4k_literal", dict(B=2, Hq=16, Lkv=4096, num_splits=4)),
-    ("mla_ragged", dict(B=2, Hq=16, Lkv=3000, num_splits=5, amp=12.0)),
-    ("mla_empty_splits", dict(B=1, Hq=16, Lkv=200, num_splits=8, amp=12.0)),
-    ("mla_h128", dict(B=1, Hq=128, Lkv=2048, num_splits=2, amp=12.0, n_needles=2)),
+    # name, overrides, decision block (32: tensor-core kernel, 64: mma.sync kernel)
+    ("mla_4k_a12", dict(B=2, Hq=32, Lkv=4096, num_splits=4, amp=12.0, n_needles=2), 64),
+    ("mla_4k_literal", dict(B=2, Hq=16, Lkv=4096, num_splits=4), 64),
+    ("mla_ragged", dict(B=2, Hq=16, Lkv=3000, num_splits=5, amp=12.0), 64),
+    ("mla_empty_splits", dict(B=1, Hq=16, Lkv=200, num_splits=8, amp=12.0), 64),
+    ("mla_h128", dict(B=1, Hq=128, Lkv=2048, num_splits=2, amp=12.0, n_needles=2), 64),
+    ("mla_h128_tc", dict(B=1, Hq=128, Lkv=2048, num_splits=2, amp=12.0, n_needles=2), 32),
+    ("mla_h128_tc_ragged", dict(B=2, Hq=128, Lkv=3000, num_splits=5, amp=12.0), 32),
+    ("mla_h128_tc_empty_splits", dict(B=1, Hq=128, Lkv=100, num_splits=8, amp=12.0), 32),
+    ("mla_h256_tc", dict(B=1, Hq=256, Lkv=1024, num_splits=2, amp=12.0), 32),
 ]
 
 
-@pytest.mark.parametrize("name,over", SMALL, ids=[s[0] for s in SMALL])
+@pytest.mark.parametrize("name,over,Bc", SMALL, ids=[s[0] for s in SMALL])
 @pytest.mark.parametrize("lam", [0.0, 1e-3, 1e-2])
-def test_mla_parity_small(name, over, lam):
-    run_mla(MLA.replace(name=name, **over), lam)
+def test_mla_parity_small(name, over, Bc, lam):
+    run_mla(MLA.replace(name=name, **over), lam, Bc=Bc)
 
 
 @pytest.mark.parametrize("cfg", ["decode_mla_64k", "decode_mla_64k_a12"])
-def test_mla_full_size_sampled(cfg):
+@pytest.mark.parametrize("Bc", [32, 64])
+def test_mla_full_size_sampled(cfg, Bc):
     """The benchmark's workload (B = 8, 128 heads, 64K keys, 32 splits),
     launched whole; two sequences and 32 of their heads compared with the
     oracle, the telemetry over everything."""
     w = synth.CONFIGS[cfg]
-    run_mla(w, 1e-3, seqs=(0, w.B - 1), heads=slice(48, 80))
+    run_mla(w, 1e-3, seqs=(0, w.B - 1), heads=slice(48, 80), Bc=Bc)
