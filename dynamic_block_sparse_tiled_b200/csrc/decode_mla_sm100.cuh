@@ -332,14 +332,18 @@ __global__ void __launch_bounds__(256, 1)
 //              after the previous P V has completed), P (bf16) over S;
 //   warp 4     TMA: Q once (nine [128 heads][64 dims] boxes), 32-key blocks of
 //              the cache through a 2-stage ring;
-//   warp 5     tcgen05 issuer and TMEM owner: S = Q C^T (M 128, N 32, K 576)
-//              into one of two S buffers, O_half += P V_half (M 128, N 256,
-//              K 32, P from TMEM, V MN-major from the stage), skipped when no
-//              head of the 128 keeps the block.
+//   warp 6     tcgen05 issuer of S = Q C^T (M 128, N 32, K 576) into one of
+//              two S buffers (once the block is loaded and the buffer's P has
+//              been read by its P V);
+//   warp 5     tcgen05 issuer of O_half += P V_half (M 128, N 256, K 32, P
+//              from TMEM, V MN-major from the stage), skipped when no head of
+//              the 128 keeps the block; owns the TMEM allocation. Two issuers
+//              so that a P V never waits behind a score product that waits
+//              for its block's load.
 namespace mla {
 struct TcCfg {
   static constexpr int DQK = 576, DV = 512, BC = 32, HM = 128;
-  static constexpr int NTHREADS = 192;
+  static constexpr int NTHREADS = 224;
   static constexpr int NBOX = DQK / 64;             // 9
   static constexpr int Q_BOX = HM * 128;            // 16 KB
   static constexpr int Q_BYTES = NBOX * Q_BOX;      // 144 KB
@@ -349,7 +353,9 @@ struct TcCfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_BAR = OFF_K + 2 * KV_BYTES;
   static constexpr int B_Q = 0, B_KF = 1, B_KE = 3, B_SF = 5, B_PR = 7, B_PVD = 9, B_DRAIN = 11;
-  static constexpr int NBAR = 12;
+  static constexpr int B_SFREE = 13;  // [2] P of the S buffer read by its P V
+  static constexpr int B_DRAIN_S = 15;  // the S issuer's drain
+  static constexpr int NBAR = 16;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // misc words: [0] tmem base, [1] abort, [2] always 0, [4..5] block kept by some head (per S buffer)
   static constexpr int MISC_BYTES = 64;
@@ -364,7 +370,7 @@ struct TcCfg {
 };
 }  // namespace mla
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
     blasst_decode_mla_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                 const __grid_constant__ CUtensorMap tmC, const MlaParams p) {
   using C = mla::TcCfg;
@@ -440,57 +446,64 @@ __global__ void __launch_bounds__(192, 1)
           ptx::mbar_wait(bar(C::B_KF + (k & 1)), (k >> 1) & 1, &misc[2], p.timeout_ns);
       }
     }
-  } else if (warp == 5) {
-    // ======================= tcgen05 issuer ==============================
+  } else if (warp == 5 || warp == 6) {
+    // ======================= tcgen05 issuers =============================
     if (lane == 0) {
       bool ok = ptx::mbar_wait(bar(C::B_Q), 0, abort_flag, p.timeout_ns);
       ptx::tc_fence_after();
-      const uint64_t q_desc = ptx::sw128_desc(sb + C::OFF_Q, 16, 1024);
-      const uint64_t k_desc = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
-      const uint64_t v_desc = ptx::sw128_desc(sb + C::OFF_K + 4 * half * C::KV_BOX, C::KV_BOX, 1024);
-      auto issue_s = [&](int n) -> bool {
-        const int st = n & 1;
-        if (!ptx::mbar_wait(bar(C::B_KF + st), (n >> 1) & 1, abort_flag, p.timeout_ns)) return false;
-        ptx::tc_fence_after();
-        const uint32_t d_tm = tmem + C::S_COL + st * C::BC;
-        const uint64_t kd = k_desc + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
+      if (warp == 6) {
+        // S(n) = Q C_n^T into S buffer n % 2
+        const uint64_t q_desc = ptx::sw128_desc(sb + C::OFF_Q, 16, 1024);
+        const uint64_t k_desc = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
+        for (int n = 0; n < nblk && ok; ++n) {
+          const int st = n & 1;
+          ok = ptx::mbar_wait(bar(C::B_KF + st), (n >> 1) & 1, abort_flag, p.timeout_ns);
+          if (ok && n >= 2)
+            ok = ptx::mbar_wait(bar(C::B_SFREE + st), ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          const uint32_t d_tm = tmem + C::S_COL + st * C::BC;
+          const uint64_t kd = k_desc + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < C::DQK / 16; ++kk) {
-          const uint64_t a = q_desc + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
-          const uint64_t bd = kd + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
-          ptx::mma_ss(d_tm, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::DQK / 16; ++kk) {
+            const uint64_t a = q_desc + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
+            const uint64_t bd = kd + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
+            ptx::mma_ss(d_tm, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          ptx::mma_commit(bar(C::B_SF + st));
         }
-        ptx::mma_commit(bar(C::B_SF + st));
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      if (ok && nblk > 1) ok = issue_s(1);
-      bool any_pv = false;
-      for (int n = 0; n < nblk && ok; ++n) {
-        const int st = n & 1;
-        ok = ptx::mbar_wait(bar(C::B_PR + st), (n >> 1) & 1, abort_flag, p.timeout_ns);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        if (misc[4 + st] != 0) {
-          // O_half += P V_half: K = the block's 32 keys in two steps of 16
-          const uint32_t p_tm = tmem + C::S_COL + st * C::BC;
-          const uint64_t vd = v_desc + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
+      } else {
+        // O_half += P(n) V_half(n); the commits free the stage, the S buffer
+        // and mark O as holding every P V up to block n
+        const uint64_t v_desc = ptx::sw128_desc(sb + C::OFF_K + 4 * half * C::KV_BOX, C::KV_BOX, 1024);
+        bool any_pv = false;
+        for (int n = 0; n < nblk && ok; ++n) {
+          const int st = n & 1;
+          ok = ptx::mbar_wait(bar(C::B_PR + st), (n >> 1) & 1, abort_flag, p.timeout_ns);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          if (misc[4 + st] != 0) {
+            const uint32_t p_tm = tmem + C::S_COL + st * C::BC;
+            const uint64_t vd = v_desc + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < C::BC / 16; ++kk)
-            ptx::mma_ts(tmem + C::O_COL, p_tm + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4),
-                        C::IDESC_PV, (any_pv || kk > 0) ? 1u : 0u);
-          any_pv = true;
+            for (int kk = 0; kk < C::BC / 16; ++kk)
+              ptx::mma_ts(tmem + C::O_COL, p_tm + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4),
+                          C::IDESC_PV, (any_pv || kk > 0) ? 1u : 0u);
+            any_pv = true;
+          }
+          ptx::mma_commit(bar(C::B_KE + st));
+          ptx::mma_commit(bar(C::B_SFREE + st));
+          ptx::mma_commit(bar(C::B_PVD + st));
         }
-        ptx::mma_commit(bar(C::B_KE + st));   // the stage may be reloaded
-        ptx::mma_commit(bar(C::B_PVD + st));  // O holds every P V up to block n
-        if (n + 2 < nblk) ok = issue_s(n + 2);  // into S buffer st: P(n) was read above
       }
       if (!ok) {
         *abort_flag = 1;
         if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
       }
-      ptx::mma_commit(bar(C::B_DRAIN));
-      ptx::mbar_wait(bar(C::B_DRAIN), 0, &misc[2], p.timeout_ns);
+      // drain: every MMA this thread issued has completed before TMEM is freed
+      const uint32_t drain = warp == 5 ? bar(C::B_DRAIN) : bar(C::B_DRAIN_S);
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, &misc[2], p.timeout_ns);
     }
   } else {
     // ======================= softmax: one head per thread ===================
