@@ -594,6 +594,7 @@ int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int
   if (!err) return BLASST_ECUDA;
   const size_t rows = static_cast<size_t>(B) * H * num_splits;
   blasst::MlaParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
   p.o_parts = static_cast<float*>(workspace);
   p.lse_parts = static_cast<float*>(workspace) + rows * C::DV;
   p.mask = skip_mask_out;

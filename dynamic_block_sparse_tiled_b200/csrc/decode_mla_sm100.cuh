@@ -38,6 +38,7 @@
 namespace blasst {
 
 struct MlaParams {
+  const __nv_bfloat16* q;  // [B, H, 576]
   float* o_parts;    // [B, H, S, 512]
   float* lse_parts;  // [B, H, S]
   uint8_t* mask;     // [B, H, nKt] or null: 0 computed, 1 skipped
@@ -345,22 +346,27 @@ struct TcCfg {
   static constexpr int DQK = 576, DV = 512, BC = 32, HM = 128;
   static constexpr int NTHREADS = 224;
   static constexpr int NBOX = DQK / 64;             // 9
+  static constexpr int QT_BOX = 4;                  // dims 0-255 of Q live in TMEM (TS operand)
   static constexpr int Q_BOX = HM * 128;            // 16 KB
-  static constexpr int Q_BYTES = NBOX * Q_BOX;      // 144 KB
+  static constexpr int Q_SM_BYTES = (NBOX - QT_BOX) * Q_BOX;  // dims 256-575 in shared memory, 80 KB
   static constexpr int KV_BOX = BC * 128;           // 4 KB
   static constexpr int KV_BYTES = NBOX * KV_BOX;    // 36 KB
+  static constexpr int NST = 4;                     // cache stages
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_BAR = OFF_K + 2 * KV_BYTES;
-  static constexpr int B_Q = 0, B_KF = 1, B_KE = 3, B_SF = 5, B_PR = 7, B_PVD = 9, B_DRAIN = 11;
-  static constexpr int B_SFREE = 13;  // [2] P of the S buffer read by its P V
-  static constexpr int B_DRAIN_S = 15;  // the S issuer's drain
-  static constexpr int NBAR = 16;
+  static constexpr int OFF_K = OFF_Q + Q_SM_BYTES;
+  static constexpr int OFF_BAR = OFF_K + NST * KV_BYTES;
+  static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + NST, B_SF = B_KE + NST;
+  static constexpr int B_PR = B_SF + 2, B_PVD = B_PR + 2, B_DRAIN = B_PVD + 2;
+  static constexpr int B_SFREE = B_DRAIN + 1;   // [2] P of the S buffer read by its P V
+  static constexpr int B_DRAIN_S = B_SFREE + 2; // the S issuer's drain
+  static constexpr int B_QT = B_DRAIN_S + 1;    // Q dims 0-255 written to TMEM (4 warps)
+  static constexpr int NBAR = B_QT + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // misc words: [0] tmem base, [1] abort, [2] always 0, [4..5] block kept by some head (per S buffer)
   static constexpr int MISC_BYTES = 64;
   static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
   static constexpr int S_COL = 0;    // S buffer b at 32 b (P: first 16 columns)
+  static constexpr int QT_COL = 64;  // Q dims 0-255, packed bf16 pairs: 128 columns
   static constexpr int O_COL = 256;  // this CTA's 256 output columns
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32acc(128, BC, false, false);
@@ -402,7 +408,8 @@ __global__ void __launch_bounds__(224, 1)
     return;
   }
   if (tid == 0) {
-    for (int i = 0; i < C::NBAR; ++i) ptx::mbar_init(bar(i), (i == C::B_PR || i == C::B_PR + 1) ? 4 : 1);
+    for (int i = 0; i < C::NBAR; ++i)
+      ptx::mbar_init(bar(i), (i == C::B_PR || i == C::B_PR + 1 || i == C::B_QT) ? 4 : 1);
     for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
     ptx::fence_mbar_init();
   }
@@ -420,16 +427,17 @@ __global__ void __launch_bounds__(224, 1)
     if (lane == 0) {
       ptx::prefetch_tmap(&tmQ);
       ptx::prefetch_tmap(&tmC);
-      ptx::mbar_arrive_expect_tx(bar(C::B_Q), C::Q_BYTES);
+      ptx::mbar_arrive_expect_tx(bar(C::B_Q), C::Q_SM_BYTES);
 #pragma unroll
-      for (int bx = 0; bx < C::NBOX; ++bx)
-        ptx::tma_load_3d(sb + C::OFF_Q + bx * C::Q_BOX, &tmQ, bx * 64, hgrp * C::HM, b, bar(C::B_Q));
+      for (int bx = C::QT_BOX; bx < C::NBOX; ++bx)
+        ptx::tma_load_3d(sb + C::OFF_Q + (bx - C::QT_BOX) * C::Q_BOX, &tmQ, bx * 64, hgrp * C::HM, b,
+                         bar(C::B_Q));
       bool ok = true;
       int n = 0;
       for (; n < nblk && ok; ++n) {
-        const int st = n & 1;
-        if (n >= 2)
-          ok = ptx::mbar_wait(bar(C::B_KE + st), ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns);
+        const int st = n % C::NST;
+        if (n >= C::NST)
+          ok = ptx::mbar_wait(bar(C::B_KE + st), ((n / C::NST) - 1) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         ptx::mbar_arrive_expect_tx(bar(C::B_KF + st), C::KV_BYTES);
 #pragma unroll
@@ -442,8 +450,8 @@ __global__ void __launch_bounds__(224, 1)
         if (p.err) atomicCAS(p.err, 0, BLASST_ETIMEOUT);
         // let the copies in flight land before the CTA exits
         ptx::mbar_wait(bar(C::B_Q), 0, &misc[2], p.timeout_ns);
-        for (int k = n - 2 < 0 ? 0 : n - 2; k < n; ++k)
-          ptx::mbar_wait(bar(C::B_KF + (k & 1)), (k >> 1) & 1, &misc[2], p.timeout_ns);
+        for (int k = n - C::NST < 0 ? 0 : n - C::NST; k < n; ++k)
+          ptx::mbar_wait(bar(C::B_KF + k % C::NST), (k / C::NST) & 1, &misc[2], p.timeout_ns);
       }
     }
   } else if (warp == 5 || warp == 6) {
@@ -452,25 +460,34 @@ __global__ void __launch_bounds__(224, 1)
       bool ok = ptx::mbar_wait(bar(C::B_Q), 0, abort_flag, p.timeout_ns);
       ptx::tc_fence_after();
       if (warp == 6) {
-        // S(n) = Q C_n^T into S buffer n % 2
+        // S(n) = Q C_n^T into S buffer n % 2: dims 0-255 with Q from TMEM,
+        // dims 256-575 with Q from shared memory
+        if (ok) ok = ptx::mbar_wait(bar(C::B_QT), 0, abort_flag, p.timeout_ns);
+        ptx::tc_fence_after();
         const uint64_t q_desc = ptx::sw128_desc(sb + C::OFF_Q, 16, 1024);
         const uint64_t k_desc = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
         for (int n = 0; n < nblk && ok; ++n) {
-          const int st = n & 1;
-          ok = ptx::mbar_wait(bar(C::B_KF + st), (n >> 1) & 1, abort_flag, p.timeout_ns);
+          const int sbuf = n & 1, st = n % C::NST;
+          ok = ptx::mbar_wait(bar(C::B_KF + st), (n / C::NST) & 1, abort_flag, p.timeout_ns);
           if (ok && n >= 2)
-            ok = ptx::mbar_wait(bar(C::B_SFREE + st), ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns);
+            ok = ptx::mbar_wait(bar(C::B_SFREE + sbuf), ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns);
           if (!ok) break;
           ptx::tc_fence_after();
-          const uint32_t d_tm = tmem + C::S_COL + st * C::BC;
+          const uint32_t d_tm = tmem + C::S_COL + sbuf * C::BC;
           const uint64_t kd = k_desc + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < C::DQK / 16; ++kk) {
-            const uint64_t a = q_desc + static_cast<uint64_t>(((kk >> 2) * C::Q_BOX + (kk & 3) * 32) >> 4);
+          for (int kk = 0; kk < 4 * C::QT_BOX; ++kk) {
             const uint64_t bd = kd + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
-            ptx::mma_ss(d_tm, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+            ptx::mma_ts(d_tm, tmem + C::QT_COL + kk * 8, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
           }
-          ptx::mma_commit(bar(C::B_SF + st));
+#pragma unroll
+          for (int kk = 4 * C::QT_BOX; kk < C::DQK / 16; ++kk) {
+            const uint64_t a =
+                q_desc + static_cast<uint64_t>((((kk >> 2) - C::QT_BOX) * C::Q_BOX + (kk & 3) * 32) >> 4);
+            const uint64_t bd = kd + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
+            ptx::mma_ss(d_tm, a, bd, C::IDESC_S, 1u);
+          }
+          ptx::mma_commit(bar(C::B_SF + sbuf));
         }
       } else {
         // O_half += P(n) V_half(n); the commits free the stage, the S buffer
@@ -478,22 +495,22 @@ __global__ void __launch_bounds__(224, 1)
         const uint64_t v_desc = ptx::sw128_desc(sb + C::OFF_K + 4 * half * C::KV_BOX, C::KV_BOX, 1024);
         bool any_pv = false;
         for (int n = 0; n < nblk && ok; ++n) {
-          const int st = n & 1;
-          ok = ptx::mbar_wait(bar(C::B_PR + st), (n >> 1) & 1, abort_flag, p.timeout_ns);
+          const int sbuf = n & 1, stg = n % C::NST;
+          ok = ptx::mbar_wait(bar(C::B_PR + sbuf), (n >> 1) & 1, abort_flag, p.timeout_ns);
           if (!ok) break;
           ptx::tc_fence_after();
-          if (misc[4 + st] != 0) {
-            const uint32_t p_tm = tmem + C::S_COL + st * C::BC;
-            const uint64_t vd = v_desc + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
+          if (misc[4 + sbuf] != 0) {
+            const uint32_t p_tm = tmem + C::S_COL + sbuf * C::BC;
+            const uint64_t vd = v_desc + static_cast<uint64_t>((stg * C::KV_BYTES) >> 4);
 #pragma unroll
             for (int kk = 0; kk < C::BC / 16; ++kk)
               ptx::mma_ts(tmem + C::O_COL, p_tm + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4),
                           C::IDESC_PV, (any_pv || kk > 0) ? 1u : 0u);
             any_pv = true;
           }
-          ptx::mma_commit(bar(C::B_KE + st));
-          ptx::mma_commit(bar(C::B_SFREE + st));
-          ptx::mma_commit(bar(C::B_PVD + st));
+          ptx::mma_commit(bar(C::B_KE + stg));
+          ptx::mma_commit(bar(C::B_SFREE + sbuf));
+          ptx::mma_commit(bar(C::B_PVD + sbuf));
         }
       }
       if (!ok) {
@@ -514,6 +531,27 @@ __global__ void __launch_bounds__(224, 1)
     float m = -INFINITY, mref = -INFINITY, l = 0.0f;
     bool ok = true;
     unsigned long long n_skip = 0, n_pv = 0;
+    {
+      // this head's query dims 0-255 into TMEM (the score product's TS operand)
+      const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (head0 + h) * C::DQK);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = qrow[8 * c + u];
+          w[4 * u] = v.x;
+          w[4 * u + 1] = v.y;
+          w[4 * u + 2] = v.z;
+          w[4 * u + 3] = v.w;
+        }
+        ptx::tmem_st32(tmem + lane_base + C::QT_COL + 32 * c, w);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::B_QT));
+    }
     for (int n = 0; n < nblk; ++n) {
       const int st = n & 1;
       ok = ptx::named_bar_and(2, 128, ptx::mbar_wait(bar(C::B_SF + st), (n >> 1) & 1, abort_flag,
@@ -626,7 +664,7 @@ __global__ void __launch_bounds__(224, 1)
           const unsigned long long pv_fl = 2ull * C::HM * C::BC * 256;
           atomicAdd(&p.stats->mma_flops, static_cast<unsigned long long>(nblk) * s_fl + n_pv * pv_fl);
           atomicAdd(&p.stats->bytes_loaded,
-                    static_cast<unsigned long long>(nblk) * C::KV_BYTES + C::Q_BYTES);
+                    static_cast<unsigned long long>(nblk) * C::KV_BYTES + C::Q_SM_BYTES + C::HM * 512);
           if (half == 0) {
             atomicAdd(&p.stats->tiles_visited, static_cast<unsigned long long>(nblk) * C::HM);
             atomicAdd(&p.stats->v_blocks_loaded, static_cast<unsigned long long>(nblk));
