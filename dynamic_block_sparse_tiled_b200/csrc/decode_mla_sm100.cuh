@@ -331,11 +331,13 @@ __global__ void __launch_bounds__(256, 1)
 //              lazy rescaling (the reference max moves only when it has grown
 //              by more than 8 in log2 units; then the O half in TMEM is scaled
 //              after the previous P V has completed), P (bf16) over S;
-//   warp 4     TMA: Q once (nine [128 heads][64 dims] boxes), 32-key blocks of
-//              the cache through a 2-stage ring;
+//   warp 4     TMA: query dims 256-575 once, 32-key blocks of the cache
+//              through a 4-stage ring;
 //   warp 6     tcgen05 issuer of S = Q C^T (M 128, N 32, K 576) into one of
-//              two S buffers (once the block is loaded and the buffer's P has
-//              been read by its P V);
+//              three S buffers (once the block is loaded and the buffer's P
+//              has been read by its P V); query dims 0-255 are a TMEM operand
+//              (written by warps 0-3 at start), dims 256-575 come from shared
+//              memory, which leaves room for a 4-stage cache ring;
 //   warp 5     tcgen05 issuer of O_half += P V_half (M 128, N 256, K 32, P
 //              from TMEM, V MN-major from the stage), skipped when no head of
 //              the 128 keeps the block; owns the TMEM allocation. Two issuers
@@ -355,24 +357,26 @@ struct TcCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_SM_BYTES;
   static constexpr int OFF_BAR = OFF_K + NST * KV_BYTES;
+  static constexpr int NSB = 3;                     // S buffers
   static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + NST, B_SF = B_KE + NST;
-  static constexpr int B_PR = B_SF + 2, B_PVD = B_PR + 2, B_DRAIN = B_PVD + 2;
-  static constexpr int B_SFREE = B_DRAIN + 1;   // [2] P of the S buffer read by its P V
-  static constexpr int B_DRAIN_S = B_SFREE + 2; // the S issuer's drain
+  static constexpr int B_PR = B_SF + NSB, B_PVD = B_PR + NSB, B_DRAIN = B_PVD + NSB;
+  static constexpr int B_SFREE = B_DRAIN + 1;   // [NSB] P of the S buffer read by its P V
+  static constexpr int B_DRAIN_S = B_SFREE + NSB; // the S issuer's drain
   static constexpr int B_QT = B_DRAIN_S + 1;    // Q dims 0-255 written to TMEM (4 warps)
   static constexpr int NBAR = B_QT + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // misc words: [0] tmem base, [1] abort, [2] always 0, [4..5] block kept by some head (per S buffer)
+  // misc words: [0] tmem base, [1] abort, [2] always 0, [4..6] block kept by some head (per S buffer)
   static constexpr int MISC_BYTES = 64;
   static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
   static constexpr int S_COL = 0;    // S buffer b at 32 b (P: first 16 columns)
-  static constexpr int QT_COL = 64;  // Q dims 0-255, packed bf16 pairs: 128 columns
+  static constexpr int QT_COL = 96;  // Q dims 0-255, packed bf16 pairs: 128 columns
   static constexpr int O_COL = 256;  // this CTA's 256 output columns
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32acc(128, BC, false, false);
   static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32acc(128, 256, false, true);
   static constexpr float TAU = 8.0f;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(NSB * BC <= QT_COL && QT_COL + 128 <= O_COL, "TMEM columns");
 };
 }  // namespace mla
 
@@ -409,7 +413,7 @@ __global__ void __launch_bounds__(224, 1)
   }
   if (tid == 0) {
     for (int i = 0; i < C::NBAR; ++i)
-      ptx::mbar_init(bar(i), (i == C::B_PR || i == C::B_PR + 1 || i == C::B_QT) ? 4 : 1);
+      ptx::mbar_init(bar(i), ((i >= C::B_PR && i < C::B_PR + C::NSB) || i == C::B_QT) ? 4 : 1);
     for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
     ptx::fence_mbar_init();
   }
@@ -467,10 +471,11 @@ __global__ void __launch_bounds__(224, 1)
         const uint64_t q_desc = ptx::sw128_desc(sb + C::OFF_Q, 16, 1024);
         const uint64_t k_desc = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
         for (int n = 0; n < nblk && ok; ++n) {
-          const int sbuf = n & 1, st = n % C::NST;
+          const int sbuf = n % C::NSB, st = n % C::NST;
           ok = ptx::mbar_wait(bar(C::B_KF + st), (n / C::NST) & 1, abort_flag, p.timeout_ns);
-          if (ok && n >= 2)
-            ok = ptx::mbar_wait(bar(C::B_SFREE + sbuf), ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns);
+          if (ok && n >= C::NSB)
+            ok = ptx::mbar_wait(bar(C::B_SFREE + sbuf), ((n / C::NSB) - 1) & 1, abort_flag,
+                                p.timeout_ns);
           if (!ok) break;
           ptx::tc_fence_after();
           const uint32_t d_tm = tmem + C::S_COL + sbuf * C::BC;
@@ -495,8 +500,8 @@ __global__ void __launch_bounds__(224, 1)
         const uint64_t v_desc = ptx::sw128_desc(sb + C::OFF_K + 4 * half * C::KV_BOX, C::KV_BOX, 1024);
         bool any_pv = false;
         for (int n = 0; n < nblk && ok; ++n) {
-          const int sbuf = n & 1, stg = n % C::NST;
-          ok = ptx::mbar_wait(bar(C::B_PR + sbuf), (n >> 1) & 1, abort_flag, p.timeout_ns);
+          const int sbuf = n % C::NSB, stg = n % C::NST;
+          ok = ptx::mbar_wait(bar(C::B_PR + sbuf), (n / C::NSB) & 1, abort_flag, p.timeout_ns);
           if (!ok) break;
           ptx::tc_fence_after();
           if (misc[4 + sbuf] != 0) {
@@ -553,8 +558,8 @@ __global__ void __launch_bounds__(224, 1)
       if (lane == 0) ptx::mbar_arrive(bar(C::B_QT));
     }
     for (int n = 0; n < nblk; ++n) {
-      const int st = n & 1;
-      ok = ptx::named_bar_and(2, 128, ptx::mbar_wait(bar(C::B_SF + st), (n >> 1) & 1, abort_flag,
+      const int st = n % C::NSB;  // S buffer
+      ok = ptx::named_bar_and(2, 128, ptx::mbar_wait(bar(C::B_SF + st), (n / C::NSB) & 1, abort_flag,
                                                       p.timeout_ns));
       if (!ok) break;
       ptx::tc_fence_after();
@@ -575,8 +580,8 @@ __global__ void __launch_bounds__(224, 1)
       const bool scale_o = move_ref && n > 0;  // O holds P V of earlier blocks
       // some head must scale O: wait (all threads) for the previous P V
       if (!ptx::named_bar_and(3, 128, !scale_o)) {
-        ok = ptx::named_bar_and(4, 128, ptx::mbar_wait(bar(C::B_PVD + ((n - 1) & 1)),
-                                                        ((n - 1) >> 1) & 1, abort_flag,
+        ok = ptx::named_bar_and(4, 128, ptx::mbar_wait(bar(C::B_PVD + ((n - 1) % C::NSB)),
+                                                        ((n - 1) / C::NSB) & 1, abort_flag,
                                                         p.timeout_ns));
         if (!ok) break;
         ptx::tc_fence_after();
@@ -632,8 +637,8 @@ __global__ void __launch_bounds__(224, 1)
     }
     if (ok) {
       // the last P V, then this split's O half and lse
-      ok = ptx::named_bar_and(2, 128, ptx::mbar_wait(bar(C::B_PVD + ((nblk - 1) & 1)),
-                                                      ((nblk - 1) >> 1) & 1, abort_flag,
+      ok = ptx::named_bar_and(2, 128, ptx::mbar_wait(bar(C::B_PVD + ((nblk - 1) % C::NSB)),
+                                                      ((nblk - 1) / C::NSB) & 1, abort_flag,
                                                       p.timeout_ns));
     }
     if (!ok) {
