@@ -357,7 +357,7 @@ struct TcCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_SM_BYTES;
   static constexpr int OFF_BAR = OFF_K + NST * KV_BYTES;
-  static constexpr int NSB = 3;                     // S buffers
+  static constexpr int NSB = 4;                     // S buffers
   static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + NST, B_SF = B_KE + NST;
   static constexpr int B_PR = B_SF + NSB, B_PVD = B_PR + NSB, B_DRAIN = B_PVD + NSB;
   static constexpr int B_SFREE = B_DRAIN + 1;   // [NSB] P of the S buffer read by its P V
@@ -365,11 +365,11 @@ struct TcCfg {
   static constexpr int B_QT = B_DRAIN_S + 1;    // Q dims 0-255 written to TMEM (4 warps)
   static constexpr int NBAR = B_QT + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // misc words: [0] tmem base, [1] abort, [2] always 0, [4..6] block kept by some head (per S buffer)
+  // misc words: [0] tmem base, [1] abort, [2] always 0, [4..7] block kept by some head (per S buffer)
   static constexpr int MISC_BYTES = 64;
   static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
   static constexpr int S_COL = 0;    // S buffer b at 32 b (P: first 16 columns)
-  static constexpr int QT_COL = 96;  // Q dims 0-255, packed bf16 pairs: 128 columns
+  static constexpr int QT_COL = 128;  // Q dims 0-255, packed bf16 pairs: 128 columns
   static constexpr int O_COL = 256;  // this CTA's 256 output columns
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32acc(128, BC, false, false);
