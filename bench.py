@@ -234,7 +234,7 @@ def measure_prefill(w, lam, steps, warmup, device, stream, flush_buf, pre=None, 
                      v_blocks=sd["v_blocks_loaded"], bytes_loaded=sd["bytes_loaded"])
 
 
-def measure_decode_mla(w, steps, device, stream, flush_buf, peaks, Bc=32):
+def measure_decode_mla(w, steps, device, stream, flush_buf, peaks, Bc=64):
     """MLA decode at lambda = 0 and at the workload's lambda: time, executed
     TFLOP/s against the bf16 peak, bytes against the copy bandwidth."""
     import torch
@@ -275,9 +275,9 @@ def measure_decode_mla(w, steps, device, stream, flush_buf, peaks, Bc=32):
                            frac=top["executed_tflops"] / peaks["bf16_tflops"],
                            hbm_frac=top["gbs"] / peaks["hbm_gbs"],
                            note=("tcgen05, 128 heads per CTA, two CTAs per split (one output half "
-                                 "each, both form the scores)") if Bc == 32 else
+                                 "each, both form the scores)") if w.Hq % 128 == 0 else
                                 ("mma.sync m16n8k16 tiles (16 heads per CTA); the cache is read "
-                                 "once from HBM, re-read from L2 by each of the 8 head groups"))
+                                 "once from HBM, re-read from L2 by each head group"))
     res["config"] = dict(B=w.B, H=w.Hq, L=w.Lkv, num_splits=w.num_splits, amplitude=w.amp, Bc=Bc)
     return res
 
@@ -745,10 +745,10 @@ def main():
         mla = {}
         for wn in ("decode_mla_64k", "decode_mla_64k_a12"):
             mla[wn] = measure_decode_mla(synth.CONFIGS[wn], max(5, args.steps), device, stream,
-                                         flush_buf, peaks, Bc=32)
-        mla["decode_mla_64k_mma_sync_bc64"] = measure_decode_mla(
-            synth.CONFIGS["decode_mla_64k"], max(5, args.steps), device, stream, flush_buf, peaks,
-            Bc=64)
+                                         flush_buf, peaks)
+        mla["decode_mla_64k_h112_mma_sync"] = measure_decode_mla(
+            synth.CONFIGS["decode_mla_64k"].replace(name="decode_mla_64k_h112", Hq=112),
+            max(5, args.steps), device, stream, flush_buf, peaks)
         extra["decode_mla_64k"] = mla
 
         # backward with the forward's decisions held fixed, 32K workload

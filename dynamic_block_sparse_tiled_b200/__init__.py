@@ -388,14 +388,13 @@ def attention_decode_mla(q, cache, *, lam=0.0, num_splits=32, Bc=None, scale=0.0
                          stats=None, stream=None, workspace=None):
     """MLA-shaped decode (one latent KV head, 576-wide rows, 512-wide values):
     allocate outputs and workspace with torch and run blasst_decode_mla
-    (Bc: 32 = the tensor-core kernel, the default when H is a multiple of
-    128; 64 = the mma.sync kernel). Returns (o [B,H,512] bf16, lse [B,H],
-    mask [B,H,ceil(L/Bc)] or None)."""
+    (64-key decision blocks; the tensor-core kernel when H is a multiple of
+    128). Returns (o [B,H,512] bf16, lse [B,H], mask [B,H,ceil(L/64)] or None)."""
     import torch
     B, H = q.shape[0], q.shape[1]
     L = cache.shape[1]
     if Bc is None:
-        Bc = 32 if H % 128 == 0 else 64
+        Bc = 64
     o = torch.empty((B, H, 512), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
     if workspace is None:

@@ -582,9 +582,10 @@ int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int
   if (!aligned16(q) || !aligned16(cache) || !aligned16(o) || !aligned16(lse)) return BLASST_EINVAL;
   if (B <= 0 || H <= 0 || L <= 0 || num_splits <= 0) return BLASST_EINVAL;
   if (!(lambda >= 0.0f && lambda < 1.0f)) return BLASST_EINVAL;
-  if (Bc != T::BC && Bc != C::BC) return BLASST_EUNSUPPORTED;
-  const bool tc = Bc == T::BC;  // tcgen05 kernel: 32-key blocks, groups of 128 heads
-  if (H % (tc ? T::HM : C::HG) != 0) return BLASST_EUNSUPPORTED;
+  static_assert(T::BC == C::BC, "both MLA kernels decide per 64-key block");
+  if (Bc != C::BC) return BLASST_EUNSUPPORTED;
+  if (H % C::HG != 0) return BLASST_EUNSUPPORTED;
+  const bool tc = H % T::HM == 0;  // tcgen05 kernel for groups of 128 heads, else mma.sync
   if (num_splits > 65535 || B > 65535 || static_cast<long long>(B) * num_splits * (H / C::HG) >
                                             0x7fffffffll)
     return BLASST_EINVAL;

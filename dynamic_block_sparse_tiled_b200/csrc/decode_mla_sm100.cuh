@@ -331,33 +331,33 @@ __global__ void __launch_bounds__(256, 1)
 //              lazy rescaling (the reference max moves only when it has grown
 //              by more than 8 in log2 units; then the O half in TMEM is scaled
 //              after the previous P V has completed), P (bf16) over S;
-//   warp 4     TMA: query dims 256-575 once, 32-key blocks of the cache
-//              through a 4-stage ring;
-//   warp 6     tcgen05 issuer of S = Q C^T (M 128, N 32, K 576) into one of
-//              three S buffers (once the block is loaded and the buffer's P
-//              has been read by its P V); query dims 0-255 are a TMEM operand
+//   warp 4     TMA: query dims 256-575 once, 64-key blocks of the cache
+//              through a 2-stage ring;
+//   warp 6     tcgen05 issuer of S = Q C^T (M 128, N 64, K 576) into one of
+//              two S buffers (once the block is loaded and the buffer's P has
+//              been read by its P V); query dims 0-255 are a TMEM operand
 //              (written by warps 0-3 at start), dims 256-575 come from shared
-//              memory, which leaves room for a 4-stage cache ring;
-//   warp 5     tcgen05 issuer of O_half += P V_half (M 128, N 256, K 32, P
+//              memory, which leaves room for two 72 KB cache stages;
+//   warp 5     tcgen05 issuer of O_half += P V_half (M 128, N 256, K 64, P
 //              from TMEM, V MN-major from the stage), skipped when no head of
 //              the 128 keeps the block; owns the TMEM allocation. Two issuers
 //              so that a P V never waits behind a score product that waits
 //              for its block's load.
 namespace mla {
 struct TcCfg {
-  static constexpr int DQK = 576, DV = 512, BC = 32, HM = 128;
+  static constexpr int DQK = 576, DV = 512, BC = 64, HM = 128;
   static constexpr int NTHREADS = 224;
   static constexpr int NBOX = DQK / 64;             // 9
   static constexpr int QT_BOX = 4;                  // dims 0-255 of Q live in TMEM (TS operand)
   static constexpr int Q_BOX = HM * 128;            // 16 KB
   static constexpr int Q_SM_BYTES = (NBOX - QT_BOX) * Q_BOX;  // dims 256-575 in shared memory, 80 KB
-  static constexpr int KV_BOX = BC * 128;           // 4 KB
-  static constexpr int KV_BYTES = NBOX * KV_BOX;    // 36 KB
-  static constexpr int NST = 4;                     // cache stages
+  static constexpr int KV_BOX = BC * 128;           // 8 KB
+  static constexpr int KV_BYTES = NBOX * KV_BOX;    // 72 KB
+  static constexpr int NST = 2;                     // cache stages
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_SM_BYTES;
   static constexpr int OFF_BAR = OFF_K + NST * KV_BYTES;
-  static constexpr int NSB = 4;                     // S buffers
+  static constexpr int NSB = 2;                     // S buffers
   static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + NST, B_SF = B_KE + NST;
   static constexpr int B_PR = B_SF + NSB, B_PVD = B_PR + NSB, B_DRAIN = B_PVD + NSB;
   static constexpr int B_SFREE = B_DRAIN + 1;   // [NSB] P of the S buffer read by its P V
@@ -365,10 +365,10 @@ struct TcCfg {
   static constexpr int B_QT = B_DRAIN_S + 1;    // Q dims 0-255 written to TMEM (4 warps)
   static constexpr int NBAR = B_QT + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // misc words: [0] tmem base, [1] abort, [2] always 0, [4..7] block kept by some head (per S buffer)
+  // misc words: [0] tmem base, [1] abort, [2] always 0, [4..5] block kept by some head (per S buffer)
   static constexpr int MISC_BYTES = 64;
   static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-  static constexpr int S_COL = 0;    // S buffer b at 32 b (P: first 16 columns)
+  static constexpr int S_COL = 0;    // S buffer b at 64 b (P: first 32 columns)
   static constexpr int QT_COL = 128;  // Q dims 0-255, packed bf16 pairs: 128 columns
   static constexpr int O_COL = 256;  // this CTA's 256 output columns
   static constexpr int TMEM_COLS = 512;
@@ -563,16 +563,20 @@ __global__ void __launch_bounds__(224, 1)
                                                       p.timeout_ns));
       if (!ok) break;
       ptx::tc_fence_after();
-      uint32_t r[32];
-      ptx::tmem_ld32(tmem + lane_base + C::S_COL + st * C::BC, r);
-      ptx::tmem_wait_ld();
       const int kbase = key_lo + n * C::BC;
-      float sv[32];
+      float sv[C::BC];
       float mb = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        sv[c] = (kbase + c < key_hi) ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
-        mb = fmaxf(mb, sv[c]);
+      for (int hc = 0; hc < C::BC / 32; ++hc) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tmem + lane_base + C::S_COL + st * C::BC + 32 * hc, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int cc = 32 * hc + c;
+          sv[cc] = (kbase + cc < key_hi) ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
+          mb = fmaxf(mb, sv[cc]);
+        }
       }
       const bool skip = n > 0 && p.log2_lambda > -INFINITY && (mb - m < p.log2_lambda);
       const float m_new = skip ? m : fmaxf(m, mb);
@@ -602,7 +606,7 @@ __global__ void __launch_bounds__(224, 1)
           ptx::tmem_st32(tmem + lane_base + C::O_COL + 32 * c, o);
         }
       }
-      uint32_t pk[16];
+      uint32_t pk[C::BC / 2];
       if (!skip) {
         m = m_new;
         if (move_ref) {
@@ -611,7 +615,7 @@ __global__ void __launch_bounds__(224, 1)
         }
         float ps = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < C::BC / 2; ++c) {
           const float p0 = ptx::ex2(sv[2 * c] - mref), p1 = ptx::ex2(sv[2 * c + 1] - mref);
           ps += p0 + p1;
           pk[c] = ptx::pack_bf16x2(p0, p1);
@@ -620,9 +624,10 @@ __global__ void __launch_bounds__(224, 1)
       } else {
         ++n_skip;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = 0u;
+        for (int c = 0; c < C::BC / 2; ++c) pk[c] = 0u;
       }
-      ptx::tmem_st16(tmem + lane_base + C::S_COL + st * C::BC, pk);
+      static_assert(C::BC == 64, "P is stored as one 32-column row");
+      ptx::tmem_st32(tmem + lane_base + C::S_COL + st * C::BC, pk);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       // does any of the 128 heads keep the block? (P V is skipped otherwise)

@@ -287,11 +287,12 @@ BLASST_API size_t blasst_decode_noalloc_max_bytes(void);
  * block of each split always computed, then the log-sum-exp merge of
  * blasst_decode. V is part of the cached rows already read for the scores, so
  * a skip saves no bytes; a block's P V is skipped for a group of heads (128
- * with Bc = 32, 16 with Bc = 64) when every head of the group drops it.
+ * when H is a multiple of 128: the tensor-core kernel; else 16: the mma.sync
+ * kernel) when every head of the group drops it.
  *   q          [B, H, 576] bf16;  cache [B, L, 576] bf16.
  *   o          [B, H, 512] bf16;  lse [B, H] fp32 (natural log).
- *   Bc         decision block: 32 (tensor-core kernel, H a multiple of 128)
- *              or 64 (mma.sync kernel, H a multiple of 16).
+ *   H          a multiple of 16.
+ *   Bc         decision block: 64 (others: BLASST_EUNSUPPORTED).
  *   num_splits splits of ceil(ceil(L/S)/Bc)*Bc keys each.
  *   scale      score scale; <= 0 selects 1/sqrt(576).
  *   workspace  >= blasst_decode_mla_workspace_bytes(B, H, num_splits).

@@ -154,10 +154,10 @@ def test_decode_mla_workspace_and_rejections(lib):
     assert ws == 8 * 128 * 32 * (512 + 1) * 4
     vp = 0x10000
     f = C.c_float
-    # decision blocks other than 32 / 64, and 32 with heads not a multiple of 128
+    # decision blocks other than 64
     assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 128, 4096, f(1e-3), 128, 4, f(0.0), vp, 1 << 30,
                                  None, None, None) == -2
-    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 64, 4096, f(1e-3), 32, 4, f(0.0), vp, 1 << 30,
+    assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 128, 4096, f(1e-3), 32, 4, f(0.0), vp, 1 << 30,
                                  None, None, None) == -2
     # heads not a multiple of 16
     assert lib.blasst_decode_mla(vp, vp, vp, vp, 2, 24, 4096, f(1e-3), 64, 4, f(0.0), vp, 1 << 30,

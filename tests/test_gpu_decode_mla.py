@@ -32,9 +32,10 @@ def _oracle_v(k):
 
 
 def run_mla(w, lam, seqs=None, heads=None, Bc=64):
-    """Run the GPU kernel on the whole workload (Bc = 32: the tensor-core
-    kernel, 64: the mma.sync kernel); compare sequences ``seqs`` and heads
-    ``heads`` (default all) with the oracle run with the same block size."""
+    """Run the GPU kernel on the whole workload (the tensor-core kernel when
+    the head count is a multiple of 128, else the mma.sync one); compare
+    sequences ``seqs`` and heads ``heads`` (default all) with the oracle run
+    with the same 64-key decision blocks."""
     bl = _lib()
     inp = synth.generate(w)
     qd = parity.to_device(inp.q[:, :, 0, :].copy())   # [B, H, 576]
@@ -73,16 +74,16 @@ def run_mla(w, lam, seqs=None, heads=None, Bc=64):
 
 
 SMALL = [
-    # name, overrides, decision block (32: tensor-core kernel, 64: mma.sync kernel)
+    # name, overrides, decision block (64; 128-head multiples run the tensor-core kernel)
     ("mla_4k_a12", dict(B=2, Hq=32, Lkv=4096, num_splits=4, amp=12.0, n_needles=2), 64),
     ("mla_4k_literal", dict(B=2, Hq=16, Lkv=4096, num_splits=4), 64),
     ("mla_ragged", dict(B=2, Hq=16, Lkv=3000, num_splits=5, amp=12.0), 64),
     ("mla_empty_splits", dict(B=1, Hq=16, Lkv=200, num_splits=8, amp=12.0), 64),
-    ("mla_h128", dict(B=1, Hq=128, Lkv=2048, num_splits=2, amp=12.0, n_needles=2), 64),
-    ("mla_h128_tc", dict(B=1, Hq=128, Lkv=2048, num_splits=2, amp=12.0, n_needles=2), 32),
-    ("mla_h128_tc_ragged", dict(B=2, Hq=128, Lkv=3000, num_splits=5, amp=12.0), 32),
-    ("mla_h128_tc_empty_splits", dict(B=1, Hq=128, Lkv=100, num_splits=8, amp=12.0), 32),
-    ("mla_h256_tc", dict(B=1, Hq=256, Lkv=1024, num_splits=2, amp=12.0), 32),
+    ("mla_h112", dict(B=1, Hq=112, Lkv=2048, num_splits=2, amp=12.0, n_needles=2), 64),
+    ("mla_h128_tc", dict(B=1, Hq=128, Lkv=2048, num_splits=2, amp=12.0, n_needles=2), 64),
+    ("mla_h128_tc_ragged", dict(B=2, Hq=128, Lkv=3000, num_splits=5, amp=12.0), 64),
+    ("mla_h128_tc_empty_splits", dict(B=1, Hq=128, Lkv=100, num_splits=8, amp=12.0), 64),
+    ("mla_h256_tc", dict(B=1, Hq=256, Lkv=1024, num_splits=2, amp=12.0), 64),
 ]
 
 
@@ -93,10 +94,16 @@ def test_mla_parity_small(name, over, Bc, lam):
 
 
 @pytest.mark.parametrize("cfg", ["decode_mla_64k", "decode_mla_64k_a12"])
-@pytest.mark.parametrize("Bc", [32, 64])
-def test_mla_full_size_sampled(cfg, Bc):
+def test_mla_full_size_sampled(cfg):
     """The benchmark's workload (B = 8, 128 heads, 64K keys, 32 splits),
     launched whole; two sequences and 32 of their heads compared with the
     oracle, the telemetry over everything."""
     w = synth.CONFIGS[cfg]
-    run_mla(w, 1e-3, seqs=(0, w.B - 1), heads=slice(48, 80), Bc=Bc)
+    run_mla(w, 1e-3, seqs=(0, w.B - 1), heads=slice(48, 80))
+
+
+def test_mla_full_size_mma_sync_kernel():
+    """The mma.sync kernel (head counts that are not multiples of 128) at the
+    workload's length: 112 heads."""
+    w = synth.CONFIGS["decode_mla_64k"].replace(name="decode_mla_64k_h112", B=2, Hq=112)
+    run_mla(w, 1e-3, seqs=(1,), heads=slice(0, 32))
