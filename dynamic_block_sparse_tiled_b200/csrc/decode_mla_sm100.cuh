@@ -363,7 +363,8 @@ struct TcCfg {
   static constexpr int B_SFREE = B_DRAIN + 1;   // [NSB] P of the S buffer read by its P V
   static constexpr int B_DRAIN_S = B_SFREE + NSB; // the S issuer's drain
   static constexpr int B_QT = B_DRAIN_S + 1;    // Q dims 0-255 written to TMEM (4 warps)
-  static constexpr int NBAR = B_QT + 1;
+  static constexpr int B_KES = B_QT + 1;        // [NST] the stage's score-only boxes free (S done)
+  static constexpr int NBAR = B_KES + NST;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // misc words: [0] tmem base, [1] abort, [2] always 0, [4..5] block kept by some head (per S buffer)
   static constexpr int MISC_BYTES = 64;
@@ -440,14 +441,31 @@ __global__ void __launch_bounds__(224, 1)
       int n = 0;
       for (; n < nblk && ok; ++n) {
         const int st = n % C::NST;
-        if (n >= C::NST)
-          ok = ptx::mbar_wait(bar(C::B_KE + st), ((n / C::NST) - 1) & 1, abort_flag, p.timeout_ns);
+        // the boxes this CTA reads only for the scores reload once the block's
+        // score product is done; its V boxes (dims [256 half, 256 half + 256))
+        // once its P V is done. One full barrier counts all nine boxes.
+        auto load_box = [&](int bx) {
+          ptx::tma_load_3d(sb + C::OFF_K + st * C::KV_BYTES + bx * C::KV_BOX, &tmC, bx * 64,
+                           key_lo + n * C::BC, b, bar(C::B_KF + st));
+        };
+        const bool reuse = n >= C::NST;
+        if (reuse)
+          ok = ptx::mbar_wait(bar(C::B_KES + st), ((n / C::NST) - 1) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         ptx::mbar_arrive_expect_tx(bar(C::B_KF + st), C::KV_BYTES);
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx)
-          ptx::tma_load_3d(sb + C::OFF_K + st * C::KV_BYTES + bx * C::KV_BOX, &tmC, bx * 64,
-                           key_lo + n * C::BC, b, bar(C::B_KF + st));
+          if (bx < 4 * half || bx >= 4 * half + 4) load_box(bx);
+        if (reuse)
+          ok = ptx::mbar_wait(bar(C::B_KE + st), ((n / C::NST) - 1) & 1, abort_flag, p.timeout_ns);
+        // the V boxes go out even when that wait gave up, so that the stage's
+        // byte count completes and the drain below can wait for it
+#pragma unroll
+        for (int bx = 4 * half; bx < 4 * half + 4; ++bx) load_box(bx);
+        if (!ok) {
+          ++n;  // block n's loads are in flight too
+          break;
+        }
       }
       if (!ok) {
         *abort_flag = 1;
@@ -493,6 +511,7 @@ __global__ void __launch_bounds__(224, 1)
             ptx::mma_ss(d_tm, a, bd, C::IDESC_S, 1u);
           }
           ptx::mma_commit(bar(C::B_SF + sbuf));
+          ptx::mma_commit(bar(C::B_KES + st));  // the stage's score-only boxes may be reloaded
         }
       } else {
         // O_half += P(n) V_half(n); the commits free the stage, the S buffer
