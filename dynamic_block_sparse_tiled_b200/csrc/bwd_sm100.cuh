@@ -28,9 +28,9 @@
 //   dV  += P^T dO         (TMEM accumulator)         bf16 TS
 //   dK  += dS^T Q         (TMEM accumulator)         bf16 SS
 //   dQ^T = K^T dS^T       (TMEM, lanes = head dims)  bf16 SS, then staged in
-//                          shared memory as a [64 rows][128 dims] fp32 tile
-//                          and added to the fp32 dQ in global memory by two
-//                          TMA reduce-adds (the add happens in L2).
+//                          shared memory as four [64 rows][32 dims] fp32
+//                          tiles and added to the fp32 dQ in global memory by
+//                          four TMA reduce-adds (the add happens in L2).
 // Computing the transposed S and dP puts the keys on TMEM lanes, so P^T can
 // feed dV straight from TMEM and every product keeps M = 128; dQ^T keeps the
 // head dims on lanes, so a warp's store of one staged dQ row covers 32
@@ -39,14 +39,17 @@
 // (every product that reads them was issued before it and the tensor core
 // completes them in order).
 //
-// Warp roles (320 threads):
-//   warps 0-3  compute: P^T and dS^T, then the dV epilogue;
-//   warps 4-7  dQ writers: drain dQ^T from TMEM, stage it, add it to global
-//              dQ with TMA reduce-adds, then the dK epilogue;
-//   warp 8     producer: K and V once, then per pair Q, dO (TMA, 3-stage
+// Warp roles (352 threads):
+//   warps 0-3, 4-7  two compute sets on alternating pairs (set = pair % 2 =
+//              the S^T, dP^T and dS^T buffer): P^T and dS^T, one key row per
+//              thread, then the set drains its pair's dQ^T (warp q: head dims
+//              [32 q, 32 q + 32)), stages it and issues the reduce-adds; at
+//              the end set 0 writes dV and set 1 writes dK;
+//   warp 8     producer: K and V once, then per pair Q, dO (TMA, 4-stage
 //              ring) and the pair's row statistics (bulk copies); builds the
 //              pair list by scanning the forward's decisions;
-//   warp 9     tcgen05 issuer; owns the TMEM allocation.
+//   warp 9     tcgen05 issuer of dV, dK and dQ^T; owns the TMEM allocation;
+//   warp 10    tcgen05 issuer of S^T and dP^T.
 // TMEM (512 columns): S^T/P^T x2 [0,128), dP^T/dQ^T x2 [128,256),
 // dV [256,384), dK [384,512).
 #pragma once
@@ -350,8 +353,8 @@ __global__ void __launch_bounds__(352, 1)
       }
     }
     if (lane == 0) {
-      // two end records (pair indices i and i + 1): the issuer and the writers
-      // stop at the first, each compute set at the first of its parity
+      // two end records (pair indices i and i + 1): the issuers stop at the
+      // first, each compute set at the first of its parity
       for (int e = 0; e < 2 && ok; ++e) {
         const int ie = i + e;
         const int s = ie % C::NST;
