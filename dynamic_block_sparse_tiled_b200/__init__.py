@@ -23,7 +23,7 @@ import threading
 __all__ = [
     "BlasstError", "Stats", "lib_path", "load_library",
     "blasst_fwd", "blasst_fwd_ex", "blasst_decode", "blasst_decode_workspace_bytes",
-    "blasst_lse_merge", "blasst_check", "blasst_selftest_exp2",
+    "blasst_lse_merge", "blasst_check", "blasst_selftest_exp2", "blasst_selftest_timeout",
     "blasst_decode_noalloc", "blasst_decode_noalloc_max_bytes", "blasst_status_string", "blasst_version",
     "blasst_bwd", "blasst_bwd_workspace_bytes", "blasst_select_blocks",
     "blasst_select_workspace_bytes", "select_blocks", "blasst_decode_mla",
@@ -133,6 +133,8 @@ def load_library(path: str | None = None):
         lib.blasst_decode_noalloc_max_bytes.restype = sz
         lib.blasst_lse_merge.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         lib.blasst_lse_merge.restype = i
+        lib.blasst_selftest_timeout.argtypes = [C.c_ulonglong, vp]
+        lib.blasst_selftest_timeout.restype = i
         lib.blasst_check.argtypes = [vp]
         lib.blasst_check.restype = i
         lib.blasst_status_string.argtypes = [i]
@@ -314,6 +316,12 @@ def blasst_selftest_exp2(x, y_mufu, y_poly, stream=None):
     """The C self-test of the two exp2 paths (fp32 CUDA tensors of equal size)."""
     _check(load_library().blasst_selftest_exp2(_ptr(x), _ptr(y_mufu), _ptr(y_poly), x.numel(),
                                                _stream(stream)), "blasst_selftest_exp2")
+
+
+def blasst_selftest_timeout(limit_ns: int, stream=None):
+    """The C self-test of the bounded-wait failure path (see blasst.h)."""
+    _check(load_library().blasst_selftest_timeout(int(limit_ns), _stream(stream)),
+           "blasst_selftest_timeout")
 
 
 def blasst_check(stream=None) -> int:

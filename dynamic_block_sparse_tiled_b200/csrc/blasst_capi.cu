@@ -212,6 +212,23 @@ __global__ void selftest_exp2_kernel(const float* x, float* y_mufu, float* y_pol
   }
 }
 
+// Bounded-wait self test: one warp waits on an mbarrier that nothing ever
+// arrives on; the wait gives up after limit_ns and the kernel records
+// BLASST_ETIMEOUT in the error word, the path every kernel's waits take.
+__global__ void selftest_timeout_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long mbar;
+  __shared__ int never;
+  const uint32_t b = blasst::ptx::smem_u32(&mbar);
+  if (threadIdx.x == 0) {
+    blasst::ptx::mbar_init(b, 1);
+    never = 0;
+    blasst::ptx::fence_mbar_init();
+  }
+  __syncwarp();
+  const bool ok = blasst::ptx::mbar_wait(b, 0, &never, limit_ns);
+  if (__all_sync(0xffffffffu, !ok) && threadIdx.x == 0 && err) atomicCAS(err, 0, BLASST_ETIMEOUT);
+}
+
 float log2_lambda_of(float lambda) {
   return lambda > 0.0f ? static_cast<float>(std::log2(static_cast<double>(lambda)))
                        : -INFINITY;
@@ -641,6 +658,14 @@ int blasst_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n, vo
   if (!x || !y_mufu || !y_poly || n <= 0) return BLASST_EINVAL;
   selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_mufu,
                                                                                      y_poly, n);
+  return cuda_status(cudaGetLastError());
+}
+
+int blasst_selftest_timeout(unsigned long long limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return BLASST_EINVAL;
+  int* err = error_word();
+  if (!err) return BLASST_ECUDA;
+  selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, limit_ns);
   return cuda_status(cudaGetLastError());
 }
 

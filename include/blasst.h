@@ -329,6 +329,14 @@ BLASST_API int blasst_check(void* stream);
 BLASST_API int blasst_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n,
                                     void* stream);
 
+/* Self-test of the failure path every kernel's waits share: launches one warp
+ * that waits on an mbarrier nothing arrives on, with a bound of limit_ns
+ * (1 ns to 10 s); the wait gives up, the kernel records BLASST_ETIMEOUT in
+ * the device error word (which blasst_check then returns and clears) and
+ * exits normally, leaving the context usable. Nothing is faulted or trapped.
+ * Returns the launch status. */
+BLASST_API int blasst_selftest_timeout(unsigned long long limit_ns, void* stream);
+
 /* Text of the last CUDA error this library saw on the calling host thread
  * (the reason behind the latest BLASST_ECUDA), or "no error". */
 BLASST_API const char* blasst_last_cuda_error(void);

@@ -288,3 +288,18 @@ def test_exp2_paths_against_float64():
     rel_m = np.abs(ym.cpu().numpy().astype(np.float64) / ref - 1.0)
     assert rel_p.max() < 1.1e-4, rel_p.max()
     assert rel_m.max() < 1e-5, rel_m.max()
+
+
+@pytest.mark.gpu
+def test_bounded_wait_failure_path_keeps_the_context_usable():
+    """A wait that nothing satisfies gives up after its bound, the kernel
+    records BLASST_ETIMEOUT, blasst_check returns it once and clears it, and
+    the next launch runs normally (no fault, no trap)."""
+    import dynamic_block_sparse_tiled_b200 as bl
+    bl.blasst_selftest_timeout(2_000_000)  # 2 ms
+    assert bl.blasst_check() == bl.BLASST_ETIMEOUT
+    assert bl.blasst_check() == 0
+    w = BASE.replace(name="after_timeout", Hq=2, Hkv=1, Lq=512, Lkv=512, amp=12.0, window=256,
+                     n_needles=2)
+    run_case(w, 1e-3)
+    assert bl.blasst_check() == 0
