@@ -73,6 +73,7 @@ KERNEL_SOURCES = {
     "prefill_32k": ("prefill_sm100.cuh", "ptx_sm100.cuh"),
     "decode_64k": ("decode_sm100.cuh", "ptx_sm100.cuh"),
     "backward_32k": ("bwd_sm100.cuh", "ptx_sm100.cuh"),
+    "decode_mla_64k": ("decode_mla_sm100.cuh", "ptx_sm100.cuh"),
 }
 
 
@@ -273,7 +274,9 @@ def measure_decode_mla(w, steps, device, stream, flush_buf, peaks, Bc=64):
     res["roofline"] = dict(bound="tensor", achieved=top["executed_tflops"],
                            peak=peaks["bf16_tflops"], unit="TFLOP/s",
                            frac=top["executed_tflops"] / peaks["bf16_tflops"],
-                           hbm_frac=top["gbs"] / peaks["hbm_gbs"],
+                           l2_to_sm_gbs=top["gbs"],
+                           traffic=profiled_traffic("decode_mla_64k") if w.name == "decode_mla_64k"
+                           else None,
                            note=("tcgen05, 128 heads per CTA, two CTAs per split (one output half "
                                  "each, both form the scores)") if w.Hq % 128 == 0 else
                                 ("mma.sync m16n8k16 tiles (16 heads per CTA); the cache is read "
