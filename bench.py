@@ -191,8 +191,16 @@ class Prefill:
                          stream=stream, block_mask_in=block_mask)
 
 
-def flush_l2(buf):
-    buf.add_(1)
+def flush_l2(buf, stream=None):
+    """Write a buffer twice the size of L2. On the timed stream: torch's
+    side streams do not synchronise with its default stream, so a flush
+    issued there would overlap the timed call instead of preceding it."""
+    import torch
+    if stream is None:
+        buf.add_(1)
+    else:
+        with torch.cuda.stream(stream):
+            buf.add_(1)
 
 
 def time_calls(fn, steps, warmup, stream, flush_buf):
@@ -203,7 +211,7 @@ def time_calls(fn, steps, warmup, stream, flush_buf):
     torch.cuda.synchronize()
     times = []
     for _ in range(steps):
-        flush_l2(flush_buf)
+        flush_l2(flush_buf, stream)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -264,23 +272,43 @@ def measure_decode_mla(w, steps, device, stream, flush_buf, peaks, Bc=64):
                                            workspace=ws, stream=stream)
         ms = statistics.mean(time_calls(run, steps, 3, stream, flush_buf))
         tf = sd["mma_flops"] / (ms * 1e-3) / 1e12
+        # algorithmic flops: every visited block's scores once (2 H 64 576),
+        # its P V (2 H 64 512) when some head keeps it. The tensor-core
+        # kernel forms each score in both CTAs of a pair (the executed count
+        # holds it twice); the mma.sync kernel executes exactly these.
+        alg_fl = sd["mma_flops"] - (sd["tiles_visited"] * 2 * 64 * 576 if w.Hq % 128 == 0 else 0)
         gbs = sd["bytes_loaded"] / (ms * 1e-3) / 1e9
-        res[str(lam)] = dict(ms=ms, executed_tflops=tf, gbs=gbs,
-                             skip_frac=sd["tiles_skipped"] / max(sd["tiles_visited"], 1))
+        res[str(lam)] = dict(ms=ms, executed_tflops=tf, algorithmic_tflops=alg_fl / (ms * 1e-3) / 1e12,
+                             gbs=gbs, skip_frac=sd["tiles_skipped"] / max(sd["tiles_visited"], 1))
     base = res["0.0"]["ms"]
     for v in res.values():
         v["speedup_vs_lambda0"] = base / v["ms"]
     top = res[str(w.lambdas[0])]
-    res["roofline"] = dict(bound="tensor", achieved=top["executed_tflops"],
-                           peak=peaks["bf16_tflops"], unit="TFLOP/s",
-                           frac=top["executed_tflops"] / peaks["bf16_tflops"],
-                           l2_to_sm_gbs=top["gbs"],
-                           traffic=profiled_traffic("decode_mla_64k") if w.name == "decode_mla_64k"
-                           else None,
-                           note=("tcgen05, 128 heads per CTA, two CTAs per split (one output half "
-                                 "each, both form the scores)") if w.Hq % 128 == 0 else
-                                ("mma.sync m16n8k16 tiles (16 heads per CTA); the cache is read "
-                                 "once from HBM, re-read from L2 by each head group"))
+    # algorithmic bytes of one call: the cache once, the queries, the split
+    # partials (O and lse) written by the decode kernel and read by the merge,
+    # the merged O and lse
+    alg = (w.B * w.Lkv * 576 * 2 + w.B * w.Hq * 576 * 2 + 2 * w.B * w.Hq * w.num_splits * 513 * 4
+           + w.B * w.Hq * (512 * 2 + 4))
+    hbm_gbs = alg / (top["ms"] * 1e-3) / 1e9
+    t_hbm = alg / (peaks["hbm_gbs"] * 1e9)
+    t_tc = top["algorithmic_tflops"] / peaks["bf16_tflops"] * top["ms"] * 1e-3
+    common = dict(l2_to_sm_gbs=top["gbs"], executed_tflops=top["executed_tflops"],
+                  tensor_frac=top["algorithmic_tflops"] / peaks["bf16_tflops"],
+                  hbm_frac=hbm_gbs / peaks["hbm_gbs"], algorithmic_bytes=int(alg),
+                  traffic=profiled_traffic("decode_mla_64k") if w.name == "decode_mla_64k" else None,
+                  note=("tcgen05, 128 heads per cluster of two CTAs (each forms half of every score "
+                        "over 288 dims, the halves exchanged through distributed shared memory, "
+                        "and accumulates one half of the output); the call also holds the split "
+                        "merge") if w.Hq % 128 == 0 else
+                       ("mma.sync m16n8k16 tiles (16 heads per CTA); the cache is read once from "
+                        "HBM, re-read from L2 by each head group"))
+    if t_hbm >= t_tc:
+        res["roofline"] = dict(bound="hbm", achieved=hbm_gbs, peak=peaks["hbm_gbs"], unit="GB/s",
+                               frac=hbm_gbs / peaks["hbm_gbs"], **common)
+    else:
+        res["roofline"] = dict(bound="tensor", achieved=top["algorithmic_tflops"],
+                               peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                               frac=top["algorithmic_tflops"] / peaks["bf16_tflops"], **common)
     res["config"] = dict(B=w.B, H=w.Hq, L=w.Lkv, num_splits=w.num_splits, amplitude=w.amp, Bc=Bc)
     return res
 
@@ -307,8 +335,8 @@ def backward_pairs(w, mask):
     return int(kb.sum())
 
 
-BWD_FLOPS_PER_PAIR = 5 * 2 * 128 * 64 * 128
-SEL_TAU, SEL_GAMMA = 0.2, 0.9  # selector route threshold and pooled-path coverage  # S^T, dP^T, dV, dK, dQ^T products
+BWD_FLOPS_PER_PAIR = 5 * 2 * 128 * 64 * 128  # S^T, dP^T, dV, dK, dQ^T products
+SEL_TAU, SEL_GAMMA = 0.2, 0.9  # selector route threshold and pooled-path coverage
 
 
 class Backward:
@@ -750,7 +778,9 @@ def main():
             mla[wn] = measure_decode_mla(synth.CONFIGS[wn], max(5, args.steps), device, stream,
                                          flush_buf, peaks)
         mla["decode_mla_64k_h112_mma_sync"] = measure_decode_mla(
-            synth.CONFIGS["decode_mla_64k"].replace(name="decode_mla_64k_h112", Hq=112),
+            synth.CONFIGS["decode_mla_64k"].replace(
+                name="decode_mla_64k_h112", Hq=112,
+                num_splits=bl.blasst_decode_mla_splits(8, 112, synth.CONFIGS["decode_mla_64k"].Lkv)),
             max(5, args.steps), device, stream, flush_buf, peaks)
         extra["decode_mla_64k"] = mla
 

@@ -115,6 +115,8 @@ def load_library(path: str | None = None):
         lib.blasst_decode_mla.restype = i
         lib.blasst_decode_mla_workspace_bytes.argtypes = [i, i, i]
         lib.blasst_decode_mla_workspace_bytes.restype = sz
+        lib.blasst_decode_mla_splits.argtypes = [i, i, i, i]
+        lib.blasst_decode_mla_splits.restype = i
         lib.blasst_select_blocks.argtypes = [C.POINTER(_SelectArgs)]
         lib.blasst_select_blocks.restype = i
         lib.blasst_select_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
@@ -236,6 +238,15 @@ def blasst_bwd(q, k, v, o, dout, lse, dq, dk, dv, *, causal: bool, Br: int, Bc: 
 
 def blasst_decode_mla_workspace_bytes(B: int, H: int, num_splits: int) -> int:
     return int(load_library().blasst_decode_mla_workspace_bytes(B, H, num_splits))
+
+
+def blasst_decode_mla_splits(B: int, H: int, L: int, num_sms: int = 0) -> int:
+    """The C entry point of the same name: a split count that fills whole
+    waves of `num_sms` SMs (<= 0: the current device's count)."""
+    S = int(load_library().blasst_decode_mla_splits(B, H, L, num_sms))
+    if S <= 0:
+        _check(S, "blasst_decode_mla_splits")
+    return S
 
 
 def blasst_decode_mla(q, cache, o, lse, *, lam: float, Bc: int, num_splits: int, workspace,
@@ -392,17 +403,20 @@ def select_blocks(q, k, *, causal=True, Br=128, Bc=128, tau=0.2, gamma=0.9, scal
     return mask, cs
 
 
-def attention_decode_mla(q, cache, *, lam=0.0, num_splits=32, Bc=None, scale=0.0, with_mask=False,
+def attention_decode_mla(q, cache, *, lam=0.0, num_splits=0, Bc=None, scale=0.0, with_mask=False,
                          stats=None, stream=None, workspace=None):
     """MLA-shaped decode (one latent KV head, 576-wide rows, 512-wide values):
     allocate outputs and workspace with torch and run blasst_decode_mla
     (64-key decision blocks; the tensor-core kernel when H is a multiple of
-    128). Returns (o [B,H,512] bf16, lse [B,H], mask [B,H,ceil(L/64)] or None)."""
+    128; num_splits <= 0 takes blasst_decode_mla_splits' choice for this
+    device). Returns (o [B,H,512] bf16, lse [B,H], mask [B,H,ceil(L/64)] or None)."""
     import torch
     B, H = q.shape[0], q.shape[1]
     L = cache.shape[1]
     if Bc is None:
         Bc = 64
+    if num_splits <= 0:
+        num_splits = blasst_decode_mla_splits(B, H, L)
     o = torch.empty((B, H, 512), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
     if workspace is None:

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -587,6 +588,34 @@ size_t blasst_decode_mla_workspace_bytes(int B, int H, int num_splits) {
   if (B <= 0 || H <= 0 || num_splits <= 0) return 0;
   const size_t rows = static_cast<size_t>(B) * H * num_splits;
   return rows * (blasst::MlaCfg::DV + 1) * sizeof(float);
+}
+
+int blasst_decode_mla_splits(int B, int H, int L, int num_sms) {
+  using C = blasst::MlaCfg;
+  using T = blasst::mla::TcCfg;
+  if (B <= 0 || H <= 0 || L <= 0 || H % C::HG != 0) return BLASST_EINVAL;
+  if (num_sms <= 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        num_sms <= 0)
+      return BLASST_ECUDA;
+  }
+  const long long per_split =
+      H % T::HM == 0 ? 2ll * B * (H / T::HM) : static_cast<long long>(B) * (H / C::HG);
+  const long long nb = (static_cast<long long>(L) + C::BC - 1) / C::BC;
+  const int s_max = static_cast<int>(nb < 1024 ? nb : 1024);
+  auto cost = [&](int S) {
+    const long long per = (static_cast<long long>(L) + S - 1) / S;
+    const long long blocks = (per + C::BC - 1) / C::BC;
+    const long long waves = (per_split * S + num_sms - 1) / num_sms;
+    return waves * blocks;
+  };
+  long long best = cost(1);
+  for (int S = 2; S <= s_max; ++S) best = std::min(best, cost(S));
+  for (int S = 1; S <= s_max; ++S)
+    if (static_cast<double>(cost(S)) <= 1.03 * static_cast<double>(best)) return S;
+  return 1;
 }
 
 int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int B, int H, int L,

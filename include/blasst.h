@@ -307,6 +307,20 @@ BLASST_API int blasst_decode_mla(const void* q, const void* cache, void* o, floa
 /* Workspace bytes of blasst_decode_mla: fp32 [B, H, S, 512] + [B, H, S]. */
 BLASST_API size_t blasst_decode_mla_workspace_bytes(int B, int H, int num_splits);
 
+/* A split count for blasst_decode_mla (64-key blocks) that fills whole waves
+ * of the GPU: every CTA of the decode kernel occupies one SM (the tensor-core
+ * kernel launches 2 B H/128 CTAs per split, the mma.sync kernel B H/16), so
+ * the launch takes about ceil(CTAs / num_sms) x (blocks per split) block
+ * times. Returns the smallest S within 3 % of the best such estimate over
+ * S = 1 .. min(ceil(L / 64), 1024) (fewer splits: less partial traffic for
+ * the merge). Host only, no device work.
+ *   num_sms  SMs to fill; <= 0 queries the current device.
+ * Returns S >= 1, or BLASST_EINVAL for B, H, L <= 0 or H not a multiple of
+ * 16, BLASST_ECUDA if the device query fails. Decisions depend on the split
+ * boundaries (each split restarts the running statistics), so the oracle
+ * must be run with the same S. */
+BLASST_API int blasst_decode_mla_splits(int B, int H, int L, int num_sms);
+
 /* Log-sum-exp merge of split partials (the second half of blasst_decode):
  *   o_parts [n_rows, num_splits, d] fp32, normalised per split;
  *   lse_parts [n_rows, num_splits] fp32, -inf marks an empty split;

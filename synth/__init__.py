@@ -156,9 +156,10 @@ CONFIGS = {
                              diffuse_heads="upper_half"),
 }
 # MLA-shaped decode (one latent KV head of 576-wide rows, 128 query heads, values
-# = the first 512 dims of the rows; the cache is K, V is not used).
+# = the first 512 dims of the rows; the cache is K, V is not used). 9 splits:
+# the library's wave-filling choice on 148 SMs (blasst_decode_mla_splits).
 CONFIGS["decode_mla_64k"] = Workload("decode_mla_64k", B=8, Hq=128, Hkv=1, Lq=1, Lkv=65536, d=576,
-                                     causal=False, Br=1, Bc=64, lambdas=(1e-3,), num_splits=32,
+                                     causal=False, Br=1, Bc=64, lambdas=(1e-3,), num_splits=9,
                                      n_needles=4, decode_window=1024)
 # Calibrated "structured" variants: amplitude 12 on the planted direction (the
 # literal amplitude 3 leaves almost no block below the threshold).

@@ -175,6 +175,34 @@ def test_decode_mla_workspace_and_rejections(lib):
                                  None, None, None) == -5
 
 
+def _mla_split_cost(B, H, L, S, sms):
+    per_split = 2 * B * (H // 128) if H % 128 == 0 else B * (H // 16)
+    blocks = -(-(-(-L // S)) // 64)
+    return -(-(per_split * S) // sms) * blocks
+
+
+@pytest.mark.parametrize("B,H,L,sms", [(8, 128, 65536, 148), (1, 128, 4096, 148), (3, 256, 100000, 132),
+                                       (2, 112, 65536, 148), (64, 128, 8192, 148), (1, 16, 64, 148)])
+def test_decode_mla_splits_fill_waves(lib, B, H, L, sms):
+    """The split count is the smallest within 3 % of the best wave-filling
+    estimate (brute force over every split count)."""
+    S = lib.blasst_decode_mla_splits(B, H, L, sms)
+    nb = -(-L // 64)
+    costs = {s: _mla_split_cost(B, H, L, s, sms) for s in range(1, min(nb, 1024) + 1)}
+    best = min(costs.values())
+    assert 1 <= S <= min(nb, 1024)
+    assert costs[S] <= 1.03 * best
+    assert all(costs[s] > 1.03 * best for s in range(1, S))
+
+
+def test_decode_mla_splits_values_and_rejections(lib):
+    # the MLA decode workload on 148 SMs: 144 CTAs of 114 blocks, one wave
+    assert lib.blasst_decode_mla_splits(8, 128, 65536, 148) == 9
+    assert lib.blasst_decode_mla_splits(0, 128, 65536, 148) == -1
+    assert lib.blasst_decode_mla_splits(8, 24, 65536, 148) == -1
+    assert lib.blasst_decode_mla_splits(8, 128, 0, 148) == -1
+
+
 def test_decode_workspace_and_rejections(lib):
     ws = lib.blasst_decode_workspace_bytes(16, 32, 128, 64)
     assert ws == 16 * 32 * 64 * (128 + 1) * 4

@@ -95,7 +95,7 @@ def test_mla_parity_small(name, over, Bc, lam):
 
 @pytest.mark.parametrize("cfg", ["decode_mla_64k", "decode_mla_64k_a12"])
 def test_mla_full_size_sampled(cfg):
-    """The benchmark's workload (B = 8, 128 heads, 64K keys, 32 splits),
+    """The benchmark's workload (B = 8, 128 heads, 64K keys, 9 splits),
     launched whole; two sequences and 32 of their heads compared with the
     oracle, the telemetry over everything."""
     w = synth.CONFIGS[cfg]
@@ -107,3 +107,16 @@ def test_mla_full_size_mma_sync_kernel():
     workload's length: 112 heads."""
     w = synth.CONFIGS["decode_mla_64k"].replace(name="decode_mla_64k_h112", B=2, Hq=112)
     run_mla(w, 1e-3, seqs=(1,), heads=slice(0, 32))
+
+
+def test_mla_workload_splits_are_the_library_choice():
+    """The benchmark's split count is what blasst_decode_mla_splits picks for
+    this device (on a 148-SM B200)."""
+    import torch
+    bl = _lib()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    w = synth.CONFIGS["decode_mla_64k"]
+    S = bl.blasst_decode_mla_splits(w.B, w.Hq, w.Lkv)
+    assert S == bl.blasst_decode_mla_splits(w.B, w.Hq, w.Lkv, sms)
+    if sms == 148:
+        assert S == w.num_splits
