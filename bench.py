@@ -870,6 +870,7 @@ def main():
                     frac=exec_tflops / peaks["bf16_tflops"],
                     traffic=profiled_traffic("prefill_32k"),
                     peak_source=f"{peaks['source']} bf16_tflops (burst; the kernel is timed alone)",
+                    frac_of_sustained=exec_tflops / peaks["bf16_tflops_sustained"],
                     algorithmic="per visited (128-row tile, 128-key block): 2*128*128*128 flops for "
                                 "S=QK^T, plus the same for O+=PV when the block is computed")
 
