@@ -422,37 +422,45 @@ def measure_decode(w, lam, steps, warmup, device, stream, flush_buf):
     return out
 
 
-def measure_e2e(w, lam, steps, warmup, device, stream):
-    """Same metric through the public API from pinned host buffers. Every
-    step uploads its inputs (Q, K, V) host -> device, runs the prefill call
-    and reads its results (O, lse) back device -> host, all inside the timed
-    region. The steps are pipelined as a serving loop runs them: an upload
-    stream, the compute stream and a readback stream over two sets of device
-    buffers, so the upload of step i+1 and the readback of step i-1 overlap
-    the prefill of step i (the PCIe link carries both directions at once).
-    The timed region opens before the first upload and closes after the last
-    readback, so the pipeline's fill and drain are inside it."""
-    import torch
-    import dynamic_block_sparse_tiled_b200 as bl
-    import synth
-    hq = torch.empty((w.B, w.Hq, w.Lq, w.d), dtype=torch.int16, pin_memory=True)
-    hk = torch.empty((w.B, w.Hkv, w.Lkv, w.d), dtype=torch.int16, pin_memory=True)
-    hv = torch.empty_like(hk, pin_memory=True)
-    synth.generate(w, out_q=hq.numpy().view(np.uint16), out_k=hk.numpy().view(np.uint16),
-                   out_v=hv.numpy().view(np.uint16))
-    dev = [dict(q=torch.empty(hq.shape, dtype=torch.bfloat16, device=device),
-                k=torch.empty(hk.shape, dtype=torch.bfloat16, device=device),
-                v=torch.empty(hv.shape, dtype=torch.bfloat16, device=device),
-                o=torch.empty(hq.shape, dtype=torch.bfloat16, device=device),
-                lse=torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=device))
-           for _ in range(2)]
-    host_out = [dict(o=torch.empty(hq.shape, dtype=torch.int16, pin_memory=True),
-                     lse=torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, pin_memory=True))
-                for _ in range(2)]
-    up = torch.cuda.Stream(device)
-    down = torch.cuda.Stream(device)
+class E2EPipeline:
+    """Prefill steps through the public API from pinned host buffers, as a
+    serving loop runs them: every step uploads its inputs (Q, K, V) host ->
+    device, runs the prefill call and reads its results (O, lse) back device
+    -> host. An upload stream, the compute stream and a readback stream work
+    over two sets of device buffers, so the upload of step i+1 and the
+    readback of step i-1 overlap the prefill of step i (the PCIe link carries
+    both directions at once). Every step processes the same synthetic batch."""
 
-    def run(n, start_event=None):
+    def __init__(self, w, lam, device, stream):
+        import torch
+        import synth
+        self.w, self.lam, self.stream = w, lam, stream
+        self.hq = torch.empty((w.B, w.Hq, w.Lq, w.d), dtype=torch.int16, pin_memory=True)
+        self.hk = torch.empty((w.B, w.Hkv, w.Lkv, w.d), dtype=torch.int16, pin_memory=True)
+        self.hv = torch.empty_like(self.hk, pin_memory=True)
+        synth.generate(w, out_q=self.hq.numpy().view(np.uint16),
+                       out_k=self.hk.numpy().view(np.uint16), out_v=self.hv.numpy().view(np.uint16))
+        self.dev = [dict(q=torch.empty(self.hq.shape, dtype=torch.bfloat16, device=device),
+                         k=torch.empty(self.hk.shape, dtype=torch.bfloat16, device=device),
+                         v=torch.empty(self.hv.shape, dtype=torch.bfloat16, device=device),
+                         o=torch.empty(self.hq.shape, dtype=torch.bfloat16, device=device),
+                         lse=torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=device))
+                    for _ in range(2)]
+        self.host_out = [dict(o=torch.empty(self.hq.shape, dtype=torch.int16, pin_memory=True),
+                              lse=torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32,
+                                              pin_memory=True))
+                         for _ in range(2)]
+        self.up = torch.cuda.Stream(device)
+        self.down = torch.cuda.Stream(device)
+        self.h2d_bytes = (self.hq.numel() + self.hk.numel() + self.hv.numel()) * 2
+        self.d2h_bytes = self.host_out[0]["o"].numel() * 2 + self.host_out[0]["lse"].numel() * 4
+
+    def run(self, n, start_event=None):
+        """Enqueue n steps; on return the compute stream waits for the last
+        readback (record an event on it to time or join the steps)."""
+        import torch
+        import dynamic_block_sparse_tiled_b200 as bl
+        w, stream, up, down = self.w, self.stream, self.up, self.down
         if start_event is not None:
             up.wait_event(start_event)
             down.wait_event(start_event)
@@ -460,20 +468,20 @@ def measure_e2e(w, lam, steps, warmup, device, stream):
         read = [None, None]      # last readback of buffer set b
         for i in range(n):
             b = i % 2
-            d, h = dev[b], host_out[b]
+            d, h = self.dev[b], self.host_out[b]
             if computed[b] is not None:   # step i-2 has finished reading set b's inputs
                 up.wait_event(computed[b])
             with torch.cuda.stream(up):
-                d["q"].view(torch.int16).copy_(hq, non_blocking=True)
-                d["k"].view(torch.int16).copy_(hk, non_blocking=True)
-                d["v"].view(torch.int16).copy_(hv, non_blocking=True)
+                d["q"].view(torch.int16).copy_(self.hq, non_blocking=True)
+                d["k"].view(torch.int16).copy_(self.hk, non_blocking=True)
+                d["v"].view(torch.int16).copy_(self.hv, non_blocking=True)
             uploaded = torch.cuda.Event()
             uploaded.record(up)
             stream.wait_event(uploaded)
             if read[b] is not None:       # step i-2's results have been read back
                 stream.wait_event(read[b])
-            bl.blasst_fwd_ex(d["q"], d["k"], d["v"], d["o"], d["lse"], causal=w.causal, lam=lam,
-                             Br=w.Br, Bc=w.Bc, stream=stream)
+            bl.blasst_fwd_ex(d["q"], d["k"], d["v"], d["o"], d["lse"], causal=w.causal,
+                             lam=self.lam, Br=w.Br, Bc=w.Bc, stream=stream)
             computed[b] = torch.cuda.Event()
             computed[b].record(stream)
             down.wait_event(computed[b])
@@ -486,19 +494,26 @@ def measure_e2e(w, lam, steps, warmup, device, stream):
             if ev is not None:
                 stream.wait_event(ev)
 
-    run(warmup)
+
+def measure_e2e(w, lam, steps, warmup, device, stream):
+    """Same metric through the public API from pinned host buffers (see
+    E2EPipeline): every step's upload and readback inside the timed region,
+    which opens before the first upload and closes after the last readback,
+    so the pipeline's fill and drain are timed too."""
+    import torch
+    pipe = E2EPipeline(w, lam, device, stream)
+    pipe.run(warmup)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    run(steps, start_event=e0)
+    pipe.run(steps, start_event=e0)
     e1.record(stream)
     e1.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
-    d2h = host_out[0]["o"].numel() * 2 + host_out[0]["lse"].numel() * 4
     return dict(value=effective_flops(w) / (ms * 1e-3) / 1e12, unit=UNIT, ms=ms,
-                h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h), steps=steps,
+                h2d_bytes_per_step=int(pipe.h2d_bytes), d2h_bytes_per_step=int(pipe.d2h_bytes),
+                steps=steps,
                 pipelined=("upload of step i+1 and readback of step i-1 overlap the prefill of "
                            "step i (three streams, two device buffer sets); fill and drain timed"))
 
