@@ -634,6 +634,54 @@ def dist_env():
     return ws, rank, local
 
 
+class Ranks:
+    """Host plumbing of the replicas (one process per GPU, nothing exchanged on
+    the data path): a barrier with device synchronisation on both sides, and
+    device times combined as the maximum over ranks. Every rank makes the same
+    calls in the same order."""
+
+    def __init__(self, backend, device):
+        self.ws, self.rank, self.local = dist_env()
+        self.device = device
+        self.cuda = device.type == "cuda"
+        if self.ws > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+    def _sync(self):
+        if self.cuda:
+            import torch
+            torch.cuda.synchronize(self.device)
+
+    def barrier(self):
+        self._sync()
+        if self.ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        self._sync()
+
+    def max(self, x):
+        if self.ws == 1:
+            return float(x)
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def aggregate(self, units_per_rank, ms_per_rank):
+        """Whole-job rate: the units all ranks processed over the slowest
+        rank's time (units per second)."""
+        return self.ws * units_per_rank / (self.max(ms_per_rank) * 1e-3)
+
+    def close(self):
+        if self.ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
 def run_reference(args):
     import synth
     ws, rank, _ = dist_env()
@@ -693,32 +741,13 @@ def main():
     import dynamic_block_sparse_tiled_b200 as bl
     bl.load_library()
     ws, rank, local = dist_env()
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local if ws > 1 else 0)
     torch.cuda.set_device(device)
+    ranks = Ranks("nccl", device)
     stream = torch.cuda.Stream(device)
     flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
     peaks = load_peaks()
     w = synth.CONFIGS[WORKLOAD]
-
-    def barrier():
-        torch.cuda.synchronize()
-        if ws > 1:
-            import torch.distributed as dist
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(x):
-        if ws == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # ---- headline: prefill 32K, lambda 1e-3, literal generator -------------
     # (the clock record spans the headline steps and the lambda = 0 and
@@ -726,19 +755,19 @@ def main():
     pre = Prefill(w, device)
     wa = synth.CONFIGS[WORKLOAD + "_a12"]
     pa = Prefill(wa, device)
-    barrier()
+    ranks.barrier()
     with ClockSampler(local) as clk:
         pre, main_r = measure_prefill(w, LAMBDA, args.steps, args.warmup, device, stream, flush_buf,
                                       pre=pre)
-        barrier()
+        ranks.barrier()
         _, dense_r = measure_prefill(w, 0.0, max(3, args.steps // 2), 3, device, stream, flush_buf,
                                      pre=pre)
         pa, a_l = measure_prefill(wa, LAMBDA, max(3, args.steps // 2), 3, device, stream, flush_buf,
                                   pre=pa)
         _, a_0 = measure_prefill(wa, 0.0, max(3, args.steps // 2), 3, device, stream, flush_buf,
                                  pre=pa)
-    ms = max_over_ranks(main_r["ms"])
-    value = ws * main_r["eff_flops"] / (ms * 1e-3) / 1e12
+    ms = ranks.max(main_r["ms"])
+    value = ranks.aggregate(main_r["eff_flops"], main_r["ms"]) / 1e12
     del pre, pa
     torch.cuda.empty_cache()
 
@@ -876,8 +905,7 @@ def main():
 
     # ---- end to end through the public API with host buffers ---------------
     e2e = measure_e2e(w, LAMBDA, max(8, args.steps), 3, device, stream)
-    e2e_ms = max_over_ranks(e2e["ms"])
-    e2e["value"] = ws * effective_flops(w) / (e2e_ms * 1e-3) / 1e12
+    e2e["value"] = ranks.aggregate(effective_flops(w), e2e["ms"]) / 1e12
     e2e.pop("ms")
 
     exec_tflops = main_r["exec_flops"] / (main_r["ms"] * 1e-3) / 1e12
@@ -905,10 +933,7 @@ def main():
             roofline=roofline, cpu_baseline={k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
             e2e=e2e, clocks=clocks, **extra)
         print(json.dumps(line), flush=True)
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
