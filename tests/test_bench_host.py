@@ -139,3 +139,44 @@ def test_traffic_records_follow_the_kernel_sources(tmp_path, monkeypatch):
     other = h[:-1] + ("1" if h[-1] != "1" else "2")  # a record of other sources
     rec.write_text(f"{key} {other} 99\n")
     assert bench.profiled_traffic(key) is None
+
+
+def test_reference_arm_json_line(monkeypatch, capsys):
+    """The reference arm (the oracle on the host cores) prints one JSON line
+    with the benchmark's keys, impl = reference, its own cpu_baseline and an
+    e2e of the line's value with no device copies (the oracle sample and the
+    input generation are stubbed: this checks the line, not the timing)."""
+    import argparse
+    import json
+
+    calls = []
+
+    def fake_sample(w, lam, budget, seed=0, inputs=None):
+        calls.append((w.name, lam, budget, seed))
+        return dict(value=0.05 + 0.01 * seed, unit=bench.UNIT, cores=16, kind="oracle",
+                    sample=f"{seed} of 8192 query tiles", seconds=2.0 + seed)
+
+    monkeypatch.setattr(synth, "generate", lambda w: None)
+    monkeypatch.setattr(bench, "oracle_sample", fake_sample)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    args = argparse.Namespace(gpus=1, steps=2, warmup=3, cpu_budget=15.0)
+    assert bench.run_reference(args) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["steps"] == 2 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == bench.WORKLOAD
+    assert abs(d["value"] - 0.055) < 1e-12                # mean over the 2 timed samples
+    assert abs(d["ms_per_step"] - 2500.0) < 1e-9
+    assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"] == dict(value=d["value"], unit=d["unit"], h2d_bytes_per_step=0,
+                            d2h_bytes_per_step=0)
+    assert len(calls) == 5                                # 3 warm-up samples, then 2 timed
+    assert [c[3] for c in calls[3:]] == [0, 1]            # one seed per timed step
+    assert all(c[2] < calls[3][2] for c in calls[:3])     # warm-up samples are smaller
