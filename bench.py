@@ -105,17 +105,19 @@ def profiled_traffic(kernel_key):
 
 class ClockSampler:
     """nvidia-smi samples (every 50 ms) of SM clock and throttle reasons while
-    running; entering waits for the first sample so the window covers the
-    timed work."""
+    running, each with nvidia-smi's own wall-clock timestamp, so a summary
+    can be taken over the time windows of one measurement leg. Entering
+    waits for the first sample so the record covers the timed work."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.samples = []  # (wall time, sm MHz, max MHz, set of active reasons)
 
     def __enter__(self):
         try:
@@ -126,16 +128,35 @@ class ClockSampler:
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
             t0 = time.monotonic()
-            while not self.lines and time.monotonic() - t0 < 10.0 and self.proc.poll() is None:
+            while not self.samples and time.monotonic() - t0 < 10.0 and self.proc.poll() is None:
                 time.sleep(0.01)
-            self.lines.clear()
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
 
+    @classmethod
+    def parse(cls, line, t_read):
+        """One csv line -> (wall time, sm MHz, max MHz, reasons) or None."""
+        import datetime
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 8:
+            return None
+        try:
+            t = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            t = t_read
+        try:
+            sm, mx = float(parts[1]), float(parts[2])
+        except ValueError:
+            return None
+        reasons = {n for n, v in zip(cls.REASONS, parts[4:8]) if v.lower() == "active"}
+        return (t, sm, mx, reasons)
+
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            s = self.parse(line, time.time())
+            if s is not None:
+                self.samples.append(s)
 
     def __exit__(self, *a):
         if self.proc:
@@ -145,25 +166,19 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+    def summary(self, windows=None):
+        """Median SM clock, max clock and active reasons over the samples that
+        fall inside any of `windows` ([(t0, t1)] in time.time() units; all
+        samples when None)."""
+        sel = [s for s in self.samples
+               if windows is None or any(a <= s[0] <= b for a, b in windows)]
+        if not sel:
             return dict(sm_mhz=None, sm_max_mhz=None, reasons=[], samples=0)
-        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(mx), reasons=sorted(reasons),
-                    samples=len(sm))
+        reasons = set()
+        for s in sel:
+            reasons |= s[3]
+        return dict(sm_mhz=statistics.median(s[1] for s in sel),
+                    sm_max_mhz=max(s[2] for s in sel), reasons=sorted(reasons), samples=len(sel))
 
 
 # ------------------------------------------------------------- GPU side
@@ -220,6 +235,46 @@ def time_calls(fn, steps, warmup, stream, flush_buf):
         e1.synchronize()
         times.append(e0.elapsed_time(e1))
     return times
+
+
+def time_interleaved(arms, rounds, per, warmup, stream, flush_buf):
+    """Device time of several arms (same kernel, different settings) measured
+    as interleaved blocks: each round times `per` calls of every arm, and
+    the arm order alternates between rounds (A B, B A, A B, ...), so a drift
+    of clocks or power over the run affects every arm alike. Returns, per
+    arm key, the mean of each block (ms) and each block's wall-clock window
+    (for the clock record)."""
+    import torch
+    for _, fn in arms:
+        for _ in range(warmup):
+            fn()
+    torch.cuda.synchronize()
+    out = {k: dict(block_ms=[], windows=[]) for k, _ in arms}
+    for r in range(rounds):
+        for k, fn in (arms if r % 2 == 0 else arms[::-1]):
+            t0 = time.time()
+            ts = time_calls(fn, per, 0, stream, flush_buf)
+            out[k]["block_ms"].append(statistics.mean(ts))
+            out[k]["windows"].append((t0, time.time()))
+    return out
+
+
+def arm_summary(t, clk):
+    """Median block time, the median SM clock over the arm's blocks, and the
+    clock-normalised time (ms x MHz = thousands of cycles)."""
+    ms = statistics.median(t["block_ms"])
+    c = clk.summary(t["windows"]) if clk is not None else dict(sm_mhz=None, reasons=[])
+    kcyc = ms * c["sm_mhz"] if c["sm_mhz"] else None
+    return dict(ms=ms, ms_blocks=t["block_ms"], sm_mhz=c["sm_mhz"], reasons=c["reasons"],
+                kcycles=kcyc)
+
+
+def speedups(res, base_key):
+    """Speedup of every arm over the base arm: plain and clock-normalised."""
+    b = res[base_key]
+    for v in res.values():
+        v["speedup_vs_lambda0"] = b["ms"] / v["ms"]
+        v["speedup_clk"] = (b["kcycles"] / v["kcycles"]) if (b["kcycles"] and v["kcycles"]) else None
 
 
 def measure_prefill(w, lam, steps, warmup, device, stream, flush_buf, pre=None, block_mask=None):
@@ -296,10 +351,10 @@ def measure_decode_mla(w, steps, device, stream, flush_buf, peaks, Bc=64):
                   tensor_frac=top["algorithmic_tflops"] / peaks["bf16_tflops"],
                   hbm_frac=hbm_gbs / peaks["hbm_gbs"], algorithmic_bytes=int(alg),
                   traffic=profiled_traffic("decode_mla_64k") if w.name == "decode_mla_64k" else None,
-                  note=("tcgen05, 128 heads per cluster of two CTAs (each forms half of every score "
-                        "over 288 dims, the halves exchanged through distributed shared memory, "
-                        "and accumulates one half of the output); the call also holds the split "
-                        "merge") if w.Hq % 128 == 0 else
+                  note=("tcgen05, 128 heads: two CTAs per (sequence, split), each forms the "
+                        "full 576-wide scores and accumulates one 256-column half of the output, "
+                        "so the score product runs twice; the call also holds the split merge")
+                  if w.Hq % 128 == 0 else
                        ("mma.sync m16n8k16 tiles (16 heads per CTA); the cache is read once from "
                         "HBM, re-read from L2 by each head group"))
     if t_hbm >= t_tc:
@@ -384,42 +439,6 @@ def measure_backward(w, lam, steps, warmup, device, stream, flush_buf, pre=None,
     return pre, bwd, dict(ms=ms, times=times, pairs=pairs, exec_flops=float(flops),
                           executed_tflops=flops / (ms * 1e-3) / 1e12,
                           skip_frac=float((mask == 1).sum()) / max(int((mask != 2).sum()), 1))
-
-
-def measure_decode(w, lam, steps, warmup, device, stream, flush_buf):
-    import torch
-    import dynamic_block_sparse_tiled_b200 as bl
-    import synth
-    inp = synth.generate(w)
-    to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
-    q, k, v = to(inp.q), to(inp.k), to(inp.v)
-    del inp
-    ws = torch.empty(bl.blasst_decode_workspace_bytes(w.B, w.Hq, w.d, w.num_splits),
-                     dtype=torch.uint8, device=device)
-    o = torch.empty((w.B, w.Hq, 1, w.d), dtype=torch.bfloat16, device=device)
-    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
-    mask = torch.empty((w.B, w.Hq, -(-w.Lkv // w.Bc)), dtype=torch.uint8, device=device)
-    out = {}
-    for lm in (0.0, lam):
-        st = bl.new_stats(device)
-        bl.blasst_decode(q, k, v, o, lse, lam=lm, Bc=w.Bc, num_splits=w.num_splits, workspace=ws,
-                         skip_mask_out=mask, stats_out=st, stream=stream)
-        rc = bl.blasst_check(stream)
-        if rc != 0:
-            raise RuntimeError(bl.blasst_status_string(rc))
-        sd = bl.stats_dict(st)
-        fn = lambda: bl.blasst_decode(q, k, v, o, lse, lam=lm, Bc=w.Bc, num_splits=w.num_splits,
-                                      workspace=ws, stream=stream)
-        times = time_calls(fn, steps, warmup, stream, flush_buf)
-        m = mask.cpu().numpy()
-        ws_bytes = ws.numel()
-        # algorithmic bytes: K always, V when some head of the group keeps the
-        # block, the split partials written then read back by the merge, q, o
-        alg = sd["bytes_loaded"] + 2 * ws_bytes + q.numel() * 2 + o.numel() * 2
-        out[lm] = dict(ms=statistics.mean(times), bytes=alg, skip_frac=float((m == 1).mean()),
-                       v_blocks=sd["v_blocks_loaded"],
-                       v_fetch_frac=sd["v_blocks_loaded"] / max(1, w.B * w.Hkv * (-(-w.Lkv // w.Bc))))
-    return out
 
 
 class E2EPipeline:
@@ -532,6 +551,109 @@ def block_sparse_pattern(w, sink_blocks=1, band_blocks=8, random_frac=0.1, seed=
         diag = min(nKt - 1, (min(qt * w.Br + w.Br, w.Lq) - 1 + off) // w.Bc)
         keep[:, :, qt, max(0, diag - band_blocks + 1):diag + 1] = True
     return (~keep).astype(np.uint8)
+
+
+# ------------------------------------------------------------ lambda legs
+def prefill_lambda_leg(w, lams, rounds, per, device, stream, flush_buf, clk, peaks, pre=None):
+    """One prefill workload at several lambdas: decisions and counters from
+    one call each, then the lambdas timed as interleaved blocks. Reports the
+    skip fraction (for workloads with diffuse heads also split into the
+    structured and the diffuse heads), executed and effective TFLOP/s, the
+    executed fraction of the bf16 peak, and the speedup over lambda = 0,
+    plain and clock-normalised."""
+    import dynamic_block_sparse_tiled_b200 as bl
+    own = pre is None
+    pre = pre or Prefill(w, device)
+    res = {}
+    for lam in lams:
+        st = bl.new_stats(device)
+        pre.run(lam, stats=st, stream=stream)
+        stream.synchronize()
+        rc = bl.blasst_check(stream)
+        if rc != 0:
+            raise RuntimeError(bl.blasst_status_string(rc))
+        sd = bl.stats_dict(st)
+        m = pre.mask.cpu().numpy()
+        vis = m != 2
+        r = dict(skip_frac=float((m == 1).sum()) / max(int(vis.sum()), 1),
+                 exec_flops=float(sd["mma_flops"]), v_blocks=sd["v_blocks_loaded"])
+        if w.diffuse_heads == "upper_half":
+            h = w.Hq // 2  # query heads of the diffuse KV heads (contiguous GQA groups)
+            r["skip_frac_structured"] = float((m[:, :h] == 1).sum()) / max(int(vis[:, :h].sum()), 1)
+            r["skip_frac_diffuse"] = float((m[:, h:] == 1).sum()) / max(int(vis[:, h:].sum()), 1)
+        res[lam] = r
+    t = time_interleaved([(lam, (lambda lam=lam: pre.run(lam, stream=stream))) for lam in lams],
+                         rounds, per, 2, stream, flush_buf)
+    eff = effective_flops(w)
+    for lam in lams:
+        r = res[lam]
+        r.update(arm_summary(t[lam], clk))
+        r["executed_tflops"] = r["exec_flops"] / (r["ms"] * 1e-3) / 1e12
+        r["effective_tflops"] = eff / (r["ms"] * 1e-3) / 1e12
+        r["frac"] = r["executed_tflops"] / peaks["bf16_tflops"]
+    speedups(res, lams[0])
+    if own:
+        del pre
+    return res
+
+
+def decode_lambda_leg(w, lam, rounds, per, device, stream, flush_buf, clk, peaks):
+    """Split-KV decode at lambda = 0 and at `lam`, interleaved: the fraction
+    of (group, block) V fetches made, the bytes the skipped fetches save, and
+    the HBM roofline on the bytes each call actually moves."""
+    import torch
+    import dynamic_block_sparse_tiled_b200 as bl
+    import synth
+    inp = synth.generate(w)
+    to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+    q, k, v = to(inp.q), to(inp.k), to(inp.v)
+    del inp
+    ws = torch.empty(bl.blasst_decode_workspace_bytes(w.B, w.Hq, w.d, w.num_splits),
+                     dtype=torch.uint8, device=device)
+    o = torch.empty((w.B, w.Hq, 1, w.d), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
+    mask = torch.empty((w.B, w.Hq, -(-w.Lkv // w.Bc)), dtype=torch.uint8, device=device)
+    lams = (0.0, lam)
+    res = {}
+    for lm in lams:
+        st = bl.new_stats(device)
+        bl.blasst_decode(q, k, v, o, lse, lam=lm, Bc=w.Bc, num_splits=w.num_splits, workspace=ws,
+                         skip_mask_out=mask, stats_out=st, stream=stream)
+        rc = bl.blasst_check(stream)
+        if rc != 0:
+            raise RuntimeError(bl.blasst_status_string(rc))
+        sd = bl.stats_dict(st)
+        m = mask.cpu().numpy()
+        # algorithmic bytes: K always, V when some head of the group keeps the
+        # block, the split partials written then read back by the merge, q, o
+        alg = sd["bytes_loaded"] + 2 * ws.numel() + q.numel() * 2 + o.numel() * 2
+        res[lm] = dict(bytes=int(alg), skip_frac=float((m == 1).mean()),
+                       v_blocks=sd["v_blocks_loaded"],
+                       v_fetch_frac=sd["v_blocks_loaded"] / max(1, w.B * w.Hkv * (-(-w.Lkv // w.Bc))))
+    t = time_interleaved(
+        [(lm, (lambda lm=lm: bl.blasst_decode(q, k, v, o, lse, lam=lm, Bc=w.Bc,
+                                              num_splits=w.num_splits, workspace=ws,
+                                              stream=stream))) for lm in lams],
+        rounds, per, 3, stream, flush_buf)
+    for lm in lams:
+        r = res[lm]
+        r.update(arm_summary(t[lm], clk))
+        r["gbs"] = r["bytes"] / (r["ms"] * 1e-3) / 1e9
+        r["frac"] = r["gbs"] / peaks["hbm_gbs"]
+    speedups(res, 0.0)
+    res[lam]["bytes_saved"] = res[0.0]["bytes"] - res[lam]["bytes"]
+    return res
+
+
+def _r(x, n=3):
+    """Round for the compact summary line (None passes through)."""
+    if x is None:
+        return None
+    if isinstance(x, float):
+        if x == 0.0 or not math.isfinite(x):
+            return x
+        return float(f"{x:.{n}g}")
+    return x
 
 
 # ------------------------------------------------------------- CPU oracle
@@ -712,13 +834,178 @@ def run_reference(args):
     return 0
 
 
+def leg_static_mask(w, args, device, stream, flush_buf):
+    """Static block-sparse input (a selector-shaped mask) on the 32K workload."""
+    import torch
+    sm_dev = torch.from_numpy(block_sparse_pattern(w)).to(device)
+    ps = Prefill(w, device)
+    steps = max(3, args.steps // 2)
+    ps, s_r = measure_prefill(w, LAMBDA, steps, 3, device, stream, flush_buf, pre=ps,
+                              block_mask=sm_dev)
+    _, s0_r = measure_prefill(w, LAMBDA, steps, 3, device, stream, flush_buf, pre=ps)
+    nvis = s_r["tiles_visited"]
+    return dict(pattern="first block + 8-block diagonal band + 10 % seeded random blocks per "
+                        "query tile", visited_tiles=nvis,
+                visited_frac_of_causal=nvis / max(1, s0_r["tiles_visited"]),
+                ms=s_r["ms"], ms_no_mask=s0_r["ms"], speedup_vs_no_mask=s0_r["ms"] / s_r["ms"],
+                executed_tflops=s_r["exec_flops"] / (s_r["ms"] * 1e-3) / 1e12)
+
+
+def leg_selector(args, device, stream, flush_buf, peaks):
+    """Pre-pass block selector (CRISP-style) on the literal and calibrated 32K
+    workloads, and the forward with and without its mask."""
+    import torch
+    import synth
+    import dynamic_block_sparse_tiled_b200 as bl
+    sel = {}
+    for wn in (WORKLOAD, WORKLOAD + "_a12"):
+        ws_ = synth.CONFIGS[wn]
+        ps = Prefill(ws_, device)
+        nq, nk = -(-ws_.Lq // ws_.Br), -(-ws_.Lkv // ws_.Bc)
+        smask = torch.empty((ws_.B, ws_.Hq, nq, nk), dtype=torch.uint8, device=device)
+        sws = torch.empty(bl.blasst_select_workspace_bytes(ws_.B, ws_.Hq, ws_.Hkv, ws_.Lq,
+                                                           ws_.Lkv, ws_.d, ws_.Br, ws_.Bc),
+                          dtype=torch.uint8, device=device)
+        run_sel = lambda: bl.blasst_select_blocks(ps.q, ps.k, smask, causal=ws_.causal,
+                                                  Br=ws_.Br, Bc=ws_.Bc, tau=SEL_TAU,
+                                                  gamma=SEL_GAMMA, workspace=sws, stream=stream)
+        run_sel()
+        stream.synchronize()
+        t_sel = statistics.mean(time_calls(run_sel, max(5, args.steps), 3, stream, flush_buf))
+        causal_tiles = causal_pairs(nq, nk) * ws_.B * ws_.Hq
+        nsel = int((smask == 0).sum().item())
+        steps = max(3, args.steps // 2)
+        ps, m_r = measure_prefill(ws_, LAMBDA, steps, 3, device, stream, flush_buf, pre=ps,
+                                  block_mask=smask)
+        _, n_r = measure_prefill(ws_, LAMBDA, steps, 3, device, stream, flush_buf, pre=ps)
+        sel_bytes = 2.0 * ws_.d * (ws_.B * ws_.Hq * ws_.Lq + ws_.B * ws_.Hkv * ws_.Lkv)
+        gbs = sel_bytes / (t_sel * 1e-3) / 1e9
+        sel[wn] = dict(selector_ms=t_sel, selected_frac_of_causal=nsel / max(causal_tiles, 1),
+                       fwd_ms_with_mask=m_r["ms"], fwd_ms_without=n_r["ms"],
+                       speedup_selector_plus_fwd=n_r["ms"] / (t_sel + m_r["ms"]),
+                       roofline=dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"],
+                                     unit="GB/s", frac=gbs / peaks["hbm_gbs"],
+                                     algorithmic="Q and K read once (bf16)"))
+        del ps, smask, sws
+        torch.cuda.empty_cache()
+    return dict(tau=SEL_TAU, gamma=SEL_GAMMA, **sel)
+
+
+def leg_mla(args, device, stream, flush_buf, peaks):
+    """MLA-shaped decode (latent cache, 128 heads), literal and calibrated,
+    and the mma.sync kernel on a 112-head shape."""
+    import synth
+    import dynamic_block_sparse_tiled_b200 as bl
+    mla = {}
+    for wn in ("decode_mla_64k", "decode_mla_64k_a12"):
+        mla[wn] = measure_decode_mla(synth.CONFIGS[wn], max(5, args.steps), device, stream,
+                                     flush_buf, peaks)
+    base = synth.CONFIGS["decode_mla_64k"]
+    mla["decode_mla_64k_h112_mma_sync"] = measure_decode_mla(
+        base.replace(name="decode_mla_64k_h112", Hq=112,
+                     num_splits=bl.blasst_decode_mla_splits(8, 112, base.Lkv)),
+        max(5, args.steps), device, stream, flush_buf, peaks)
+    return mla
+
+
+def leg_backward(w, wa, args, device, stream, flush_buf, peaks):
+    """Backward with the forward's decisions held fixed (32K literal at
+    lambda = 1e-3; calibrated at lambda = 1e-3 against lambda = 0)."""
+    import torch
+    steps = max(3, args.steps // 2)
+    pb = Prefill(w, device)
+    pb, bb, b_l = measure_backward(w, LAMBDA, steps, 3, device, stream, flush_buf, pre=pb)
+    del pb, bb
+    torch.cuda.empty_cache()
+    pb = Prefill(wa, device)
+    pb, bb, ba_l = measure_backward(wa, LAMBDA, steps, 3, device, stream, flush_buf, pre=pb)
+    _, _, ba_0 = measure_backward(wa, 0.0, steps, 3, device, stream, flush_buf, pre=pb, bwd=bb)
+    del pb, bb
+    torch.cuda.empty_cache()
+    return dict(
+        ms=b_l["ms"], pairs=b_l["pairs"], skip_frac=b_l["skip_frac"],
+        executed_tflops=b_l["executed_tflops"],
+        roofline=dict(bound="tensor", achieved=b_l["executed_tflops"], peak=peaks["bf16_tflops"],
+                      unit="TFLOP/s", frac=b_l["executed_tflops"] / peaks["bf16_tflops"],
+                      traffic=profiled_traffic("backward_32k"),
+                      algorithmic="per computed (64-row tile, 128-key block) pair: 5 products "
+                                  "of 2*128*64*128 flops (S^T, dP^T, dV, dK, dQ^T)"),
+        a12=dict(ms=ba_l["ms"], ms_lambda0=ba_0["ms"], speedup_vs_lambda0=ba_0["ms"] / ba_l["ms"],
+                 skip_frac=ba_l["skip_frac"], executed_tflops=ba_l["executed_tflops"]),
+        note="dq, dk, dv in fp32; one call = the row pass (rowsum(dO*O), dq cleared) and the "
+             "pair kernel")
+
+
+def detail(name, obj):
+    """A leg's full record, on stderr (stdout carries the one summary line)."""
+    def conv(x):
+        if isinstance(x, dict):
+            return {str(k): conv(v) for k, v in x.items()}
+        if isinstance(x, (list, tuple)):
+            return [conv(v) for v in x]
+        if isinstance(x, (np.integer,)):
+            return int(x)
+        if isinstance(x, (np.floating,)):
+            return float(x)
+        return x
+    print(json.dumps({"detail": name, **conv(obj)}), file=sys.stderr, flush=True)
+
+
+def compact_legs(legs):
+    """The legs' key figures for the summary line (full records: stderr)."""
+    out = {}
+
+    def lam_arm(r, frac=False):
+        d = dict(skip=_r(r["skip_frac"]), x=_r(r["speedup_vs_lambda0"]), xc=_r(r["speedup_clk"]))
+        if frac:
+            d["frac"] = _r(r["frac"])
+        for k, kk in (("skip_frac_structured", "skip_s"), ("skip_frac_diffuse", "skip_d")):
+            if k in r:
+                d[kk] = _r(r[k])
+        return d
+
+    for key, lam in (("p32k", LAMBDA), ("p32k_a12", LAMBDA), ("p256k", 1e-3),
+                     ("p256k_a12", 1e-3)):
+        if key in legs:
+            out[key] = lam_arm(legs[key][lam], frac=True)
+    for key in ("p128k", "p128k_a12"):
+        if key in legs:
+            out[key] = {f"{lam:g}": [_r(r["skip_frac"]), _r(r["speedup_vs_lambda0"]),
+                                     _r(r["speedup_clk"])]
+                        for lam, r in legs[key].items() if lam != 0.0}
+    for key in ("dec", "dec_a12"):
+        if key in legs:
+            r, r0 = legs[key][LAMBDA], legs[key][0.0]
+            out[key] = dict(ms=_r(r["ms"]), gbs=_r(r["gbs"], 4), frac=_r(r["frac"]),
+                            frac_l0=_r(r0["frac"]), x=_r(r["speedup_vs_lambda0"]),
+                            xc=_r(r["speedup_clk"]), skip=_r(r["skip_frac"]),
+                            vfetch=_r(r["v_fetch_frac"]), saved_gb=_r(r["bytes_saved"] / 1e9))
+    if "mla" in legs:
+        rf = legs["mla"]["decode_mla_64k"]["roofline"]
+        out["mla"] = dict(ms=_r(legs["mla"]["decode_mla_64k"][str(1e-3)]["ms"]), bound=rf["bound"],
+                          frac=_r(rf["frac"]), tensor_frac=_r(rf["tensor_frac"]))
+    if "bwd" in legs:
+        b = legs["bwd"]
+        tr = b["roofline"]["traffic"]
+        out["bwd"] = dict(ms=_r(b["ms"]), frac=_r(b["roofline"]["frac"]),
+                          traffic_gb=_r(tr / 1e9) if tr else None,
+                          a12_x=_r(b["a12"]["speedup_vs_lambda0"]))
+    if "sel" in legs:
+        s = legs["sel"][WORKLOAD]
+        out["sel"] = dict(ms=_r(s["selector_ms"]), frac=_r(s["roofline"]["frac"]))
+    if "static" in legs:
+        out["static"] = dict(x=_r(legs["static"]["speedup_vs_no_mask"]))
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="blasst", choices=["blasst", "reference"])
-    ap.add_argument("--quick", action="store_true", help="skip the 128K and decode legs")
+    ap.add_argument("--quick", action="store_true",
+                    help="headline, its lambda = 0 pair and the end-to-end number only")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--case", default=None,
                     help="profiling driver: run only this workload's kernel --calls times, untimed "
@@ -748,160 +1035,59 @@ def main():
     flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
     peaks = load_peaks()
     w = synth.CONFIGS[WORKLOAD]
-
-    # ---- headline: prefill 32K, lambda 1e-3, literal generator -------------
-    # (the clock record spans the headline steps and the lambda = 0 and
-    # calibrated-variant legs of the same kernel right after them)
-    pre = Prefill(w, device)
     wa = synth.CONFIGS[WORKLOAD + "_a12"]
-    pa = Prefill(wa, device)
-    ranks.barrier()
+    legs = {}
+
     with ClockSampler(local) as clk:
-        pre, main_r = measure_prefill(w, LAMBDA, args.steps, args.warmup, device, stream, flush_buf,
-                                      pre=pre)
+        # ---- headline: prefill 32K, lambda 1e-3, literal generator ---------
+        pre = Prefill(w, device)
         ranks.barrier()
-        _, dense_r = measure_prefill(w, 0.0, max(3, args.steps // 2), 3, device, stream, flush_buf,
-                                     pre=pre)
-        pa, a_l = measure_prefill(wa, LAMBDA, max(3, args.steps // 2), 3, device, stream, flush_buf,
-                                  pre=pa)
-        _, a_0 = measure_prefill(wa, 0.0, max(3, args.steps // 2), 3, device, stream, flush_buf,
-                                 pre=pa)
-    ms = ranks.max(main_r["ms"])
-    value = ranks.aggregate(main_r["eff_flops"], main_r["ms"]) / 1e12
-    del pre, pa
-    torch.cuda.empty_cache()
+        t_head = time.time()
+        pre, main_r = measure_prefill(w, LAMBDA, args.steps, args.warmup, device, stream,
+                                      flush_buf, pre=pre)
+        ranks.barrier()
+        head_win = [(t_head, time.time())]
+        ms = ranks.max(main_r["ms"])
+        value = ranks.aggregate(main_r["eff_flops"], main_r["ms"]) / 1e12
 
-    extra = {}
-    extra["structured_a12"] = dict(
-        skip_frac=a_l["skip_frac"], ms=a_l["ms"], ms_lambda0=a_0["ms"],
-        speedup_vs_lambda0=a_0["ms"] / a_l["ms"],
-        effective_tflops=a_l["eff_flops"] / (a_l["ms"] * 1e-3) / 1e12,
-        executed_tflops=a_l["exec_flops"] / (a_l["ms"] * 1e-3) / 1e12,
-        note="calibrated variant: planted amplitude 12 instead of 3 (the literal generator leaves "
-             "almost no block under the threshold)")
-
-    if not args.quick:
-        w3 = synth.CONFIGS["prefill_128k_a12"]
-        p3 = Prefill(w3, device)
-        curve = {}
-        for lam in (0.0, 1e-4, 1e-3, 1e-2):
-            _, r3 = measure_prefill(w3, lam, 3, 3, device, stream, flush_buf, pre=p3)
-            curve[str(lam)] = dict(ms=r3["ms"], skip_frac=r3["skip_frac"],
-                                   effective_tflops=r3["eff_flops"] / (r3["ms"] * 1e-3) / 1e12,
-                                   executed_tflops=r3["exec_flops"] / (r3["ms"] * 1e-3) / 1e12)
-        base = curve["0.0"]["ms"]
-        for v in curve.values():
-            v["speedup_vs_lambda0"] = base / v["ms"]
-        extra["prefill_128k_a12_lambda_curve"] = curve
-        del p3
+        # ---- lambda = 0 against lambda = 1e-3, interleaved, same inputs ----
+        legs["p32k"] = prefill_lambda_leg(w, (0.0, LAMBDA), 6, 3, device, stream, flush_buf, clk,
+                                          peaks, pre=pre)
+        del pre
         torch.cuda.empty_cache()
-
-        # static block-sparse input (a selector's mask) on the 32K workload
-        import torch as _t
-        sm = block_sparse_pattern(w)
-        sm_dev = _t.from_numpy(sm).to(device)
-        ps = Prefill(w, device)
-        ps, s_r = measure_prefill(w, LAMBDA, max(3, args.steps // 2), 3, device, stream, flush_buf,
-                                  pre=ps, block_mask=sm_dev)
-        _, s0_r = measure_prefill(w, LAMBDA, max(3, args.steps // 2), 3, device, stream, flush_buf,
-                                  pre=ps)
-        nvis = s_r["tiles_visited"]
-        extra["static_block_sparse_32k"] = dict(
-            pattern="first block + 8-block diagonal band + 10 % seeded random blocks per query tile",
-            visited_tiles=nvis, visited_frac_of_causal=nvis / max(1, s0_r["tiles_visited"]),
-            ms=s_r["ms"], ms_no_mask=s0_r["ms"], speedup_vs_no_mask=s0_r["ms"] / s_r["ms"],
-            executed_tflops=s_r["exec_flops"] / (s_r["ms"] * 1e-3) / 1e12)
-        del ps, sm_dev
-        torch.cuda.empty_cache()
-
-        # pre-pass block selector (CRISP-style) feeding the static mask
-        sel = {}
-        for wn in (WORKLOAD, WORKLOAD + "_a12"):
-            ws_ = synth.CONFIGS[wn]
-            ps = Prefill(ws_, device)
-            nq, nk = -(-ws_.Lq // ws_.Br), -(-ws_.Lkv // ws_.Bc)
-            smask = torch.empty((ws_.B, ws_.Hq, nq, nk), dtype=torch.uint8, device=device)
-            sws = torch.empty(bl.blasst_select_workspace_bytes(ws_.B, ws_.Hq, ws_.Hkv, ws_.Lq,
-                                                               ws_.Lkv, ws_.d, ws_.Br, ws_.Bc),
-                              dtype=torch.uint8, device=device)
-            run_sel = lambda: bl.blasst_select_blocks(ps.q, ps.k, smask, causal=ws_.causal,
-                                                      Br=ws_.Br, Bc=ws_.Bc, tau=SEL_TAU,
-                                                      gamma=SEL_GAMMA, workspace=sws,
-                                                      stream=stream)
-            run_sel()
-            stream.synchronize()
-            t_sel = statistics.mean(time_calls(run_sel, max(5, args.steps), 3, stream, flush_buf))
-            causal_tiles = causal_pairs(-(-ws_.Lq // ws_.Br), -(-ws_.Lkv // ws_.Bc)) * ws_.B * ws_.Hq
-            nsel = int((smask == 0).sum().item())
-            ps, m_r = measure_prefill(ws_, LAMBDA, max(3, args.steps // 2), 3, device, stream,
-                                      flush_buf, pre=ps, block_mask=smask)
-            _, n_r = measure_prefill(ws_, LAMBDA, max(3, args.steps // 2), 3, device, stream,
-                                     flush_buf, pre=ps)
-            sel_bytes = 2.0 * ws_.d * (ws_.B * ws_.Hq * ws_.Lq + ws_.B * ws_.Hkv * ws_.Lkv)
-            gbs = sel_bytes / (t_sel * 1e-3) / 1e9
-            sel[wn] = dict(selector_ms=t_sel, selected_frac_of_causal=nsel / max(causal_tiles, 1),
-                           fwd_ms_with_mask=m_r["ms"], fwd_ms_without=n_r["ms"],
-                           speedup_selector_plus_fwd=n_r["ms"] / (t_sel + m_r["ms"]),
-                           roofline=dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"],
-                                         unit="GB/s", frac=gbs / peaks["hbm_gbs"],
-                                         algorithmic="Q and K read once (bf16)"))
-            del ps, smask, sws
+        # The other legs measure per-GPU properties of the kernels; replicas
+        # (N > 1) time the headline and the end-to-end loop only.
+        if ws == 1:
+            legs["p32k_a12"] = prefill_lambda_leg(wa, (0.0, LAMBDA), 6, 3, device, stream,
+                                                  flush_buf, clk, peaks)
             torch.cuda.empty_cache()
-        extra["selector_32k"] = dict(tau=SEL_TAU, gamma=SEL_GAMMA, **sel)
-
-        # MLA-shaped decode (latent cache, 128 heads), literal and calibrated
-        mla = {}
-        for wn in ("decode_mla_64k", "decode_mla_64k_a12"):
-            mla[wn] = measure_decode_mla(synth.CONFIGS[wn], max(5, args.steps), device, stream,
-                                         flush_buf, peaks)
-        mla["decode_mla_64k_h112_mma_sync"] = measure_decode_mla(
-            synth.CONFIGS["decode_mla_64k"].replace(
-                name="decode_mla_64k_h112", Hq=112,
-                num_splits=bl.blasst_decode_mla_splits(8, 112, synth.CONFIGS["decode_mla_64k"].Lkv)),
-            max(5, args.steps), device, stream, flush_buf, peaks)
-        extra["decode_mla_64k"] = mla
-
-        # backward with the forward's decisions held fixed, 32K workload
-        pb = Prefill(w, device)
-        pb, bb, b_l = measure_backward(w, LAMBDA, max(3, args.steps // 2), 3, device, stream,
-                                       flush_buf, pre=pb)
-        del pb, bb
-        torch.cuda.empty_cache()
-        pb = Prefill(wa, device)
-        pb, bb, ba_l = measure_backward(wa, LAMBDA, max(3, args.steps // 2), 3, device, stream,
-                                        flush_buf, pre=pb)
-        _, _, ba_0 = measure_backward(wa, 0.0, max(3, args.steps // 2), 3, device, stream,
-                                      flush_buf, pre=pb, bwd=bb)
-        del pb, bb
-        torch.cuda.empty_cache()
-        extra["backward_32k"] = dict(
-            ms=b_l["ms"], pairs=b_l["pairs"], skip_frac=b_l["skip_frac"],
-            executed_tflops=b_l["executed_tflops"],
-            roofline=dict(bound="tensor", achieved=b_l["executed_tflops"],
-                          peak=peaks["bf16_tflops"], unit="TFLOP/s",
-                          frac=b_l["executed_tflops"] / peaks["bf16_tflops"],
-                          traffic=profiled_traffic("backward_32k"),
-                          algorithmic="per computed (64-row tile, 128-key block) pair: 5 products "
-                                      "of 2*128*64*128 flops (S^T, dP^T, dV, dK, dQ^T)"),
-            a12=dict(ms=ba_l["ms"], ms_lambda0=ba_0["ms"], speedup_vs_lambda0=ba_0["ms"] / ba_l["ms"],
-                     skip_frac=ba_l["skip_frac"], executed_tflops=ba_l["executed_tflops"]),
-            note="dq, dk, dv in fp32; one call = the row pass (rowsum(dO*O), dq cleared) and the "
-                 "pair kernel")
-
-        wd = synth.CONFIGS["decode_64k"]
-        dres = measure_decode(wd, LAMBDA, max(5, args.steps), 3, device, stream, flush_buf)
-        d = dres[LAMBDA]
-        d0 = dres[0.0]
-        gbs = d["bytes"] / (d["ms"] * 1e-3) / 1e9
-        extra["decode_64k"] = dict(
-            ms=d["ms"], ms_lambda0=d0["ms"], speedup_vs_lambda0=d0["ms"] / d["ms"],
-            skip_frac=d["skip_frac"], v_fetch_frac=d["v_fetch_frac"],
-            roofline=dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
-                          frac=gbs / peaks["hbm_gbs"], traffic=profiled_traffic("decode_64k"),
-                          achieved_lambda0=d0["bytes"] / (d0["ms"] * 1e-3) / 1e9,
-                          peak_source=f"{peaks['source']} hbm_gbs (copy)",
-                          vs_8tbs=gbs / 8000.0))
-        torch.cuda.empty_cache()
+        if ws == 1 and not args.quick:
+            lam4 = (0.0, 1e-4, 1e-3, 1e-2)
+            for key, wn in (("p128k", "prefill_128k"), ("p128k_a12", "prefill_128k_a12")):
+                legs[key] = prefill_lambda_leg(synth.CONFIGS[wn], lam4, 4, 1, device, stream,
+                                               flush_buf, clk, peaks)
+                torch.cuda.empty_cache()
+            for key, wn in (("p256k", "prefill_256k"), ("p256k_a12", "prefill_256k_a12")):
+                legs[key] = prefill_lambda_leg(synth.CONFIGS[wn], (0.0, 1e-3), 4, 1, device,
+                                               stream, flush_buf, clk, peaks)
+                torch.cuda.empty_cache()
+            for key, wn in (("dec", "decode_64k"), ("dec_a12", "decode_64k_a12")):
+                legs[key] = decode_lambda_leg(synth.CONFIGS[wn], LAMBDA, 6, 5, device, stream,
+                                              flush_buf, clk, peaks)
+                torch.cuda.empty_cache()
+            legs["static"] = leg_static_mask(w, args, device, stream, flush_buf)
+            torch.cuda.empty_cache()
+            legs["sel"] = leg_selector(args, device, stream, flush_buf, peaks)
+            legs["mla"] = leg_mla(args, device, stream, flush_buf, peaks)
+            torch.cuda.empty_cache()
+            legs["bwd"] = leg_backward(w, wa, args, device, stream, flush_buf, peaks)
+            torch.cuda.empty_cache()
+            if rank == 0:
+                d = legs["dec"][LAMBDA]
+                legs["dec"]["roofline"] = dict(
+                    bound="hbm", achieved=d["gbs"], peak=peaks["hbm_gbs"], unit="GB/s",
+                    frac=d["frac"], traffic=profiled_traffic("decode_64k"),
+                    peak_source=f"{peaks['source']} hbm_gbs (copy)", vs_8tbs=d["gbs"] / 8000.0)
 
     # ---- end to end through the public API with host buffers ---------------
     e2e = measure_e2e(w, LAMBDA, max(8, args.steps), 3, device, stream)
@@ -912,14 +1098,19 @@ def main():
     roofline = dict(bound="tensor", achieved=exec_tflops, peak=peaks["bf16_tflops"], unit="TFLOP/s",
                     frac=exec_tflops / peaks["bf16_tflops"],
                     traffic=profiled_traffic("prefill_32k"),
-                    peak_source=f"{peaks['source']} bf16_tflops (burst; the kernel is timed alone)",
-                    frac_of_sustained=exec_tflops / peaks["bf16_tflops_sustained"],
-                    algorithmic="per visited (128-row tile, 128-key block): 2*128*128*128 flops for "
-                                "S=QK^T, plus the same for O+=PV when the block is computed")
+                    frac_of_sustained=exec_tflops / peaks["bf16_tflops_sustained"])
 
     if rank == 0:
+        for k, v in legs.items():
+            detail(k, v)
+        detail("roofline_notes", dict(
+            peak_source=f"{peaks['source']} bf16_tflops (burst; the kernel is timed alone)",
+            algorithmic="per visited (128-row tile, 128-key block): 2*128*128*128 flops for "
+                        "S=QK^T, plus the same for O+=PV when the block is computed",
+            e2e_pipelined=e2e.pop("pipelined")))
         cpu = oracle_sample(w, LAMBDA, args.cpu_budget)
-        clocks = clk.summary()
+        clocks = clk.summary(head_win)
+        l0 = legs["p32k"]
         line = dict(
             metric=METRIC, value=value, unit=UNIT, n_gpus=ws, steps=args.steps, warmup=args.warmup,
             ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
@@ -928,11 +1119,22 @@ def main():
                         causal=w.causal, Br=w.Br, Bc=w.Bc, amplitude=w.amp,
                         parallelism=f"replicas{ws}", l2="flushed between steps; inputs > L2",
                         **{"lambda": LAMBDA}),
+            roofline=roofline,
+            cpu_baseline={k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            e2e=e2e, clocks={k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
             skip_frac=main_r["skip_frac"], executed_tflops=exec_tflops,
-            ms_lambda0=dense_r["ms"], speedup_vs_lambda0=dense_r["ms"] / main_r["ms"],
-            roofline=roofline, cpu_baseline={k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
-            e2e=e2e, clocks=clocks, **extra)
-        print(json.dumps(line), flush=True)
+            ms_lambda0=l0[0.0]["ms"], speedup_vs_lambda0=l0[LAMBDA]["speedup_vs_lambda0"],
+            speedup_vs_lambda0_clk=l0[LAMBDA]["speedup_clk"],
+            legs=compact_legs(legs))
+        for k in ("value", "ms_per_step", "executed_tflops", "ms_lambda0", "speedup_vs_lambda0",
+                  "speedup_vs_lambda0_clk"):
+            line[k] = _r(line[k], 4)
+        for k in ("achieved", "frac", "frac_of_sustained"):
+            line["roofline"][k] = _r(line["roofline"][k], 4)
+        line["e2e"]["value"] = _r(line["e2e"]["value"], 4)
+        line["e2e"].pop("steps", None)
+        line["cpu_baseline"]["value"] = _r(line["cpu_baseline"]["value"], 4)
+        print(json.dumps(line, separators=(",", ":")), flush=True)
     ranks.close()
     return 0
 

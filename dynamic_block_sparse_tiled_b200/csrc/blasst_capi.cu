@@ -509,28 +509,36 @@ size_t blasst_decode_workspace_bytes(int B, int Hq, int d, int num_splits) {
   return o_bytes + rows * sizeof(float);
 }
 
-int blasst_lse_merge(const float* o_parts, const float* lse_parts, void* o, float* lse, int n_rows,
-                     int d, int num_splits, int out_dtype, void* stream) {
-  if (!o_parts || !lse_parts || !o || !lse || n_rows <= 0 || d <= 0 || num_splits <= 0)
-    return BLASST_EINVAL;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+}  // extern "C"
+
+namespace {
+
+// The merge kernel launch. `err` (nullable) is the device error word: when it
+// holds an error on entry (a bounded wait of the split kernel before it gave
+// up), the kernel writes NaN outputs and -inf lse instead of merging partials
+// that may not have been written.
+int launch_lse_merge(const float* o_parts, const float* lse_parts, void* o, float* lse,
+                     int n_rows, int d, int num_splits, int out_dtype, const int* err,
+                     cudaStream_t s) {
   const int threads = d >= 128 ? 128 : ((d + 31) / 32) * 32;
   if (out_dtype == BLASST_BF16) {
     blasst::blasst_lse_merge_kernel<__nv_bfloat16><<<n_rows, threads, 0, s>>>(
-        o_parts, lse_parts, static_cast<__nv_bfloat16*>(o), lse, d, num_splits);
+        o_parts, lse_parts, static_cast<__nv_bfloat16*>(o), lse, d, num_splits, err);
   } else if (out_dtype == BLASST_FP32) {
     blasst::blasst_lse_merge_kernel<float><<<n_rows, threads, 0, s>>>(
-        o_parts, lse_parts, static_cast<float*>(o), lse, d, num_splits);
+        o_parts, lse_parts, static_cast<float*>(o), lse, d, num_splits, err);
   } else {
     return BLASST_EINVAL;
   }
   return cuda_status(cudaGetLastError());
 }
 
-int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
-                  int B, int Hq, int Hkv, int Lkv, int d, float lambda, int Bc, int num_splits,
-                  void* workspace, size_t workspace_bytes, uint8_t* skip_mask_out,
-                  blasst_stats* stats_out, void* stream) {
+// Argument checks of blasst_decode that need no workspace (shared with the
+// allocation-free entry point, which checks them before the size of its
+// fixed array).
+int decode_args_status(const void* q, const void* k_cache, const void* v_cache, const void* o,
+                       const float* lse, int B, int Hq, int Hkv, int Lkv, int d, float lambda,
+                       int Bc, int num_splits) {
   if (!q || !k_cache || !v_cache || !o || !lse) return BLASST_EINVAL;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
       !aligned16(lse))
@@ -543,6 +551,29 @@ int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void*
   const int g = Hq / Hkv;
   if (g != 1 && g != 2 && g != 4 && g != 8) return BLASST_EUNSUPPORTED;
   if (num_splits > 65535 || B > 65535 || Hkv > 65535) return BLASST_EINVAL;
+  return BLASST_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int blasst_lse_merge(const float* o_parts, const float* lse_parts, void* o, float* lse, int n_rows,
+                     int d, int num_splits, int out_dtype, void* stream) {
+  if (!o_parts || !lse_parts || !o || !lse || n_rows <= 0 || d <= 0 || num_splits <= 0)
+    return BLASST_EINVAL;
+  return launch_lse_merge(o_parts, lse_parts, o, lse, n_rows, d, num_splits, out_dtype, nullptr,
+                          static_cast<cudaStream_t>(stream));
+}
+
+int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                  int B, int Hq, int Hkv, int Lkv, int d, float lambda, int Bc, int num_splits,
+                  void* workspace, size_t workspace_bytes, uint8_t* skip_mask_out,
+                  blasst_stats* stats_out, void* stream) {
+  const int arc = decode_args_status(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, d, lambda, Bc,
+                                     num_splits);
+  if (arc != BLASST_OK) return arc;
+  const int g = Hq / Hkv;
   const size_t need = blasst_decode_workspace_bytes(B, Hq, d, num_splits);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return BLASST_EWORKSPACE;
 
@@ -580,8 +611,8 @@ int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void*
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int rc = dispatch_decode(d, Bc, g, mk, mv, p, s);
   if (rc != BLASST_OK) return rc;
-  return blasst_lse_merge(p.o_parts, p.lse_parts, o, lse, B * Hq, d, num_splits, BLASST_BF16,
-                          stream);
+  return launch_lse_merge(p.o_parts, p.lse_parts, o, lse, B * Hq, d, num_splits, BLASST_BF16, err,
+                          s);
 }
 
 size_t blasst_decode_mla_workspace_bytes(int B, int H, int num_splits) {
@@ -679,8 +710,8 @@ int blasst_decode_mla(const void* q, const void* cache, void* o, float* lse, int
   }
   int rc = cuda_status(cudaGetLastError());
   if (rc != BLASST_OK) return rc;
-  return blasst_lse_merge(p.o_parts, p.lse_parts, o, lse, B * H, C::DV, num_splits, BLASST_BF16,
-                          stream);
+  return launch_lse_merge(p.o_parts, p.lse_parts, o, lse, B * H, C::DV, num_splits, BLASST_BF16,
+                          err, s);
 }
 
 int blasst_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n, void* stream) {
@@ -764,13 +795,19 @@ int blasst_decode_noalloc(const void* q, const void* k_cache, const void* v_cach
                           float* lse, int B, int Hq, int Hkv, int Lkv, int d, float lambda, int Bc,
                           int num_splits, uint8_t* skip_mask_out, blasst_stats* stats_out,
                           void* stream) {
-  if (B <= 0 || Hq <= 0 || d <= 0 || num_splits <= 0) return BLASST_EINVAL;
+  // The shape and pointer checks of blasst_decode come first, so an
+  // unsupported shape is reported as such rather than as a size problem.
+  const int arc = decode_args_status(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, d, lambda, Bc,
+                                     num_splits);
+  if (arc != BLASST_OK) return arc;
   const size_t need = blasst_decode_workspace_bytes(B, Hq, d, num_splits);
   if (need == 0 || need > kNoAllocScratchBytes) return BLASST_EWORKSPACE;
   void* scratch = decode_scratch();
   if (!scratch) return BLASST_ECUDA;
   // Every partial the merge reads is written by the split kernel of the same
-  // call (empty splits included), so nothing in the array needs clearing.
+  // call (empty splits included), so nothing in the array needs clearing. If
+  // a bounded wait of that kernel gives up, the merge sees the device error
+  // word and writes NaN / -inf instead of reading partials it did not write.
   return blasst_decode(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, d, lambda, Bc, num_splits,
                        scratch, kNoAllocScratchBytes, skip_mask_out, stats_out, stream);
 }

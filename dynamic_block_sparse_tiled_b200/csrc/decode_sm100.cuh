@@ -565,11 +565,23 @@ __global__ void __launch_bounds__(320, 1)
 
 // o = sum_s w_s o_s / sum_s w_s, lse = M + ln(sum_s w_s), w_s = exp(lse_s - M).
 // One CTA per row; thread x handles output dims x, x + blockDim, ...
+// `err` (nullable): the device error word. If it is set when the kernel
+// starts (a bounded wait of the split kernel gave up, so some partials were
+// never written), the row gets NaN outputs and lse = -inf instead.
 template <typename OutT>
 __global__ void blasst_lse_merge_kernel(const float* __restrict__ o_parts,
                                         const float* __restrict__ lse_parts, OutT* __restrict__ o,
-                                        float* __restrict__ lse, int d, int S) {
+                                        float* __restrict__ lse, int d, int S,
+                                        const int* __restrict__ err) {
   const int row = blockIdx.x;
+  if (err != nullptr && *reinterpret_cast<const volatile int*>(err) != 0) {
+    for (int x = threadIdx.x; x < d; x += blockDim.x) {
+      if constexpr (sizeof(OutT) == 2) o[static_cast<size_t>(row) * d + x] = __float2bfloat16_rn(NAN);
+      else o[static_cast<size_t>(row) * d + x] = NAN;
+    }
+    if (threadIdx.x == 0) lse[row] = -INFINITY;
+    return;
+  }
   const float* lp = lse_parts + static_cast<size_t>(row) * S;
   float M = -INFINITY;
   for (int s = 0; s < S; ++s) M = fmaxf(M, lp[s]);

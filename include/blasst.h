@@ -241,7 +241,11 @@ BLASST_API size_t blasst_decode_workspace_bytes(int B, int Hq, int d, int num_sp
  *   skip_mask_out nullable uint8 [B, Hq, ceil(Lkv/Bc)] (0 computed, 1 skipped).
  *   stats_out  nullable device blasst_stats.
  * A KV block's V rows are read only if at least one query head of its GQA
- * group keeps the block; heads that skip it add nothing. */
+ * group keeps the block; heads that skip it add nothing.
+ * If a bounded wait of the split kernel gives up (blasst_check then returns
+ * BLASST_ETIMEOUT), the merge writes NaN to o and -inf to lse rather than
+ * merging partials that were never written; the same holds for any decode
+ * call made while the device error word still holds an earlier error. */
 BLASST_API int blasst_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                   int B, int Hq, int Hkv, int Lkv, int d, float lambda, int Bc, int num_splits,
                   void* workspace, size_t workspace_bytes, uint8_t* skip_mask_out,
@@ -263,7 +267,12 @@ BLASST_API int blasst_decode(const void* q, const void* k_cache, const void* v_c
  *     cudaGetSymbolAddress with that device current); make that first call
  *     before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents;
- *     every value a call reads back is written earlier in the same call.
+ *     every partial a call merges is written earlier in the same call, so
+ *     nothing needs clearing between calls. If a bounded wait of the split
+ *     kernel gives up (blasst_check then returns BLASST_ETIMEOUT), some
+ *     partials of that call are never written: its merge sees the device
+ *     error word and writes NaN to o and -inf to lse instead (so does any
+ *     decode call made while the word still holds an error).
  *     Calls that may run concurrently on the GPU (different streams, or
  *     different host threads on the same device) race on the array: order
  *     them on one stream. */

@@ -180,3 +180,97 @@ def test_reference_arm_json_line(monkeypatch, capsys):
     assert len(calls) == 5                                # 3 warm-up samples, then 2 timed
     assert [c[3] for c in calls[3:]] == [0, 1]            # one seed per timed step
     assert all(c[2] < calls[3][2] for c in calls[:3])     # warm-up samples are smaller
+
+
+def test_clock_samples_are_selected_by_window():
+    lines = [
+        "2026/12/02 10:00:00.000, 1900, 1965, 700.1, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/02 10:00:00.050, 1700, 1965, 990.3, Not Active, Not Active, Not Active, Active",
+        "2026/12/02 10:00:00.100, 1800, 1965, 900.0, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+    ]
+    clk = bench.ClockSampler(0)
+    for ln in lines:
+        s = bench.ClockSampler.parse(ln, 0.0)
+        if s is not None:
+            clk.samples.append(s)
+    assert len(clk.samples) == 3
+    t0 = clk.samples[0][0]
+    full = clk.summary()
+    assert full["sm_mhz"] == 1800 and full["sm_max_mhz"] == 1965
+    assert full["reasons"] == ["sw_power_cap"] and full["samples"] == 3
+    first = clk.summary([(t0 - 0.001, t0 + 0.001)])
+    assert first["sm_mhz"] == 1900 and first["reasons"] == [] and first["samples"] == 1
+    two = clk.summary([(t0 + 0.04, t0 + 0.06), (t0 + 0.09, t0 + 0.11)])
+    assert two["sm_mhz"] == 1750 and two["samples"] == 2
+    assert clk.summary([(t0 + 5, t0 + 6)])["sm_mhz"] is None
+
+
+def test_interleaved_rounds_alternate_the_arm_order(monkeypatch):
+    import torch
+    calls = []
+
+    def fake_time_calls(fn, steps, warmup, stream, flush_buf):
+        for _ in range(warmup):
+            fn()
+        out = []
+        for _ in range(steps):
+            out.append(float(fn()))
+        return out
+
+    monkeypatch.setattr(bench, "time_calls", fake_time_calls)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+
+    def arm(name, ms):
+        def fn():
+            calls.append(name)
+            return ms
+        return fn
+
+    t = bench.time_interleaved([("a", arm("a", 2.0)), ("b", arm("b", 1.0))], rounds=4, per=2,
+                               warmup=1, stream=None, flush_buf=None)
+    assert calls == ["a", "b"] + ["a", "a", "b", "b", "b", "b", "a", "a"] * 2
+    assert t["a"]["block_ms"] == [2.0] * 4 and t["b"]["block_ms"] == [1.0] * 4
+    assert len(t["a"]["windows"]) == 4
+
+    class Clk:
+        def summary(self, windows):
+            return dict(sm_mhz=1000.0 if windows is t["a"]["windows"] else 2000.0, reasons=[])
+
+    res = {0.0: bench.arm_summary(t["a"], Clk()), 1e-3: bench.arm_summary(t["b"], Clk())}
+    bench.speedups(res, 0.0)
+    assert res[1e-3]["speedup_vs_lambda0"] == 2.0
+    # same cycles on both arms: the clock-normalised speedup is 1
+    assert res[1e-3]["speedup_clk"] == 1.0 and res[0.0]["speedup_clk"] == 1.0
+
+
+def test_summary_line_legs_stay_compact():
+    def arm(skip, x, **kw):
+        return dict(skip_frac=skip, speedup_vs_lambda0=x, speedup_clk=x * 0.99123, frac=0.61234,
+                    ms=9.1234567, **kw)
+    diffuse = dict(skip_frac_structured=0.91234, skip_frac_diffuse=0.00123)
+    legs = {"p32k": {0.0: arm(0.0, 1.0), 1e-3: arm(0.0, 1.0123)},
+            "p32k_a12": {0.0: arm(0.0, 1.0), 1e-3: arm(0.95312, 1.62345)}}
+    for k in ("p128k", "p128k_a12"):
+        legs[k] = {lam: arm(0.75123, 1.45123) for lam in (0.0, 1e-4, 1e-3, 1e-2)}
+    for k in ("p256k", "p256k_a12"):
+        legs[k] = {lam: arm(0.51234, 1.31234, **diffuse) for lam in (0.0, 1e-3)}
+    for k in ("dec", "dec_a12"):
+        d = dict(ms=0.69123, gbs=6300.123, frac=0.96234, speedup_vs_lambda0=1.00123,
+                 speedup_clk=1.00234, skip_frac=0.51234, v_fetch_frac=0.41234,
+                 bytes_saved=1.23456e9)
+        legs[k] = {0.0: d, 1e-3: d}
+    legs["mla"] = {"decode_mla_64k": {"roofline": dict(bound="hbm", frac=0.39123,
+                                                       tensor_frac=0.35123),
+                                      str(1e-3): dict(ms=0.24981)}}
+    legs["bwd"] = dict(ms=25.5123, roofline=dict(frac=0.52123, traffic=12.45e9),
+                       a12=dict(speedup_vs_lambda0=7.5123))
+    legs["sel"] = {"prefill_32k": dict(selector_ms=0.19234, roofline=dict(frac=0.84123))}
+    legs["static"] = dict(speedup_vs_no_mask=3.2123)
+    c = bench.compact_legs(legs)
+    assert set(c) == set(legs)
+    assert c["p256k"]["skip_s"] == 0.912 and c["p256k"]["skip_d"] == 0.00123
+    assert c["p128k"]["0.001"] == [0.751, 1.45, 1.44]
+    assert c["dec_a12"]["saved_gb"] == 1.23
+    import json
+    assert len(json.dumps(c, separators=(",", ":"))) < 1200

@@ -222,6 +222,30 @@ def test_decode_workspace_and_rejections(lib):
     assert rc == -1
 
 
+def test_decode_noalloc_checks_the_shape_before_the_size(lib):
+    """The allocation-free decode reports an unsupported or invalid shape as
+    such, even when its partials would not fit the fixed array either."""
+    vp = 0x10000
+    cap = lib.blasst_decode_noalloc_max_bytes()
+    # d = 256 is not built: EUNSUPPORTED, although 64*32*64*257*4 bytes > 32 MiB
+    assert lib.blasst_decode_workspace_bytes(64, 32, 256, 64) > cap
+    rc = lib.blasst_decode_noalloc(vp, vp, vp, vp, vp, 64, 32, 8, 65536, 256, C.c_float(1e-3), 128,
+                                   64, None, None, None)
+    assert rc == -2
+    # Hq not a multiple of Hkv: EINVAL
+    rc = lib.blasst_decode_noalloc(vp, vp, vp, vp, vp, 64, 32, 7, 65536, 128, C.c_float(1e-3), 128,
+                                   64, None, None, None)
+    assert rc == -1
+    # a misaligned pointer: EINVAL
+    rc = lib.blasst_decode_noalloc(vp + 2, vp, vp, vp, vp, 1, 32, 8, 1024, 128, C.c_float(1e-3),
+                                   128, 4, None, None, None)
+    assert rc == -1
+    # a valid shape that does not fit: EWORKSPACE (before any device call)
+    rc = lib.blasst_decode_noalloc(vp, vp, vp, vp, vp, 64, 32, 8, 65536, 128, C.c_float(1e-3), 128,
+                                   64, None, None, None)
+    assert rc == -5
+
+
 def test_merge_rejects_bad_arguments(lib):
     assert lib.blasst_lse_merge(None, None, None, None, 1, 128, 2, 0, None) == -1
     assert lib.blasst_lse_merge(0x1000, 0x2000, 0x3000, 0x4000, 4, 128, 2, 9, None) == -1

@@ -101,7 +101,24 @@ def run_bwd_case(w, lam, static=None, gpu_decisions=False):
         assert np.all(g[z] == 0.0), f"{w.name} {name}: nonzero rows that no kept pair reaches"
     print(w.name, {k: {m: f"{x:.2e}" for m, x in e.items()} for k, e in errs.items()},
           "empty rows", int(q_zero.sum()), "unreached keys", int(k_zero.sum()))
+    _gate_rejects_perturbations(w.name, (gq, rq), (gk, rk))
     return errs
+
+
+def _gate_rejects_perturbations(what, dq_pair, dk_pair):
+    """The gates are tight enough to see small mistakes: the GPU's dk scaled
+    by 1.02, and one dq row (the largest) scaled by 1.05, must both fail."""
+    gq, rq = dq_pair
+    gk, rk = dk_pair
+    if not np.any(rk):
+        return
+    with pytest.raises(AssertionError):
+        parity.assert_grad_within(gk * 1.02, rk, f"{what} dk x 1.02")
+    flat = gq.reshape(-1, gq.shape[-1]).copy()
+    i = int(np.argmax(np.linalg.norm(rq.reshape(flat.shape), axis=1)))
+    flat[i] *= 1.05
+    with pytest.raises(AssertionError):
+        parity.assert_grad_within(flat.reshape(gq.shape), rq, f"{what} dq row x 1.05")
 
 
 CASES = [
@@ -206,3 +223,4 @@ def test_backward_full_size_sampled():
     e = {n: parity.assert_grad_within(a, b_, f"32K {n}")
          for n, a, b_ in (("dq", gq, rq), ("dk", gk, rk), ("dv", gv, rv))}
     print("32K sampled", {k_: {m: f"{x:.2e}" for m, x in v_.items()} for k_, v_ in e.items()})
+    _gate_rejects_perturbations("32K sampled", (gq, rq), (gk, rk))

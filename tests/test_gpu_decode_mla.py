@@ -60,9 +60,9 @@ def run_mla(w, lam, seqs=None, heads=None, Bc=64):
         n_vis, n_dis, ok, dis = parity.compare_masks(mask_g[b:b + 1, heads], ref["mask"],
                                                      ref["margin"], lam32)
         assert ok, f"MLA mask: {n_dis}/{n_vis} disagree outside the tie band"
-        row_ok = ~dis.any(axis=-1)
         stats = parity.compare_outputs(o_g[b:b + 1, heads], lse_g[b:b + 1, heads],
-                                       ref["o"][..., :512], ref["lse"], row_ok)
+                                       ref["o"][..., :512], ref["lse"], None, dis.any(axis=-1),
+                                       max_tie_rows=n_dis)
         parity.assert_within(stats, f"{w.name} seq {b}")
         worst = {k_: max(worst[k_], stats[k_]) for k_ in worst}
         skip.append(float((ref["mask"] == 1).mean()))
