@@ -92,33 +92,39 @@ def run_bwd_case(w, lam, static=None, gpu_decisions=False):
                                  tile_mask=fmask)
     gq, gk, gv = (t.cpu().numpy().astype(np.float64) for t in (dq, dk, dv))
     q_zero, k_zero = _structural_zeros(w, fmask)
+    scale = 1.0 / np.sqrt(w.d)
+    aq, ak, av = parity.grad_abs_scales(inp.q, inp.k, inp.v, dout, causal=w.causal, scale=scale,
+                                        tile_mask=fmask, Br=w.Br, Bc=w.Bc)
     errs = {}
-    for name, g, r, z in (("dq", gq, rq, q_zero), ("dk", gk, rk, k_zero), ("dv", gv, rv, k_zero)):
+    for name, g, r, z, a in (("dq", gq, rq, q_zero, aq), ("dk", gk, rk, k_zero, ak),
+                             ("dv", gv, rv, k_zero, av)):
         assert np.all(np.isfinite(g)), f"{w.name} {name} not finite"
-        errs[name] = parity.assert_grad_within(g, r, f"{w.name} {name}")
+        errs[name] = parity.assert_grad_within(g, r, f"{w.name} {name}", abs_scale=a)
         # rows that no kept pair reaches are exact zeros on both sides
         assert np.all(r[z] == 0.0)
         assert np.all(g[z] == 0.0), f"{w.name} {name}: nonzero rows that no kept pair reaches"
     print(w.name, {k: {m: f"{x:.2e}" for m, x in e.items()} for k, e in errs.items()},
           "empty rows", int(q_zero.sum()), "unreached keys", int(k_zero.sum()))
-    _gate_rejects_perturbations(w.name, (gq, rq), (gk, rk))
+    _gate_rejects_perturbations(w.name, (gq, rq, aq), (gk, rk, ak))
     return errs
 
 
-def _gate_rejects_perturbations(what, dq_pair, dk_pair):
+def _gate_rejects_perturbations(what, dq_set, dk_set):
     """The gates are tight enough to see small mistakes: the GPU's dk scaled
-    by 1.02, and one dq row (the largest) scaled by 1.05, must both fail."""
-    gq, rq = dq_pair
-    gk, rk = dk_pair
+    by 1.02 must fail, and so must one dq element moved by 4u of its
+    componentwise scale (twice the allowance)."""
+    gq, rq, aq = dq_set
+    gk, rk, ak = dk_set
     if not np.any(rk):
         return
     with pytest.raises(AssertionError):
-        parity.assert_grad_within(gk * 1.02, rk, f"{what} dk x 1.02")
-    flat = gq.reshape(-1, gq.shape[-1]).copy()
-    i = int(np.argmax(np.linalg.norm(rq.reshape(flat.shape), axis=1)))
-    flat[i] *= 1.05
+        parity.assert_grad_within(gk * 1.02, rk, f"{what} dk x 1.02", abs_scale=ak)
+    flat = gq.reshape(-1).copy()
+    a = np.asarray(aq, np.float64).reshape(-1)
+    i = int(np.argmax(a))
+    flat[i] += 2 * parity.GRAD_ABS_FACTOR * a[i]
     with pytest.raises(AssertionError):
-        parity.assert_grad_within(flat.reshape(gq.shape), rq, f"{what} dq row x 1.05")
+        parity.assert_grad_within(flat.reshape(gq.shape), rq, f"{what} dq element", abs_scale=aq)
 
 
 CASES = [
@@ -220,7 +226,10 @@ def test_backward_full_size_sampled():
     gq = dq.reshape(-1, w.d)[rows].cpu().numpy().astype(np.float64)
     gk = dk[0, hk, w.Lkv - w.Bc:].cpu().numpy().astype(np.float64)
     gv = dv[0, hk, w.Lkv - w.Bc:].cpu().numpy().astype(np.float64)
-    e = {n: parity.assert_grad_within(a, b_, f"32K {n}")
-         for n, a, b_ in (("dq", gq, rq), ("dk", gk, rk), ("dv", gv, rv))}
+    aq, ak, av = parity.grad_abs_scales(inp.q, inp.k, inp.v, dout, causal=True,
+                                        scale=1.0 / np.sqrt(w.d), tile_mask=tm, Br=w.Br, Bc=w.Bc,
+                                        rows=rows, key_range=(0, hk, w.Lkv - w.Bc, w.Lkv))
+    e = {n: parity.assert_grad_within(a, b_, f"32K {n}", abs_scale=s_)
+         for n, a, b_, s_ in (("dq", gq, rq, aq), ("dk", gk, rk, ak), ("dv", gv, rv, av))}
     print("32K sampled", {k_: {m: f"{x:.2e}" for m, x in v_.items()} for k_, v_ in e.items()})
-    _gate_rejects_perturbations("32K sampled", (gq, rq), (gk, rk))
+    _gate_rejects_perturbations("32K sampled", (gq, rq, aq), (gk, rk, ak))
