@@ -26,7 +26,9 @@
 //   warp 9     TMA producer for V: loads V of block j only after the vote on
 //              block j says some row group keeps it; writes the skip mask;
 //   warp 10    tcgen05 issuer for S = Q K^T into one of three TMEM S buffers,
-//              three blocks ahead; owns the TMEM allocation;
+//              three blocks ahead (one wait per block: the P V issuer's
+//              commit after that buffer's previous block, kept or not);
+//              owns the TMEM allocation;
 //   warp 11    tcgen05 issuer for O += P V. P (bf16) overwrites the first
 //              Bc/2 columns of its block's S buffer, so an S buffer is reused
 //              once the softmax is done with it and, for a kept block, its
@@ -107,19 +109,19 @@ struct PrefillCfg {
   static constexpr int B_VF = B_KE + NK;
   static constexpr int B_VE = B_VF + NV;
   static constexpr int B_SF = B_VE + NV;   // [NS] S written (tcgen05 commit)
-  static constexpr int B_SC = B_SF + NS;   // [NS] block done with by softmax, PV issuer, V producer
-  static constexpr int B_PV = B_SC + NS;   // [NS] P V of the buffer's block done
+  static constexpr int B_FREE = B_SF + NS;  // [NS] block done with: P V issuer (its commit, after
+                                           // the softmax's P signal) and V producer
+  static constexpr int B_PV = B_FREE + NS;  // [NS] every P V up to the block done
   static constexpr int B_DEC = B_PV + NS;  // [NSLOT] decision (V producer)
   static constexpr int B_P = B_DEC + NSLOT;  // [NSLOT] P ready or block skipped (PV issuer)
   static constexpr int B_HS = B_P + NSLOT;   // [2] running statistics handed to set s
   static constexpr int B_DRAIN = B_HS + 2;   // [2] QK issuer, PV issuer
   static constexpr int NBAR = B_DRAIN + 2;
-  static constexpr int SC_COUNT = 4 + 2;     // a softmax set's 4 warps, PV issuer, V producer
+  static constexpr int FREE_COUNT = 2;       // P V issuer's commit, V producer
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // misc words: [0] tmem base, [1] abort, [3] always 0 (for waits only a timeout
   // ends), [4..7] decisions, [8..15] votes [set][warp of set] (Br = 64),
-  // [16..17] softmax abort word per set, [20..21] last kept block handed to set
-  // s, [24..29] kept blocks per S buffer handed to set s ([s][3])
+  // [16..17] softmax abort word per set
   static constexpr int MISC_BYTES = 128;
   static constexpr int OFF_ST = OFF_MISC + MISC_BYTES;  // [2 sets][2: m, mref][128 rows] floats
   static constexpr int OFF_LSUM = OFF_ST + 2 * 2 * 128 * 4;  // [2 sets][128 rows] floats
@@ -163,8 +165,6 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* dec_val = misc + 4;
   volatile int* votes = misc + 8;
   volatile int* sm_abort = misc + 16;
-  volatile int* st_last = misc + 20;
-  volatile int* st_cnt = misc + 24;
   volatile float* st_rows = reinterpret_cast<volatile float*>(smem + C::OFF_ST);
   volatile float* lsum = reinterpret_cast<volatile float*>(smem + C::OFF_LSUM);
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 0; i < C::NS; ++i) {
       ptx::mbar_init(bar(C::B_SF + i), 1);
-      ptx::mbar_init(bar(C::B_SC + i), C::SC_COUNT);
+      ptx::mbar_init(bar(C::B_FREE + i), C::FREE_COUNT);
       ptx::mbar_init(bar(C::B_PV + i), 1);
     }
     for (int i = 0; i < C::NSLOT; ++i) {
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(384, 1)
         ok = ptx::mbar_wait(bar(C::B_DEC + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         const int keepmask = dec_val[slot];
-        ptx::mbar_arrive(bar(C::B_SC + (j % C::NS)));  // decision slot read
+        ptx::mbar_arrive(bar(C::B_FREE + (j % C::NS)));  // decision slot read
         // skip-mask entries and counters for block j (off the softmax path)
         const unsigned long long tile_flops = 2ull * 128ull * BC * D;
         st_flops += tile_flops + (keepmask ? tile_flops : 0ull);
@@ -419,22 +419,16 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       for (int j = 0; j < C::NS && j < nblk && ok; ++j) ok = issue_qk(j);
-      // S buffer j % NS takes block j+NS once block j is done with: the
-      // softmax has read S_j (and written P_j), the PV issuer and the V
-      // producer have read decision j (so decision slots and the P / DEC
-      // barriers are never more than NS blocks ahead of their readers), and,
-      // when block j was kept, its P V has completed.
-      int kept[C::NS] = {};
+      // S buffer j % NS takes block j+NS once block j is done with, one wait:
+      // the P V issuer commits after every block (kept or not) once the
+      // softmax has signalled P_j, so its commit arrives when P_j V_j (if
+      // any) has completed; the V producer arrives when it has read decision
+      // j (decision slots and the P / DEC barriers are then never more than
+      // NS blocks ahead of their readers). No decision is read here.
       for (int j = 0; j + C::NS < nblk && ok; ++j) {
-        const int bsl = j % C::NS;
-        ok = ptx::mbar_wait(bar(C::B_SC + bsl), (j / C::NS) & 1, abort_flag, p.timeout_ns);
+        ok = ptx::mbar_wait(bar(C::B_FREE + j % C::NS), (j / C::NS) & 1, abort_flag,
+                            p.timeout_ns);
         if (!ok) break;
-        if (dec_val[j % C::NSLOT] != 0) {
-          ++kept[bsl];
-          ok = ptx::mbar_wait(bar(C::B_PV + bsl), (kept[bsl] - 1) & 1, abort_flag,
-                              p.timeout_ns);
-          if (!ok) break;
-        }
         ok = issue_qk(j + C::NS);
       }
       if (!ok) {
@@ -458,7 +452,6 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         ptx::tc_fence_after();
         const bool keep = dec_val[slot] != 0;
-        ptx::mbar_arrive(bar(C::B_SC + (j % C::NS)));  // decision slot read
         if (keep) {
           const int vs = pv_count % C::NV;
           ok = ptx::mbar_wait(bar(C::B_VF + vs), (pv_count / C::NV) & 1, abort_flag,
@@ -473,9 +466,11 @@ __global__ void __launch_bounds__(384, 1)
             ptx::mma_ts(tmem + C::O_COL, p_tm + kk * 8,
                         vd + static_cast<uint64_t>(kk * (2048 >> 4)), C::IDESC_PV, 1u);
           ptx::mma_commit(bar(C::B_VE + vs));
-          ptx::mma_commit(bar(C::B_PV + (j % C::NS)));
           ++pv_count;
         }
+        // buffer j % NS reusable, and every P V up to block j done
+        ptx::mma_commit(bar(C::B_FREE + j % C::NS));
+        ptx::mma_commit(bar(C::B_PV + j % C::NS));
       }
       if (!ok) {
         *abort_flag = 1;
@@ -549,18 +544,11 @@ __global__ void __launch_bounds__(384, 1)
 
       // ---- running statistics after block j-1 (from the other set) -------
       float m = -INFINITY, mref = -INFINITY;
-      int last_kept = -1;
-      int cnt[C::NS];
-#pragma unroll
-      for (int i = 0; i < C::NS; ++i) cnt[i] = 0;
       if (j > 0) {
         const bool ok2 = lane0_wait(bar(C::B_HS + set), ((j - 1) >> 1) & 1);
         ok = ok && ok2;
         m = st_in[t];
         mref = st_in[128 + t];
-        last_kept = st_last[set];
-#pragma unroll
-        for (int i = 0; i < C::NS; ++i) cnt[i] = st_cnt[set * 4 + i];
       }
 
       // ---- the vote: every row of the tile (group) must find block j
@@ -613,10 +601,6 @@ __global__ void __launch_bounds__(384, 1)
       st_out[t] = m_new;
       st_out[128 + t] = mref_new;
       if (leader) {
-        st_last[1 - set] = keepmask ? j : last_kept;
-#pragma unroll
-        for (int i = 0; i < C::NS; ++i)
-          st_cnt[(1 - set) * 4 + i] = cnt[i] + ((keepmask && i == sbuf) ? 1 : 0);
         dec_val[j % C::NSLOT] = keepmask;
         ptx::mbar_arrive(bar(C::B_DEC + (j % C::NSLOT)));
       }
@@ -629,10 +613,10 @@ __global__ void __launch_bounds__(384, 1)
           l = (lref == -INFINITY) ? 0.0f : l * ptx::ex2(lref - mref_new);
           lref = mref_new;
         }
-        if (__any_sync(0xffffffffu, need) && last_kept >= 0) {
-          // O must be quiescent: wait for the last issued P V.
-          const int lb = last_kept % C::NS;
-          const bool ok3 = lane0_wait(bar(C::B_PV + lb), (cnt[lb] - 1) & 1);
+        if (__any_sync(0xffffffffu, need) && j > 0) {
+          // O must be quiescent: every P V up to block j-1 has completed (the
+          // first block is always kept, so O holds its P V by then).
+          const bool ok3 = lane0_wait(bar(C::B_PV + (j - 1) % C::NS), ((j - 1) / C::NS) & 1);
           if (!ok3) {
             *abort_flag = 1;
             if (lane == 0) sm_abort[set] = 1;
@@ -704,7 +688,6 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) {
         ptx::mbar_arrive(bar(C::B_P + (j % C::NSLOT)));
-        ptx::mbar_arrive(bar(C::B_SC + sbuf));
       }
     }
 
@@ -718,15 +701,12 @@ __global__ void __launch_bounds__(384, 1)
     const int fin = nblk & 1;
     // (a static mask can leave no block at all: then O = 0, lse = -inf)
     const float mref_fin = nblk > 0 ? st_rows[fin * 256 + 128 + t] : -INFINITY;
-    const int last_fin = nblk > 0 ? st_last[fin] : -1;
     const float l_mine =
         (lref == -INFINITY || mref_fin == -INFINITY) ? 0.0f : l * ptx::ex2(lref - mref_fin);
     lsum[set * 128 + t] = l_mine;
     bool ok = __shfl_sync(0xffffffffu, (lane == 0 && *abort_flag == 0) ? 1 : 0, 0) != 0;
-    if (ok && last_fin >= 0) {
-      const int lb = last_fin % C::NS;
-      ok = lane0_wait(bar(C::B_PV + lb), (st_cnt[fin * 4 + lb] - 1) & 1);
-    }
+    if (ok && nblk > 0)  // every P V has completed
+      ok = lane0_wait(bar(C::B_PV + (nblk - 1) % C::NS), ((nblk - 1) / C::NS) & 1);
     ptx::tc_fence_after();
     ptx::named_bar_sync(3, C::NSOFT);
     const float ltot = lsum[t] + lsum[128 + t];
