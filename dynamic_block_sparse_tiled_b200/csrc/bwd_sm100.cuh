@@ -238,11 +238,12 @@ __global__ void __launch_bounds__(352, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: key block j of KV head (b, hk). Under a causal mask block
-  // 0 meets the most query tiles, so ascending j runs the longest CTAs first.
-  const int nbhk = p.B * p.Hkv;
-  const int j = static_cast<int>(blockIdx.x) / nbhk;
-  const int bhk = static_cast<int>(blockIdx.x) % nbhk;
+  // ---- work item: key block j of KV head (b, hk), KV-head major: the CTAs
+  // in flight work on one KV head, so the query rows they read (Q, dO) and
+  // add into (dQ) are those of one GQA group. Under a causal mask block 0
+  // meets the most query tiles, so ascending j runs the longest CTAs first.
+  const int j = static_cast<int>(blockIdx.x) % p.nKb;
+  const int bhk = static_cast<int>(blockIdx.x) / p.nKb;
   const int b = bhk / p.Hkv;
   const int hk = bhk % p.Hkv;
 
@@ -310,18 +311,23 @@ __global__ void __launch_bounds__(352, 1)
       const int num = j * C::BK - p.off - (C::BQ - 1);
       t_lo = num <= 0 ? 0 : (num + C::BQ - 1) / C::BQ;
     }
+    // Query tiles from the last one down, 32 at a time, the group's heads
+    // interleaved within each 32-tile chunk: the CTAs of a KV head start on
+    // the same last rows and move down together, so the Q, dO and dQ rows
+    // they touch at any time stay few and in L2. (The gradients are sums
+    // over pairs: their order only changes the fp32 rounding order.)
     int i = 0;  // pairs issued
-    for (int hh = 0; hh < p.g && ok; ++hh) {
-      const int hq = hk * p.g + hh;
-      const int bh = b * p.Hq + hq;
-      for (int t0 = t_lo; t0 < p.nT && ok; t0 += 32) {
-        const int t = t0 + lane;
-        const uint32_t km = t < p.nT ? bwd_keep_bits(p, bh, t, j) : 0u;
+    for (int tc = p.nT - 1; tc >= t_lo && ok; tc -= 32) {
+      for (int hh = 0; hh < p.g && ok; ++hh) {
+        const int hq = hk * p.g + hh;
+        const int bh = b * p.Hq + hq;
+        const int t = tc - lane;  // lane 0: the highest tile of the chunk
+        const uint32_t km = t >= t_lo ? bwd_keep_bits(p, bh, t, j) : 0u;
         uint32_t bal = __ballot_sync(0xffffffffu, km != 0u);
         while (bal != 0u) {
           const int l = __ffs(bal) - 1;
           bal &= bal - 1u;
-          const int tt = t0 + l;
+          const int tt = tc - l;
           const uint32_t kmv = __shfl_sync(0xffffffffu, km, l);
           bool okl = true;
           if (lane == 0) {
