@@ -109,15 +109,19 @@ struct PrefillCfg {
   static constexpr int B_VF = B_KE + NK;
   static constexpr int B_VE = B_VF + NV;
   static constexpr int B_SF = B_VE + NV;   // [NS] S written (tcgen05 commit)
-  static constexpr int B_FREE = B_SF + NS;  // [NS] block done with: P V issuer (its commit, after
-                                           // the softmax's P signal) and V producer
-  static constexpr int B_PV = B_FREE + NS;  // [NS] every P V up to the block done
+  static constexpr int B_PV = B_SF + NS;   // [NS] every P V up to the block done
   static constexpr int B_DEC = B_PV + NS;  // [NSLOT] decision (V producer)
   static constexpr int B_P = B_DEC + NSLOT;  // [NSLOT] P ready or block skipped (PV issuer)
   static constexpr int B_HS = B_P + NSLOT;   // [2] running statistics handed to set s
   static constexpr int B_DRAIN = B_HS + 2;   // [2] QK issuer, PV issuer
   static constexpr int NBAR = B_DRAIN + 2;
-  static constexpr int FREE_COUNT = 2;       // P V issuer's commit, V producer
+  // B_KF + s completes for block j (j % NK == s) when K_j has landed and
+  // block j - NK is done with: the K producer's arrival (with the bytes), the
+  // P V issuer's commit after block j - NK (kept or not, once the softmax has
+  // signalled it: P_{j-NK} V has read S buffer s) and the V producer's
+  // arrival once it has read decision j - NK. One wait per block for the S
+  // issuer. (The first NK phases get the two block-done arrivals at set-up.)
+  static constexpr int KF_COUNT = 3;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // misc words: [0] tmem base, [1] abort, [3] always 0 (for waits only a timeout
   // ends), [4..7] decisions, [8..15] votes [set][warp of set] (Br = 64),
@@ -142,6 +146,7 @@ struct PrefillCfg {
   static_assert(TMEM_COLS <= 512, "TMEM budget");
   static_assert(SMEM_BYTES_LISTED <= 227 * 1024, "shared memory budget");
   static_assert(NSLOT > NS, "decision slots must outlive the S look-ahead");
+  static_assert(NK == NS, "K stage s and S buffer s are released together");
 };
 
 __device__ __forceinline__ void record_error(int* err, int code) {
@@ -171,6 +176,16 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+
+  // A CTA that starts while the device error word holds an error (a bounded
+  // wait of this launch, or of an earlier one not yet read by blasst_check,
+  // gave up) does nothing: the launch then ends within one wave of waits
+  // instead of every CTA waiting out its own bounds.
+  // (misc[0] holds the TMEM base only once it is allocated, below)
+  if (threadIdx.x == 0)
+    misc[0] = (p.err != nullptr && *reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
+  __syncthreads();
+  if (misc[0] != 0) return;
 
   // ---- work item ----------------------------------------------------------
   // KV-head major: the CTAs in flight share one KV head's K/V in L2; within
@@ -270,7 +285,7 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(C::B_Q), 1);
     for (int i = 0; i < C::NK; ++i) {
-      ptx::mbar_init(bar(C::B_KF + i), 1);
+      ptx::mbar_init(bar(C::B_KF + i), C::KF_COUNT);
       ptx::mbar_init(bar(C::B_KE + i), 1);
     }
     for (int i = 0; i < C::NV; ++i) {
@@ -279,7 +294,6 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 0; i < C::NS; ++i) {
       ptx::mbar_init(bar(C::B_SF + i), 1);
-      ptx::mbar_init(bar(C::B_FREE + i), C::FREE_COUNT);
       ptx::mbar_init(bar(C::B_PV + i), 1);
     }
     for (int i = 0; i < C::NSLOT; ++i) {
@@ -292,6 +306,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 1; i < C::MISC_BYTES / 4; ++i)
       if (i != 2) misc[i] = 0;
+    for (int i = 0; i < C::NK; ++i)
+      for (int a = 1; a < C::KF_COUNT; ++a) ptx::mbar_arrive(bar(C::B_KF + i));
     ptx::fence_mbar_init();
   }
   if (warp == C::WARP_MMA) {
@@ -347,7 +363,7 @@ __global__ void __launch_bounds__(384, 1)
         ok = ptx::mbar_wait(bar(C::B_DEC + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         const int keepmask = dec_val[slot];
-        ptx::mbar_arrive(bar(C::B_FREE + (j % C::NS)));  // decision slot read
+        ptx::mbar_arrive(bar(C::B_KF + (j % C::NK)));  // decision j read: for block j + NK
         // skip-mask entries and counters for block j (off the softmax path)
         const unsigned long long tile_flops = 2ull * 128ull * BC * D;
         st_flops += tile_flops + (keepmask ? tile_flops : 0ull);
@@ -418,19 +434,11 @@ __global__ void __launch_bounds__(384, 1)
         ptx::mma_commit(bar(C::B_SF + (j % C::NS)));
         return true;
       };
-      for (int j = 0; j < C::NS && j < nblk && ok; ++j) ok = issue_qk(j);
-      // S buffer j % NS takes block j+NS once block j is done with, one wait:
-      // the P V issuer commits after every block (kept or not) once the
-      // softmax has signalled P_j, so its commit arrives when P_j V_j (if
-      // any) has completed; the V producer arrives when it has read decision
-      // j (decision slots and the P / DEC barriers are then never more than
-      // NS blocks ahead of their readers). No decision is read here.
-      for (int j = 0; j + C::NS < nblk && ok; ++j) {
-        ok = ptx::mbar_wait(bar(C::B_FREE + j % C::NS), (j / C::NS) & 1, abort_flag,
-                            p.timeout_ns);
-        if (!ok) break;
-        ok = issue_qk(j + C::NS);
-      }
+      // S buffer j % NS takes block j once block j - NS is done with, in the
+      // same wait as K_j (see KF_COUNT): decision slots and the P / DEC
+      // barriers are then never more than NS blocks ahead of their readers.
+      // No decision is read here.
+      for (int j = 0; j < nblk && ok; ++j) ok = issue_qk(j);
       if (!ok) {
         *abort_flag = 1;
         record_error(p.err, BLASST_ETIMEOUT);
@@ -468,8 +476,9 @@ __global__ void __launch_bounds__(384, 1)
           ptx::mma_commit(bar(C::B_VE + vs));
           ++pv_count;
         }
-        // buffer j % NS reusable, and every P V up to block j done
-        ptx::mma_commit(bar(C::B_FREE + j % C::NS));
+        // buffer j % NS reusable (for block j + NS), and every P V up to
+        // block j done
+        ptx::mma_commit(bar(C::B_KF + j % C::NK));
         ptx::mma_commit(bar(C::B_PV + j % C::NS));
       }
       if (!ok) {
@@ -551,6 +560,21 @@ __global__ void __launch_bounds__(384, 1)
         mref = st_in[128 + t];
       }
 
+      // ---- new running statistics, handed to the other set ---------------
+      // A skipped block leaves every row's running max as it was: the test
+      // that skips it finds the row's block max below the running max. So the
+      // running max after block j is the prefix max of the visited blocks'
+      // maxima whatever the votes, and so is the lazy reference that follows
+      // it. The other set gets both before this set votes: the vote stays off
+      // the chain from block to block.
+      const float m_new = ((gvis >> gi) & 1) ? fmaxf(m, mbh) : m;
+      const bool need = m_new > mref + C::TAU;  // (only ever in a kept group)
+      const float mref_new = need ? m_new : mref;
+      st_out[t] = m_new;
+      st_out[128 + t] = mref_new;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::B_HS + (1 - set)));
+
       // ---- the vote: every row of the tile (group) must find block j
       //      negligible; a block beyond a row's causal range votes skip -----
       bool rowskip = true;
@@ -593,19 +617,11 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
 
-      // ---- new running statistics, handed to the other set ---------------
       const bool my_keep = (keepmask >> gi) & 1;
-      const float m_new = my_keep ? fmaxf(m, mbh) : m;
-      const bool need = my_keep && (m_new > mref + C::TAU);
-      const float mref_new = need ? m_new : mref;
-      st_out[t] = m_new;
-      st_out[128 + t] = mref_new;
       if (leader) {
         dec_val[j % C::NSLOT] = keepmask;
         ptx::mbar_arrive(bar(C::B_DEC + (j % C::NSLOT)));
       }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(C::B_HS + (1 - set)));
 
       if (keepmask) {
         // l and O follow the reference mref_new

@@ -341,7 +341,10 @@ BLASST_API int blasst_lse_merge(const float* o_parts, const float* lse_parts, vo
 
 /* Synchronises `stream`, then returns (and clears) the device error word:
  * BLASST_OK, BLASST_ETIMEOUT if a kernel's bounded wait gave up, or
- * BLASST_ECUDA if the stream reported a CUDA error. */
+ * BLASST_ECUDA if the stream reported a CUDA error. While the word holds an
+ * error, prefill CTAs that start return without computing (so a failing
+ * launch ends within one wave of bounded waits) and decode merges write NaN:
+ * outputs of calls made after an error and before this check are undefined. */
 BLASST_API int blasst_check(void* stream);
 
 /* Self-test of the two exponentials the prefill kernel uses, so that a test

@@ -180,6 +180,40 @@ def pin_margins_independent_of_lambda(orc):
         prev = res["mask"]
 
 
+def pin_running_max_is_prefix_max(orc):
+    """A skipped block leaves the running max unchanged (its block max lies
+    below it on every row), so the running max before block j is the prefix
+    max of the visited blocks' row maxima, whatever was skipped. The margins
+    mu_j = max_r (m_blk - m_run) recomputed here from that prefix max alone,
+    with the oracle's conventions for rows without keys, must equal the
+    oracle's (which updates m_run only on computed blocks) while it skips."""
+    for causal in (True, False):
+        q, k, v, kw = _skipping_case(seed=23, causal=causal)
+        Br, Bc = kw["Br"], kw["Bc"]
+        B, Hq, Lq, d = q.shape
+        Hkv, Lkv = k.shape[1], k.shape[2]
+        g = Hq // Hkv
+        s = np.einsum("bhid,bhjd->bhij", q, np.repeat(k, g, axis=1)) / np.sqrt(d)
+        if causal:
+            s = np.where(np.arange(Lkv)[None, :] <= np.arange(Lq)[:, None] + (Lkv - Lq), s, -np.inf)
+        nQt, nKt = -(-Lq // Br), -(-Lkv // Bc)
+        res = orc.prefill(q, k, v, lam=1e-2, **kw)
+        _, _, mask, margin = _dense_from(res)
+        assert np.any(mask == 1), "case did not skip anything"
+        for qt in range(nQt):
+            rows = s[:, :, qt * Br:min((qt + 1) * Br, Lq), :]
+            run = np.full(rows.shape[:3], -np.inf)
+            for kt in range(nKt):
+                vis = mask[:, :, qt, kt] != 2
+                mb = rows[..., kt * Bc:min((kt + 1) * Bc, Lkv)].max(-1)
+                dr = np.where(mb == -np.inf, -np.inf, np.where(run == -np.inf, np.inf, mb - run))
+                mu = dr.max(-1)
+                got = margin[:, :, qt, kt]
+                np.testing.assert_allclose(np.where(vis, got, 0.0), np.where(vis, mu, 0.0),
+                                           rtol=0, atol=1e-9)
+                run = np.where(vis[..., None], np.maximum(run, mb), run)
+
+
 def pin_shift_invariance(orc):
     """paras 2/4: the reference point of the exponentials does not change the
     result (lazy rescale with a large slack, or one fixed reference), and the
@@ -643,6 +677,7 @@ ALL_PINS = [
     pin_first_block_always_computed,
     pin_kept_set_equivalence,
     pin_margins_independent_of_lambda,
+    pin_running_max_is_prefix_max,
     pin_shift_invariance,
     pin_permutation_invariance,
     pin_error_bound,
