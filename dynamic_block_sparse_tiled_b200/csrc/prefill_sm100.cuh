@@ -105,8 +105,7 @@ struct PrefillCfg {
   // barrier indices
   static constexpr int B_Q = 0;
   static constexpr int B_KF = 1;
-  static constexpr int B_KE = B_KF + NK;
-  static constexpr int B_VF = B_KE + NK;
+  static constexpr int B_VF = B_KF + NK;
   static constexpr int B_VE = B_VF + NV;
   static constexpr int B_SF = B_VE + NV;   // [NS] S written (tcgen05 commit)
   static constexpr int B_PV = B_SF + NS;   // [NS] every P V up to the block done
@@ -286,7 +285,6 @@ __global__ void __launch_bounds__(384, 1)
     ptx::mbar_init(bar(C::B_Q), 1);
     for (int i = 0; i < C::NK; ++i) {
       ptx::mbar_init(bar(C::B_KF + i), C::KF_COUNT);
-      ptx::mbar_init(bar(C::B_KE + i), 1);
     }
     for (int i = 0; i < C::NV; ++i) {
       ptx::mbar_init(bar(C::B_VF + i), 1);
@@ -339,7 +337,9 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; j < nblk && ok; ++j) {
         const int ks = j % C::NK;
         if (j >= C::NK)
-          ok = ptx::mbar_wait(bar(C::B_KE + ks), ((j / C::NK) - 1) & 1, abort_flag,
+          // stage ks held K_{j-NK}: free once S_{j-NK} is written (S buffer
+          // ks, NS == NK)
+          ok = ptx::mbar_wait(bar(C::B_SF + ks), ((j / C::NK) - 1) & 1, abort_flag,
                               p.timeout_ns);
         if (!ok) break;
         load_kv(&tmK, sb + C::OFF_K + ks * C::KV_BYTES, kt_of(j), bar(C::B_KF + ks));
@@ -415,12 +415,11 @@ __global__ void __launch_bounds__(384, 1)
       // cannot carry (shared addresses < 256 KB).
       const uint64_t q_desc = ptx::sw128_desc(sb + C::OFF_Q, 16, 1024);
       const uint64_t k_desc = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
-      auto issue_qk = [&](int j) -> bool {
-        const int ks = j % C::NK;
-        if (!ptx::mbar_wait(bar(C::B_KF + ks), (j / C::NK) & 1, abort_flag, p.timeout_ns))
+      auto issue_qk = [&](int j, int ks, uint32_t par) -> bool {
+        if (!ptx::mbar_wait(bar(C::B_KF + ks), par, abort_flag, p.timeout_ns))
           return false;
         ptx::tc_fence_after();
-        const uint32_t d_tm = tmem + C::S_COL + (j % C::NS) * BC;
+        const uint32_t d_tm = tmem + C::S_COL + ks * BC;
         const uint64_t kd = k_desc + static_cast<uint64_t>(ks * (C::KV_BYTES >> 4));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -430,15 +429,20 @@ __global__ void __launch_bounds__(384, 1)
               kd + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
           ptx::mma_ss(d_tm, a, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        ptx::mma_commit(bar(C::B_KE + ks));
-        ptx::mma_commit(bar(C::B_SF + (j % C::NS)));
+        ptx::mma_commit(bar(C::B_SF + ks));
         return true;
       };
       // S buffer j % NS takes block j once block j - NS is done with, in the
       // same wait as K_j (see KF_COUNT): decision slots and the P / DEC
       // barriers are then never more than NS blocks ahead of their readers.
-      // No decision is read here.
-      for (int j = 0; j < nblk && ok; ++j) ok = issue_qk(j);
+      // No decision is read here. The loop runs over the NK (= NS) stages at
+      // a time, so stage, buffer and barrier addresses are constants.
+      uint32_t par = 0;
+      for (int j0 = 0; j0 < nblk && ok; j0 += C::NK, par ^= 1u) {
+#pragma unroll
+        for (int u = 0; u < C::NK; ++u)
+          if (j0 + u < nblk && ok) ok = issue_qk(j0 + u, u, par);
+      }
       if (!ok) {
         *abort_flag = 1;
         record_error(p.err, BLASST_ETIMEOUT);
