@@ -88,11 +88,11 @@ struct PrefillCfg {
   static constexpr int NG = BM / BR;   // vote groups
   static constexpr int WPG = BR / 32;  // TMEM lane quarters (warps of a set) per vote group
   static constexpr int NCH = BC / 32;  // 32-column chunks of a block row
-  static constexpr int KEEPC = NCH < 2 ? NCH : 2;  // chunks kept in registers from the max pass
   static constexpr int NK = 3;
   static constexpr int NV = 2;
-  static constexpr int NS = 3;     // S buffers (fp32, BC columns; P aliases the first BC/2)
-  static constexpr int NSLOT = 4;  // decision slots (> NS, see the QK issuer)
+  static constexpr int NS = 2;     // S buffers (fp32, BC columns), one per softmax set
+  static constexpr int NPV = 4;    // "every P V up to block j done" barriers (j % 4)
+  static constexpr int NSLOT = 4;  // decision slots
   static constexpr int DBOX = D / 64;
   static constexpr int Q_BOX = BM * 128;
   static constexpr int KV_BOX = BC * 128;
@@ -104,23 +104,26 @@ struct PrefillCfg {
   static constexpr int OFF_BAR = OFF_V + NV * KV_BYTES;
   // barrier indices
   static constexpr int B_Q = 0;
+  // B_KF + s completes for block j (j % NK == s) when K_j has landed and S
+  // buffer j % NS may take S_j: the K producer's arrival (with the bytes), the
+  // four warps of the softmax set of block j-2 once S_{j-2} is in registers,
+  // and the PV issuer and the V producer once each has read decision j-3 (so
+  // the decision slots, P and DEC barriers never run more than three blocks
+  // ahead of their readers). The S issuer waits once per block. The first
+  // phases get the arrivals of the blocks before 0 at set-up.
   static constexpr int B_KF = 1;
-  static constexpr int B_VF = B_KF + NK;
+  static constexpr int KF_COUNT = 7;
+  // B_KE + s: K stage s free again (the four warps of the set that read S_j)
+  static constexpr int B_KE = B_KF + NK;
+  static constexpr int B_VF = B_KE + NK;
   static constexpr int B_VE = B_VF + NV;
-  static constexpr int B_SF = B_VE + NV;   // [NS] S written (tcgen05 commit)
-  static constexpr int B_PV = B_SF + NS;   // [NS] every P V up to the block done
-  static constexpr int B_DEC = B_PV + NS;  // [NSLOT] decision (V producer)
-  static constexpr int B_P = B_DEC + NSLOT;  // [NSLOT] P ready or block skipped (PV issuer)
-  static constexpr int B_HS = B_P + NSLOT;   // [2] running statistics handed to set s
-  static constexpr int B_DRAIN = B_HS + 2;   // [2] QK issuer, PV issuer
+  static constexpr int B_SF = B_VE + NV;      // [NS] S written (tcgen05 commit)
+  static constexpr int B_PV = B_SF + NS;   // [NPV] every P V up to the block done
+  static constexpr int B_DEC = B_PV + NPV;    // [NSLOT] decision (V producer)
+  static constexpr int B_P = B_DEC + NSLOT;   // [NSLOT] P ready or block skipped (PV issuer)
+  static constexpr int B_HS = B_P + NSLOT;  // [2] running statistics handed to set s
+  static constexpr int B_DRAIN = B_HS + 2;      // [2] QK issuer, PV issuer
   static constexpr int NBAR = B_DRAIN + 2;
-  // B_KF + s completes for block j (j % NK == s) when K_j has landed and
-  // block j - NK is done with: the K producer's arrival (with the bytes), the
-  // P V issuer's commit after block j - NK (kept or not, once the softmax has
-  // signalled it: P_{j-NK} V has read S buffer s) and the V producer's
-  // arrival once it has read decision j - NK. One wait per block for the S
-  // issuer. (The first NK phases get the two block-done arrivals at set-up.)
-  static constexpr int KF_COUNT = 3;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // misc words: [0] tmem base, [1] abort, [3] always 0 (for waits only a timeout
   // ends), [4..7] decisions, [8..15] votes [set][warp of set] (Br = 64),
@@ -133,8 +136,9 @@ struct PrefillCfg {
   static constexpr int OFF_SCAN = OFF_LIST + MAX_LIST * 4;    // [NTHREADS] counts
   static constexpr int SMEM_BYTES = OFF_LIST + 1024;                   // + alignment slack
   static constexpr int SMEM_BYTES_LISTED = OFF_SCAN + NTHREADS * 4 + 1024;
-  static constexpr int S_COL = 0;          // S buffer b at column b * BC (P: first BC/2)
-  static constexpr int O_COL = NS * BC;    // O accumulator
+  static constexpr int S_COL = 0;          // S buffer b (set b) at column b * BC
+  static constexpr int P_COL = NS * BC;    // P buffer b (bf16 pairs, BC/2 columns) after them
+  static constexpr int O_COL = P_COL + NS * (BC / 2);  // O accumulator
   static constexpr int TMEM_COLS = pow2_at_least(O_COL + D);
   static constexpr uint32_t IDESC_QK = ptx::idesc_f32acc(1, 128, BC, false);
   static constexpr uint32_t IDESC_PV = ptx::idesc_f32acc(1, 128, D, true);
@@ -143,9 +147,9 @@ struct PrefillCfg {
   static_assert(BC == 64 || BC == 128, "KV block");
   static_assert(BR == 64 || BR == 128, "query tile");
   static_assert(TMEM_COLS <= 512, "TMEM budget");
+  static_assert(NK == 3 && NS == 2, "the K-full barrier counts the readers of block j - NK");
+  static_assert(NSLOT > NK, "decision slots must outlive the readers' lag");
   static_assert(SMEM_BYTES_LISTED <= 227 * 1024, "shared memory budget");
-  static_assert(NSLOT > NS, "decision slots must outlive the S look-ahead");
-  static_assert(NK == NS, "K stage s and S buffer s are released together");
 };
 
 __device__ __forceinline__ void record_error(int* err, int code) {
@@ -285,6 +289,7 @@ __global__ void __launch_bounds__(384, 1)
     ptx::mbar_init(bar(C::B_Q), 1);
     for (int i = 0; i < C::NK; ++i) {
       ptx::mbar_init(bar(C::B_KF + i), C::KF_COUNT);
+      ptx::mbar_init(bar(C::B_KE + i), 4);
     }
     for (int i = 0; i < C::NV; ++i) {
       ptx::mbar_init(bar(C::B_VF + i), 1);
@@ -292,8 +297,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 0; i < C::NS; ++i) {
       ptx::mbar_init(bar(C::B_SF + i), 1);
-      ptx::mbar_init(bar(C::B_PV + i), 1);
     }
+    for (int i = 0; i < C::NPV; ++i) ptx::mbar_init(bar(C::B_PV + i), 1);
     for (int i = 0; i < C::NSLOT; ++i) {
       ptx::mbar_init(bar(C::B_DEC + i), 1);
       ptx::mbar_init(bar(C::B_P + i), 4);
@@ -304,8 +309,10 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 1; i < C::MISC_BYTES / 4; ++i)
       if (i != 2) misc[i] = 0;
+    // blocks 0 .. NS-1 have no S_{j-2} reader and blocks 0 .. NK-1 no
+    // decision j-3: those arrivals are made here
     for (int i = 0; i < C::NK; ++i)
-      for (int a = 1; a < C::KF_COUNT; ++a) ptx::mbar_arrive(bar(C::B_KF + i));
+      for (int a = 0; a < (i < C::NS ? 4 : 0) + 2; ++a) ptx::mbar_arrive(bar(C::B_KF + i));
     ptx::fence_mbar_init();
   }
   if (warp == C::WARP_MMA) {
@@ -337,9 +344,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; j < nblk && ok; ++j) {
         const int ks = j % C::NK;
         if (j >= C::NK)
-          // stage ks held K_{j-NK}: free once S_{j-NK} is written (S buffer
-          // ks, NS == NK)
-          ok = ptx::mbar_wait(bar(C::B_SF + ks), ((j / C::NK) - 1) & 1, abort_flag,
+          ok = ptx::mbar_wait(bar(C::B_KE + ks), ((j / C::NK) - 1) & 1, abort_flag,
                               p.timeout_ns);
         if (!ok) break;
         load_kv(&tmK, sb + C::OFF_K + ks * C::KV_BYTES, kt_of(j), bar(C::B_KF + ks));
@@ -363,7 +368,7 @@ __global__ void __launch_bounds__(384, 1)
         ok = ptx::mbar_wait(bar(C::B_DEC + slot), (j / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         const int keepmask = dec_val[slot];
-        ptx::mbar_arrive(bar(C::B_KF + (j % C::NK)));  // decision j read: for block j + NK
+        ptx::mbar_arrive(bar(C::B_KF + (j % C::NK)));  // decision j read (block j + NK)
         // skip-mask entries and counters for block j (off the softmax path)
         const unsigned long long tile_flops = 2ull * 128ull * BC * D;
         st_flops += tile_flops + (keepmask ? tile_flops : 0ull);
@@ -415,11 +420,12 @@ __global__ void __launch_bounds__(384, 1)
       // cannot carry (shared addresses < 256 KB).
       const uint64_t q_desc = ptx::sw128_desc(sb + C::OFF_Q, 16, 1024);
       const uint64_t k_desc = ptx::sw128_desc(sb + C::OFF_K, 16, 1024);
-      auto issue_qk = [&](int j, int ks, uint32_t par) -> bool {
-        if (!ptx::mbar_wait(bar(C::B_KF + ks), par, abort_flag, p.timeout_ns))
+      auto issue_qk = [&](int j) -> bool {
+        const int ks = j % C::NK;
+        if (!ptx::mbar_wait(bar(C::B_KF + ks), (j / C::NK) & 1, abort_flag, p.timeout_ns))
           return false;
         ptx::tc_fence_after();
-        const uint32_t d_tm = tmem + C::S_COL + ks * BC;
+        const uint32_t d_tm = tmem + C::S_COL + (j % C::NS) * BC;
         const uint64_t kd = k_desc + static_cast<uint64_t>(ks * (C::KV_BYTES >> 4));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -429,20 +435,16 @@ __global__ void __launch_bounds__(384, 1)
               kd + static_cast<uint64_t>(((kk >> 2) * C::KV_BOX + (kk & 3) * 32) >> 4);
           ptx::mma_ss(d_tm, a, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        ptx::mma_commit(bar(C::B_SF + ks));
+        ptx::mma_commit(bar(C::B_SF + (j % C::NS)));
         return true;
       };
-      // S buffer j % NS takes block j once block j - NS is done with, in the
-      // same wait as K_j (see KF_COUNT): decision slots and the P / DEC
-      // barriers are then never more than NS blocks ahead of their readers.
-      // No decision is read here. The loop runs over the NK (= NS) stages at
-      // a time, so stage, buffer and barrier addresses are constants.
-      uint32_t par = 0;
-      for (int j0 = 0; j0 < nblk && ok; j0 += C::NK, par ^= 1u) {
-#pragma unroll
-        for (int u = 0; u < C::NK; ++u)
-          if (j0 + u < nblk && ok) ok = issue_qk(j0 + u, u, par);
-      }
+      // S_j goes into the buffer of its softmax set (j % 2) once that set has
+      // read S_{j-2} into registers (right after its row max: neither its
+      // exponentials nor P V hold the buffer) and the PV issuer and the V
+      // producer are past block j-3, all in one wait (B_KF). That also keeps
+      // the Q K^T products from running far ahead of the P V ones, which
+      // helps the dense step.
+      for (int j = 0; j < nblk && ok; ++j) ok = issue_qk(j);
       if (!ok) {
         *abort_flag = 1;
         record_error(p.err, BLASST_ETIMEOUT);
@@ -464,13 +466,14 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         ptx::tc_fence_after();
         const bool keep = dec_val[slot] != 0;
+        ptx::mbar_arrive(bar(C::B_KF + (j % C::NK)));  // decision j read (block j + NK)
         if (keep) {
           const int vs = pv_count % C::NV;
           ok = ptx::mbar_wait(bar(C::B_VF + vs), (pv_count / C::NV) & 1, abort_flag,
                               p.timeout_ns);
           if (!ok) break;
           ptx::tc_fence_after();
-          const uint32_t p_tm = tmem + C::S_COL + (j % C::NS) * BC;
+          const uint32_t p_tm = tmem + C::P_COL + (j % C::NS) * (BC / 2);
           const uint64_t vd = v_desc + static_cast<uint64_t>(vs * (C::KV_BYTES >> 4));
           ptx::mma_ts(tmem + C::O_COL, p_tm, vd, C::IDESC_PV, pv_count > 0 ? 1u : 0u);
 #pragma unroll
@@ -480,10 +483,8 @@ __global__ void __launch_bounds__(384, 1)
           ptx::mma_commit(bar(C::B_VE + vs));
           ++pv_count;
         }
-        // buffer j % NS reusable (for block j + NS), and every P V up to
-        // block j done
-        ptx::mma_commit(bar(C::B_KF + j % C::NK));
-        ptx::mma_commit(bar(C::B_PV + j % C::NS));
+        // every P V up to block j done (P buffer reuse, lazy rescale, epilogue)
+        ptx::mma_commit(bar(C::B_PV + j % C::NPV));
       }
       if (!ok) {
         *abort_flag = 1;
@@ -519,13 +520,14 @@ __global__ void __launch_bounds__(384, 1)
     };
 
     for (int j = set; j < nblk; j += 2) {
-      const int sbuf = j % C::NS;
+      const int sbuf = j % C::NS;  // == set
       const uint32_t s_tm = tmem + lane_base + C::S_COL + sbuf * BC;
+      const uint32_t p_tm = tmem + lane_base + C::P_COL + sbuf * (BC / 2);
       bool ok = lane0_wait(bar(C::B_SF + sbuf), (j / C::NS) & 1);
       ptx::tc_fence_after();
 
-      // ---- row max of block j (masked), first chunks kept in registers ---
-      uint32_t sk[C::KEEPC * 32];
+      // ---- row max of block j (masked); the row's S stays in registers ----
+      uint32_t sk[C::NCH * 32];
       float mbh = -INFINITY;
       const int kt = kt_of(j);
       const uint32_t gvis = groups_at(j);
@@ -535,8 +537,7 @@ __global__ void __launch_bounds__(384, 1)
         float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
-          uint32_t tmp[32];
-          uint32_t* sr = c < C::KEEPC ? sk + 32 * c : tmp;
+          uint32_t* sr = sk + 32 * c;
           ptx::tmem_ld32p(s_tm + 32 * c, sr);
           ptx::tmem_wait_ld();
           if (need_mask) {
@@ -554,6 +555,14 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbh = fmaxf(ptx::fmax3(mc[0], mc[1], mc[2]), mc[3]) * sl2;
       }
+      // S_j is in registers: its buffer may take S_{j+2}, and K_j's stage
+      // (read by the finished Q K_j^T) may take K_{j+NK}
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(bar(C::B_KF + (j + 2) % C::NK));
+        ptx::mbar_arrive(bar(C::B_KE + j % C::NK));
+      }
 
       // ---- running statistics after block j-1 (from the other set) -------
       float m = -INFINITY, mref = -INFINITY;
@@ -564,15 +573,8 @@ __global__ void __launch_bounds__(384, 1)
         mref = st_in[128 + t];
       }
 
-      // ---- new running statistics, handed to the other set ---------------
-      // A skipped block leaves every row's running max as it was: the test
-      // that skips it finds the row's block max below the running max. So the
-      // running max after block j is the prefix max of the visited blocks'
-      // maxima whatever the votes, and so is the lazy reference that follows
-      // it. The other set gets both before this set votes: the vote stays off
-      // the chain from block to block.
       const float m_new = ((gvis >> gi) & 1) ? fmaxf(m, mbh) : m;
-      const bool need = m_new > mref + C::TAU;  // (only ever in a kept group)
+      const bool need = m_new > mref + C::TAU;
       const float mref_new = need ? m_new : mref;
       st_out[t] = m_new;
       st_out[128 + t] = mref_new;
@@ -621,10 +623,31 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
 
+      // ---- new running statistics, handed to the other set ---------------
       const bool my_keep = (keepmask >> gi) & 1;
       if (leader) {
         dec_val[j % C::NSLOT] = keepmask;
         ptx::mbar_arrive(bar(C::B_DEC + (j % C::NSLOT)));
+      }
+
+      // A skipped block has no P to write: it goes to the P V issuer at once.
+      if (!keepmask) {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_P + (j % C::NSLOT)));
+      }
+
+      // This set's P buffer was last read by the P V of block j-2. The wait is
+      // taken at every block (kept or not), so each set awaits its "P V done"
+      // phases in order. It stays exact after a skipped block was handed on:
+      // the P V issuer can then pass block j+1 but not j+2 (this set's next),
+      // and the phase of j-2 + NPV (NPV = 4) needs it past j+2.
+      if (j >= 2) {
+        const bool okp = lane0_wait(bar(C::B_PV + (j - 2) % C::NPV), ((j - 2) / C::NPV) & 1);
+        if (!okp) {
+          *abort_flag = 1;
+          if (lane == 0) sm_abort[set] = 1;
+          record_error(p.err, BLASST_ETIMEOUT);
+        }
       }
 
       if (keepmask) {
@@ -636,7 +659,7 @@ __global__ void __launch_bounds__(384, 1)
         if (__any_sync(0xffffffffu, need) && j > 0) {
           // O must be quiescent: every P V up to block j-1 has completed (the
           // first block is always kept, so O holds its P V by then).
-          const bool ok3 = lane0_wait(bar(C::B_PV + (j - 1) % C::NS), ((j - 1) / C::NS) & 1);
+          const bool ok3 = lane0_wait(bar(C::B_PV + (j - 1) % C::NPV), ((j - 1) / C::NPV) & 1);
           if (!ok3) {
             *abort_flag = 1;
             if (lane == 0) sm_abort[set] = 1;
@@ -657,24 +680,14 @@ __global__ void __launch_bounds__(384, 1)
           ptx::tmem_wait_st();
         }
 
-        // ---- P = exp2(s * scale*log2e - mref) as bf16 over S's first half -
+        // ---- P = exp2(s * scale*log2e - mref) as bf16 into the P buffer ----
         const float neg = -mref_new;
         float rs[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) rs[i] = 0.0f;
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
-          uint32_t tmp[32];
-          uint32_t* sr = c < C::KEEPC ? sk + 32 * c : tmp;
-          if (c >= C::KEEPC) {
-            ptx::tmem_ld32p(s_tm + 32 * c, sr);
-            ptx::tmem_wait_ld();
-            if (need_mask) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (col0 + 32 * c + i > last_col) sr[i] = __float_as_uint(-INFINITY);
-            }
-          }
+          const uint32_t* sr = sk + 32 * c;
           uint32_t pk[16];
           // (with a static mask a row may have no key yet: it adds nothing)
           if (my_keep && (!LISTED || mref_new > -INFINITY)) {
@@ -698,16 +711,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = 0u;
           }
-          // P columns [16c, 16c+16) overwrite S columns already in registers
-          ptx::tmem_st16(s_tm + 16 * c, pk);
+          ptx::tmem_st16(p_tm + 16 * c, pk);
         }
         l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-      }
-      __syncwarp();
-      if (lane == 0) {
-        ptx::mbar_arrive(bar(C::B_P + (j % C::NSLOT)));
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_P + (j % C::NSLOT)));
       }
     }
 
@@ -726,7 +736,7 @@ __global__ void __launch_bounds__(384, 1)
     lsum[set * 128 + t] = l_mine;
     bool ok = __shfl_sync(0xffffffffu, (lane == 0 && *abort_flag == 0) ? 1 : 0, 0) != 0;
     if (ok && nblk > 0)  // every P V has completed
-      ok = lane0_wait(bar(C::B_PV + (nblk - 1) % C::NS), ((nblk - 1) / C::NS) & 1);
+      ok = lane0_wait(bar(C::B_PV + (nblk - 1) % C::NPV), ((nblk - 1) / C::NPV) & 1);
     ptx::tc_fence_after();
     ptx::named_bar_sync(3, C::NSOFT);
     const float ltot = lsum[t] + lsum[128 + t];
