@@ -110,20 +110,27 @@ struct BwdCfg {
   // barriers
   static constexpr int B_KV = 0;
   static constexpr int B_QF = 1;               // [NST] stage loaded (+ record)
-  static constexpr int B_QE = B_QF + NST;      // [NST] stage free: issuer commit + the set's 4 dQ adds read
+  static constexpr int B_QE = B_QF + NST;      // [NST] stage free (QE_COUNT)
   static constexpr int B_SF = B_QE + NST;      // [2] S^T ready
   static constexpr int B_PR = B_SF + 2;        // [2] P^T in TMEM (4 warps of a compute set)
   static constexpr int B_DPF = B_PR + 2;       // [2] dP^T ready
   static constexpr int B_DSR = B_DPF + 2;      // [2] dS^T in shared memory (4 warps of a set)
-  static constexpr int B_DSE = B_DSR + 2;      // [2] dS^T buffer free (issuer commit)
-  static constexpr int B_DQF = B_DSE + 2;      // [2] dQ^T ready
-  static constexpr int B_DQE = B_DQF + 2;      // [2] dQ^T drained (4 warps of a set)
-  static constexpr int B_ZERO = B_DQE + 2;     // dV, dK accumulators cleared (8 compute warps)
-  static constexpr int B_SFREE = B_ZERO + 1;   // [2] dV of the buffer's pair done (P^T read)
-  static constexpr int B_ACC = B_SFREE + 2;    // dV, dK final
+  static constexpr int B_DQF = B_DSR + 2;      // [2] dQ^T ready (the set then knows dK and
+                                               // dQ^T of the pair have read its dS^T buffer)
+  static constexpr int B_ZERO = B_DQF + 2;     // dV, dK accumulators cleared (8 compute warps)
+  static constexpr int B_ACC = B_ZERO + 1;     // dV, dK final
   static constexpr int B_DRAIN = B_ACC + 1;    // [2] the two issuers' drains
   static constexpr int NBAR = B_DRAIN + 2;
-  static constexpr int QE_COUNT = 1 + 4;
+  // stage free: the 4 warps of the pair's set once their dQ adds have read
+  // the staged tiles (after dQ^T was ready, so every product that read the
+  // stage's Q and dO is done: the tensor core completes in order)
+  static constexpr int QE_COUNT = 4;
+  // stage loaded for pair i, and the buffers of pair i-2 free for pair i: the
+  // producer's arrival (with the bytes), the dV issuer's commit after dV of
+  // pair i-2 (its P^T read) and the 4 warps of that pair's set once they have
+  // drained its dQ^T (the dP^T / dQ^T buffer). The S^T / dP^T issuer waits
+  // once per pair. Pairs 0 and 1 get the pair-before arrivals at set-up.
+  static constexpr int QF_COUNT = 1 + 1 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // misc words: [0] tmem base, [1] abort, [3] always 0 (waits only a timeout ends)
   static constexpr int MISC_BYTES = 64;
@@ -250,7 +257,7 @@ __global__ void __launch_bounds__(352, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(C::B_KV), 1);
     for (int i = 0; i < C::NST; ++i) {
-      ptx::mbar_init(bar(C::B_QF + i), 1);
+      ptx::mbar_init(bar(C::B_QF + i), C::QF_COUNT);
       ptx::mbar_init(bar(C::B_QE + i), C::QE_COUNT);
     }
     for (int i = 0; i < 2; ++i) {
@@ -258,17 +265,14 @@ __global__ void __launch_bounds__(352, 1)
       ptx::mbar_init(bar(C::B_PR + i), 4);
       ptx::mbar_init(bar(C::B_DPF + i), 1);
       ptx::mbar_init(bar(C::B_DSR + i), 4);
-      ptx::mbar_init(bar(C::B_DSE + i), 1);
       ptx::mbar_init(bar(C::B_DQF + i), 1);
-      ptx::mbar_init(bar(C::B_DQE + i), 4);
     }
     ptx::mbar_init(bar(C::B_ZERO), 8);
     ptx::mbar_init(bar(C::B_ACC), 1);
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(bar(C::B_SFREE + i), 1);
-      ptx::mbar_init(bar(C::B_DRAIN + i), 1);
-    }
+    for (int i = 0; i < 2; ++i) ptx::mbar_init(bar(C::B_DRAIN + i), 1);
     for (int i = 1; i < C::MISC_BYTES / 4; ++i) misc[i] = 0;
+    for (int i = 0; i < 2; ++i)
+      for (int a = 1; a < C::QF_COUNT; ++a) ptx::mbar_arrive(bar(C::B_QF + i));
     ptx::fence_mbar_init();
   }
   if (warp == C::WARP_MMA) {
@@ -374,8 +378,12 @@ __global__ void __launch_bounds__(352, 1)
       if (!ok) {
         fail();
         // let the copies already in flight land before the CTA exits
+        // (a stage's phase also counts the other roles' arrivals for the pair
+        // two back, which an abort may leave out: 1 ms each is ample for the
+        // copies themselves)
+        const uint64_t drain_ns = p.timeout_ns < 1000000ull ? p.timeout_ns : 1000000ull;
         for (int k = i - C::NST < 0 ? 0 : i - C::NST; k < i; ++k)
-          ptx::mbar_wait(bar(C::B_QF + k % C::NST), (k / C::NST) & 1, &misc[3], p.timeout_ns);
+          ptx::mbar_wait(bar(C::B_QF + k % C::NST), (k / C::NST) & 1, &misc[3], drain_ns);
         ptx::mbar_wait(bar(C::B_KV), 0, &misc[3], p.timeout_ns);
       }
     }
@@ -425,11 +433,7 @@ __global__ void __launch_bounds__(352, 1)
         const uint64_t st = static_cast<uint64_t>(i % C::NST) * QST;
         if (warp == C::WARP_SP) {
           // S^T = K Q^T and dP^T = V dO^T: M = 128 keys, N = 64 rows, K = 128 dims
-          if (i >= 2 && !ptx::mbar_wait(bar(C::B_SFREE + bs), ((i - 2) >> 1) & 1, abort_flag,
-                                        p.timeout_ns)) {
-            ok = false;
-            break;
-          }
+          // (the buffers of pair i-2 are free: counted by the stage's barrier)
           ptx::tc_fence_after();
           const uint32_t s_tm = tmem + C::S_COL + bs * 64;
 #pragma unroll
@@ -439,12 +443,6 @@ __global__ void __launch_bounds__(352, 1)
             ptx::mma_ss(s_tm, a, bq, C::IDESC_S, kk > 0 ? 1u : 0u);
           }
           ptx::mma_commit(bar(C::B_SF + bs));
-          if (i >= 2 && !ptx::mbar_wait(bar(C::B_DQE + bs), ((i - 2) >> 1) & 1, abort_flag,
-                                        p.timeout_ns)) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
           const uint32_t dp_tm = tmem + C::DP_COL + bs * 64;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -465,7 +463,8 @@ __global__ void __launch_bounds__(352, 1)
           for (int kk = 0; kk < 4; ++kk)
             ptx::mma_ts(tmem + C::DV_COL, p_tm + kk * 8,
                         dDO_mn + st + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DV, 1u);
-          ptx::mma_commit(bar(C::B_SFREE + bs));
+          // P^T of pair i read: its S^T buffer may take pair i+2
+          ptx::mma_commit(bar(C::B_QF + (i + 2) % C::NST));
           // dK += dS^T Q (M = 128 keys, N = 128 dims, K = 64 rows) and
           // dQ^T = K^T dS^T (M = 128 dims, N = 64 rows, K = 128 keys)
           if (!ptx::mbar_wait(bar(C::B_DSR + bs), (i >> 1) & 1, abort_flag, p.timeout_ns)) {
@@ -486,8 +485,6 @@ __global__ void __launch_bounds__(352, 1)
                         dsm + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_DQ,
                         kk > 0 ? 1u : 0u);
           ptx::mma_commit(bar(C::B_DQF + bs));
-          ptx::mma_commit(bar(C::B_QE + i % C::NST));
-          ptx::mma_commit(bar(C::B_DSE + bs));
         }
       }
       if (warp == C::WARP_MMA) ptx::mma_commit(bar(C::B_ACC));
@@ -588,10 +585,8 @@ __global__ void __launch_bounds__(352, 1)
       ok = warp_wait(bar(C::B_DPF + bs), (i >> 1) & 1);
       if (!ok) break;
       ptx::tc_fence_after();
-      if (i >= 2) {
-        ok = warp_wait(bar(C::B_DSE + bs), ((i - 2) >> 1) & 1);
-        if (!ok) break;
-      }
+      // (dS^T of pair i-2 has been read: this set waited for that pair's dQ^T,
+      // committed after its dK and dQ^T products)
       uint8_t* dsrow = smem + C::OFF_DS + bs * C::DS_BYTES + kl * 128;
       const float* dr = rs + C::BQ;
 #pragma unroll
@@ -634,7 +629,8 @@ __global__ void __launch_bounds__(352, 1)
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(C::B_DQE + bs));
+        // dQ^T drained: the dP^T / dQ^T buffer may take pair i+2
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_QF + (i + 2) % C::NST));
         const int slot = (quad < 2 ? C::OFF_Q + quad * C::DQS_BYTES
                                    : C::OFF_DO + (quad - 2) * C::DQS_BYTES) + s * C::Q_BYTES;
         float* tile = reinterpret_cast<float*>(smem + slot);
