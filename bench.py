@@ -259,14 +259,24 @@ def time_interleaved(arms, rounds, per, warmup, stream, flush_buf):
     return out
 
 
-def arm_summary(t, clk):
+def kernel_mhz(sd):
+    """Mean SM clock while the kernel ran, from its own telemetry (summed CTA
+    cycles over summed CTA nanoseconds), or None where the call has none."""
+    cyc, ns = sd.get("sm_cycles", 0), sd.get("sm_ns", 0)
+    return cyc / ns * 1e3 if cyc > 0 and ns > 0 else None
+
+
+def arm_summary(t, clk, k_mhz=None):
     """Median block time, the median SM clock over the arm's blocks, and the
-    clock-normalised time (ms x MHz = thousands of cycles)."""
+    clock-normalised time (ms x MHz = thousands of cycles). With the kernel's
+    own clock (``k_mhz``) the cycles use it: the nvidia-smi sampler (every 50
+    ms) can miss short blocks or sample between calls."""
     ms = statistics.median(t["block_ms"])
     c = clk.summary(t["windows"]) if clk is not None else dict(sm_mhz=None, reasons=[])
-    kcyc = ms * c["sm_mhz"] if c["sm_mhz"] else None
+    mhz = k_mhz or c["sm_mhz"]
+    kcyc = ms * mhz if mhz else None
     return dict(ms=ms, ms_blocks=t["block_ms"], sm_mhz=c["sm_mhz"], reasons=c["reasons"],
-                kcycles=kcyc)
+                kernel_mhz=k_mhz, kcycles=kcyc)
 
 
 def speedups(res, base_key):
@@ -287,12 +297,14 @@ def measure_prefill(w, lam, steps, warmup, device, stream, flush_buf, pre=None, 
     if rc != 0:
         raise RuntimeError(bl.blasst_status_string(rc))
     sd = bl.stats_dict(st)
-    times = time_calls(lambda: pre.run(lam, stream=stream, block_mask=block_mask), steps, warmup,
-                       stream, flush_buf)
+    kst = bl.new_stats(device)  # the timed calls' own SM cycles and nanoseconds
+    times = time_calls(lambda: pre.run(lam, stream=stream, block_mask=block_mask, stats=kst),
+                       steps, warmup, stream, flush_buf)
     mask = pre.mask.cpu().numpy()
     vis = int((mask != 2).sum())
     skip = int((mask == 1).sum())
     return pre, dict(ms=statistics.mean(times), ms_min=min(times), times=times,
+                     kernel_mhz=kernel_mhz(bl.stats_dict(kst)),
                      exec_flops=float(sd["mma_flops"]), eff_flops=effective_flops(w),
                      skip_frac=skip / max(vis, 1), tiles_visited=vis, tiles_skipped=skip,
                      v_blocks=sd["v_blocks_loaded"], bytes_loaded=sd["bytes_loaded"])
@@ -582,12 +594,13 @@ def prefill_lambda_leg(w, lams, rounds, per, device, stream, flush_buf, clk, pea
             r["skip_frac_structured"] = float((m[:, :h] == 1).sum()) / max(int(vis[:, :h].sum()), 1)
             r["skip_frac_diffuse"] = float((m[:, h:] == 1).sum()) / max(int(vis[:, h:].sum()), 1)
         res[lam] = r
-    t = time_interleaved([(lam, (lambda lam=lam: pre.run(lam, stream=stream))) for lam in lams],
-                         rounds, per, 2, stream, flush_buf)
+    kst = {lam: bl.new_stats(device) for lam in lams}
+    t = time_interleaved([(lam, (lambda lam=lam: pre.run(lam, stream=stream, stats=kst[lam])))
+                          for lam in lams], rounds, per, 2, stream, flush_buf)
     eff = effective_flops(w)
     for lam in lams:
         r = res[lam]
-        r.update(arm_summary(t[lam], clk))
+        r.update(arm_summary(t[lam], clk, kernel_mhz(bl.stats_dict(kst[lam]))))
         r["executed_tflops"] = r["exec_flops"] / (r["ms"] * 1e-3) / 1e12
         r["effective_tflops"] = eff / (r["ms"] * 1e-3) / 1e12
         r["frac"] = r["executed_tflops"] / peaks["bf16_tflops"]
@@ -1121,7 +1134,8 @@ def main():
                         **{"lambda": LAMBDA}),
             roofline=roofline,
             cpu_baseline={k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
-            e2e=e2e, clocks={k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            e2e=e2e, clocks=dict({k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+                                 sm_mhz_kernel=_r(main_r["kernel_mhz"], 4)),
             skip_frac=main_r["skip_frac"], executed_tflops=exec_tflops,
             ms_lambda0=l0[0.0]["ms"], speedup_vs_lambda0=l0[LAMBDA]["speedup_vs_lambda0"],
             speedup_vs_lambda0_clk=l0[LAMBDA]["speedup_clk"],

@@ -57,7 +57,8 @@ class BlasstError(RuntimeError):
 class Stats(C.Structure):
     _fields_ = [("tiles_visited", C.c_ulonglong), ("tiles_skipped", C.c_ulonglong),
                 ("v_blocks_loaded", C.c_ulonglong), ("mma_flops", C.c_ulonglong),
-                ("bytes_loaded", C.c_ulonglong)]
+                ("bytes_loaded", C.c_ulonglong), ("sm_cycles", C.c_ulonglong),
+                ("sm_ns", C.c_ulonglong)]
 
 
 class _FwdArgs(C.Structure):
@@ -342,9 +343,9 @@ def blasst_check(stream=None) -> int:
 
 # -------------------------------------------------------------- conveniences
 def new_stats(device="cuda"):
-    """A zeroed device-side blasst_stats (5 x uint64, as an int64 tensor)."""
+    """A zeroed device-side blasst_stats (uint64 fields, as an int64 tensor)."""
     import torch
-    return torch.zeros(5, dtype=torch.int64, device=device)
+    return torch.zeros(len(Stats._fields_), dtype=torch.int64, device=device)
 
 
 def stats_dict(st) -> dict:

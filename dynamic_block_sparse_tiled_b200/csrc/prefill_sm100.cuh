@@ -127,7 +127,8 @@ struct PrefillCfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // misc words: [0] tmem base, [1] abort, [3] always 0 (for waits only a timeout
   // ends), [4..7] decisions, [8..15] votes [set][warp of set] (Br = 64),
-  // [16..17] softmax abort word per set
+  // [16..17] softmax abort word per set, [24..27] the CTA's start (clock64,
+  // %globaltimer) for the telemetry
   static constexpr int MISC_BYTES = 128;
   static constexpr int OFF_ST = OFF_MISC + MISC_BYTES;  // [2 sets][2: m, mref][128 rows] floats
   static constexpr int OFF_LSUM = OFF_ST + 2 * 2 * 128 * 4;  // [2 sets][128 rows] floats
@@ -309,6 +310,10 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 1; i < C::MISC_BYTES / 4; ++i)
       if (i != 2) misc[i] = 0;
+    // (in shared memory: no register stays live across the kernel for it)
+    reinterpret_cast<volatile unsigned long long*>(misc + 24)[0] =
+        static_cast<unsigned long long>(clock64());
+    reinterpret_cast<volatile unsigned long long*>(misc + 24)[1] = ptx::globaltimer_ns();
     // blocks 0 .. NS-1 have no S_{j-2} reader and blocks 0 .. NK-1 no
     // decision j-3: those arrivals are made here
     for (int i = 0; i < C::NK; ++i)
@@ -784,6 +789,12 @@ __global__ void __launch_bounds__(384, 1)
   __syncwarp();  // role warps reconverge (only their lane 0 worked)
   ptx::tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0 && p.stats) {
+    const volatile unsigned long long* t0 =
+        reinterpret_cast<const volatile unsigned long long*>(misc + 24);
+    atomicAdd(&p.stats->sm_cycles, static_cast<unsigned long long>(clock64()) - t0[0]);
+    atomicAdd(&p.stats->sm_ns, static_cast<unsigned long long>(ptx::globaltimer_ns()) - t0[1]);
+  }
   if (warp == C::WARP_MMA) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);

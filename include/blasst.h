@@ -73,6 +73,13 @@ typedef struct blasst_stats {
   unsigned long long v_blocks_loaded; /* KV blocks whose V was fetched */
   unsigned long long mma_flops;       /* tensor-core / FMA flops actually executed (2 per MAC) */
   unsigned long long bytes_loaded;    /* Q, K, V bytes requested from global memory */
+  /* bf16 prefill only (other calls leave them as they are): summed over the
+   * launch's CTAs, the SM clock cycles (clock64) and the nanoseconds
+   * (%globaltimer) from each CTA's start to its end. Their ratio is the mean
+   * SM clock while the kernel ran, which a sampler outside the GPU can miss
+   * on short calls. */
+  unsigned long long sm_cycles;
+  unsigned long long sm_ns;
 } blasst_stats;
 
 /* Forward prefill pass, bf16 in / bf16 out, fp32 lse, on the legacy default
