@@ -59,6 +59,10 @@ def run_case(w, lam, items=None, check_stats=True, static_mask=None):
         sd = bl.stats_dict(st)
         assert sd["tiles_visited"] == int((mask_g != 2).sum())
         assert sd["tiles_skipped"] == int((mask_g == 1).sum())
+        if w.dtype != "fp32":
+            # the bf16 kernel's own cycle and time spans: a plausible SM clock
+            assert sd["sm_cycles"] > 0 and sd["sm_ns"] > 0
+            assert 300.0 < sd["sm_cycles"] / sd["sm_ns"] * 1e3 < 2500.0
     return dict(stats, n_vis=n_vis, n_dis=n_dis, skip=float((ref["mask"] == 1).sum()) / max(n_vis, 1))
 
 
