@@ -24,6 +24,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -77,14 +78,24 @@ KERNEL_SOURCES = {
 }
 
 
+def code_only(text):
+    """C/C++ source without its comments and empty lines, runs of blanks as
+    one, so that an edit of the comments or the layout leaves a kernel's hash
+    as it was."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"\s+", " ", re.sub(r"//.*$", "", ln)).strip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash(kernel_key):
-    """Hash of the source files that make up one kernel."""
+    """Hash of the code (comments stripped) of the source files that make up
+    one kernel."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dynamic_block_sparse_tiled_b200", "csrc")
     for name in KERNEL_SOURCES[kernel_key]:
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -12,27 +12,27 @@
 // output accumulator; the skip test always uses the exact running max.
 //
 // One CTA owns 128 query rows of one (batch, query head) and walks the KV
-// blocks of its KV head. Warp roles (384 threads):
+// blocks of its KV head. TMEM holds two S buffers (fp32, one per softmax
+// set), two P buffers (bf16, one per set) and O. Warp roles (384 threads):
 //   warps 0-3  softmax of the even blocks, warps 4-7 softmax of the odd
 //              blocks; thread t of a set owns row t (TMEM lane t) over all
-//              Bc columns of its blocks. The two sets alternate, so on each
-//              SM sub-partition one warp runs the exponentials of block j
-//              while the other reads S, takes the row max and votes on block
-//              j+1: the latency-bound and the MUFU-bound phases overlap.
-//              The running statistics pass from one set to the other through
-//              shared memory right after each vote (the vote on j+1 needs the
-//              running max after j, nothing else of block j);
+//              Bc columns of its blocks and holds the whole S row in
+//              registers after the max pass, so the S buffer is free again at
+//              once. The two sets alternate, so on each SM sub-partition one
+//              warp runs the exponentials of block j while the other reads S,
+//              takes the row max and votes on block j+1. The running max after
+//              block j is the prefix max of the visited blocks' maxima whatever
+//              the votes (a skipped block lies below it on every row), so each
+//              set hands the running statistics to the other right after its
+//              row max, before its own vote;
 //   warp 8     TMA producer for Q and K (3-stage ring, ahead of the votes);
 //   warp 9     TMA producer for V: loads V of block j only after the vote on
 //              block j says some row group keeps it; writes the skip mask;
-//   warp 10    tcgen05 issuer for S = Q K^T into one of three TMEM S buffers,
-//              three blocks ahead (one wait per block: the P V issuer's
-//              commit after that buffer's previous block, kept or not);
+//   warp 10    tcgen05 issuer for S = Q K^T: one wait and one commit per
+//              block (the K-full barrier also counts the set that freed the S
+//              buffer and the P V issuer and V producer past block j-3);
 //              owns the TMEM allocation;
-//   warp 11    tcgen05 issuer for O += P V. P (bf16) overwrites the first
-//              Bc/2 columns of its block's S buffer, so an S buffer is reused
-//              once the softmax is done with it and, for a kept block, its
-//              P V has completed.
+//   warp 11    tcgen05 issuer for O += P V, P from its set's TMEM P buffer.
 // With Br = 64 the 128 rows form two independent vote groups that share the
 // MMAs: a group that skips contributes zero rows of P and leaves its running
 // statistics untouched.

@@ -274,3 +274,12 @@ def test_summary_line_legs_stay_compact():
     assert c["dec_a12"]["saved_gb"] == 1.23
     import json
     assert len(json.dumps(c, separators=(",", ":"))) < 1200
+
+
+def test_kernel_hash_ignores_comments():
+    """A traffic record stays valid across comment edits, not code edits."""
+    a = "int f(int x) {  // one\n  /* two\n three */ return x + 1;\n}\n"
+    b = "// header\nint f(int x) {\n\n  return x + 1;   // other\n}\n"
+    c = "int f(int x) {\n  return x + 2;\n}\n"
+    assert bench.code_only(a) == bench.code_only(b)
+    assert bench.code_only(a) != bench.code_only(c)
