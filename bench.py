@@ -467,11 +467,15 @@ def measure_backward(w, lam, steps, warmup, device, stream, flush_buf, pre=None,
 class E2EPipeline:
     """Prefill steps through the public API from pinned host buffers, as a
     serving loop runs them: every step uploads its inputs (Q, K, V) host ->
-    device, runs the prefill call and reads its results (O, lse) back device
-    -> host. An upload stream, the compute stream and a readback stream work
-    over two sets of device buffers, so the upload of step i+1 and the
-    readback of step i-1 overlap the prefill of step i (the PCIe link carries
-    both directions at once). Every step processes the same synthetic batch."""
+    device, runs the prefill and reads its results (O, lse) back device ->
+    host. An upload stream, the compute stream and a readback stream work
+    over two sets of device buffers, and each step goes in chunks of one KV
+    head group (its g query heads and one K / V head; contiguous slices when
+    B = 1), each its own prefill call: the upload of the next chunk and the
+    readback of the previous one overlap the prefill of a chunk (the PCIe
+    link carries both directions at once), so the pipeline fills and drains
+    in one chunk's copies rather than a whole step's. Every step processes
+    the same synthetic batch."""
 
     def __init__(self, w, lam, device, stream):
         import torch
@@ -496,6 +500,11 @@ class E2EPipeline:
         self.down = torch.cuda.Stream(device)
         self.h2d_bytes = (self.hq.numel() + self.hk.numel() + self.hv.numel()) * 2
         self.d2h_bytes = self.host_out[0]["o"].numel() * 2 + self.host_out[0]["lse"].numel() * 4
+        g = w.Hq // w.Hkv
+        # (query heads, KV heads) of each chunk: one KV head group each when the
+        # slices are contiguous (B = 1), else the whole step
+        self.chunks = ([(slice(h * g, (h + 1) * g), slice(h, h + 1)) for h in range(w.Hkv)]
+                       if w.B == 1 else [(slice(0, w.Hq), slice(0, w.Hkv))])
 
     def run(self, n, start_event=None):
         """Enqueue n steps; on return the compute stream waits for the last
@@ -506,35 +515,39 @@ class E2EPipeline:
         if start_event is not None:
             up.wait_event(start_event)
             down.wait_event(start_event)
-        computed = [None, None]  # last prefill that used buffer set b
-        read = [None, None]      # last readback of buffer set b
+        nc = len(self.chunks)
+        computed = [[None] * nc, [None] * nc]  # last prefill of chunk c in buffer set b
+        read = [[None] * nc, [None] * nc]      # last readback of chunk c of set b
         for i in range(n):
             b = i % 2
             d, h = self.dev[b], self.host_out[b]
-            if computed[b] is not None:   # step i-2 has finished reading set b's inputs
-                up.wait_event(computed[b])
-            with torch.cuda.stream(up):
-                d["q"].view(torch.int16).copy_(self.hq, non_blocking=True)
-                d["k"].view(torch.int16).copy_(self.hk, non_blocking=True)
-                d["v"].view(torch.int16).copy_(self.hv, non_blocking=True)
-            uploaded = torch.cuda.Event()
-            uploaded.record(up)
-            stream.wait_event(uploaded)
-            if read[b] is not None:       # step i-2's results have been read back
-                stream.wait_event(read[b])
-            bl.blasst_fwd_ex(d["q"], d["k"], d["v"], d["o"], d["lse"], causal=w.causal,
-                             lam=self.lam, Br=w.Br, Bc=w.Bc, stream=stream)
-            computed[b] = torch.cuda.Event()
-            computed[b].record(stream)
-            down.wait_event(computed[b])
-            with torch.cuda.stream(down):
-                h["o"].copy_(d["o"].view(torch.int16), non_blocking=True)
-                h["lse"].copy_(d["lse"], non_blocking=True)
-            read[b] = torch.cuda.Event()
-            read[b].record(down)
-        for ev in read:
-            if ev is not None:
-                stream.wait_event(ev)
+            for c, (qs, ks) in enumerate(self.chunks):
+                if computed[b][c] is not None:  # step i-2 has finished reading these inputs
+                    up.wait_event(computed[b][c])
+                with torch.cuda.stream(up):
+                    d["q"][:, qs].view(torch.int16).copy_(self.hq[:, qs], non_blocking=True)
+                    d["k"][:, ks].view(torch.int16).copy_(self.hk[:, ks], non_blocking=True)
+                    d["v"][:, ks].view(torch.int16).copy_(self.hv[:, ks], non_blocking=True)
+                uploaded = torch.cuda.Event()
+                uploaded.record(up)
+                stream.wait_event(uploaded)
+                if read[b][c] is not None:      # step i-2's results have been read back
+                    stream.wait_event(read[b][c])
+                bl.blasst_fwd_ex(d["q"][:, qs], d["k"][:, ks], d["v"][:, ks], d["o"][:, qs],
+                                 d["lse"][:, qs], causal=w.causal, lam=self.lam, Br=w.Br,
+                                 Bc=w.Bc, stream=stream)
+                computed[b][c] = torch.cuda.Event()
+                computed[b][c].record(stream)
+                down.wait_event(computed[b][c])
+                with torch.cuda.stream(down):
+                    h["o"][:, qs].copy_(d["o"][:, qs].view(torch.int16), non_blocking=True)
+                    h["lse"][:, qs].copy_(d["lse"][:, qs], non_blocking=True)
+                read[b][c] = torch.cuda.Event()
+                read[b][c].record(down)
+        for evs in read:
+            for ev in evs:
+                if ev is not None:
+                    stream.wait_event(ev)
 
 
 def measure_e2e(w, lam, steps, warmup, device, stream):
@@ -556,8 +569,10 @@ def measure_e2e(w, lam, steps, warmup, device, stream):
     return dict(value=effective_flops(w) / (ms * 1e-3) / 1e12, unit=UNIT, ms=ms,
                 h2d_bytes_per_step=int(pipe.h2d_bytes), d2h_bytes_per_step=int(pipe.d2h_bytes),
                 steps=steps,
-                pipelined=("upload of step i+1 and readback of step i-1 overlap the prefill of "
-                           "step i (three streams, two device buffer sets); fill and drain timed"))
+                chunks=len(pipe.chunks),
+                pipelined=("each step in chunks of one KV head group, one prefill call each: the "
+                           "next chunk's upload and the previous chunk's readback overlap a chunk's "
+                           "prefill (three streams, two device buffer sets); fill and drain timed"))
 
 
 def block_sparse_pattern(w, sink_blocks=1, band_blocks=8, random_frac=0.1, seed=0):
@@ -1131,7 +1146,7 @@ def main():
             peak_source=f"{peaks['source']} bf16_tflops (burst; the kernel is timed alone)",
             algorithmic="per visited (128-row tile, 128-key block): 2*128*128*128 flops for "
                         "S=QK^T, plus the same for O+=PV when the block is computed",
-            e2e_pipelined=e2e.pop("pipelined")))
+            e2e_pipelined=e2e.pop("pipelined"), e2e_chunks_per_step=e2e.pop("chunks")))
         cpu = oracle_sample(w, LAMBDA, args.cpu_budget)
         clocks = clk.summary(head_win)
         l0 = legs["p32k"]
