@@ -259,3 +259,15 @@ def test_python_binding_fails_loudly_without_cuda_tensors():
     with pytest.raises(ValueError):
         bl.attention_prefill(q, q, q)
     del np
+
+
+def test_stats_struct_matches_the_header():
+    """The binding's blasst_stats has the header's fields, in order (the
+    device writes them by offset)."""
+    import dynamic_block_sparse_tiled_b200 as bl
+    hdr = open(HEADER).read()
+    body = re.search(r"typedef struct blasst_stats \{(.*?)\} blasst_stats;", hdr, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"unsigned long long (\w+);", body)
+    assert fields == [f[0] for f in bl.Stats._fields_]
+    assert C.sizeof(bl.Stats) == 8 * len(fields)
